@@ -1,0 +1,311 @@
+"""Pins for the CPU oracle: each check ties the oracle to something other than
+itself -- a hand-derived fixture, a closed form, brute force, an invariant of
+the mathematics, or a library routine."""
+import os
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import oracle as O
+from lfsr_seeded_moe_b200 import synth
+
+GOLD = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _read_rows(name):
+    rows = []
+    with open(os.path.join(GOLD, name)) as f:
+        for line in f:
+            line = line.strip()
+            if line and not line.startswith("#"):
+                rows.append(line)
+    return rows
+
+
+class _M:
+    """A packed matrix as plain NumPy arrays."""
+
+    def __init__(self, seeds, coefs, codes, eb, P):
+        self.seeds, self.coefs, self.codes, self.exp_bias, self.P = seeds, coefs, codes, eb, P
+
+
+# ------------------------------------------------------------------ LFSR
+
+def test_period_is_maximal_and_visits_every_state():
+    # maximal length: from any non-zero seed the register returns after exactly
+    # 65,535 steps, visiting every non-zero state once (the pages search all
+    # 65,535 seeds, so the register must be maximal)
+    s = O.states(1, 65536)
+    assert s[65535] == 1
+    body = s[:65535].astype(np.int64)
+    assert np.all(body != 0)
+    assert len(np.unique(body)) == 65535
+    for seed in (2, 0x1234, 0xFFFF, 0x8000):
+        assert O.lfsr_period(seed) == 65535
+
+
+def test_zero_seed_is_fixed():
+    assert np.all(O.states(0, 40) == 0)
+    assert O.lfsr_period(0) == 0
+
+
+def test_states_match_hand_derivation():
+    rows = [r.split() for r in _read_rows("lfsr_seed1.txt")]
+    want = np.array([int(h, 16) for _, h in rows], np.uint16)
+    assert np.array_equal(O.states(1, len(want)), want)
+
+
+def test_states_are_windows_of_the_output_bit_stream():
+    # s_t = (W >> t) & 0xFFFF where bit 16+k of W is the recurrence
+    # W_k ^ W_{k+2} ^ W_{k+3} ^ W_{k+5} on the bit stream (not register stepping)
+    rng = np.random.default_rng(7)
+    for seed in list(rng.integers(1, 65536, 200)) + [1, 0xFFFF]:
+        bits = [(int(seed) >> i) & 1 for i in range(16)]
+        for k in range(40):
+            bits.append(bits[k] ^ bits[k + 2] ^ bits[k + 3] ^ bits[k + 5])
+        W = sum(b << i for i, b in enumerate(bits))
+        st = O.states(int(seed), 41)
+        for t in range(41):
+            assert int(st[t]) == (W >> t) & 0xFFFF
+
+
+# ----------------------------------------------------------------- basis
+
+def test_basis_fill_order_and_offset_match_hand_blocks():
+    for line in _read_rows("blocks_seed1.txt"):
+        cs, ws = line.split("|")
+        c = [int(v) for v in cs.split()]
+        want = np.array([float(v) for v in ws.split()])
+        got = O.regen_block(1, c, code=15, bias=0)
+        assert np.array_equal(got, want), (c, got, want)
+
+
+def test_basis_values_are_centred_states():
+    U = O.basis(0x1234, 4)
+    st = O.states(0x1234, 33).astype(np.float64)
+    for r in range(8):
+        for j in range(4):
+            assert U[r, j] == (st[1 + 8 * j + r] - 32768.0) / 32768.0
+    assert np.all(U >= -1.0) and np.all(U < 1.0)
+
+
+def test_p3_basis_is_first_three_columns_of_p4():
+    for seed in (1, 77, 0xBEEF, 65535):
+        assert np.array_equal(O.basis(seed, 3), O.basis(seed, 4)[:, :3])
+
+
+def test_regen_is_linear_and_scaled_by_powers_of_two():
+    rng = np.random.default_rng(3)
+    for _ in range(50):
+        seed = int(rng.integers(1, 65536))
+        a = rng.integers(-4, 4, 4)
+        b = rng.integers(-4, 4, 4)
+        wa = O.regen_block(seed, a, 3, -2)
+        wb = O.regen_block(seed, b, 3, -2)
+        assert np.array_equal(O.regen_block(seed, a + b, 3, -2), wa + wb)
+        assert np.array_equal(O.regen_block(seed, a, 4, -2), 2.0 * wa)
+        assert np.array_equal(O.regen_block(seed, a, 0, 1), wa)
+
+
+def test_zero_seed_closed_form():
+    # every state is 0 -> every basis entry is -1 -> w_r = -2^(code+bias) sum(c)
+    for c, code, bias in [((1, 2, 3, 4), 5, -5), ((-8, 7, 0, 1), 15, -12), ((3, -2, 1), 0, 4)]:
+        w = O.regen_block(0, c, code, bias)
+        assert np.all(w == -(2.0 ** (code + bias)) * sum(c))
+
+
+# --------------------------------------------------------------- packing
+
+def test_packed_field_positions():
+    for line in _read_rows("pack_examples.txt"):
+        head, cc, wv = line.split("|")
+        P, coefs, codes, parity, bias = head.split()
+        P, coefs, codes, parity, bias = int(P), int(coefs, 16), int(codes, 16), int(parity), int(bias)
+        want_w = float(wv)
+        nb = 2  # two blocks so both code nibbles exist
+        seeds = np.zeros((1, nb), np.uint16)
+        cf = np.zeros((1, nb), np.uint16)
+        cf[0, parity] = coefs
+        cd = np.array([[codes]], np.uint8) if P == 4 else None
+        m = _M(seeds, cf, cd, np.array([bias], np.int32), P)
+        w = O.decompress(m, np.float64)
+        assert np.all(w[0, 8 * parity: 8 * parity + 8] == want_w), (line, w)
+
+
+def test_bits_per_weight_match_the_published_pack_sizes():
+    # "120.8 B routed expert weights ... 68.0 GB, at 4.5 bits each" (P4) and
+    # 60.4 GB expert bytes for P3 (Qwen3.8-Flash-Next-NanoSeedLM-P4 card, "The family")
+    n_weights = 120.8e9
+    p4 = O.packed_bytes(8, 16 * 1024, 4) - 4 * 8   # streams only
+    p3 = O.packed_bytes(8, 16 * 1024, 3) - 4 * 8
+    bpw4 = p4 * 8 / (8 * 16 * 1024)
+    bpw3 = p3 * 8 / (8 * 16 * 1024)
+    assert bpw4 == 4.5 and bpw3 == 4.0
+    assert round(n_weights * bpw4 / 8 / 1e9, 1) == 68.0
+    assert round(n_weights * bpw3 / 8 / 1e9, 1) == 60.4
+
+
+def test_decompress_is_exact_in_fp32():
+    for P in (3, 4):
+        m = synth.seed_matrix(64, 256, P, (101, P)).numpy()
+        for bias in (-100, -12, 0, 100):
+            m.exp_bias = np.full(64, bias, np.int32)
+            w32 = O.decompress(m, np.float32)
+            w64 = O.decompress(m, np.float64)
+            assert np.array_equal(w32.astype(np.float64), w64)
+
+
+# --------------------------------------------------------------- matvec
+
+@pytest.mark.parametrize("P", [3, 4])
+def test_seed_matvec_equals_dense_fp64_product(P):
+    N, K, M = 96, 512, 3
+    m = synth.seed_matrix(N, K, P, (102, P)).numpy()
+    x = synth.bf16_bits(synth.activations((102, P), M, K)).numpy().view(np.uint16)
+    y = O.seed_matvec(m, x)
+    w = O.decompress(m, np.float64)
+    y_dense = O.dense_matvec(w, O.bf16_to_f64(x))
+    assert np.max(np.abs(y - y_dense)) <= 1e-12 * np.max(np.abs(y_dense))
+
+
+def test_bf16_rounding_matches_torch_rne():
+    rng = np.random.default_rng(11)
+    v = rng.standard_normal(20000).astype(np.float32)
+    # exact ties: low 16 bits 0x8000
+    ties = (rng.integers(0, 2**31, 2000, dtype=np.int64).astype(np.uint32) & 0x7FFF0000) | 0x8000
+    ties = (ties & 0x7F7FFFFF).view(np.float32)
+    v = np.concatenate([v, ties, -ties, np.float32([1.0, -2.5, 3e38, 1e-30])])
+    got = O.f64_to_bf16(v.astype(np.float64))
+    want = torch.from_numpy(v).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    assert np.array_equal(got, want)
+    assert np.array_equal(O.bf16_to_f64(want), torch.from_numpy(want.view(np.int16)).view(torch.bfloat16).double().numpy())
+
+
+def test_bf16_weights_matvec_matches_rounded_dense_product():
+    m = synth.seed_matrix(40, 256, 3, (104,)).numpy()
+    x = np.random.default_rng(1).standard_normal((2, 256))
+    w = O.decompress(m, np.float32)
+    wb = torch.from_numpy(w).to(torch.bfloat16).double().numpy()
+    y = O.seed_matvec_bf16w(m, x)
+    y_ref = x @ wb.T
+    assert np.max(np.abs(y - y_ref)) <= 1e-12 * np.max(np.abs(y_ref))
+
+
+# -------------------------------------------------------------- routing
+
+def test_route_topk_matches_sort_and_softmax():
+    rng = np.random.default_rng(5)
+    logits = rng.standard_normal((50, 100)).astype(np.float32)
+    logits[3, :] = 0.25                      # all tied -> ids 0..7
+    logits[4, 10] = logits[4, 20] = 9.0      # a tie at the top -> 10 before 20
+    ids, w = O.route_topk(logits, 8)
+    for t in range(50):
+        order = np.lexsort((np.arange(100), -logits[t].astype(np.float64)))[:8]
+        assert np.array_equal(ids[t], order)
+        sel = logits[t, order].astype(np.float64)
+        sm = np.exp(sel - sel.max())
+        assert np.allclose(w[t], sm / sm.sum(), rtol=1e-14, atol=0)
+    assert np.array_equal(ids[3], np.arange(8))
+    assert np.allclose(w[3], 1 / 8)
+    assert ids[4, 0] == 10 and ids[4, 1] == 20
+
+
+# ---------------------------------------------------------------- FFN
+
+@pytest.mark.parametrize("mode", [0, 1])
+def test_moe_ffn_equals_dense_composition(mode):
+    E, hidden, inter, P, T, k = 6, 64, 48, 4, 3, 2
+    L = synth.moe_layer(0, E, hidden, inter, P, config=103)
+    g, u, d = (getattr(L, n).numpy() for n in ("gate", "up", "down"))
+    x = synth.bf16_bits(synth.activations((103,), T, hidden)).numpy().view(np.uint16)
+    logits = synth.router_logits((103,), T, E).numpy()
+    ids, w = O.route_topk(logits, k)
+    y = O.moe_ffn(g, u, d, E, hidden, inter, x, ids, w, mode=mode)
+
+    def dense(m):
+        wt = O.decompress(m, np.float64)
+        if mode == 1:
+            wt = torch.from_numpy(wt.astype(np.float32)).to(torch.bfloat16).double().numpy()
+        return wt
+
+    Wg, Wu, Wd = dense(g), dense(u), dense(d)
+    xf = O.bf16_to_f64(x)
+    y_ref = np.zeros((T, hidden))
+    for t in range(T):
+        for q in range(k):
+            e = ids[t, q]
+            gg = Wg[e * inter:(e + 1) * inter] @ xf[t]
+            uu = Wu[e * inter:(e + 1) * inter] @ xf[t]
+            h = gg / (1 + np.exp(-gg)) * uu
+            if mode == 1:
+                h = torch.from_numpy(h.astype(np.float32)).to(torch.bfloat16).double().numpy() \
+                    if np.all(np.abs(h) < 3e38) else h
+            y_ref[t] += w[t, q] * (Wd[e * hidden:(e + 1) * hidden] @ h)
+    tol = 1e-12 if mode == 0 else 1e-2 / 256  # mode 1: h rounded from fp32 vs fp64 may tie-flip
+    assert O.normwise_rel_err(y, y_ref) <= tol
+
+
+def test_silu_closed_forms():
+    assert O.silu(0.0) == 0.0
+    assert abs(O.silu(40.0) - 40.0) < 1e-12
+    assert abs(O.silu(-40.0)) < 1e-15
+    assert abs(O.silu(1.0) - 1.0 / (1.0 + np.exp(-1.0))) < 1e-16
+
+
+def test_layer_stack_chaining_normalises():
+    E, hidden, inter, P, L, k = 4, 32, 16, 4, 3, 2
+    layers = []
+    for li in range(L):
+        m = synth.moe_layer(li, E, hidden, inter, P, config=105)
+        layers.append(tuple(getattr(m, n).numpy() for n in ("gate", "up", "down")))
+    logits = np.stack([synth.router_logits((105, li), 1, E).numpy() for li in range(L)])
+    x0 = synth.bf16_bits(synth.activations((105,), 1, hidden)).numpy().view(np.uint16)
+    y, xs = O.layer_stack(layers, logits, x0, hidden, inter, E, k)
+    assert len(xs) == L and np.array_equal(xs[0], x0)
+    for li in range(1, L):
+        xf = O.bf16_to_f64(xs[li])
+        assert abs(np.sqrt(np.mean(xf * xf)) - 1.0) < 1e-2
+
+
+# --------------------------------------------------------------- search
+
+@pytest.mark.parametrize("P", [3, 4])
+def test_search_recovers_a_planted_block_with_zero_error(P):
+    rng = np.random.default_rng(20 + P)
+    for _ in range(2):
+        seed = int(rng.integers(1, 65536))
+        c = rng.integers(-8, 8, P)
+        c[int(rng.integers(0, P))] |= 1          # an odd entry makes the code identifiable
+        code = int(rng.integers(0, 16))
+        bias = -12
+        w = O.regen_block(seed, c, code, bias)
+        s, cc, cd, err = O.search_block(w, P, bias)
+        assert (s, cd, err) == (seed, code, 0.0)
+        assert np.array_equal(cc, c)
+
+
+def test_search_without_the_planted_seed_has_positive_error():
+    w = O.regen_block(40000, [3, -5, 1, 7], 9, -12)
+    s, c, code, err = O.search_block(w, 4, -12, 1, 39999)
+    assert err > 0 and s != 40000
+
+
+def test_search_matches_brute_force_on_a_tiny_range():
+    # brute force over 32 seeds x 16 codes x all 16^3 coefficient vectors (P=3)
+    rng = np.random.default_rng(9)
+    w = rng.standard_normal(8) * 0.01
+    bias = -12
+    s, c, code, err = O.search_block(w, 3, bias, 100, 131)
+    grid = np.stack(np.meshgrid(*[np.arange(-8, 8)] * 3, indexing="ij"), -1).reshape(-1, 3)
+    best = np.inf
+    for seed in range(100, 132):
+        U = O.basis(seed, 3)
+        V = grid @ U.T                                   # [4096][8]
+        for cd in range(16):
+            e = np.sum((w[None, :] - 2.0 ** (cd + bias) * V) ** 2, axis=1)
+            best = min(best, e.min())
+    # the search rounds least-squares coefficients, so it can only be >= the true optimum;
+    # on random blocks rounding the LS solution is close to optimal
+    assert err >= best - 1e-18
+    assert err <= 4.0 * best
