@@ -1,0 +1,416 @@
+"""Benchmark of the seed-decompress MoE decode path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--batch T] [--impl ours|reference]
+
+A step is one decode step of T tokens (default 1) through a 45-layer stack of
+seed-packed MoE layers (100 experts per layer, hidden 2048, expert
+intermediate 1408, P=4, top-8 routing from N(0,1) logits): per layer routing,
+gate/up + SiLU, down + weighted sum, then the RMS chaining into the next
+layer, all through the library's C ABI (nslm_moe_stack_decode) captured in a
+CUDA graph.  The 21.9 GB of packed experts stay resident in HBM; a token reads
+1.75 GB of them, far more than the 126 MB L2, so no flush is needed.
+
+The JSON line also carries the seed-GEMV sweep (packed-byte GB/s per expert
+shape, rotating copies to defeat L2), a roofline object for the per-layer
+decode FFN, the end-to-end number through the C ABI with host buffers, the
+clocks seen during the timed region and the CPU oracle's time on a sample.
+
+--impl reference times the CPU oracle (the plain C definition of the method)
+on this host's cores on a bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+E, HIDDEN, INTER, P, K_TOP, LAYERS = 100, 2048, 1408, 4, 8, 45
+WORKLOAD = "45-layer seed-expert MoE decode: 100 experts/layer, hidden 2048, inter 1408, P=4, top-8"
+METRIC = "MoE seed-FFN decode tokens/s"
+GEMV_METRIC = "seed-GEMV packed-byte HBM GB/s (% of peak)"
+GEMV_SHAPES = [(2048, 4096), (4096, 2048), (1408, 2048), (2048, 1408)]
+FALLBACK_HBM_GBS = 6650.0
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        d = json.load(open(path))
+        return float(d["hbm_gbs"]), "measured"
+    return FALLBACK_HBM_GBS, "fallback"
+
+
+def layer_packed_bytes_per_token() -> int:
+    per_expert = 2 * (INTER * (HIDDEN // 8) * 4.5 + 4 * INTER) + (HIDDEN * (INTER // 8) * 4.5 + 4 * HIDDEN)
+    return int(K_TOP * per_expert)
+
+
+# ------------------------------------------------------------------ clocks
+
+class ClockSampler:
+    """Samples SM clocks and throttle reasons with nvidia-smi while running."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except OSError:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx = float(parts[2])
+            except ValueError:
+                continue
+            for nm, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(nm)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": mx, "reasons": [], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# --------------------------------------------------------------- oracle leg
+
+def oracle_layer_seconds(n_layers: int, T: int = 1, seed_tag: int = 0):
+    """Time the CPU oracle on n_layers decode layers of T tokens (routed experts only)."""
+    import numpy as np
+
+    from lfsr_seeded_moe_b200 import synth
+    from oracle import oracle as O
+
+    total = 0.0
+    for li in range(n_layers):
+        logits = synth.router_logits((4, li, seed_tag), T, E).numpy()
+        ids, w = O.route_topk(logits, K_TOP)
+        experts = sorted(set(int(e) for e in ids.reshape(-1)))
+        # a compact stack with only the routed experts, drawn on the host
+        remap = {e: i for i, e in enumerate(experts)}
+        sl = [synth.expert_slice(li, e, E, HIDDEN, INTER, P, config=4) for e in experts]
+
+        def stack(name):
+            class _S:
+                pass
+            s = _S()
+            parts = [getattr(x, name).numpy() for x in sl]
+            s.seeds = np.concatenate([q.seeds for q in parts])
+            s.coefs = np.concatenate([q.coefs for q in parts])
+            s.codes = np.concatenate([q.codes for q in parts])
+            s.exp_bias = np.concatenate([q.exp_bias for q in parts])
+            s.P = P
+            return s
+
+        g, u, d = stack("gate"), stack("up"), stack("down")
+        x = synth.bf16_bits(synth.activations((4, seed_tag), T, HIDDEN)).numpy().view(np.uint16)
+        ids_c = np.vectorize(lambda e: remap[int(e)])(ids).astype(np.int32)
+        t0 = time.perf_counter()
+        O.moe_ffn(g, u, d, len(experts), HIDDEN, INTER, x, ids_c, w, mode=0)
+        total += time.perf_counter() - t0
+    return total
+
+
+def cpu_baseline(budget_s: float = 15.0, T: int = 1):
+    from oracle import oracle as O
+
+    t1 = oracle_layer_seconds(1, T, seed_tag=1)
+    n = max(1, min(LAYERS, int(budget_s / max(t1, 1e-3))))
+    t = oracle_layer_seconds(n, T, seed_tag=2) if n > 1 else t1
+    per_layer = t / n
+    tok_s = T / (per_layer * LAYERS)
+    return {"value": tok_s, "unit": "tokens/s", "cores": O.threads_used(), "kind": "oracle",
+            "sample": f"{n} layer(s) x {T} token(s) of the 45-layer stack, oracle fp64, scaled to 45 layers "
+                      f"({per_layer:.3f} s per layer)"}
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    from oracle import oracle as O
+
+    T = args.batch
+    for _ in range(args.warmup):
+        oracle_layer_seconds(1, T, seed_tag=100)
+    times = [oracle_layer_seconds(1, T, seed_tag=200 + i) for i in range(args.steps)]
+    per_layer = sum(times) / len(times)
+    tok_s = T / (per_layer * LAYERS)
+    line = {
+        "impl": "reference", "metric": METRIC, "value": tok_s, "unit": "tokens/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": per_layer * LAYERS * 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded SplitMix64 fields)",
+        "config": {"workload": WORKLOAD, "batch_tokens": T, "layers": LAYERS,
+                   "sample": "each step: one layer of the stack on the CPU oracle, scaled x45"},
+        "cpu_baseline": {"value": tok_s, "unit": "tokens/s", "cores": O.threads_used(), "kind": "oracle",
+                         "sample": f"{args.steps} step(s) of one decode layer, scaled to 45 layers"},
+        "e2e": {"value": tok_s, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line))
+    return 0
+
+
+# ------------------------------------------------------------------- GPU leg
+
+def gemv_sweep(torch, nslm, synth, dev, hbm):
+    out = []
+    for Pv in (4, 3):
+        for (N, K) in GEMV_SHAPES:
+            m0 = synth.seed_matrix(N, K, Pv, (11, N, K, Pv), device=dev)
+            nbytes = m0.packed_bytes()
+            ncopy = min(400, max(2, int(4 * 126e6 // nbytes) + 1))
+            mats = [synth.seed_matrix(N, K, Pv, (11, N, K, Pv, c), device=dev) for c in range(ncopy)]
+            structs = [nslm.matrix(m) for m in mats]
+            x = synth.activations((11,), 1, K).to(dev)
+            y = torch.empty(1, N, device=dev)
+            nslm.nslm_seed_gemv(structs[0], x, 1, y)
+            torch.cuda.synchronize()
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g):
+                for c in range(ncopy):
+                    nslm.nslm_seed_gemv(structs[c], x, 1, y)
+            for _ in range(3):
+                g.replay()
+            torch.cuda.synchronize()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            reps = 5
+            e0.record()
+            for _ in range(reps):
+                g.replay()
+            e1.record()
+            torch.cuda.synchronize()
+            t = e0.elapsed_time(e1) * 1e-3 / (reps * ncopy)
+            gbs = nbytes / t / 1e9
+            out.append({"P": Pv, "N": N, "K": K, "us": round(t * 1e6, 3), "GB_s": round(gbs, 1),
+                        "pct_of_hbm": round(100 * gbs / hbm, 2), "weights_per_s": N * K / t})
+            del g, mats, structs
+            torch.cuda.empty_cache()
+    return out
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--batch", type=int, default=1, help="decode tokens per step (1..8)")
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-gemv", action="store_true")
+    ap.add_argument("--no-cpu", action="store_true")
+    args = ap.parse_args()
+    if args.impl == "reference":
+        return run_reference(args)
+
+    import torch
+    import torch.distributed as dist
+
+    from lfsr_seeded_moe_b200 import nslm, synth
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    hbm, peak_kind = peaks()
+    T = args.batch
+
+    # --- resident expert stack (each rank holds its own replica)
+    layers = [synth.moe_layer(l, E, HIDDEN, INTER, P, device=dev, config=4) for l in range(LAYERS)]
+    arr = nslm.moe_layers([(L.gate, L.up, L.down) for L in layers])
+    S = 8  # distinct step inputs, cycled
+    logits = [torch.stack([synth.router_logits((4, l, rank, s), T, E) for l in range(LAYERS)]).to(dev).contiguous()
+              for s in range(S)]
+    xs = [synth.activations((4, rank, s), T, HIDDEN).to(dev).contiguous() for s in range(S)]
+    y = torch.empty(T, HIDDEN, device=dev)
+    wsb = nslm.nslm_workspace_bytes(nslm.NSLM_OP_MOE_STACK, T, E, HIDDEN, INTER, K_TOP, LAYERS)
+    ws = torch.empty(wsb, dtype=torch.uint8, device=dev)
+
+    cs = torch.cuda.Stream()
+    graphs = []
+    with torch.cuda.stream(cs):
+        nslm.nslm_moe_stack_decode(arr, LAYERS, E, K_TOP, logits[0], xs[0], T, y, ws, wsb, stream=cs)
+        launches_per_step = nslm.nslm_last_launch_count()
+    torch.cuda.synchronize()
+    for s in range(S):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            nslm.nslm_moe_stack_decode(arr, LAYERS, E, K_TOP, logits[s], xs[s], T, y, ws, wsb)
+        graphs.append(g)
+
+    for i in range(max(3, args.warmup)):
+        graphs[i % S].replay()
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(dev.index if dev.index is not None else 0) as clk:
+        torch.cuda.synchronize()
+        e0.record()
+        for i in range(args.steps):
+            graphs[i % S].replay()
+        e1.record()
+        torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    elapsed = e0.elapsed_time(e1) * 1e-3
+    if world > 1:
+        t = torch.tensor([elapsed], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        elapsed = float(t.item())
+    value = world * args.steps * T / elapsed
+
+    # --- end to end through the C ABI: pinned host inputs in, result out, every step
+    hx = [x.cpu().pin_memory() for x in xs]
+    hl = [lg.cpu().pin_memory() for lg in logits]
+    hy = torch.empty(T, HIDDEN, dtype=torch.float32).pin_memory()
+    dx = torch.empty_like(xs[0])
+    dl = torch.empty_like(logits[0])
+    h2d = hx[0].numel() * hx[0].element_size() + hl[0].numel() * hl[0].element_size()
+    d2h = hy.numel() * hy.element_size()
+    for i in range(3):
+        dx.copy_(hx[i % S], non_blocking=True)
+        dl.copy_(hl[i % S], non_blocking=True)
+        nslm.nslm_moe_stack_decode(arr, LAYERS, E, K_TOP, dl, dx, T, y, ws, wsb)
+        hy.copy_(y, non_blocking=True)
+    torch.cuda.synchronize()
+    f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    f0.record()
+    for i in range(args.steps):
+        dx.copy_(hx[i % S], non_blocking=True)
+        dl.copy_(hl[i % S], non_blocking=True)
+        nslm.nslm_moe_stack_decode(arr, LAYERS, E, K_TOP, dl, dx, T, y, ws, wsb)
+        hy.copy_(y, non_blocking=True)
+    f1.record()
+    torch.cuda.synchronize()
+    e2e_t = f0.elapsed_time(f1) * 1e-3
+    if world > 1:
+        t = torch.tensor([e2e_t], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_t = float(t.item())
+    e2e = {"value": world * args.steps * T / e2e_t, "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+           "d2h_bytes_per_step": d2h}
+
+    # --- roofline: the per-layer decode FFN (route-plan + gate/up + down launches)
+    ids = torch.empty(T, K_TOP, dtype=torch.int32, device=dev)
+    wts = torch.empty(T, K_TOP, device=dev)
+    nslm.nslm_moe_route_topk(logits[0][0], T, E, K_TOP, ids, wts)
+    fsb = nslm.nslm_workspace_bytes(nslm.NSLM_OP_MOE_FFN, T, E, HIDDEN, INTER, K_TOP)
+    fws = torch.empty(fsb, dtype=torch.uint8, device=dev)
+    st = [(nslm.matrix(L.gate), nslm.matrix(L.up), nslm.matrix(L.down)) for L in layers]
+    nreps = 4 * LAYERS
+    g = torch.cuda.CUDAGraph()
+    torch.cuda.synchronize()
+    with torch.cuda.graph(g):
+        for i in range(nreps):
+            nslm.nslm_moe_seed_ffn(*st[i % LAYERS], E, xs[0], ids, wts, T, K_TOP, y, fws, fsb)
+    g.replay()
+    torch.cuda.synchronize()
+    r0, r1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    r0.record()
+    g.replay()
+    r1.record()
+    torch.cuda.synchronize()
+    layer_s = r0.elapsed_time(r1) * 1e-3 / nreps
+    # distinct experts read per layer (T tokens may share experts)
+    uniq = len(set(ids.cpu().numpy().reshape(-1).tolist()))
+    per_expert = layer_packed_bytes_per_token() / K_TOP
+    layer_bytes = int(uniq * per_expert)
+    achieved = layer_bytes / layer_s / 1e9
+    traffic = None
+    tr_path = os.path.join(ROOT, "profiles", "ffn_decode_layer_traffic.txt")
+    if os.path.exists(tr_path) and T == 1:
+        for ln in open(tr_path):
+            if ln.startswith("dram_bytes_per_layer_call:"):
+                try:
+                    traffic = int(ln.split(":")[1].split()[0])
+                except ValueError:
+                    traffic = None
+    roofline = {"bound": "hbm", "kernel": "decode FFN layer (route-plan + gate/up + down)",
+                "achieved": round(achieved, 1), "peak": hbm, "unit": "GB/s",
+                "frac": round(achieved / hbm, 4), "traffic": traffic,
+                "algorithmic_bytes_per_launch": layer_bytes, "us_per_launch": round(layer_s * 1e6, 3),
+                "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)" if peak_kind == "measured" else "fallback"}
+    del g
+    torch.cuda.empty_cache()
+
+    gemv = None
+    if not args.no_gemv:
+        gemv = {"metric": GEMV_METRIC, "shapes": gemv_sweep(torch, nslm, synth, dev, hbm),
+                "note": "batch 1, each shape timed over rotating copies (> 4x L2) in a CUDA graph"}
+
+    line = {
+        "metric": METRIC, "value": round(value, 2), "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(elapsed / args.steps * 1e3, 4),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+        "data": "synthetic (seeded SplitMix64 packed fields, bf16 N(0,1) activations, N(0,1) router logits)",
+        "config": {"workload": WORKLOAD, "batch_tokens": T, "layers": LAYERS, "experts": E,
+                   "hidden": HIDDEN, "inter": INTER, "P": P, "top_k": K_TOP,
+                   "packed_GB_resident": round(sum(L.gate.packed_bytes() + L.up.packed_bytes() + L.down.packed_bytes()
+                                                   for L in layers) / 1e9, 3),
+                   "l2": "inputs larger than L2 (1.75 GB of weights read per token)",
+                   "parallelism": f"replicas x{world}", "graph": "one CUDA graph per step"},
+        "clocks": clk.summary(),
+        "e2e": e2e,
+        "gpu_launches": launches_per_step * args.steps,
+        "roofline": roofline,
+    }
+    if gemv is not None:
+        line["gemv"] = gemv
+    if rank == 0 and world == 1 and not args.no_cpu:
+        line["cpu_baseline"] = cpu_baseline()
+    if rank == 0:
+        print(json.dumps(line))
+    graphs.clear()
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

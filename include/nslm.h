@@ -1,0 +1,176 @@
+/*
+ * nslm.h -- C ABI of libnslm, a B200 (sm_100a) library for SeedLM
+ * seed-decompress matrix multiplies on routed mixture-of-experts layers.
+ *
+ * The method (sources, by page title and section):
+ *  - "NanoSeedLM: LLM inference using pseudo-random numbers" (barnson.org),
+ *    "Where this started": a weight matrix is cut into blocks of 8 weights;
+ *    each block is a 16-bit LFSR seed, P tiny int4 coefficients and a shared
+ *    exponent; running the LFSR from the seed gives an 8 x P basis U and the
+ *    block is 2^e * U * c.  "What I changed: September 2026": the seed is the
+ *    initial register state, and the weights are rebuilt inside the GPU
+ *    kernels, in registers, every time (never decompressed to memory).
+ *  - "K2-Horizon-MoVA-36B-A4B -- NanoSeedLM p4mx-q4v", "This upload": the
+ *    tensors NAME.seeds (U16), NAME.coefs (U16), NAME.codes (U8) and
+ *    NAME.exp_bias (I32); 100 routed FFN experts per layer, P = 4.
+ *  - "Qwen3.8-Flash-Next-NanoSeedLM-P4", "The family": P = 4 costs 4.5 bits
+ *    per weight, P = 3 costs 4.0 bits per weight.
+ *
+ * Definitions the pages leave open, fixed by this library:
+ *  - LFSR: 16-bit Fibonacci register, polynomial x^16 + x^14 + x^13 + x^11 + 1;
+ *    a step shifts right by one and enters s0^s2^s3^s5 at bit 15.
+ *  - Basis: U[r][j] = (s_{1+8j+r} - 32768) / 32768, where s_0 is the seed and
+ *    s_t the state after t steps; r = 0..7 (weight), j = 0..P-1 (coefficient).
+ *  - Block: w_r = 2^(code + exp_bias[row]) * sum_j c_j U[r][j]; c_j is a
+ *    two's-complement nibble in [-8, 7]; code an unsigned nibble in [0, 15].
+ *    Every such weight is exactly representable in fp32.
+ *  - Packed layout of an N x K matrix (nb = K / 8 blocks per row, row-major,
+ *    little-endian), block b of row i covering W[i][8b .. 8b+7]:
+ *      seeds    uint16 [N][nb]
+ *      coefs    uint16 [N][nb]   c_j in bits 4j..4j+3; for P = 3 the exponent
+ *                                code is in bits 12..15
+ *      codes    uint8  [N][nb/2] P = 4 only: block 2m's code in the low
+ *                                nibble of byte m, block 2m+1's in the high
+ *                                nibble; NULL for P = 3
+ *      exp_bias int32  [N]       must lie in [-100, 100]
+ *
+ * Conventions for every entry point:
+ *  - Every pointer is a DEVICE pointer unless its comment says HOST.  The
+ *    caller owns every buffer, the workspace included; the library never
+ *    allocates, frees or synchronises.  All work is enqueued on `stream`
+ *    (a cudaStream_t; NULL means the legacy default stream) and completes
+ *    asynchronously.
+ *  - Arguments are checked on the host before anything is launched; a bad
+ *    argument returns a negative status and launches nothing.  A launch
+ *    failure returns NSLM_ERR_CUDA (the CUDA error is consumed).
+ *  - Device arrays must be 16-byte aligned; K must be a multiple of 16 for
+ *    P = 4 and of 8 for P = 3.
+ *  - No function prints, aborts or throws.
+ */
+#ifndef NSLM_H
+#define NSLM_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* A cudaStream_t, declared without the CUDA headers. */
+typedef struct CUstream_st *nslm_stream_t;
+
+/* Status codes. */
+#define NSLM_OK 0
+#define NSLM_ERR_ARG (-1)         /* null pointer, bad enum or count */
+#define NSLM_ERR_ALIGN (-2)       /* a device pointer is not 16-byte aligned */
+#define NSLM_ERR_SHAPE (-3)       /* N, K, P or a size outside what is supported */
+#define NSLM_ERR_WORKSPACE (-4)   /* workspace missing or smaller than required */
+#define NSLM_ERR_CUDA (-5)        /* a CUDA call or launch failed */
+#define NSLM_ERR_UNSUPPORTED (-7) /* the current device is not sm_100 */
+
+/* One packed seed matrix (see the layout above).  For a stack of E experts,
+ * N = E * rows and expert e owns rows [e * rows, (e + 1) * rows). */
+typedef struct {
+    const uint16_t *seeds;
+    const uint16_t *coefs;
+    const uint8_t *codes;    /* NULL when P == 3 */
+    const int32_t *exp_bias;
+    int32_t N;
+    int32_t K;
+    int32_t P;               /* 3 or 4 */
+} nslm_seed_matrix;
+
+/* One MoE layer: gate and up are [E * inter][hidden], down is [E * hidden][inter]. */
+typedef struct {
+    nslm_seed_matrix gate;
+    nslm_seed_matrix up;
+    nslm_seed_matrix down;
+} nslm_moe_layer;
+
+/* Workspace sizing: op codes for nslm_workspace_bytes. */
+#define NSLM_OP_GEMV 0
+#define NSLM_OP_GROUPED_GEMM 1
+#define NSLM_OP_MOE_FFN 2
+#define NSLM_OP_MOE_STACK 3
+
+/* Bytes of workspace an operation needs (0 if none).  T = tokens, E =
+ * experts, hidden/inter = FFN sizes, k = experts per token, L = layers (only
+ * NSLM_OP_MOE_STACK uses L; pass 0 otherwise).  Host-only, never fails. */
+size_t nslm_workspace_bytes(int32_t op, int32_t T, int32_t E, int32_t hidden,
+                            int32_t inter, int32_t k, int32_t L);
+
+/* Seed GEMV, the decode matrix-vector product ("Where this started": the
+ * weights are regenerated from the seeds inside the multiply).
+ *   y[m][i] = sum_k W[i][k] * x[m][k],  m < M, i < N.
+ * x: bf16 bit patterns [M][K]; y: fp32 [M][N]; 1 <= M <= 8.
+ * Accumulates in fp32; results match the fp64 product to about 1e-6
+ * relative.  Uses no workspace (ws may be NULL). */
+int32_t nslm_seed_gemv(const nslm_seed_matrix *W, const uint16_t *x_bf16, int32_t M,
+                       float *y, void *ws, size_t ws_bytes, nslm_stream_t stream);
+
+/* Grouped seed GEMM over stacked experts, the batched (prefill) product of
+ * "Qwen3.8-Flash-Next" prompt processing ("The prompt time ... the grouped
+ * expert GEMMs", NanoSeedLM documentation index, Results).
+ *   For every expert e and every row t in [offsets[e], offsets[e+1]):
+ *     y[t][i] = sum_k W_e[i][k] * x[t][k],  i < rows = W->N / E.
+ * x: bf16 [R][K], rows grouped by expert; offsets: int32 [E + 1] (DEVICE),
+ * non-decreasing, offsets[0] = 0, offsets[E] = R; y: fp32 [R][rows].
+ * Weights are regenerated into bf16 (round to nearest even) tiles and
+ * multiplied on the tensor cores with fp32 accumulation.
+ * Workspace: nslm_workspace_bytes(NSLM_OP_GROUPED_GEMM, R, E, K, rows, 1, 0). */
+int32_t nslm_seed_grouped_gemm(const nslm_seed_matrix *W, int32_t E, const uint16_t *x_bf16,
+                               const int32_t *offsets, int32_t R, float *y, void *ws,
+                               size_t ws_bytes, nslm_stream_t stream);
+
+/* Router: for each token, the k largest of E logits (descending; ties go to
+ * the lower expert id) and the softmax of the k selected logits.
+ * logits: fp32 [T][E]; ids: int32 [T][k]; w: fp32 [T][k]; 1 <= k <= 8,
+ * k <= E <= 1024.  ("Why K2-Horizon-MoVA": 100 routed experts, top 8.) */
+int32_t nslm_moe_route_topk(const float *logits, int32_t T, int32_t E, int32_t k,
+                            int32_t *ids, float *w, nslm_stream_t stream);
+
+/* Routed expert FFN for T tokens ("Why K2-Horizon-MoVA": routed FFN experts,
+ * top 8; gate and up projections, SiLU, down projection):
+ *   y[t] = sum_q w[t][q] * Down_e( SiLU(Gate_e x[t]) * (Up_e x[t]) ),  e = ids[t][q]
+ * with SiLU(g) = g / (1 + exp(-g)).  gate/up: [E * inter][hidden];
+ * down: [E * hidden][inter], all with the same P.  x: bf16 [T][hidden];
+ * ids: int32 [T][k] in [0, E); w: fp32 [T][k]; y: fp32 [T][hidden].
+ * T <= 8 runs the decode path (fp32 weights and hidden activations);
+ * larger T runs the tensor-core path (bf16 weights, bf16 hidden activation).
+ * Workspace: nslm_workspace_bytes(NSLM_OP_MOE_FFN, T, E, hidden, inter, k, 0). */
+int32_t nslm_moe_seed_ffn(const nslm_seed_matrix *gate, const nslm_seed_matrix *up,
+                          const nslm_seed_matrix *down, int32_t E, const uint16_t *x_bf16,
+                          const int32_t *ids, const float *w, int32_t T, int32_t k, float *y,
+                          void *ws, size_t ws_bytes, nslm_stream_t stream);
+
+/* A stack of L MoE layers for T <= 8 decode tokens.  Layer l routes with
+ * logits[l] (fp32 [L][T][E]) and runs nslm_moe_seed_ffn on its input; the
+ * next layer's input is bf16(y / sqrt(mean(y^2) + 1e-6)) per token (the pages
+ * put attention between MoE layers; this normalisation stands in for it).
+ * layers: HOST array of L layers (device pointers inside), all with the same
+ * E, hidden, inter and P.  x0: bf16 [T][hidden]; y: fp32 [T][hidden], the
+ * last layer's output.
+ * Workspace: nslm_workspace_bytes(NSLM_OP_MOE_STACK, T, E, hidden, inter, k, L). */
+int32_t nslm_moe_stack_decode(const nslm_moe_layer *layers, int32_t L, int32_t E, int32_t k,
+                              const float *logits, const uint16_t *x0_bf16, int32_t T,
+                              float *y, void *ws, size_t ws_bytes, nslm_stream_t stream);
+
+/* Test exports: the regenerated weights themselves, written out densely.
+ * w_out: fp32 [N][K] (exact) or bf16 bit patterns [N][K] (round to nearest
+ * even of the exact value).  Not on the hot path. */
+int32_t nslm_debug_decompress(const nslm_seed_matrix *W, float *w_out, nslm_stream_t stream);
+int32_t nslm_debug_decompress_bf16(const nslm_seed_matrix *W, uint16_t *w_out,
+                                   nslm_stream_t stream);
+
+/* A static, human-readable name for a status code. */
+const char *nslm_status_string(int32_t status);
+
+/* Number of kernel launches the last successful call on this host thread
+ * enqueued (for accounting in benchmarks). */
+int32_t nslm_last_launch_count(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* NSLM_H */

@@ -1,0 +1,302 @@
+// abi.cu -- host-side validation, workspace sizing and the remaining C entry
+// points of libnslm (routing, expert FFN, layer stack, debug decompression).
+#include <algorithm>
+#include <mutex>
+#include <numeric>
+
+#include "chunk.cuh"
+#include "common.cuh"
+#include "moe.cuh"
+
+namespace nslm {
+
+thread_local int32_t g_launches = 0;
+
+namespace {
+constexpr int kMaxDevices = 64;
+int g_cc_major[kMaxDevices];  // 0 = not queried yet
+int g_sms[kMaxDevices];
+struct SmemEntry {
+  const void *kernel;
+  int device;
+  size_t bytes;
+};
+SmemEntry g_smem[256];
+int g_smem_n = 0;
+std::mutex g_mu;
+
+int current_device() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return -1;
+  return dev;
+}
+}  // namespace
+
+int32_t check_device() {
+  const int dev = current_device();
+  if (dev < 0 || dev >= kMaxDevices) return cuda_status(cudaErrorNoDevice);
+  if (g_cc_major[dev] == 0) {
+    int major = 0, sms = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+      return cuda_status(cudaErrorNoDevice);
+    g_sms[dev] = sms;
+    g_cc_major[dev] = major;
+  }
+  return g_cc_major[dev] == 10 ? NSLM_OK : NSLM_ERR_UNSUPPORTED;
+}
+
+int32_t num_sms() {
+  const int dev = current_device();
+  if (dev < 0 || dev >= kMaxDevices) return 148;
+  if (g_cc_major[dev] == 0) check_device();
+  return g_sms[dev] > 0 ? g_sms[dev] : 148;
+}
+
+int32_t ensure_smem(const void *kernel, size_t bytes) {
+  if (bytes <= 48 * 1024) return NSLM_OK;
+  const int dev = current_device();
+  std::lock_guard<std::mutex> lock(g_mu);
+  for (int i = 0; i < g_smem_n; ++i)
+    if (g_smem[i].kernel == kernel && g_smem[i].device == dev && g_smem[i].bytes >= bytes) return NSLM_OK;
+  const int32_t st = cuda_status(
+      cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes));
+  if (st) return st;
+  for (int i = 0; i < g_smem_n; ++i)
+    if (g_smem[i].kernel == kernel && g_smem[i].device == dev) {
+      g_smem[i].bytes = bytes;
+      return NSLM_OK;
+    }
+  if (g_smem_n < 256) g_smem[g_smem_n++] = SmemEntry{kernel, dev, bytes};
+  return NSLM_OK;
+}
+
+int32_t check_matrix(const nslm_seed_matrix *W) {
+  if (!W) return NSLM_ERR_ARG;
+  if (W->P != 3 && W->P != 4) return NSLM_ERR_SHAPE;
+  if (W->N < 0 || W->K <= 0) return NSLM_ERR_SHAPE;
+  if (W->K % (W->P == 4 ? 16 : 8) != 0) return NSLM_ERR_SHAPE;
+  if (W->N > 0) {
+    if (!W->seeds || !W->coefs || !W->exp_bias) return NSLM_ERR_ARG;
+    if (W->P == 4 && !W->codes) return NSLM_ERR_ARG;
+    if (!aligned16(W->seeds) || !aligned16(W->coefs) || !aligned16(W->exp_bias)) return NSLM_ERR_ALIGN;
+    if (W->P == 4 && !aligned16(W->codes)) return NSLM_ERR_ALIGN;
+  }
+  return NSLM_OK;
+}
+
+ChunkLayout chunk_layout(int32_t K, int32_t N, int32_t target_ctas, int32_t max_threads) {
+  ChunkLayout L{};
+  const int nb = K / 8;
+  L.C = ceil_div(nb, 8);
+  // candidates: Cpad = C (rows a multiple of 32/gcd), or C rounded up to a
+  // multiple of 8 or of 32; pick the least idle lanes that still gives at
+  // least target_ctas row groups, else the most row groups
+  int best_cpad = -1, best_r = 0;
+  double best_score = -1e30;
+  const int cands[3] = {L.C, ceil_div(L.C, 8) * 8, ceil_div(L.C, 32) * 32};
+  for (int cpad : cands) {
+    int rmin = 32 / std::gcd(cpad, 32);
+    if (rmin * cpad > 1024) continue;
+    int r = rmin;
+    while (r * 2 * cpad <= max_threads && ceil_div(N, r * 2) >= target_ctas) r *= 2;
+    const double idle = double(cpad - L.C) / cpad;
+    const int groups = ceil_div(std::max(N, 1), r);
+    const double fill = std::min(1.0, double(groups) / target_ctas);
+    const double score = fill * (1.0 - idle);
+    if (score > best_score + 1e-9) { best_score = score; best_cpad = cpad; best_r = r; }
+  }
+  if (best_cpad < 0) { best_cpad = ceil_div(L.C, 32) * 32; best_r = 1; }
+  L.Cpad = best_cpad;
+  L.R = best_r;
+  L.threads = L.R * L.Cpad;
+  return L;
+}
+
+// --------------------------------------------------------- debug kernels
+
+template <int P>
+__global__ void decompress_kernel(const nslm_seed_matrix W, float *w32, uint16_t *wbf) {
+  __shared__ StreamTables tab;
+  build_stream_tables(&tab);
+  __syncthreads();
+  const int nb = W.K / 8;
+  const size_t nblk = (size_t)W.N * nb;
+  for (size_t b = (size_t)blockIdx.x * blockDim.x + threadIdx.x; b < nblk;
+       b += (size_t)gridDim.x * blockDim.x) {
+    const size_t row = b / nb, col = b - row * nb;
+    const uint32_t seed = W.seeds[b];
+    const uint32_t q = W.coefs[b];
+    uint32_t lo, hi;
+    stream_word(&tab, seed, lo, hi);
+    float F[8];
+    block_ints(lo, hi, coef_bytes<P>(q), F);
+    uint32_t code;
+    if (P == 4) code = (W.codes[row * (nb / 2) + col / 2] >> (4 * (col & 1))) & 0xFu;
+    else code = q >> 12;
+    const float scale = block_scale(code, row_scale_key(W.exp_bias[row]));
+    const size_t base = row * (size_t)W.K + col * 8;
+#pragma unroll
+    for (int r = 0; r < 8; ++r) {
+      const float w = F[r] * scale;  // exact: a 21-bit integer times a power of two
+      if (w32) w32[base + r] = w;
+      if (wbf) wbf[base + r] = __bfloat16_as_ushort(__float2bfloat16_rn(w));
+    }
+  }
+}
+
+static int32_t decompress(const nslm_seed_matrix *W, float *w32, uint16_t *wbf, nslm_stream_t stream) {
+  g_launches = 0;
+  int32_t st = check_matrix(W);
+  if (st) return st;
+  if (!w32 && !wbf) return NSLM_ERR_ARG;
+  if ((st = check_device())) return st;
+  if (W->N == 0) return NSLM_OK;
+  const size_t nblk = (size_t)W->N * (W->K / 8);
+  const int threads = 256;
+  const int grid = (int)std::min<size_t>((nblk + threads - 1) / threads, (size_t)num_sms() * 8);
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (W->P == 4) decompress_kernel<4><<<grid, threads, 0, s>>>(*W, w32, wbf);
+  else decompress_kernel<3><<<grid, threads, 0, s>>>(*W, w32, wbf);
+  st = launch_status();
+  if (st == NSLM_OK) g_launches = 1;
+  return st;
+}
+
+}  // namespace nslm
+
+using namespace nslm;
+
+extern "C" {
+
+const char *nslm_status_string(int32_t status) {
+  switch (status) {
+    case NSLM_OK: return "ok";
+    case NSLM_ERR_ARG: return "invalid argument";
+    case NSLM_ERR_ALIGN: return "device pointer not 16-byte aligned";
+    case NSLM_ERR_SHAPE: return "unsupported shape";
+    case NSLM_ERR_WORKSPACE: return "workspace missing or too small";
+    case NSLM_ERR_CUDA: return "CUDA error";
+    case NSLM_ERR_UNSUPPORTED: return "device is not sm_100";
+    default: return "unknown status";
+  }
+}
+
+int32_t nslm_last_launch_count(void) { return g_launches; }
+
+size_t nslm_workspace_bytes(int32_t op, int32_t T, int32_t E, int32_t hidden, int32_t inter,
+                            int32_t k, int32_t L) {
+  (void)E;
+  (void)hidden;
+  switch (op) {
+    case NSLM_OP_GEMV: return 0;
+    case NSLM_OP_GROUPED_GEMM: return 0;
+    case NSLM_OP_MOE_FFN:
+      if (T <= kMaxT)
+        return ffn_workspace(nullptr, std::max(T, 1), std::max(k, 1), std::max(hidden, 0),
+                             std::max(inter, 0), 1).bytes;
+      return 0;
+    case NSLM_OP_MOE_STACK:
+      return ffn_workspace(nullptr, std::max(T, 1), std::max(k, 1), std::max(hidden, 0),
+                           std::max(inter, 0), std::max(L, 1)).bytes;
+    default: return 0;
+  }
+}
+
+int32_t nslm_debug_decompress(const nslm_seed_matrix *W, float *w_out, nslm_stream_t stream) {
+  if (!w_out) return NSLM_ERR_ARG;
+  return decompress(W, w_out, nullptr, stream);
+}
+
+int32_t nslm_debug_decompress_bf16(const nslm_seed_matrix *W, uint16_t *w_out, nslm_stream_t stream) {
+  if (!w_out) return NSLM_ERR_ARG;
+  return decompress(W, nullptr, w_out, stream);
+}
+
+int32_t nslm_moe_route_topk(const float *logits, int32_t T, int32_t E, int32_t k, int32_t *ids,
+                            float *w, nslm_stream_t stream) {
+  g_launches = 0;
+  if (!logits || !ids || !w) return NSLM_ERR_ARG;
+  if (T < 0 || k < 1 || k > kMaxK || E < k || E > 1024) return NSLM_ERR_SHAPE;
+  int32_t st = check_device();
+  if (st) return st;
+  if (T == 0) return NSLM_OK;
+  // routes chunks of up to 8 tokens per CTA; plans are not needed here, so
+  // each chunk writes only ids and w
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  for (int t0 = 0; t0 < T; t0 += kMaxT) {
+    const int tn = std::min(kMaxT, T - t0);
+    st = launch_route_plan(logits + (size_t)t0 * E, nullptr, nullptr, tn, E, k, 1, nullptr,
+                           ids + (size_t)t0 * k, w + (size_t)t0 * k, nullptr, 0, s);
+    if (st) return st;
+    ++g_launches;
+  }
+  return NSLM_OK;
+}
+
+int32_t nslm_moe_seed_ffn(const nslm_seed_matrix *gate, const nslm_seed_matrix *up,
+                          const nslm_seed_matrix *down, int32_t E, const uint16_t *x_bf16,
+                          const int32_t *ids, const float *w, int32_t T, int32_t k, float *y,
+                          void *ws, size_t ws_bytes, nslm_stream_t stream) {
+  g_launches = 0;
+  FfnDims d{};
+  int32_t st = check_ffn_shapes(gate, up, down, E, d);
+  if (st) return st;
+  if (!x_bf16 || !ids || !w || !y) return NSLM_ERR_ARG;
+  if (k < 1 || k > kMaxK || T < 0) return NSLM_ERR_SHAPE;
+  if (!aligned16(x_bf16) || !aligned16(y)) return NSLM_ERR_ALIGN;
+  if (T == 0) return NSLM_OK;
+  if (T > kMaxT) return NSLM_ERR_SHAPE;  // the tensor-core path takes larger batches
+  const size_t need = nslm_workspace_bytes(NSLM_OP_MOE_FFN, T, E, d.hidden, d.inter, k, 0);
+  if (!ws || ws_bytes < need) return NSLM_ERR_WORKSPACE;
+  if (!aligned16(ws)) return NSLM_ERR_ALIGN;
+  if ((st = check_device())) return st;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const FfnWorkspace fw = ffn_workspace(reinterpret_cast<char *>(ws), T, k, d.hidden, d.inter, 1);
+  if ((st = launch_route_plan(nullptr, ids, w, T, E, k, 1, fw.plans, nullptr, nullptr, fw.counters,
+                              d.hidden, s)))
+    return st;
+  int launches = 1;
+  st = launch_decode_layer(d, gate, up, down, fw.plans, x_bf16, nullptr, T, k, fw, y, s, launches);
+  if (st == NSLM_OK) g_launches = launches;
+  return st;
+}
+
+int32_t nslm_moe_stack_decode(const nslm_moe_layer *layers, int32_t L, int32_t E, int32_t k,
+                              const float *logits, const uint16_t *x0_bf16, int32_t T, float *y,
+                              void *ws, size_t ws_bytes, nslm_stream_t stream) {
+  g_launches = 0;
+  if (!layers || !logits || !x0_bf16 || !y) return NSLM_ERR_ARG;
+  if (L < 1 || T < 1 || T > kMaxT || k < 1 || k > kMaxK || E < k || E > 1024) return NSLM_ERR_SHAPE;
+  FfnDims d{};
+  int32_t st = check_ffn_shapes(&layers[0].gate, &layers[0].up, &layers[0].down, E, d);
+  if (st) return st;
+  for (int l = 1; l < L; ++l) {
+    FfnDims dl{};
+    if ((st = check_ffn_shapes(&layers[l].gate, &layers[l].up, &layers[l].down, E, dl))) return st;
+    if (dl.hidden != d.hidden || dl.inter != d.inter || dl.P != d.P) return NSLM_ERR_SHAPE;
+  }
+  if (!aligned16(x0_bf16) || !aligned16(y) || !aligned16(logits)) return NSLM_ERR_ALIGN;
+  const size_t need = nslm_workspace_bytes(NSLM_OP_MOE_STACK, T, E, d.hidden, d.inter, k, L);
+  if (!ws || ws_bytes < need) return NSLM_ERR_WORKSPACE;
+  if (!aligned16(ws)) return NSLM_ERR_ALIGN;
+  if ((st = check_device())) return st;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const FfnWorkspace fw = ffn_workspace(reinterpret_cast<char *>(ws), T, k, d.hidden, d.inter, L);
+  if ((st = launch_route_plan(logits, nullptr, nullptr, T, E, k, L, fw.plans, nullptr, nullptr,
+                              fw.counters, d.hidden, s)))
+    return st;
+  int launches = 1;
+  for (int l = 0; l < L; ++l) {
+    const uint16_t *xin = (l == 0) ? x0_bf16 : nullptr;
+    const float *yprev = (l == 0) ? nullptr : fw.y_mid;
+    float *yout = (l == L - 1) ? y : fw.y_mid;
+    st = launch_decode_layer(d, &layers[l].gate, &layers[l].up, &layers[l].down, fw.plans + l, xin,
+                             yprev, T, k, fw, yout, s, launches);
+    if (st) return st;
+  }
+  g_launches = launches;
+  return NSLM_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,58 @@
+// moe.cuh -- internal declarations of the MoE decode path (not part of the ABI).
+#pragma once
+#include <cstddef>
+#include <cstdint>
+#include <algorithm>
+#include <cuda_runtime.h>
+
+#include "../../include/nslm.h"
+
+namespace nslm {
+
+constexpr int kMaxT = 8;                 // decode path: at most 8 tokens
+constexpr int kMaxK = 8;                 // at most 8 experts per token
+constexpr int kMaxPairs = kMaxT * kMaxK;
+
+// One layer's routing grouped by expert.  A slot is one expert together with
+// the (token, slot-in-token) pairs routed to it, at most T pairs per slot.
+struct SlotPlan {
+  int32_t n_slots;
+  int32_t n_pairs;
+  int32_t expert[kMaxPairs];
+  int32_t start[kMaxPairs + 1];  // pairs of slot s: pair[start[s] .. start[s+1])
+  int32_t pair[kMaxPairs];       // pair index t * k + q, sorted by expert
+  int32_t ids[kMaxPairs];        // routed expert ids [T][k]
+  float w[kMaxPairs];            // routing weights [T][k]
+};
+constexpr size_t kPlanBytes = (sizeof(SlotPlan) + 255) / 256 * 256;
+
+struct FfnDims {
+  int32_t E, hidden, inter, P;
+};
+
+int32_t check_ffn_shapes(const nslm_seed_matrix *gate, const nslm_seed_matrix *up,
+                         const nslm_seed_matrix *down, int32_t E, FfnDims &d);
+
+// Workspace of the decode path, carved from the caller's buffer (base may be
+// null to size it).  counters must be zero before the first down kernel; the
+// routing kernel zeroes them and the down kernel leaves them zero.
+struct FfnWorkspace {
+  SlotPlan *plans;     // [L]
+  int32_t *counters;   // [hidden]
+  float *h;            // [T*k][inter]
+  float *y_part;       // [slot groups][T][hidden]
+  float *y_mid;        // [T][hidden] (layer stack)
+  size_t bytes;
+};
+FfnWorkspace ffn_workspace(char *base, int T, int k, int hidden, int inter, int L);
+
+int32_t launch_route_plan(const float *logits, const int32_t *ids, const float *w, int T, int E,
+                          int k, int L, SlotPlan *plans, int32_t *ids_out, float *w_out,
+                          int32_t *counters, int n_counters, cudaStream_t s);
+int32_t launch_decode_layer(const FfnDims &d, const nslm_seed_matrix *gate,
+                            const nslm_seed_matrix *up, const nslm_seed_matrix *down,
+                            const SlotPlan *plan, const uint16_t *x_bf16, const float *y_prev,
+                            int T, int k, const FfnWorkspace &w, float *y, cudaStream_t s,
+                            int &launches);
+
+}  // namespace nslm

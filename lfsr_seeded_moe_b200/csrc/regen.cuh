@@ -1,0 +1,138 @@
+// regen.cuh -- device-side SeedLM block regeneration for sm_100a.
+//
+// A block of 8 weights is a 16-bit LFSR seed, P int4 coefficients and a 4-bit
+// exponent code ("NanoSeedLM: LLM inference using pseudo-random numbers",
+// "Where this started").  With s_t the register state t steps after the seed
+// (the seed is s_0: "What I changed: September 2026"), the weights are
+//
+//   w_r = 2^(code + bias) * sum_j c_j * (s_{1+8j+r} - 32768) / 32768
+//       = 2^(code + bias - 15) * A_r,   A_r = sum_j c_j * (s_{1+8j+r} - 32768),
+//
+// an integer A_r with |A_r| <= 2^20 times a power of two, so fp32 holds w_r
+// exactly.  This file rebuilds A_r without stepping the register:
+//
+// 1. Stream word.  The register is a Fibonacci LFSR (x^16 + x^14 + x^13 +
+//    x^11 + 1), so the states are 16-bit windows of one bit stream:
+//    s_t = (W >> t) & 0xFFFF, where W holds the seed in bits 0..15 and the
+//    new bit 16+k = W_k ^ W_{k+2} ^ W_{k+3} ^ W_{k+5} ("'LFSR is free'": the
+//    24 or 32 bits that follow a seed are a linear function of it, so states
+//    become shifts of a 64-bit word).  The 8P new bits are linear over GF(2)
+//    in the seed, so they are the XOR of two 256-entry table rows, one per
+//    seed byte (computed at compile time; each CTA copies the 2 KB into
+//    shared memory).
+//
+// 2. Byte dot products.  For a window Z = W >> (1 + t), the integer
+//    d_t = sum_j c_j * byte_j(Z) is one dp4a (unsigned stream bytes times
+//    signed coefficient bytes).  Because s_{1+8j+r} = byte_j(W >> (1+r)) +
+//    256 * byte_j(W >> (9+r)),
+//        sum_j c_j * s_{1+8j+r} = d_r + 256 * d_{r+8},
+//    so 16 funnel shifts and 16 dp4a give all 8 A_r.  The centring term
+//    -32768 * sum_j c_j and a float "magic" offset ride in the dp4a
+//    accumulator, so A_r + 1.5 * 2^23 lands in an fp32 bit pattern and one
+//    subtraction recovers A_r exactly (no int-to-float convert).
+//
+// Measured on this B200 (warp instructions per clock per SM): LOP3/SHF/PRMT
+// share one pipe at 2.0, DP4A/IMAD another at 2.0, and a mix of the two
+// reaches 3.4; the inner loop is written to alternate the two pipes.
+#pragma once
+#include <cstdint>
+#include <cuda_runtime.h>
+
+namespace nslm {
+
+constexpr uint32_t kMagicBits = 0x4B400000u;  // 1.5 * 2^23 as fp32
+constexpr float kMagic = 12582912.0f;
+
+// ---------------------------------------------------------------- stream
+
+// Smem tables: for a seed s, the 32 bits that follow it in the stream are
+// tab[s & 0xFF] ^ tab[256 + (s >> 8)].
+struct StreamTables {
+  uint32_t t[512];
+};
+
+// The table contents, computed at compile time from the bit recurrence
+// (bit 16+k = bit k ^ bit k+2 ^ bit k+3 ^ bit k+5): entry v < 256 holds the 32
+// bits that follow start value v, entry 256 + v those that follow v << 8.
+struct StreamTableInit {
+  uint32_t t[512];
+  constexpr StreamTableInit() : t() {
+    for (int i = 0; i < 512; ++i) {
+      uint64_t w = i < 256 ? (uint64_t)i : (uint64_t)(i - 256) << 8;
+      for (int k = 0; k < 32; ++k) {
+        uint64_t b = ((w >> k) ^ (w >> (k + 2)) ^ (w >> (k + 3)) ^ (w >> (k + 5))) & 1u;
+        w |= b << (16 + k);
+      }
+      t[i] = (uint32_t)(w >> 16);
+    }
+  }
+};
+static __device__ const StreamTableInit kStreamTab{};
+
+// Copy the tables into shared memory with all threads of the CTA (the caller
+// synchronises afterwards).
+__device__ __forceinline__ void build_stream_tables(StreamTables *tab) {
+  for (int i = threadIdx.x; i < 512; i += blockDim.x) tab->t[i] = kStreamTab.t[i];
+}
+
+// W = seed | next32 << 16, returned as (lo = bits 0..31, hi = bits 32..47).
+__device__ __forceinline__ void stream_word(const StreamTables *tab, uint32_t seed,
+                                            uint32_t &lo, uint32_t &hi) {
+  uint32_t nxt = tab->t[seed & 0xFFu] ^ tab->t[256u + ((seed >> 8) & 0xFFu)];
+  lo = __byte_perm(seed, nxt, 0x5410);  // seed bytes 0,1 then next bytes 0,1
+  hi = nxt >> 16;
+}
+
+// ----------------------------------------------------------- coefficients
+
+// Packed coefficient nibbles -> four signed bytes [c0, c1, c2, c3]
+// (P = 3: byte 3 is 0; the top nibble there is the exponent code).
+template <int P>
+__device__ __forceinline__ uint32_t coef_bytes(uint32_t q16) {
+  uint32_t v = (q16 | (q16 << 12)) & 0x0F0F0F0Fu;            // [c0, c2, c1, c3]
+  v = __byte_perm(v, 0u, P == 4 ? 0x3120 : 0x4120);          // [c0, c1, c2, c3|0]
+  // two's-complement nibble -> byte: a set bit 3 adds 0xF0 (no carry out)
+  return v + (v & 0x08080808u) * 30u;
+}
+
+__device__ __forceinline__ int32_t dp4a_us(uint32_t a_u8x4, uint32_t b_s8x4, int32_t acc) {
+  int32_t d;
+  asm("dp4a.u32.s32 %0, %1, %2, %3;" : "=r"(d) : "r"(a_u8x4), "r"(b_s8x4), "r"(acc));
+  return d;
+}
+
+__device__ __forceinline__ int32_t dp4a_ss(uint32_t a_s8x4, uint32_t b_s8x4, int32_t acc) {
+  int32_t d;
+  asm("dp4a.s32.s32 %0, %1, %2, %3;" : "=r"(d) : "r"(a_s8x4), "r"(b_s8x4), "r"(acc));
+  return d;
+}
+
+// ----------------------------------------------------------------- block
+
+// The 8 weights of a block as fp32 (w_r = A_r exactly, before the power-of-
+// two scale): F[r] = (float)A_r.
+__device__ __forceinline__ void block_ints(uint32_t lo, uint32_t hi, uint32_t cb,
+                                           float (&F)[8]) {
+  int32_t csum = dp4a_ss(cb, 0x01010101u, 0);
+  int32_t base = (int32_t)kMagicBits - 32768 * csum;
+#pragma unroll
+  for (int r = 0; r < 8; ++r) {
+    uint32_t z0 = __funnelshift_r(lo, hi, 1 + r);   // W >> (1 + r)
+    uint32_t z1 = __funnelshift_r(lo, hi, 9 + r);   // W >> (9 + r)
+    int32_t d0 = dp4a_us(z0, cb, base);
+    int32_t d1 = dp4a_us(z1, cb, 0);
+    int32_t bits = d0 + 256 * d1;                   // bit pattern of kMagic + A_r
+    F[r] = __int_as_float(bits) - kMagic;
+  }
+}
+
+// Scale 2^(code + bias - 15) as an fp32 bit pattern: rowk = (bias + 112) << 23.
+__device__ __forceinline__ float block_scale(uint32_t code, uint32_t rowk) {
+  return __uint_as_float(rowk + (code << 23));
+}
+
+__device__ __forceinline__ uint32_t row_scale_key(int32_t bias) {
+  return (uint32_t)(bias + 112) << 23;
+}
+
+}  // namespace nslm

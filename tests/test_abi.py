@@ -1,0 +1,86 @@
+"""The C ABI on the CPU: the library loads, exports every declared symbol, and
+rejects bad arguments with the documented status codes before launching
+anything (these checks run on the host; no pointer is dereferenced)."""
+import ctypes
+
+import pytest
+
+from lfsr_seeded_moe_b200 import nslm
+
+
+def test_every_declared_symbol_is_exported():
+    names = nslm.declared_functions()
+    assert len(names) >= 10
+    lib = nslm.raw()
+    for n in names:
+        assert hasattr(lib, n), n
+
+
+def test_status_strings():
+    for code in (0, -1, -2, -3, -4, -5, -7):
+        assert nslm.nslm_status_string(code) not in ("", "unknown status")
+    assert nslm.nslm_status_string(12345) == "unknown status"
+
+
+def _mat(N=64, K=256, P=4, base=0x10000, codes=True):
+    return nslm.nslm_seed_matrix(base, base + 0x100000, base + 0x200000 if codes else 0,
+                                 base + 0x300000, N, K, P)
+
+
+def _gemv(W, x=0x7000000, M=1, y=0x8000000):
+    return nslm.raw().nslm_seed_gemv(ctypes.byref(W), x, M, y, 0, 0, 0)
+
+
+def test_gemv_argument_checks():
+    assert _gemv(_mat(P=5)) == nslm.NSLM_ERR_SHAPE
+    assert _gemv(_mat(K=24, P=4)) == nslm.NSLM_ERR_SHAPE      # P=4 needs K % 16 == 0
+    assert _gemv(_mat(K=12, P=3)) == nslm.NSLM_ERR_SHAPE      # K % 8
+    assert _gemv(_mat(), M=0) == nslm.NSLM_ERR_SHAPE
+    assert _gemv(_mat(), M=9) == nslm.NSLM_ERR_SHAPE
+    assert _gemv(_mat(), x=0) == nslm.NSLM_ERR_ARG
+    assert _gemv(_mat(), y=0x8000004) == nslm.NSLM_ERR_ALIGN
+    assert _gemv(_mat(codes=False)) == nslm.NSLM_ERR_ARG      # P=4 needs codes
+    assert _gemv(_mat(base=0x10008)) == nslm.NSLM_ERR_ALIGN
+    assert _gemv(_mat(K=65536), M=1) == nslm.NSLM_ERR_SHAPE   # activations exceed shared memory
+    assert nslm.raw().nslm_seed_gemv(None, 0x7000000, 1, 0x8000000, 0, 0, 0) == nslm.NSLM_ERR_ARG
+
+
+def test_ffn_argument_checks():
+    E, hidden, inter = 4, 256, 128
+    g = _mat(E * inter, hidden)
+    u = _mat(E * inter, hidden)
+    d = _mat(E * hidden, inter)
+    ws_need = nslm.nslm_workspace_bytes(nslm.NSLM_OP_MOE_FFN, 1, E, hidden, inter, 2)
+    assert ws_need > 0
+    f = nslm.raw().nslm_moe_seed_ffn
+    ok = dict(x=0x7000000, ids=0x7100000, w=0x7200000, T=1, k=2, y=0x7300000, ws=0x7400000, wsb=ws_need)
+
+    def call(gg=g, uu=u, dd=d, E_=E, **kw):
+        a = dict(ok, **kw)
+        return f(ctypes.byref(gg), ctypes.byref(uu), ctypes.byref(dd), E_, a["x"], a["ids"], a["w"],
+                 a["T"], a["k"], a["y"], a["ws"], a["wsb"], 0)
+
+    assert call(dd=_mat(E * hidden, inter + 8)) == nslm.NSLM_ERR_SHAPE
+    assert call(E_=3) == nslm.NSLM_ERR_SHAPE                  # rows not divisible by E
+    assert call(k=9) == nslm.NSLM_ERR_SHAPE
+    assert call(T=9) == nslm.NSLM_ERR_SHAPE
+    assert call(wsb=ws_need - 1) == nslm.NSLM_ERR_WORKSPACE
+    assert call(ws=0) == nslm.NSLM_ERR_WORKSPACE
+    assert call(x=0) == nslm.NSLM_ERR_ARG
+    assert call(T=0) == nslm.NSLM_OK                           # nothing to do, nothing launched
+    assert nslm.nslm_last_launch_count() == 0
+
+
+def test_route_argument_checks():
+    f = nslm.raw().nslm_moe_route_topk
+    assert f(0x1000, 1, 100, 9, 0x2000, 0x3000, 0) == nslm.NSLM_ERR_SHAPE
+    assert f(0x1000, 1, 4, 8, 0x2000, 0x3000, 0) == nslm.NSLM_ERR_SHAPE
+    assert f(0x1000, 1, 2000, 8, 0x2000, 0x3000, 0) == nslm.NSLM_ERR_SHAPE
+    assert f(0, 1, 100, 8, 0x2000, 0x3000, 0) == nslm.NSLM_ERR_ARG
+
+
+def test_workspace_sizes_are_monotone():
+    a = nslm.nslm_workspace_bytes(nslm.NSLM_OP_MOE_STACK, 1, 100, 2048, 1408, 8, 45)
+    b = nslm.nslm_workspace_bytes(nslm.NSLM_OP_MOE_STACK, 8, 100, 2048, 1408, 8, 45)
+    assert 0 < a < b
+    assert nslm.nslm_workspace_bytes(nslm.NSLM_OP_GEMV, 1, 1, 1, 1, 1) == 0

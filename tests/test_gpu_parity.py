@@ -1,0 +1,196 @@
+"""GPU parity: the CUDA library (through its C ABI) against the CPU oracle.
+
+Regenerated weights must be bit-exact; products must be within 2e-3 of the
+fp64 oracle in the normwise relative error max|y - ref| / max|ref|.
+"""
+import numpy as np
+import pytest
+import torch
+
+from oracle import oracle as O
+from lfsr_seeded_moe_b200 import synth
+
+pytestmark = pytest.mark.gpu
+
+TOL = 2e-3          # the stated bar (fp32 accumulate vs fp64 oracle)
+TIGHT = 1e-5        # what the fp32 decode path actually reaches; a regression guard
+
+
+@pytest.fixture(scope="module")
+def nslm():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from lfsr_seeded_moe_b200 import nslm as n
+    return n
+
+
+def _out(*shape):
+    """Output buffer pre-filled with NaN, so an entry the kernel never wrote fails."""
+    return torch.full(shape, float("nan"), dtype=torch.float32, device="cuda")
+
+
+def _dev(m):
+    return m.to("cuda")
+
+
+def _x(tag, M, K):
+    xb = synth.activations(tag, M, K)
+    return xb.cuda().contiguous(), synth.bf16_bits(xb).numpy().view(np.uint16)
+
+
+def _all_seed_matrix(P, bias_lo=-100, bias_hi=100):
+    """512 x 1024 matrix whose 65,536 blocks hold every seed value 0..65535 once."""
+    N, K = 512, 1024
+    m = synth.seed_matrix(N, K, P, (900, P))
+    m.seeds = torch.arange(65536, dtype=torch.int32).to(torch.int16).reshape(N, K // 8).contiguous()
+    m.exp_bias = torch.linspace(bias_lo, bias_hi, N).round().to(torch.int32)
+    return m
+
+
+@pytest.mark.parametrize("P", [3, 4])
+def test_decompress_fp32_bit_exact_all_seeds(nslm, P):
+    m = _all_seed_matrix(P)
+    md = _dev(m)
+    w = _out(m.N, m.K)
+    nslm.nslm_debug_decompress(md, w)
+    torch.cuda.synchronize()
+    ref = O.decompress(m.numpy(), np.float32)
+    got = w.cpu().numpy()
+    assert np.array_equal(got.view(np.uint32), ref.view(np.uint32))
+
+
+@pytest.mark.parametrize("P", [3, 4])
+def test_decompress_bf16_bit_exact_all_seeds(nslm, P):
+    m = _all_seed_matrix(P, -20, 10)
+    md = _dev(m)
+    w = torch.empty(m.N, m.K, dtype=torch.int16, device="cuda")
+    nslm.nslm_debug_decompress_bf16(md, w)
+    torch.cuda.synchronize()
+    ref = O.decompress_bf16(m.numpy())
+    assert np.array_equal(w.cpu().numpy().view(np.uint16), ref)
+
+
+GEMV_SHAPES = [(512, 1024), (2048, 4096), (4096, 2048), (1408, 2048), (2048, 1408)]
+
+
+@pytest.mark.parametrize("P", [3, 4])
+@pytest.mark.parametrize("N,K", GEMV_SHAPES)
+def test_gemv_matches_oracle(nslm, P, N, K):
+    m = synth.seed_matrix(N, K, P, (901, N, K, P))
+    x, xh = _x((901, K), 1, K)
+    y = _out(1, N)
+    nslm.nslm_seed_gemv(_dev(m), x, 1, y)
+    torch.cuda.synchronize()
+    ref = O.seed_matvec(m.numpy(), xh)
+    err = O.normwise_rel_err(y.cpu().numpy(), ref)
+    assert err <= TOL and err <= TIGHT, err
+
+
+@pytest.mark.parametrize("M", [2, 3, 8])
+@pytest.mark.parametrize("P", [3, 4])
+def test_gemv_multi_token(nslm, M, P):
+    N, K = 704, 2048
+    m = synth.seed_matrix(N, K, P, (902, M, P))
+    x, xh = _x((902, M), M, K)
+    y = _out(M, N)
+    nslm.nslm_seed_gemv(_dev(m), x, M, y)
+    torch.cuda.synchronize()
+    ref = O.seed_matvec(m.numpy(), xh)
+    err = O.normwise_rel_err(y.cpu().numpy(), ref)
+    assert err <= TIGHT, err
+
+
+@pytest.mark.parametrize("P,N,K", [(3, 999, 1000), (4, 1001, 1008), (3, 1, 8), (4, 3, 16),
+                                   (4, 130, 4096 + 64 + 16), (3, 77, 520)])
+def test_gemv_ragged_shapes(nslm, P, N, K):
+    m = synth.seed_matrix(N, K, P, (903, N, K, P))
+    x, xh = _x((903, K), 2, K)
+    y = _out(2, N)
+    nslm.nslm_seed_gemv(_dev(m), x, 2, y)
+    torch.cuda.synchronize()
+    ref = O.seed_matvec(m.numpy(), xh)
+    assert O.normwise_rel_err(y.cpu().numpy(), ref) <= TIGHT
+
+
+def test_gemv_extreme_fields(nslm):
+    # seed 0 (all-zero register), all codes 15, coefficients -8 and 7, bias -100 and +90
+    N, K, P = 64, 512, 4
+    m = synth.seed_matrix(N, K, P, (904,))
+    m.seeds[::3] = 0
+    m.coefs[1::2] = torch.tensor(0x8888, dtype=torch.int32).to(torch.int16)
+    m.coefs[::2] = 0x7777
+    m.codes[:] = torch.tensor(0xFF, dtype=torch.uint8)
+    m.exp_bias = torch.tensor([90 if i % 2 else -100 for i in range(N)], dtype=torch.int32)
+    x, xh = _x((904,), 1, K)
+    y = _out(1, N)
+    nslm.nslm_seed_gemv(_dev(m), x, 1, y)
+    torch.cuda.synchronize()
+    ref = O.seed_matvec(m.numpy(), xh)
+    for rows in (slice(0, None, 2), slice(1, None, 2)):  # two magnitudes: compare each
+        assert O.normwise_rel_err(y.cpu().numpy()[:, rows], ref[:, rows]) <= TIGHT
+
+
+def test_route_topk_matches_oracle(nslm):
+    T, E, k = 64, 100, 8
+    logits = synth.router_logits((905,), T, E)
+    logits[3, :] = 0.5                          # all tied
+    logits[4, 7] = logits[4, 90] = 5.0          # tie at the top
+    ids = torch.empty(T, k, dtype=torch.int32, device="cuda")
+    w = _out(T, k)
+    nslm.nslm_moe_route_topk(logits.cuda(), T, E, k, ids, w)
+    torch.cuda.synchronize()
+    rid, rw = O.route_topk(logits.numpy(), k)
+    assert np.array_equal(ids.cpu().numpy(), rid)
+    assert np.max(np.abs(w.cpu().numpy() - rw)) <= 1e-6
+
+
+def _ffn_case(nslm, E, hidden, inter, P, T, k, tag, zipf=None):
+    L = synth.moe_layer(0, E, hidden, inter, P, config=tag)
+    x, xh = _x((tag, T), T, hidden)
+    logits = synth.router_logits((tag,), T, E, zipf)
+    rid, rw = O.route_topk(logits.numpy(), k)
+    ids = torch.from_numpy(rid).cuda()
+    w = torch.from_numpy(rw.astype(np.float32)).cuda()
+    y = _out(T, hidden)
+    wsb = nslm.nslm_workspace_bytes(nslm.NSLM_OP_MOE_FFN, T, E, hidden, inter, k)
+    ws = torch.empty(wsb, dtype=torch.uint8, device="cuda")
+    nslm.nslm_moe_seed_ffn(_dev(L.gate), _dev(L.up), _dev(L.down), E, x, ids, w, T, k, y, ws, wsb)
+    torch.cuda.synchronize()
+    g, u, d = (getattr(L, n).numpy() for n in ("gate", "up", "down"))
+    ref = O.moe_ffn(g, u, d, E, hidden, inter, xh, rid, rw.astype(np.float32).astype(np.float64), mode=0)
+    return y.cpu().numpy(), ref
+
+
+def test_ffn_decode_one_token_full_layer(nslm):
+    # one MoE layer decode: 100 experts, hidden 2048, intermediate 1408, P=4, top-8
+    y, ref = _ffn_case(nslm, 100, 2048, 1408, 4, 1, 8, 906)
+    assert O.normwise_rel_err(y, ref) <= TIGHT
+
+
+@pytest.mark.parametrize("T", [2, 5, 8])
+@pytest.mark.parametrize("P", [3, 4])
+def test_ffn_decode_batch(nslm, T, P):
+    y, ref = _ffn_case(nslm, 16, 256, 128, P, T, 4, 907 + T)
+    assert O.normwise_rel_err(y, ref) <= TIGHT
+
+
+def test_ffn_decode_ragged_and_zipf(nslm):
+    y, ref = _ffn_case(nslm, 12, 272, 120, 3, 3, 8, 908, zipf=1.1)
+    assert O.normwise_rel_err(y, ref) <= TIGHT
+
+
+@pytest.mark.parametrize("T", [1, 3])
+def test_stack_decode_matches_oracle(nslm, T):
+    Lyr, E, hidden, inter, P, k = 4, 8, 256, 128, 4, 2
+    layers = [synth.moe_layer(l, E, hidden, inter, P, config=909) for l in range(Lyr)]
+    logits = torch.stack([synth.router_logits((909, l), T, E) for l in range(Lyr)])
+    x, xh = _x((909, T), T, hidden)
+    dl = [(_dev(m.gate), _dev(m.up), _dev(m.down)) for m in layers]
+    y = _out(T, hidden)
+    wsb = nslm.nslm_workspace_bytes(nslm.NSLM_OP_MOE_STACK, T, E, hidden, inter, k, Lyr)
+    ws = torch.empty(wsb, dtype=torch.uint8, device="cuda")
+    nslm.nslm_moe_stack_decode(dl, Lyr, E, k, logits.cuda().contiguous(), x, T, y, ws, wsb)
+    torch.cuda.synchronize()
+    hl = [tuple(getattr(m, n).numpy() for n in ("gate", "up", "down")) for m in layers]
+    ref, _ = O.layer_stack(hl, logits.numpy(), xh, hidden, inter, E, k, mode=0)
+    assert O.normwise_rel_err(y.cpu().numpy(), ref) <= TOL
