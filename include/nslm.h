@@ -144,6 +144,32 @@ int32_t nslm_moe_seed_ffn(const nslm_seed_matrix *gate, const nslm_seed_matrix *
                           const int32_t *ids, const float *w, int32_t T, int32_t k, float *y,
                           void *ws, size_t ws_bytes, nslm_stream_t stream);
 
+/* The decode path of nslm_moe_seed_ffn (T <= 8) for callers that may not
+ * allocate device memory: the scratch it needs lives in a 1 MiB array built
+ * into the library (one per GPU that loads it, kept until the process exits),
+ * so no workspace is passed and nothing is allocated.  The pages have no
+ * counterpart; this is an interface convenience, not part of the method.
+ *
+ * Which callers this is for: code embedded in a host application whose
+ * allocator owns the GPU's memory, latency-critical loops that cannot take an
+ * allocation's implicit synchronisation, and callers that only receive input
+ * and output pointers.
+ *
+ * Arguments, layout and results are those of nslm_moe_seed_ffn without ws and
+ * ws_bytes.  Returns NSLM_ERR_WORKSPACE if the problem's workspace
+ * (nslm_workspace_bytes(NSLM_OP_MOE_FFN, T, E, hidden, inter, k, 0)) exceeds
+ * 1 MiB; T > 8 returns NSLM_ERR_SHAPE.
+ * The first call on a device, made with that device current, looks up the
+ * array's device address (cudaGetSymbolAddress) and caches it; make that first
+ * call before capturing any stream.  All calls share the one array: calls
+ * whose work overlaps on the GPU (e.g. on two streams at once) race and give
+ * wrong results.  Each call rewrites what it reads, so the contents left by an
+ * earlier call do no harm. */
+int32_t nslm_moe_seed_ffn_static(const nslm_seed_matrix *gate, const nslm_seed_matrix *up,
+                                 const nslm_seed_matrix *down, int32_t E, const uint16_t *x_bf16,
+                                 const int32_t *ids, const float *w, int32_t T, int32_t k,
+                                 float *y, nslm_stream_t stream);
+
 /* A stack of L MoE layers for T <= 8 decode tokens.  Layer l routes with
  * logits[l] (fp32 [L][T][E]) and runs nslm_moe_seed_ffn on its input; the
  * next layer's input is bf16(y / sqrt(mean(y^2) + 1e-6)) per token (the pages

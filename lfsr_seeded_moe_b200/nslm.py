@@ -65,6 +65,7 @@ def _load():
         "nslm_seed_grouped_gemm": (i32, [mp, i32, vp, vp, i32, vp, vp, sz, vp]),
         "nslm_moe_route_topk": (i32, [vp, i32, i32, i32, vp, vp, vp]),
         "nslm_moe_seed_ffn": (i32, [mp, mp, mp, i32, vp, vp, vp, i32, i32, vp, vp, sz, vp]),
+        "nslm_moe_seed_ffn_static": (i32, [mp, mp, mp, i32, vp, vp, vp, i32, i32, vp, vp]),
         "nslm_moe_stack_decode": (i32, [ctypes.POINTER(nslm_moe_layer), i32, i32, i32, vp, vp, i32,
                                         vp, vp, sz, vp]),
         "nslm_debug_decompress": (i32, [mp, vp, vp]),
@@ -161,6 +162,16 @@ def nslm_moe_seed_ffn(gate, up, down, E: int, x_bf16, ids, w, T: int, k: int, y,
            _lib.nslm_moe_seed_ffn(ctypes.byref(_mat(gate)), ctypes.byref(_mat(up)),
                                   ctypes.byref(_mat(down)), E, _p(x_bf16), _p(ids), _p(w), T, k,
                                   _p(y), _p(ws), ws_bytes, _s(stream)))
+
+
+def nslm_moe_seed_ffn_static(gate, up, down, E: int, x_bf16, ids, w, T: int, k: int, y,
+                             stream=None) -> None:
+    """nslm_moe_seed_ffn without a workspace argument, for callers that may not
+    allocate device memory: the library's built-in 1 MiB scratch array is used."""
+    _check("nslm_moe_seed_ffn_static",
+           _lib.nslm_moe_seed_ffn_static(ctypes.byref(_mat(gate)), ctypes.byref(_mat(up)),
+                                         ctypes.byref(_mat(down)), E, _p(x_bf16), _p(ids), _p(w), T,
+                                         k, _p(y), _s(stream)))
 
 
 def moe_layers(layers) -> "ctypes.Array":
