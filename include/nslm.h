@@ -117,7 +117,10 @@ int32_t nslm_seed_gemv(const nslm_seed_matrix *W, const uint16_t *x_bf16, int32_
  * x: bf16 [R][K], rows grouped by expert; offsets: int32 [E + 1] (DEVICE),
  * non-decreasing, offsets[0] = 0, offsets[E] = R; y: fp32 [R][rows].
  * Weights are regenerated into bf16 (round to nearest even) tiles and
- * multiplied on the tensor cores with fp32 accumulation.
+ * multiplied on the tensor cores (tcgen05) with fp32 accumulation.  Requires
+ * K % 64 == 0 and 1 <= E <= 1024; rows outside [0, R) are never read.  A
+ * tensor-core wait that does not complete within about two seconds stops the
+ * kernel and sets the first int32 of the workspace to 1 (0 otherwise).
  * Workspace: nslm_workspace_bytes(NSLM_OP_GROUPED_GEMM, R, E, K, rows, 1, 0). */
 int32_t nslm_seed_grouped_gemm(const nslm_seed_matrix *W, int32_t E, const uint16_t *x_bf16,
                                const int32_t *offsets, int32_t R, float *y, void *ws,
@@ -137,7 +140,9 @@ int32_t nslm_moe_route_topk(const float *logits, int32_t T, int32_t E, int32_t k
  * down: [E * hidden][inter], all with the same P.  x: bf16 [T][hidden];
  * ids: int32 [T][k] in [0, E); w: fp32 [T][k]; y: fp32 [T][hidden].
  * T <= 8 runs the decode path (fp32 weights and hidden activations);
- * larger T runs the tensor-core path (bf16 weights, bf16 hidden activation).
+ * larger T runs the tensor-core path (bf16 weights, bf16 hidden activation;
+ * hidden and inter multiples of 64, E <= 1024; the first int32 of the
+ * workspace is set to 1 if a tensor-core wait timed out).
  * Workspace: nslm_workspace_bytes(NSLM_OP_MOE_FFN, T, E, hidden, inter, k, 0). */
 int32_t nslm_moe_seed_ffn(const nslm_seed_matrix *gate, const nslm_seed_matrix *up,
                           const nslm_seed_matrix *down, int32_t E, const uint16_t *x_bf16,

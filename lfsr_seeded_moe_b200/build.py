@@ -7,6 +7,7 @@ rebuilt when any source under csrc/ or include/ is newer than it.
 """
 from __future__ import annotations
 
+import concurrent.futures
 import glob
 import os
 import subprocess
@@ -43,15 +44,21 @@ def build(force: bool = False, verbose: bool = False, extra_flags=None) -> str:
     if not force and up_to_date():
         return LIB
     os.makedirs(OUT_DIR, exist_ok=True)
-    objs = []
+    jobs = []
     for src in sources():
         obj = os.path.join(OUT_DIR, os.path.basename(src)[:-3] + ".o")
         cmd = [NVCC, *ARCH, *FLAGS, *(extra_flags or []), "-I", os.path.join(ROOT, "include"),
                "-c", src, "-o", obj]
         if verbose:
             print(" ".join(cmd), file=sys.stderr)
-        subprocess.run(cmd, check=True)
-        objs.append(obj)
+        jobs.append((cmd, obj))
+    # translation units compile independently: run them in parallel
+    with concurrent.futures.ThreadPoolExecutor(max_workers=max(1, os.cpu_count() or 1)) as ex:
+        for r in ex.map(lambda j: subprocess.run(j[0], capture_output=True, text=True), jobs):
+            if r.stdout or r.stderr:
+                print(r.stdout + r.stderr, file=sys.stderr, end="")
+            r.check_returncode()
+    objs = [o for _, o in jobs]
     tmp = LIB + f".tmp{os.getpid()}"
     cmd = [NVCC, *ARCH, "-shared", "-o", tmp, *objs]  # static cudart (nvcc default)
     if verbose:

@@ -6,6 +6,7 @@
 
 #include "chunk.cuh"
 #include "common.cuh"
+#include "grouped.cuh"
 #include "moe.cuh"
 
 namespace nslm {
@@ -190,12 +191,13 @@ size_t nslm_workspace_bytes(int32_t op, int32_t T, int32_t E, int32_t hidden, in
   (void)hidden;
   switch (op) {
     case NSLM_OP_GEMV: return 0;
-    case NSLM_OP_GROUPED_GEMM: return 0;
+    case NSLM_OP_GROUPED_GEMM: return grouped_ws_bytes(std::max(E, 1));
     case NSLM_OP_MOE_FFN:
       if (T <= kMaxT)
         return ffn_workspace(nullptr, std::max(T, 1), std::max(k, 1), std::max(hidden, 0),
                              std::max(inter, 0), 1).bytes;
-      return 0;
+      return batched_workspace(nullptr, T, std::max(k, 1), std::max(E, 1), std::max(hidden, 0),
+                               std::max(inter, 0)).bytes;
     case NSLM_OP_MOE_STACK:
       return ffn_workspace(nullptr, std::max(T, 1), std::max(k, 1), std::max(hidden, 0),
                            std::max(inter, 0), std::max(L, 1)).bytes;
@@ -246,12 +248,18 @@ int32_t nslm_moe_seed_ffn(const nslm_seed_matrix *gate, const nslm_seed_matrix *
   if (k < 1 || k > kMaxK || T < 0) return NSLM_ERR_SHAPE;
   if (!aligned16(x_bf16) || !aligned16(y)) return NSLM_ERR_ALIGN;
   if (T == 0) return NSLM_OK;
-  if (T > kMaxT) return NSLM_ERR_SHAPE;  // the tensor-core path takes larger batches
+  if (T > kMaxT && (d.hidden % 64 || d.inter % 64 || E > 1024)) return NSLM_ERR_SHAPE;
   const size_t need = nslm_workspace_bytes(NSLM_OP_MOE_FFN, T, E, d.hidden, d.inter, k, 0);
   if (!ws || ws_bytes < need) return NSLM_ERR_WORKSPACE;
   if (!aligned16(ws)) return NSLM_ERR_ALIGN;
   if ((st = check_device())) return st;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (T > kMaxT) {  // tensor-core path: bf16 weights, bf16 hidden activation
+    int launches = 0;
+    st = launch_batched_ffn(d, gate, up, down, x_bf16, ids, w, T, k, y, ws, s, launches);
+    if (st == NSLM_OK) g_launches = launches;
+    return st;
+  }
   const FfnWorkspace fw = ffn_workspace(reinterpret_cast<char *>(ws), T, k, d.hidden, d.inter, 1);
   if ((st = launch_route_plan(nullptr, ids, w, T, E, k, 1, fw.plans, nullptr, nullptr, fw.counters,
                               d.hidden, s)))
