@@ -230,6 +230,55 @@ def gemv_sweep(torch, nslm, synth, dev, hbm):
     return out
 
 
+def batched_sweep(torch, nslm, synth, dev, hbm, bf16_peak):
+    """Batched MoE layer on the tensor-core path: 100 experts, 2048/1408, P=3, top-8."""
+    Pb, nl = 3, 4
+    layers = [synth.moe_layer(l, E, HIDDEN, INTER, Pb, device=dev, config=3) for l in range(nl)]
+    per_expert = 2 * (INTER * (HIDDEN // 8) * 4 + 4 * INTER) + (HIDDEN * (INTER // 8) * 4 + 4 * HIDDEN)
+    out = []
+    for T in (64, 512):
+        for zipf in (None, 1.1):
+            logits = synth.router_logits((3, T, zipf is not None), T, E, zipf).to(dev)
+            ids = torch.empty(T, K_TOP, dtype=torch.int32, device=dev)
+            w = torch.empty(T, K_TOP, device=dev)
+            nslm.nslm_moe_route_topk(logits, T, E, K_TOP, ids, w)
+            x = synth.activations((3, T), T, HIDDEN).to(dev)
+            y = torch.empty(T, HIDDEN, device=dev)
+            wsb = nslm.nslm_workspace_bytes(nslm.NSLM_OP_MOE_FFN, T, E, HIDDEN, INTER, K_TOP)
+            ws = torch.zeros(wsb, dtype=torch.uint8, device=dev)
+            st = [(nslm.matrix(L.gate), nslm.matrix(L.up), nslm.matrix(L.down)) for L in layers]
+            nslm.nslm_moe_seed_ffn(*st[0], E, x, ids, w, T, K_TOP, y, ws, wsb)
+            torch.cuda.synchronize()
+            reps = 2 * nl
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g):
+                for i in range(reps):
+                    nslm.nslm_moe_seed_ffn(*st[i % nl], E, x, ids, w, T, K_TOP, y, ws, wsb)
+            g.replay()
+            torch.cuda.synchronize()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            g.replay()
+            g.replay()
+            e1.record()
+            torch.cuda.synchronize()
+            t = e0.elapsed_time(e1) * 1e-3 / (2 * reps)
+            status = int(ws[:4].view(torch.int32).item())
+            uniq = len(set(ids.cpu().numpy().reshape(-1).tolist()))
+            nbytes = uniq * per_expert
+            flops = 2.0 * T * K_TOP * 3 * INTER * HIDDEN
+            out.append({"T": T, "routing": "zipf1.1" if zipf else "uniform", "experts_touched": uniq,
+                        "us_per_layer": round(t * 1e6, 2), "tokens_per_s_per_layer": round(T / t, 1),
+                        "packed_GB_s": round(nbytes / t / 1e9, 1), "pct_of_hbm": round(100 * nbytes / t / 1e9 / hbm, 2),
+                        "mma_TFLOP_s": round(flops / t / 1e12, 1),
+                        "pct_of_bf16_peak": round(100 * flops / t / 1e12 / bf16_peak, 2) if bf16_peak else None,
+                        "status": status})
+            del g
+    del layers
+    torch.cuda.empty_cache()
+    return out
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -238,6 +287,7 @@ def main():
     ap.add_argument("--batch", type=int, default=1, help="decode tokens per step (1..8)")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-gemv", action="store_true")
+    ap.add_argument("--no-batched", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
     args = ap.parse_args()
     if args.impl == "reference":
@@ -378,6 +428,16 @@ def main():
     del g
     torch.cuda.empty_cache()
 
+    batched = None
+    if not args.no_batched:
+        bf16_peak = None
+        pk = os.path.join(ROOT, "MEASURED_PEAKS.json")
+        if os.path.exists(pk):
+            bf16_peak = float(json.load(open(pk)).get("bf16_tflops", 0.0)) or None
+        batched = {"workload": "one batched MoE layer on the tensor-core path: 100 experts, 2048/1408, P=3, top-8",
+                   "results": batched_sweep(torch, nslm, synth, dev, hbm, bf16_peak),
+                   "note": "4 resident layers rotated in a CUDA graph; packed bytes = experts touched"}
+
     gemv = None
     if not args.no_gemv:
         gemv = {"metric": GEMV_METRIC, "shapes": gemv_sweep(torch, nslm, synth, dev, hbm),
@@ -401,6 +461,8 @@ def main():
     }
     if gemv is not None:
         line["gemv"] = gemv
+    if batched is not None:
+        line["batched"] = batched
     if rank == 0 and world == 1 and not args.no_cpu:
         line["cpu_baseline"] = cpu_baseline()
     if rank == 0:

@@ -146,9 +146,10 @@ __device__ __forceinline__ float regen_chunk_block(const StreamTables *tab, cons
   const int32_t base = (int32_t)kMagic2Bits - 32768 * dp4a_ss(cb2, 0x01010101u, 0);
 #pragma unroll
   for (int r = 0; r < 8; ++r) {
-    const int32_t d0 = dp4a_us(__funnelshift_r(lo, hi, 1 + r), cb2, base);  // bytes of W >> (1+r)
-    const int32_t d1 = dp4a_us(__funnelshift_r(lo, hi, 9 + r), cb2, 0);     // bytes of W >> (9+r)
-    G[r] = __int_as_float(d0 + 256 * d1);  // bits of Mg + 2 A_r ulps = Mg + A_r
+    // bytes of W >> (9+r) weigh 256, bytes of W >> (1+r) weigh 1; the sum is
+    // the bit pattern of Mg + 2 A_r ulps = Mg + A_r
+    const int32_t d1 = dp4a_us(__funnelshift_r(lo, hi, 9 + r), cb2, 0);
+    G[r] = __int_as_float(dp4a_us(__funnelshift_r(lo, hi, 1 + r), cb2, imad(d1, 256, base)));
   }
   const uint32_t code = (P == 4) ? ((f.codes >> (4 * i)) & 0xFu) : (q >> 12);
   return block_scale(code, rowk);

@@ -9,7 +9,8 @@
 // expert and up to `bn` of that expert's token rows.  For every 64-wide K
 // slice, all threads regenerate the 128 x 64 weight tile from its seeds as
 // bf16 (round to nearest even of the exact fp32 weight) straight into shared
-// memory, copy the matching token rows, and one thread issues tcgen05.mma
+// memory (512 threads, each owning two blocks of two rows per slice), copy the
+// matching token rows, and one thread issues tcgen05.mma
 // (bf16 x bf16 -> fp32 in tensor memory).  Two shared-memory stages let the
 // tensor core work on one slice while the threads regenerate the next.  The
 // weights are never written to global memory.
@@ -28,7 +29,8 @@ namespace nslm {
 
 constexpr int kBM = 128;        // weight rows per tile (MMA M)
 constexpr int kBK = 64;         // K per stage: 8 blocks, 128 bytes of bf16 per row
-constexpr int kGThreads = 512;
+constexpr int kGThreads = 512;                 // producer threads
+constexpr int kCtaThreads = kGThreads + 32;    // + one warp that issues the MMAs
 constexpr int kStages = 2;
 constexpr long long kWaitCycles = 4000000000LL;  // ~2 s: a wait longer than this is an error
 
@@ -55,51 +57,108 @@ struct GroupedParams {
 // core-matrix rows.  seeds2/coefs2 hold the two blocks' 16-bit fields, code2
 // their two exponent nibbles.
 template <int P>
-__device__ __forceinline__ void regen_pair_bf16(const StreamTables *tab, uint32_t seeds2, uint32_t coefs2,
-                                                uint32_t code2, uint32_t rowk, uint4 *dst0, uint4 *dst1) {
+__device__ __forceinline__ void regen_pair_bf16(const StreamTablesX32 *tab, uint32_t lane4, uint32_t seeds2,
+                                                uint32_t coefs2, uint32_t code2, uint32_t rowk, uint4 *dst0,
+                                                uint4 *dst1) {
 #pragma unroll
   for (int h = 0; h < 2; ++h) {
     const uint32_t seed = h ? (seeds2 >> 16) : (seeds2 & 0xFFFFu);
     const uint32_t q = h ? (coefs2 >> 16) : (coefs2 & 0xFFFFu);
     uint32_t lo, hi;
-    stream_word(tab, seed, lo, hi);
+    stream_word_x32(tab, lane4, seed, lo, hi);
     const uint32_t cb2 = coef_bytes2<P>(q);
     const int32_t base = (int32_t)kMagic2Bits - 32768 * dp4a_ss(cb2, 0x01010101u, 0);
     const uint32_t code = (P == 4) ? ((code2 >> (4 * h)) & 0xFu) : (q >> 12);
     const float s = block_scale(code, rowk);
-    const float2 s2 = make_float2(s, s), off2 = make_float2(-kMagic2 * s, -kMagic2 * s);
+    const float off = -kMagic2 * s;
     uint32_t packed[4];
 #pragma unroll
     for (int r = 0; r < 8; r += 2) {
-      const int32_t a0 = dp4a_us(__funnelshift_r(lo, hi, 1 + r), cb2, base) +
-                         256 * dp4a_us(__funnelshift_r(lo, hi, 9 + r), cb2, 0);
-      const int32_t a1 = dp4a_us(__funnelshift_r(lo, hi, 2 + r), cb2, base) +
-                         256 * dp4a_us(__funnelshift_r(lo, hi, 10 + r), cb2, 0);
+      const int32_t a0 = dp4a_us(__funnelshift_r(lo, hi, 1 + r), cb2,
+                                 imad(dp4a_us(__funnelshift_r(lo, hi, 9 + r), cb2, 0), 256, base));
+      const int32_t a1 = dp4a_us(__funnelshift_r(lo, hi, 2 + r), cb2,
+                                 imad(dp4a_us(__funnelshift_r(lo, hi, 10 + r), cb2, 0), 256, base));
       // (Mg + A) * s - Mg * s = A * s exactly (power-of-two scale)
-      const float2 w = __ffma2_rn(make_float2(__int_as_float(a0), __int_as_float(a1)), s2, off2);
-      const __nv_bfloat162 b = __floats2bfloat162_rn(w.x, w.y);
+      const __nv_bfloat162 b =
+          __floats2bfloat162_rn(fmaf(__int_as_float(a0), s, off), fmaf(__int_as_float(a1), s, off));
       packed[r >> 1] = *reinterpret_cast<const uint32_t *>(&b);
     }
     *(h ? dst1 : dst0) = make_uint4(packed[0], packed[1], packed[2], packed[3]);
   }
 }
 
+// Tile shapes: every thread owns two tasks per K slice -- two consecutive
+// blocks (16 weights) of the same row of both 128-row sub-tiles.  GATEUP tiles are
+// 128 rows of gate and the same 128 rows of up (two accumulators); the other
+// modes use 256-row tiles (two M=128 halves, two accumulators).
+template <int MODE> struct TileShape {
+  static constexpr int kRows = (MODE == GMODE_GATEUP) ? kBM : 2 * kBM;
+};
+
+// Pipeline (no CTA-wide barrier in the main loop):
+//   each of the 512 producer threads, per K slice: wait empty[stage] -> start async copies of its
+//     token-row chunks -> regenerate its two tasks' blocks (weight fields were
+//     prefetched two slices earlier) -> wait for its copies -> proxy fence ->
+//     arrive full[stage]
+//   the MMA warp (lane 0), per K slice: wait full[stage] -> (first slice of a tile: wait
+//     acc_empty) -> issue the MMAs -> commit empty[stage] (and acc_full after
+//     the tile's last slice)
+//   warps 0-3, per tile: wait acc_full -> read D from tensor memory -> store
+//     -> arrive acc_empty
+// Every wait is bounded; a thread that gives up raises a shared abort flag
+// that all threads check before each slice.
+struct SliceFields {  // packed fields of one thread's two tasks for one K slice
+  uint32_t s2[2], q2[2], c2[2];
+};
+
+template <int P>
+__device__ __forceinline__ void load_slice(const uint32_t *const (&sp)[2], const uint32_t *const (&qp)[2],
+                                           const uint8_t *const (&cp)[2], const bool (&ok)[2], int kt,
+                                           SliceFields &f) {
+#pragma unroll
+  for (int j = 0; j < 2; ++j) {
+    f.s2[j] = ok[j] ? __ldcs(sp[j] + 4 * kt) : 0u;
+    f.q2[j] = ok[j] ? __ldcs(qp[j] + 4 * kt) : 0u;
+    f.c2[j] = (P == 4 && ok[j]) ? (uint32_t)__ldcs(cp[j] + 4 * kt) : 0u;
+  }
+}
+
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void *src, uint32_t src_bytes) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(src_bytes) : "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() {
+  asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
+}
+
 template <int P, int MODE>
-__global__ void __launch_bounds__(kGThreads, 1) grouped_seed_gemm_kernel(const GroupedParams p) {
-  constexpr int NA = (MODE == GMODE_GATEUP) ? 2 : 1;
+__global__ void __launch_bounds__(kCtaThreads, 1) grouped_seed_gemm_kernel(const GroupedParams p) {
+  constexpr int kRows = TileShape<MODE>::kRows;
   extern __shared__ __align__(1024) uint8_t gsm[];
-  StreamTables *tab = reinterpret_cast<StreamTables *>(gsm);
-  uint8_t *a_base = gsm + 2048;                                   // [stage][NA][128 rows x 128 B]
-  uint8_t *b_base = a_base + (size_t)kStages * NA * kBM * 128;    // [stage][bn rows x 128 B]
-  __shared__ __align__(8) uint64_t mbar[kStages];
+  StreamTablesX32 *tab = reinterpret_cast<StreamTablesX32 *>(gsm);
+  uint8_t *a_base = gsm + sizeof(StreamTablesX32);               // [stage][sub 0..1][128 rows x 128 B]
+  uint8_t *b_base = a_base + (size_t)kStages * 2 * kBM * 128;    // [stage][bn rows x 128 B]
+  __shared__ __align__(8) uint64_t full_bar[kStages];
+  __shared__ __align__(8) uint64_t empty_bar[kStages];
+  __shared__ __align__(8) uint64_t acc_full_bar, acc_empty_bar;
   __shared__ uint32_t tmem_base_s;
+  __shared__ volatile int s_abort;
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  build_stream_tables(tab);
+  const bool issuer_warp = tid >= kGThreads;
+  // a producer's tasks: row trow, block pair bp, of sub-tiles 0 and 1
+  const int trow = tid & (kBM - 1), bp = (tid >> 7) & 3;
+  build_stream_tables_x32(tab);
   if (warp == 0) umma::tmem_alloc(umma::smem_u32(&tmem_base_s), (uint32_t)p.tmem_cols);
+  const uint32_t lane4 = 4u * (uint32_t)lane;
   if (tid == 0) {
-    for (int s = 0; s < kStages; ++s) umma::mbar_init(umma::smem_u32(&mbar[s]), 1);
+    for (int s = 0; s < kStages; ++s) {
+      umma::mbar_init(umma::smem_u32(&full_bar[s]), kGThreads);
+      umma::mbar_init(umma::smem_u32(&empty_bar[s]), 1);
+    }
+    umma::mbar_init(umma::smem_u32(&acc_full_bar), 1);
+    umma::mbar_init(umma::smem_u32(&acc_empty_bar), 128);
     umma::mbar_init_fence();
+    s_abort = 0;
   }
   umma::fence_before_sync();
   __syncthreads();
@@ -108,11 +167,50 @@ __global__ void __launch_bounds__(kGThreads, 1) grouped_seed_gemm_kernel(const G
 
   const int total_tiles = p.tile_start[p.E];
   const int ksteps = p.K / kBK;
-  uint32_t it = 0;  // stage iterations issued by this CTA
-  bool abort = false;
-  for (int t = blockIdx.x; t < total_tiles && !abort; t += gridDim.x) {
-    // the expert owning tile t: the last e with tile_start[e] <= t
-    int lo_e = 0, hi_e = p.E - 1;
+  uint32_t it = 0;      // K slices produced (or consumed) by this CTA
+  uint32_t ntile = 0;   // tiles finished by this CTA
+
+  if (issuer_warp) {  // ---- the MMA warp: lane 0 waits for each slice and issues it
+    if (lane == 0) {
+      for (int t = blockIdx.x; t < total_tiles && !s_abort; t += gridDim.x, ++ntile) {
+        int lo_e = 0, hi_e = p.E - 1;
+        while (lo_e < hi_e) {
+          const int mid = (lo_e + hi_e + 1) >> 1;
+          if (p.tile_start[mid] <= t) lo_e = mid; else hi_e = mid - 1;
+        }
+        const int e = lo_e;
+        const int nt = (t - p.tile_start[e]) / p.mtiles;
+        const int r_begin = max(0, p.offsets[e]) + nt * p.bn;
+        const int n_valid = max(0, min(p.bn, min(p.R, p.offsets[e + 1]) - r_begin));
+        const uint32_t idesc = umma::idesc_bf16_f32(kBM, max(16, (n_valid + 15) & ~15));
+        for (int kt = 0; kt < ksteps; ++kt, ++it) {
+          const int stage = it & 1;
+          bool go = umma::mbar_wait_bounded(umma::smem_u32(&full_bar[stage]), (it >> 1) & 1, kWaitCycles);
+          if (go && kt == 0 && ntile > 0)  // the epilogue has drained the last tile's accumulators
+            go = umma::mbar_wait_bounded(umma::smem_u32(&acc_empty_bar), (ntile - 1) & 1, kWaitCycles);
+          if (!go) { s_abort = 1; break; }
+          umma::fence_after_sync();
+          const uint32_t asa = umma::smem_u32(a_base + (size_t)stage * 2 * kBM * 128);
+          const uint32_t bsa = umma::smem_u32(b_base + (size_t)stage * p.bn * 128);
+#pragma unroll
+          for (int s = 0; s < kBK / 16; ++s) {
+            const uint64_t bd = umma::smem_desc_kmajor(bsa + s * 256, 128, 1024);
+#pragma unroll
+            for (int a = 0; a < 2; ++a) {
+              const uint64_t ad = umma::smem_desc_kmajor(asa + a * kBM * 128 + s * 256, 128, 1024);
+              umma::mma_bf16(tmem + (uint32_t)(a * p.bn), ad, bd, idesc, (kt | s) != 0);
+            }
+          }
+          umma::commit(umma::smem_u32(&empty_bar[stage]));
+          if (kt == ksteps - 1) umma::commit(umma::smem_u32(&acc_full_bar));
+        }
+      }
+    }
+    __syncwarp();
+  } else
+  for (int t = blockIdx.x; t < total_tiles; t += gridDim.x, ++ntile) {
+    if (s_abort) break;
+    int lo_e = 0, hi_e = p.E - 1;  // the last e with tile_start[e] <= t
     while (lo_e < hi_e) {
       const int mid = (lo_e + hi_e + 1) >> 1;
       if (p.tile_start[mid] <= t) lo_e = mid; else hi_e = mid - 1;
@@ -124,107 +222,139 @@ __global__ void __launch_bounds__(kGThreads, 1) grouped_seed_gemm_kernel(const G
     const int r_begin = seg_begin + nt * p.bn;
     const int n_valid = max(0, min(p.bn, seg_end - r_begin));
     const int N = max(16, (n_valid + 15) & ~15);
-    const int m0 = mt * kBM;
-    const uint32_t idesc = umma::idesc_bf16_f32(kBM, N);
+    const int m0 = mt * kRows;
 
+    // the two tasks' weight rows for the whole tile
+    const uint32_t *sp[2];
+    const uint32_t *qp[2];
+    const uint8_t *cpp[2];
+    bool ok[2];
+    uint32_t rowk[2];
+#pragma unroll
+    for (int j = 0; j < 2; ++j) {
+      const nslm_seed_matrix &W = (MODE == GMODE_GATEUP && j) ? p.A1 : p.A0;
+      const int grow = m0 + (MODE == GMODE_GATEUP ? 0 : j * kBM) + trow;
+      ok[j] = grow < p.rows;
+      const size_t wr = (size_t)e * p.rows + (ok[j] ? grow : 0);
+      sp[j] = reinterpret_cast<const uint32_t *>(W.seeds + wr * p.nb) + bp;
+      qp[j] = reinterpret_cast<const uint32_t *>(W.coefs + wr * p.nb) + bp;
+      cpp[j] = (P == 4) ? W.codes + wr * (p.nb / 2) + bp : nullptr;
+      rowk[j] = row_scale_key(__ldg(W.exp_bias + wr));
+    }
+    const size_t a_off = ((trow >> 3) * 8 + 2 * bp) * 128 + (trow & 7) * 16;
+    // token rows this thread copies: chunks (n, kc) for n = trow, trow + 128 and kc = bp, bp + 4
+    const uint16_t *brow[2];
+    uint32_t bbytes[2], bdst[2][2];
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+      const int n = trow + 128 * i;
+#pragma unroll
+      for (int h = 0; h < 2; ++h) bdst[i][h] = ((n >> 3) * 8 + bp + 4 * h) * 128 + (n & 7) * 16;
+      const bool v = n < n_valid;
+      const int xr = v ? (p.row_of ? p.row_of[r_begin + n] : r_begin + n) : 0;
+      brow[i] = p.x + (size_t)xr * p.K;
+      bbytes[i] = v ? 16u : 0u;  // zero-fill rows past n_valid
+    }
+
+    SliceFields f0, f1;
+    load_slice<P>(sp, qp, cpp, ok, 0, f0);
+    if (ksteps > 1) load_slice<P>(sp, qp, cpp, ok, 1, f1);
     for (int kt = 0; kt < ksteps; ++kt, ++it) {
       const int stage = it & 1;
-      bool ok = true;
-      if (it >= 2) ok = umma::mbar_wait_bounded(umma::smem_u32(&mbar[stage]), ((it >> 1) - 1) & 1, kWaitCycles);
-      if (__syncthreads_or(!ok)) { abort = true; break; }
-
-      // ---- A: NA x 128 rows x 8 blocks, two blocks per task
-      for (int u = tid; u < NA * kBM * 4; u += kGThreads) {
-        const int a = u / (kBM * 4), rem = u - a * (kBM * 4);
-        const int row = rem & (kBM - 1), bp = rem >> 7;  // block pair 0..3
-        const nslm_seed_matrix &W = a ? p.A1 : p.A0;
-        uint8_t *tile = a_base + (size_t)(stage * NA + a) * kBM * 128;
-        uint4 *dst0 = reinterpret_cast<uint4 *>(tile + ((row >> 3) * 8 + 2 * bp) * 128 + (row & 7) * 16);
-        uint4 *dst1 = reinterpret_cast<uint4 *>(tile + ((row >> 3) * 8 + 2 * bp + 1) * 128 + (row & 7) * 16);
-        const int grow = m0 + row;
-        if (grow < p.rows) {
-          const size_t r = (size_t)e * p.rows + grow;
-          const int b = kt * 8 + 2 * bp;
-          const uint32_t s2 = __ldcs(reinterpret_cast<const uint32_t *>(W.seeds + r * p.nb + b));
-          const uint32_t q2 = __ldcs(reinterpret_cast<const uint32_t *>(W.coefs + r * p.nb + b));
-          const uint32_t c2 = (P == 4) ? (uint32_t)__ldcs(W.codes + r * (p.nb / 2) + b / 2) : 0u;
-          regen_pair_bf16<P>(tab, s2, q2, c2, row_scale_key(__ldg(W.exp_bias + r)), dst0, dst1);
-        } else {
-          *dst0 = make_uint4(0, 0, 0, 0);
-          *dst1 = make_uint4(0, 0, 0, 0);
-        }
-      }
-      // ---- B: N token rows x 8 chunks of 16 bytes (zeros past n_valid)
+      if (it >= 2 && !umma::mbar_wait_bounded(umma::smem_u32(&empty_bar[stage]), ((it >> 1) - 1) & 1, kWaitCycles))
+        s_abort = 1;
+      if (s_abort) break;
+      uint8_t *atile = a_base + (size_t)stage * 2 * kBM * 128;
       uint8_t *btile = b_base + (size_t)stage * p.bn * 128;
-      for (int u = tid; u < N * 8; u += kGThreads) {
-        const int n = u % N, kc = u / N;
-        uint4 v = make_uint4(0, 0, 0, 0);
-        if (n < n_valid) {
-          const int sr = r_begin + n;
-          const int xr = p.row_of ? p.row_of[sr] : sr;
-          v = __ldg(reinterpret_cast<const uint4 *>(p.x + (size_t)xr * p.K + kt * kBK + kc * 8));
+      // token rows for this slice: asynchronous copies, overlapped with the regeneration
+      const uint32_t bsa = umma::smem_u32(btile);
+#pragma unroll
+      for (int i = 0; i < 2; ++i) {
+        if (trow + 128 * i < N) {
+#pragma unroll
+          for (int h = 0; h < 2; ++h)
+            cp_async16(bsa + bdst[i][h], brow[i] + kt * kBK + (bp + 4 * h) * 8, bbytes[i]);
         }
-        *reinterpret_cast<uint4 *>(btile + ((n >> 3) * 8 + kc) * 128 + (n & 7) * 16) = v;
       }
+      const SliceFields cur = f0;
+      f0 = f1;
+      if (kt + 2 < ksteps) load_slice<P>(sp, qp, cpp, ok, kt + 2, f1);
+      // rows past the matrix carry zero coefficient fields, which regenerate
+      // to exactly zero weights: no branch
+#pragma unroll
+      for (int j = 0; j < 2; ++j) {
+        uint4 *dst0 = reinterpret_cast<uint4 *>(atile + j * kBM * 128 + a_off);
+        uint4 *dst1 = reinterpret_cast<uint4 *>(atile + j * kBM * 128 + a_off + 128);
+        regen_pair_bf16<P>(tab, lane4, cur.s2[j], cur.q2[j], cur.c2[j], rowk[j], dst0, dst1);
+      }
+      cp_async_wait_all();
       umma::fence_proxy_async();
-      __syncthreads();
-      if (tid == 0) {
+      umma::mbar_arrive(umma::smem_u32(&full_bar[stage]));
+
+    }
+    if (s_abort) break;
+
+    // ---- epilogue (warps 0-3): read D from tensor memory once the tile's MMAs are done
+    if (warp < 4) {
+      __syncwarp();
+      const bool acc_ok = umma::mbar_wait_bounded(umma::smem_u32(&acc_full_bar), ntile & 1, kWaitCycles);
+      if (!acc_ok) s_abort = 1;
+      // tcgen05.ld is warp-collective: the whole warp takes one decision
+      if (__all_sync(0xffffffffu, acc_ok && !s_abort)) {
         umma::fence_after_sync();
-        const uint32_t bsa = umma::smem_u32(btile);
+        const uint32_t lane_addr = tmem + ((uint32_t)(32 * warp) << 16);
+        if (MODE == GMODE_GATEUP) {
+          const int row = m0 + 32 * warp + lane;
+          const bool rok = row < p.rows;
+          for (int c = 0; c * 8 < N; ++c) {
+            float g[8], up[8];
+            umma::tmem_ld8(lane_addr + (uint32_t)(c * 8), g);
+            umma::tmem_ld8(lane_addr + (uint32_t)(p.bn + c * 8), up);
 #pragma unroll
-        for (int s = 0; s < kBK / 16; ++s) {
-          const uint64_t bd = umma::smem_desc_kmajor(bsa + s * 256, 128, 1024);
+            for (int j = 0; j < 8; ++j) {
+              const int n = c * 8 + j;
+              if (!rok || n >= n_valid) continue;
+              const size_t sr = (size_t)(r_begin + n);
+              p.h[sr * p.rows + row] = __bfloat16_as_ushort(__float2bfloat16_rn(g[j] / (1.f + expf(-g[j])) * up[j]));
+            }
+          }
+        } else {
 #pragma unroll
-          for (int a = 0; a < NA; ++a) {
-            const uint32_t asa = umma::smem_u32(a_base + (size_t)(stage * NA + a) * kBM * 128);
-            const uint64_t ad = umma::smem_desc_kmajor(asa + s * 256, 128, 1024);
-            umma::mma_bf16(tmem + (uint32_t)(a * p.bn), ad, bd, idesc, (kt | s) != 0);
+          for (int mh = 0; mh < 2; ++mh) {
+            const int row = m0 + mh * kBM + 32 * warp + lane;
+            const bool rok = row < p.rows;
+            for (int c = 0; c * 8 < N; ++c) {
+              float v[8];
+              umma::tmem_ld8(lane_addr + (uint32_t)(mh * p.bn + c * 8), v);
+#pragma unroll
+              for (int j = 0; j < 8; ++j) {
+                const int n = c * 8 + j;
+                if (!rok || n >= n_valid) continue;
+                const size_t sr = (size_t)(r_begin + n);
+                if (MODE == GMODE_GEMM) {
+                  p.y[sr * p.rows + row] = v[j];
+                } else {
+                  const int pr = p.pair_of[sr];
+                  p.part[(size_t)pr * p.rows + row] = p.pair_w[pr] * v[j];
+                }
+              }
+            }
           }
         }
-        umma::commit(umma::smem_u32(&mbar[stage]));
+        umma::fence_before_sync();
+        umma::mbar_arrive(umma::smem_u32(&acc_empty_bar));
       }
     }
-    if (abort) break;
-
-    // ---- epilogue: wait for the tile's last MMAs, read D from tensor memory
-    const uint32_t last = it - 1;
-    const bool ok = umma::mbar_wait_bounded(umma::smem_u32(&mbar[last & 1]), (last >> 1) & 1, kWaitCycles);
-    if (__syncthreads_or(!ok)) { abort = true; break; }
-    umma::fence_after_sync();
-    const int q = warp & 3;                     // lane quarter this warp may read
-    const int row = m0 + 32 * q + lane;
-    const bool row_ok = row < p.rows;
-    const uint32_t lane_addr = tmem + ((uint32_t)(32 * q) << 16);
-    for (int c = warp >> 2; c * 8 < N; c += kGThreads / 128) {
-      float v[8], v2[8];
-      umma::tmem_ld8(lane_addr + (uint32_t)(c * 8), v);
-      if (MODE == GMODE_GATEUP) umma::tmem_ld8(lane_addr + (uint32_t)(p.bn + c * 8), v2);
-#pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        const int n = c * 8 + j;
-        if (!row_ok || n >= n_valid) continue;
-        const size_t sr = (size_t)(r_begin + n);
-        if (MODE == GMODE_GEMM) {
-          p.y[sr * p.rows + row] = v[j];
-        } else if (MODE == GMODE_GATEUP) {
-          const float g = v[j], up = v2[j];
-          p.h[sr * p.rows + row] = __bfloat16_as_ushort(__float2bfloat16_rn(g / (1.f + expf(-g)) * up));
-        } else {
-          const int pr = p.pair_of[sr];
-          p.part[(size_t)pr * p.rows + row] = p.pair_w[pr] * v[j];
-        }
-      }
-    }
-    umma::fence_before_sync();
-    __syncthreads();
   }
 
-  if (abort) {
+  cp_async_wait_all();
+  __syncthreads();
+  if (s_abort) {
     if (tid == 0) atomicExch(p.status, 1);
     // let MMAs still in flight finish (bounded) before the tensor memory is freed
-    if (it > 0) {
+    if (tid == kGThreads && it > 0) {
       const uint32_t last = it - 1;
-      umma::mbar_wait_bounded(umma::smem_u32(&mbar[last & 1]), (last >> 1) & 1, kWaitCycles);
+      umma::mbar_wait_bounded(umma::smem_u32(&empty_bar[last & 1]), (last >> 1) & 1, kWaitCycles);
     }
   }
   umma::fence_before_sync();
@@ -333,17 +463,16 @@ static int tmem_cols_for(int ncols) {
   return c;
 }
 
-static size_t grouped_smem(int NA, int bn) {
-  return 2048 + (size_t)kStages * NA * kBM * 128 + (size_t)kStages * bn * 128;
+static size_t grouped_smem(int bn) {
+  return sizeof(StreamTablesX32) + (size_t)kStages * 2 * kBM * 128 + (size_t)kStages * bn * 128;
 }
 
 template <int P, int MODE>
 static int32_t launch_grouped_t(const GroupedParams &p, cudaStream_t s) {
-  constexpr int NA = (MODE == GMODE_GATEUP) ? 2 : 1;
-  const size_t smem = grouped_smem(NA, p.bn);
+  const size_t smem = grouped_smem(p.bn);
   auto kern = grouped_seed_gemm_kernel<P, MODE>;
   if (int32_t st = ensure_smem((const void *)kern, smem)) return st;
-  kern<<<num_sms(), kGThreads, smem, s>>>(p);
+  kern<<<num_sms(), kCtaThreads, smem, s>>>(p);
   return launch_status();
 }
 
@@ -358,9 +487,10 @@ int32_t launch_grouped(const GroupedParams &p, int P, int mode, cudaStream_t s) 
   return launch_grouped_t<3, GMODE_DOWN>(p, s);
 }
 
+// Token rows per tile (up to 256: two accumulators of 256 fp32 columns fill the
+// 512 tensor-memory columns); experts with more rows take several tiles.
 static int choose_bn(int max_rows_per_expert) {
-  const int r = std::max(16, (std::min(max_rows_per_expert, 256) + 15) & ~15);
-  return r;
+  return std::max(16, (std::min(max_rows_per_expert, 256) + 15) & ~15);
 }
 
 BatchedPlan batched_workspace(char *base, int T, int k, int E, int hidden, int inter) {
@@ -388,7 +518,8 @@ int32_t launch_batched_ffn(const FfnDims &d, const nslm_seed_matrix *gate, const
   if (d.hidden % kBK || d.inter % kBK || d.E > 1024) return NSLM_ERR_SHAPE;
   const BatchedPlan bp = batched_workspace(reinterpret_cast<char *>(ws), T, k, d.E, d.hidden, d.inter);
   const int bn = choose_bn(T);  // an expert gets at most T pairs (one per token)
-  const int mt_gu = ceil_div(d.inter, kBM), mt_dn = ceil_div(d.hidden, kBM);
+  const int mt_gu = ceil_div(d.inter, TileShape<GMODE_GATEUP>::kRows);
+  const int mt_dn = ceil_div(d.hidden, TileShape<GMODE_DOWN>::kRows);
   batched_plan_kernel<<<1, 1024, 0, s>>>(ids, T, d.E, k, bn, mt_gu, mt_dn, bp);
   if (int32_t st = launch_status()) return st;
   ++launches;
@@ -406,7 +537,7 @@ int32_t launch_batched_ffn(const FfnDims &d, const nslm_seed_matrix *gate, const
     GroupedParams p{};
     p.A0 = *down; p.E = d.E; p.rows = d.hidden; p.K = d.inter; p.nb = d.inter / 8;
     p.R = TK; p.x = bp.h; p.row_of = nullptr; p.offsets = bp.offsets; p.tile_start = bp.tiles_dn;
-    p.mtiles = mt_dn; p.bn = bn; p.tmem_cols = tmem_cols_for(bn); p.status = bp.status;
+    p.mtiles = mt_dn; p.bn = bn; p.tmem_cols = tmem_cols_for(2 * bn); p.status = bp.status;
     p.part = bp.part; p.pair_of = bp.pair_of; p.pair_w = w;
     if (int32_t st = launch_grouped(p, d.P, GMODE_DOWN, s)) return st;
     ++launches;
@@ -449,13 +580,13 @@ extern "C" int32_t nslm_seed_grouped_gemm(const nslm_seed_matrix *W, int32_t E,
   int32_t *tile_start = status + 1;
   const int rows = W->N / E;
   const int bn = choose_bn(R);
-  const int mtiles = ceil_div(rows, kBM);
+  const int mtiles = ceil_div(rows, TileShape<GMODE_GEMM>::kRows);
   tile_prefix_kernel<<<1, 1024, 0, s>>>(offsets, E, mtiles, bn, R, tile_start, status);
   if ((st = launch_status())) return st;
   GroupedParams p{};
   p.A0 = *W; p.E = E; p.rows = rows; p.K = W->K; p.nb = W->K / 8; p.R = R; p.x = x_bf16;
   p.row_of = nullptr; p.offsets = offsets; p.tile_start = tile_start; p.mtiles = mtiles; p.bn = bn;
-  p.tmem_cols = tmem_cols_for(bn); p.status = status; p.y = y;
+  p.tmem_cols = tmem_cols_for(2 * bn); p.status = status; p.y = y;
   st = launch_grouped(p, W->P, GMODE_GEMM, s);
   if (st == NSLM_OK) g_launches = 2;
   return st;

@@ -75,6 +75,28 @@ __device__ __forceinline__ void build_stream_tables(StreamTables *tab) {
   for (int i = threadIdx.x; i < 512; i += blockDim.x) tab->t[i] = kStreamTab.t[i];
 }
 
+// The same tables replicated 32 times and interleaved by lane: entry i of copy
+// c at word i * 32 + c.  Lane l reads copy l, so the 32 lanes of a warp never
+// hit the same bank whatever seeds they hold (64 KB of shared memory).
+struct StreamTablesX32 {
+  uint32_t t[512 * 32];
+};
+
+__device__ __forceinline__ void build_stream_tables_x32(StreamTablesX32 *tab) {
+  for (int i = threadIdx.x; i < 512 * 32; i += blockDim.x) tab->t[i] = kStreamTab.t[i >> 5];
+}
+
+// W = seed | next32 << 16 from the replicated tables; lane4 = 4 * (lane id).
+__device__ __forceinline__ void stream_word_x32(const StreamTablesX32 *tab, uint32_t lane4, uint32_t seed,
+                                                uint32_t &lo, uint32_t &hi) {
+  const char *base = reinterpret_cast<const char *>(tab->t) + lane4;
+  const uint32_t a = *reinterpret_cast<const uint32_t *>(base + ((seed & 0xFFu) << 7));
+  const uint32_t b = *reinterpret_cast<const uint32_t *>(base + (((seed >> 8) & 0xFFu) << 7) + 256 * 128);
+  const uint32_t nxt = a ^ b;
+  lo = __byte_perm(seed, nxt, 0x5410);
+  hi = nxt >> 16;
+}
+
 // W = seed | next32 << 16, returned as (lo = bits 0..31, hi = bits 32..47).
 __device__ __forceinline__ void stream_word(const StreamTables *tab, uint32_t seed,
                                             uint32_t &lo, uint32_t &hi) {
@@ -104,6 +126,13 @@ __device__ __forceinline__ int32_t dp4a_us(uint32_t a_u8x4, uint32_t b_s8x4, int
 __device__ __forceinline__ int32_t dp4a_ss(uint32_t a_s8x4, uint32_t b_s8x4, int32_t acc) {
   int32_t d;
   asm("dp4a.s32.s32 %0, %1, %2, %3;" : "=r"(d) : "r"(a_s8x4), "r"(b_s8x4), "r"(acc));
+  return d;
+}
+
+// a * b + c in one integer multiply-add.
+__device__ __forceinline__ int32_t imad(int32_t a, int32_t b, int32_t c) {
+  int32_t d;
+  asm("mad.lo.s32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
   return d;
 }
 

@@ -89,15 +89,21 @@ __device__ __forceinline__ void mbar_init(uint32_t mbar, uint32_t count) {
 __device__ __forceinline__ void mbar_init_fence() {
   asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
 }
+// One bounded wait: the thread may be suspended by the hardware for up to
+// about 1 ms (instead of spinning) until the phase completes.
 __device__ __forceinline__ bool mbar_try_wait(uint32_t mbar, uint32_t parity) {
   uint32_t done;
   asm volatile(
-      "{\n\t.reg .pred P1;\n\tmbarrier.try_wait.parity.shared::cta.b64 P1, [%1], %2;\n\t"
+      "{\n\t.reg .pred P1;\n\tmbarrier.try_wait.parity.shared::cta.b64 P1, [%1], %2, %3;\n\t"
       "selp.b32 %0, 1, 0, P1;\n\t}"
       : "=r"(done)
-      : "r"(mbar), "r"(parity)
+      : "r"(mbar), "r"(parity), "r"(1000000u)
       : "memory");
   return done != 0;
+}
+
+__device__ __forceinline__ void mbar_arrive(uint32_t mbar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(mbar) : "memory");
 }
 
 // Wait for the phase of the given parity to complete, for at most ~max_cycles

@@ -63,7 +63,13 @@ def test_ffn_argument_checks():
     assert call(dd=_mat(E * hidden, inter + 8)) == nslm.NSLM_ERR_SHAPE
     assert call(E_=3) == nslm.NSLM_ERR_SHAPE                  # rows not divisible by E
     assert call(k=9) == nslm.NSLM_ERR_SHAPE
-    assert call(T=9) == nslm.NSLM_ERR_SHAPE
+    # T > 8 takes the tensor-core path: it needs its own (larger) workspace ...
+    assert call(T=9) == nslm.NSLM_ERR_WORKSPACE
+    big = nslm.nslm_workspace_bytes(nslm.NSLM_OP_MOE_FFN, 9, E, hidden, inter, 2)
+    assert big > ws_need
+    # ... and hidden / inter multiples of 64
+    g72, u72, d72 = _mat(E * 72, hidden), _mat(E * 72, hidden), _mat(E * hidden, 72)
+    assert call(gg=g72, uu=u72, dd=d72, T=9, wsb=1 << 30) == nslm.NSLM_ERR_SHAPE
     assert call(wsb=ws_need - 1) == nslm.NSLM_ERR_WORKSPACE
     assert call(ws=0) == nslm.NSLM_ERR_WORKSPACE
     assert call(x=0) == nslm.NSLM_ERR_ARG
