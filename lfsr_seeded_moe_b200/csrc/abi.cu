@@ -72,6 +72,31 @@ int32_t ensure_smem(const void *kernel, size_t bytes) {
   return NSLM_OK;
 }
 
+struct OccEntry {
+  const void *kernel;
+  int device, threads;
+  size_t smem;
+  int ctas;
+};
+static OccEntry g_occ[256];
+static int g_occ_n = 0;
+
+int32_t max_active_ctas(const void *kernel, int threads, size_t smem) {
+  const int dev = current_device();
+  std::lock_guard<std::mutex> lock(g_mu);
+  for (int i = 0; i < g_occ_n; ++i)
+    if (g_occ[i].kernel == kernel && g_occ[i].device == dev && g_occ[i].threads == threads && g_occ[i].smem == smem)
+      return g_occ[i].ctas;
+  int n = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kernel, threads, smem) != cudaSuccess) {
+    (void)cudaGetLastError();
+    n = 1;
+  }
+  n = n < 1 ? 1 : n;
+  if (g_occ_n < 256) g_occ[g_occ_n++] = OccEntry{kernel, dev, threads, smem, n};
+  return n;
+}
+
 int32_t check_matrix(const nslm_seed_matrix *W) {
   if (!W) return NSLM_ERR_ARG;
   if (W->P != 3 && W->P != 4) return NSLM_ERR_SHAPE;
@@ -265,7 +290,7 @@ int32_t nslm_moe_seed_ffn(const nslm_seed_matrix *gate, const nslm_seed_matrix *
                               d.hidden, s)))
     return st;
   int launches = 1;
-  st = launch_decode_layer(d, gate, up, down, fw.plans, x_bf16, nullptr, T, k, fw, y, s, launches);
+  st = launch_decode_layer(d, gate, up, down, fw.plans, x_bf16, nullptr, T, k, fw, y, false, s, launches);
   if (st == NSLM_OK) g_launches = launches;
   return st;
 }
@@ -299,8 +324,9 @@ int32_t nslm_moe_stack_decode(const nslm_moe_layer *layers, int32_t L, int32_t E
     const uint16_t *xin = (l == 0) ? x0_bf16 : nullptr;
     const float *yprev = (l == 0) ? nullptr : fw.y_mid;
     float *yout = (l == L - 1) ? y : fw.y_mid;
+    // layer l > 0: the routing kernel ran at least two kernels back
     st = launch_decode_layer(d, &layers[l].gate, &layers[l].up, &layers[l].down, fw.plans + l, xin,
-                             yprev, T, k, fw, yout, s, launches);
+                             yprev, T, k, fw, yout, l > 0, s, launches);
     if (st) return st;
   }
   g_launches = launches;

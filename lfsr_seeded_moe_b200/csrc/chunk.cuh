@@ -15,6 +15,7 @@
 #pragma once
 #include <cuda_bf16.h>
 
+#include "../../include/nslm.h"
 #include "regen.cuh"
 
 namespace nslm {
@@ -45,6 +46,24 @@ __device__ __forceinline__ void xs_store_block(float4 *xs4, float2 *xn2, int m, 
   xs4[xs_index(m, b & 7, 1, b >> 3, cpad)] = hi;
   const float sum = ((lo.x + lo.y) + (lo.z + lo.w)) + ((hi.x + hi.y) + (hi.z + hi.w));
   xn2[xn_index(m, b & 7, b >> 3, cpad)] = make_float2(-kMagic2 * sum, 0.f);
+}
+
+// Chunk-major layout, for kernels in which every lane reads one chunk slot:
+//   xs4[17 q + 2 i + h] = x[64 q + 8 i + 4 h .. +3]
+//   xn2[9 q + i]        = (-Mg * sum of block 8 q + i, 0)
+// A lane's 24 reads are then immediate offsets from two base addresses, and
+// the odd strides (17 x 16 bytes, 9 x 8 bytes) put consecutive slots in
+// distinct banks.
+constexpr int kCmX4 = 17, kCmXn = 9;
+__host__ __device__ inline size_t cm_bytes(int slots) {
+  return (size_t)slots * (kCmX4 * sizeof(float4) + kCmXn * sizeof(float2));
+}
+__device__ __forceinline__ void cm_store_block(float4 *xs4, float2 *xn2, int b, float4 lo, float4 hi) {
+  const int q = b >> 3, i = b & 7;
+  xs4[kCmX4 * q + 2 * i] = lo;
+  xs4[kCmX4 * q + 2 * i + 1] = hi;
+  const float sum = ((lo.x + lo.y) + (lo.z + lo.w)) + ((hi.x + hi.y) + (hi.z + hi.w));
+  xn2[kCmXn * q + i] = make_float2(-kMagic2 * sum, 0.f);
 }
 
 // 8 bf16 values (one 16-byte word) -> two float4.
@@ -80,6 +99,26 @@ __device__ __forceinline__ void stage_f32(float4 *xs4, float2 *xn2, const float 
     for (int b = threadIdx.x; b < nb; b += blockDim.x)
       xs_store_block(xs4, xn2, m, b, cpad, __ldcg(row + 2 * b), __ldcg(row + 2 * b + 1));
   }
+}
+
+// Asynchronous global -> shared copies (cp.async): 16 bytes with zero fill
+// past src_bytes, 16 bytes, 4 bytes; commit / wait on this thread's groups.
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void *src, uint32_t src_bytes) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(src_bytes) : "memory");
+}
+__device__ __forceinline__ void cp_async16(void *dst, const void *src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"((uint32_t)__cvta_generic_to_shared(dst)),
+               "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async4(void *dst, const void *src) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"((uint32_t)__cvta_generic_to_shared(dst)),
+               "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+__device__ __forceinline__ void cp_async_wait_all() {
+  asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
 }
 
 // Fields of the 8 blocks of a chunk: seeds and coefs as 4 words of two
@@ -122,14 +161,64 @@ __device__ __forceinline__ void load_chunk(const uint16_t *__restrict__ seeds_ro
   }
 }
 
-// Two's-complement nibbles -> doubled signed bytes [2c0, 2c1, 2c2, 2c3]
+// Shared-memory landing slots for the fields of one whole chunk per thread
+// (structure of arrays over the n threads of a CTA, so that a warp's 16-byte
+// reads are contiguous): seeds, coefs, codes word, exponent bias.
+struct FieldSlots {
+  uint4 *s, *q;
+  uint32_t *c;
+  int32_t *b;
+  __host__ __device__ static size_t bytes(int n) { return (size_t)n * 40; }
+  __device__ __forceinline__ FieldSlots(void *base, int n) {
+    s = reinterpret_cast<uint4 *>(base);
+    q = s + n;
+    c = reinterpret_cast<uint32_t *>(q + n);
+    b = reinterpret_cast<int32_t *>(c + n);
+  }
+};
+
+// Start the copies of chunk ch of row `grow` (whole chunks) into slot i.
+template <int P>
+__device__ __forceinline__ void fetch_chunk(const nslm_seed_matrix &W, size_t grow, int nb, int ch,
+                                            const FieldSlots &fs, int i) {
+  cp_async16(fs.s + i, W.seeds + grow * nb + ch * 8);
+  cp_async16(fs.q + i, W.coefs + grow * nb + ch * 8);
+  if (P == 4) cp_async4(fs.c + i, W.codes + grow * (nb / 2) + ch * 4);
+  cp_async4(fs.b + i, W.exp_bias + grow);
+}
+
+// Read slot i back (after the copies have completed).
+template <int P>
+__device__ __forceinline__ void read_chunk(const FieldSlots &fs, int i, ChunkFields &f, uint32_t &rowk) {
+  const uint4 s = fs.s[i], q = fs.q[i];
+  f.s[0] = s.x; f.s[1] = s.y; f.s[2] = s.z; f.s[3] = s.w;
+  f.q[0] = q.x; f.q[1] = q.y; f.q[2] = q.z; f.q[3] = q.w;
+  f.codes = (P == 4) ? fs.c[i] : 0u;
+  rowk = row_scale_key(fs.b[i]);
+}
+
+// Two's-complement nibbles -> doubled signed bytes in the order dp2a pairs
+// them with the 16-bit halves of a funnel shift: [2c0, 2c2, 2c1, 2c3]
 // (P = 3: byte 3 is 0; the top nibble there is the exponent code).
 template <int P>
-__device__ __forceinline__ uint32_t coef_bytes2(uint32_t q16) {
-  uint32_t v = (q16 | (q16 << 12)) & 0x0F0F0F0Fu;       // [c0, c2, c1, c3] as nibbles
-  v = __byte_perm(v, 0u, P == 4 ? 0x3120 : 0x4120);     // [c0, c1, c2, c3|0]
+__device__ __forceinline__ uint32_t coef_pairs2(uint32_t q16) {
+  const uint32_t v = (q16 | (q16 << 12)) & (P == 4 ? 0x0F0F0F0Fu : 0x000F0F0Fu);
   // 2c mod 256 per byte: 2q, plus 224 where bit 3 is set (no carry out)
   return (v << 1) + (v & 0x08080808u) * 28u;
+}
+
+// G[r] = Mg + A_r (exact fp32) from the stream (v, nxt) of a block and its
+// coefficient pairs.  W >> (1+r) holds the states s_{1+r} and s_{17+r} in its
+// two 16-bit halves (j = 0, 2) and W >> (9+r) holds s_{9+r} and s_{25+r}
+// (j = 1, 3), so two dp2a give sum_j 2 c_j s_{1+8j+r}; the accumulator starts
+// at the bits of Mg minus 2 * 32768 * sum_j c_j, and the fp32 step at Mg is 0.5.
+__device__ __forceinline__ void block_magic(uint32_t v, uint32_t nxt, uint32_t cp2, float (&G)[8]) {
+  const int32_t base = (int32_t)kMagic2Bits - 32768 * dp4a_ss(cp2, 0x01010101u, 0);
+#pragma unroll
+  for (int r = 0; r < 8; ++r) {
+    const uint32_t z = (r == 7) ? nxt : __funnelshift_r(v, nxt, 25 + r);  // W >> (9+r)
+    G[r] = __int_as_float(dp2a_hi_us(z, cp2, dp2a_lo_us(__funnelshift_r(v, nxt, 17 + r), cp2, base)));
+  }
 }
 
 // Regenerate block i (0..7) of a loaded chunk: G[r] = Mg + A_r (exact fp32);
@@ -138,19 +227,11 @@ template <int P>
 __device__ __forceinline__ float regen_chunk_block(const StreamTables *tab, const ChunkFields &f,
                                                    int i, uint32_t rowk, float (&G)[8]) {
   const uint32_t sw = f.s[i >> 1], qw = f.q[i >> 1];
-  const uint32_t seed = (i & 1) ? (sw >> 16) : (sw & 0xFFFFu);
   const uint32_t q = (i & 1) ? (qw >> 16) : (qw & 0xFFFFu);
-  uint32_t lo, hi;
-  stream_word(tab, seed, lo, hi);
-  const uint32_t cb2 = coef_bytes2<P>(q);
-  const int32_t base = (int32_t)kMagic2Bits - 32768 * dp4a_ss(cb2, 0x01010101u, 0);
-#pragma unroll
-  for (int r = 0; r < 8; ++r) {
-    // bytes of W >> (9+r) weigh 256, bytes of W >> (1+r) weigh 1; the sum is
-    // the bit pattern of Mg + 2 A_r ulps = Mg + A_r
-    const int32_t d1 = dp4a_us(__funnelshift_r(lo, hi, 9 + r), cb2, 0);
-    G[r] = __int_as_float(dp4a_us(__funnelshift_r(lo, hi, 1 + r), cb2, imad(d1, 256, base)));
-  }
+  uint32_t v, nxt;
+  if (i & 1) stream_pair_of<1>(tab, sw, v, nxt);
+  else stream_pair_of<0>(tab, sw, v, nxt);
+  block_magic(v, nxt, coef_pairs2<P>(q), G);
   const uint32_t code = (P == 4) ? ((f.codes >> (4 * i)) & 0xFu) : (q >> 12);
   return block_scale(code, rowk);
 }
@@ -218,11 +299,166 @@ __device__ __forceinline__ void chunk_dot2(const StreamTables *tab, const ChunkF
   }
 }
 
+// <G, x> - Mg * sum(x) for one staged block, as a packed pair of partial sums.
+__device__ __forceinline__ float2 block_dot2(const float (&G)[8], const float4 &xa, const float4 &xb,
+                                             const float2 &xn) {
+  float2 p = __ffma2_rn(make_float2(G[0], G[1]), make_float2(xa.x, xa.y), xn);
+  p = __ffma2_rn(make_float2(G[2], G[3]), make_float2(xa.z, xa.w), p);
+  p = __ffma2_rn(make_float2(G[4], G[5]), make_float2(xb.x, xb.y), p);
+  return __ffma2_rn(make_float2(G[6], G[7]), make_float2(xb.z, xb.w), p);
+}
+
+// One chunk against one staged vector whose chunk slot is at xa (float4 pair
+// stride `stride` between the 16 half-blocks) and xn (stride `stride` between
+// the 8 block offsets): acc += sum_b scale_b * <w_b, x_b> as a packed pair.
+// nvalid: blocks of the chunk inside the row (8 unless the row is ragged).
+template <int P, bool VEC>
+__device__ __forceinline__ void chunk_dot_at(const StreamTables *tab, const ChunkFields &f, int nvalid,
+                                             uint32_t rowk, const float4 *xa, const float2 *xn,
+                                             int stride, float2 &acc) {
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    if (!VEC && i >= nvalid) break;
+    float G[8];
+    const float s = regen_chunk_block<P>(tab, f, i, rowk, G);
+    const float2 d = block_dot2(G, xa[(2 * i) * stride], xa[(2 * i + 1) * stride], xn[i * stride]);
+    acc = __ffma2_rn(make_float2(s, s), d, acc);
+  }
+}
+
+// Two chunks (the gate and up rows of one expert) against the same staged
+// vector, interleaved block by block.
+template <int P, bool VEC>
+__device__ __forceinline__ void chunk_dot2_at(const StreamTables *tab, const ChunkFields &fa,
+                                              const ChunkFields &fb, int nvalid, uint32_t rowka,
+                                              uint32_t rowkb, const float4 *xa, const float2 *xn,
+                                              int stride, float2 &acca, float2 &accb) {
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    if (!VEC && i >= nvalid) break;
+    float Ga[8], Gb[8];
+    const float sa = regen_chunk_block<P>(tab, fa, i, rowka, Ga);
+    const float sb = regen_chunk_block<P>(tab, fb, i, rowkb, Gb);
+    const float4 x0 = xa[(2 * i) * stride], x1 = xa[(2 * i + 1) * stride];
+    const float2 x2 = xn[i * stride];
+    acca = __ffma2_rn(make_float2(sa, sa), block_dot2(Ga, x0, x1, x2), acca);
+    accb = __ffma2_rn(make_float2(sb, sb), block_dot2(Gb, x0, x1, x2), accb);
+  }
+}
+
+// Packed fp32x2 products (FFMA2) or scalar FFMA chains in the chunk-major dots.
+constexpr bool kPackedDot = true;
+
+// scale * (<G, x> - Mg * sum(x)) added to acc, for one staged block.
+__device__ __forceinline__ void block_fma(const float (&G)[8], float s, const float4 &xa, const float4 &xb,
+                                          const float2 &xn, float2 &acc) {
+  if (kPackedDot) {
+    acc = __ffma2_rn(make_float2(s, s), block_dot2(G, xa, xb, xn), acc);
+  } else {
+    float a = fmaf(G[0], xa.x, xn.x);
+    a = fmaf(G[1], xa.y, a);
+    a = fmaf(G[2], xa.z, a);
+    a = fmaf(G[3], xa.w, a);
+    a = fmaf(G[4], xb.x, a);
+    a = fmaf(G[5], xb.y, a);
+    a = fmaf(G[6], xb.z, a);
+    a = fmaf(G[7], xb.w, a);
+    acc.x = fmaf(s, a, acc.x);
+  }
+}
+
+// One chunk against the staged slot at xa (16 float4) / xn (8 float2) of the
+// chunk-major layout: acc += sum_b scale_b * <w_b, x_b>.
+template <int P, bool VEC>
+__device__ __forceinline__ void chunk_dot_cm(const StreamTables *tab, const ChunkFields &f, int nvalid,
+                                             uint32_t rowk, const float4 *xa, const float2 *xn, float2 &acc) {
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    if (!VEC && i >= nvalid) break;
+    float G[8];
+    const float s = regen_chunk_block<P>(tab, f, i, rowk, G);
+    block_fma(G, s, xa[2 * i], xa[2 * i + 1], xn[i], acc);
+  }
+}
+
+// The gate and up chunks of one row against the same staged slot.
+template <int P, bool VEC>
+__device__ __forceinline__ void chunk_dot2_cm(const StreamTables *tab, const ChunkFields &fa,
+                                              const ChunkFields &fb, int nvalid, uint32_t rowka,
+                                              uint32_t rowkb, const float4 *xa, const float2 *xn,
+                                              float2 &acca, float2 &accb) {
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    if (!VEC && i >= nvalid) break;
+    float Ga[8], Gb[8];
+    const float sa = regen_chunk_block<P>(tab, fa, i, rowka, Ga);
+    const float sb = regen_chunk_block<P>(tab, fb, i, rowkb, Gb);
+    const float4 x0 = xa[2 * i], x1 = xa[2 * i + 1];
+    const float2 x2 = xn[i];
+    block_fma(Ga, sa, x0, x1, x2, acca);
+    block_fma(Gb, sb, x0, x1, x2, accb);
+  }
+}
+
 // Sum of a float over the 32 lanes of a warp (fixed order: deterministic).
 __device__ __forceinline__ float warp_sum(float v) {
 #pragma unroll
   for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
   return v;
+}
+
+// ------------------------------------------------------- activation staging
+
+// Stage the activations of M tokens (rows[m]) into vectors m of the chunk
+// layout.  Source is either bf16 x [T][K], or fp32 y [T][K] normalised per
+// token to bf16(y / sqrt(mean(y^2) + 1e-6)).
+template <bool CM>
+static __device__ __noinline__ void stage_activations(float4 *xs4, float2 *xn2, const uint16_t *__restrict__ x_bf16,
+                                  const float *__restrict__ y_prev, const int *rows, int M, int K,
+                                  int cpad, float *scratch /* >= 33 floats */) {
+  const int tid = threadIdx.x, nthr = blockDim.x, nb = K >> 3;
+  if (x_bf16) {
+    if (!CM) {
+      stage_bf16(xs4, xn2, x_bf16, rows, M, K, cpad);
+      return;
+    }
+    // chunk-major: one vector
+    const uint4 *row = reinterpret_cast<const uint4 *>(x_bf16 + (size_t)rows[0] * K);
+    for (int b = tid; b < nb; b += nthr) {
+      float4 lo, hi;
+      bf16x8_to_f32(__ldg(row + b), lo, hi);
+      cm_store_block(xs4, xn2, b, lo, hi);
+    }
+    return;
+  }
+  for (int m = 0; m < M; ++m) {
+    const float4 *row = reinterpret_cast<const float4 *>(y_prev + (size_t)rows[m] * K);
+    float ss = 0.f;
+    for (int i = tid; i < 2 * nb; i += nthr) {
+      const float4 v = __ldcg(row + i);
+      ss = fmaf(v.x, v.x, fmaf(v.y, v.y, fmaf(v.z, v.z, fmaf(v.w, v.w, ss))));
+    }
+    ss = warp_sum(ss);
+    if ((tid & 31) == 0) scratch[tid >> 5] = ss;
+    __syncthreads();
+    if (tid == 0) {
+      float t = 0.f;
+      for (int w = 0; w < (nthr + 31) / 32; ++w) t += scratch[w];
+      scratch[32] = sqrtf(t / (float)K + 1e-6f);
+    }
+    __syncthreads();
+    const float r = scratch[32];
+    for (int b = tid; b < nb; b += nthr) {
+      float4 lo = __ldcg(row + 2 * b), hi = __ldcg(row + 2 * b + 1);
+#define NSLM_NORM(v) __bfloat162float(__float2bfloat16_rn(__fdiv_rn((v), r)))
+      lo = make_float4(NSLM_NORM(lo.x), NSLM_NORM(lo.y), NSLM_NORM(lo.z), NSLM_NORM(lo.w));
+      hi = make_float4(NSLM_NORM(hi.x), NSLM_NORM(hi.y), NSLM_NORM(hi.z), NSLM_NORM(hi.w));
+#undef NSLM_NORM
+      if (CM) cm_store_block(xs4, xn2, b, lo, hi);
+      else xs_store_block(xs4, xn2, m, b, cpad, lo, hi);
+    }
+    __syncthreads();  // scratch is reused by the next token
+  }
 }
 
 // Row sums of per-thread partials: red[v * nthr + r * cpad + c] holds value v of

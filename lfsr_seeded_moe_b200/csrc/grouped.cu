@@ -64,23 +64,18 @@ __device__ __forceinline__ void regen_pair_bf16(const StreamTablesX32 *tab, uint
   for (int h = 0; h < 2; ++h) {
     const uint32_t seed = h ? (seeds2 >> 16) : (seeds2 & 0xFFFFu);
     const uint32_t q = h ? (coefs2 >> 16) : (coefs2 & 0xFFFFu);
-    uint32_t lo, hi;
-    stream_word_x32(tab, lane4, seed, lo, hi);
-    const uint32_t cb2 = coef_bytes2<P>(q);
-    const int32_t base = (int32_t)kMagic2Bits - 32768 * dp4a_ss(cb2, 0x01010101u, 0);
+    uint32_t v, nxt;
+    stream_pair_x32(tab, lane4, seed, v, nxt);
+    float G[8];
+    block_magic(v, nxt, coef_pairs2<P>(q), G);
     const uint32_t code = (P == 4) ? ((code2 >> (4 * h)) & 0xFu) : (q >> 12);
     const float s = block_scale(code, rowk);
     const float off = -kMagic2 * s;
     uint32_t packed[4];
 #pragma unroll
     for (int r = 0; r < 8; r += 2) {
-      const int32_t a0 = dp4a_us(__funnelshift_r(lo, hi, 1 + r), cb2,
-                                 imad(dp4a_us(__funnelshift_r(lo, hi, 9 + r), cb2, 0), 256, base));
-      const int32_t a1 = dp4a_us(__funnelshift_r(lo, hi, 2 + r), cb2,
-                                 imad(dp4a_us(__funnelshift_r(lo, hi, 10 + r), cb2, 0), 256, base));
       // (Mg + A) * s - Mg * s = A * s exactly (power-of-two scale)
-      const __nv_bfloat162 b =
-          __floats2bfloat162_rn(fmaf(__int_as_float(a0), s, off), fmaf(__int_as_float(a1), s, off));
+      const __nv_bfloat162 b = __floats2bfloat162_rn(fmaf(G[r], s, off), fmaf(G[r + 1], s, off));
       packed[r >> 1] = *reinterpret_cast<const uint32_t *>(&b);
     }
     *(h ? dst1 : dst0) = make_uint4(packed[0], packed[1], packed[2], packed[3]);
@@ -123,12 +118,6 @@ __device__ __forceinline__ void load_slice(const uint32_t *const (&sp)[2], const
   }
 }
 
-__device__ __forceinline__ void cp_async16(uint32_t dst, const void *src, uint32_t src_bytes) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(src_bytes) : "memory");
-}
-__device__ __forceinline__ void cp_async_wait_all() {
-  asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
-}
 
 template <int P, int MODE>
 __global__ void __launch_bounds__(kCtaThreads, 1) grouped_seed_gemm_kernel(const GroupedParams p) {

@@ -25,6 +25,7 @@
 
 #include "chunk.cuh"
 #include "common.cuh"
+#include "decode1.cuh"
 #include "moe.cuh"
 
 namespace nslm {
@@ -133,48 +134,6 @@ __global__ void __launch_bounds__(256) route_plan_kernel(const float *__restrict
   }
 }
 
-// ------------------------------------------------------- activation staging
-
-// Stage the activations of M tokens (rows[m]) into vectors m of the chunk
-// layout.  Source is either bf16 x [T][K], or fp32 y [T][K] normalised per
-// token to bf16(y / sqrt(mean(y^2) + 1e-6)).
-__device__ void stage_activations(float4 *xs4, float2 *xn2, const uint16_t *__restrict__ x_bf16,
-                                  const float *__restrict__ y_prev, const int *rows, int M, int K,
-                                  int cpad, float *scratch /* >= 33 floats */) {
-  if (x_bf16) {
-    stage_bf16(xs4, xn2, x_bf16, rows, M, K, cpad);
-    return;
-  }
-  const int tid = threadIdx.x, nthr = blockDim.x, nb = K >> 3;
-  for (int m = 0; m < M; ++m) {
-    const float4 *row = reinterpret_cast<const float4 *>(y_prev + (size_t)rows[m] * K);
-    float ss = 0.f;
-    for (int i = tid; i < 2 * nb; i += nthr) {
-      const float4 v = __ldcg(row + i);
-      ss = fmaf(v.x, v.x, fmaf(v.y, v.y, fmaf(v.z, v.z, fmaf(v.w, v.w, ss))));
-    }
-    ss = warp_sum(ss);
-    if ((tid & 31) == 0) scratch[tid >> 5] = ss;
-    __syncthreads();
-    if (tid == 0) {
-      float t = 0.f;
-      for (int w = 0; w < (nthr + 31) / 32; ++w) t += scratch[w];
-      scratch[32] = sqrtf(t / (float)K + 1e-6f);
-    }
-    __syncthreads();
-    const float r = scratch[32];
-    for (int b = tid; b < nb; b += nthr) {
-      float4 lo = __ldcg(row + 2 * b), hi = __ldcg(row + 2 * b + 1);
-#define NSLM_NORM(v) __bfloat162float(__float2bfloat16_rn(__fdiv_rn((v), r)))
-      lo = make_float4(NSLM_NORM(lo.x), NSLM_NORM(lo.y), NSLM_NORM(lo.z), NSLM_NORM(lo.w));
-      hi = make_float4(NSLM_NORM(hi.x), NSLM_NORM(hi.y), NSLM_NORM(hi.z), NSLM_NORM(hi.w));
-#undef NSLM_NORM
-      xs_store_block(xs4, xn2, m, b, cpad, lo, hi);
-    }
-    __syncthreads();  // scratch is reused by the next token
-  }
-}
-
 // ------------------------------------------------------------- gate / up
 
 struct GateUpParams {
@@ -263,7 +222,7 @@ __global__ void __launch_bounds__(256) ffn_gate_up_kernel(const GateUpParams p) 
   }
   build_stream_tables(tab);
   __syncthreads();
-  stage_activations(xs4, xn2, p.x_bf16, p.y_prev, s_tok, M, p.hidden, cpad, scratch);
+  stage_activations<false>(xs4, xn2, p.x_bf16, p.y_prev, s_tok, M, p.hidden, cpad, scratch);
   __syncthreads();
 #define NSLM_GU(MM) gate_up_body<P, MM, VEC, CPAD>(p, tab, xs4, xn2, red, s_sum, s_pair, fg, fu, rowkg, rowku, active, ch, g)
   if (MT == 1) {
@@ -543,8 +502,10 @@ static int32_t launch_decode_layer_t(const FfnDims &d, const nslm_seed_matrix *g
 int32_t launch_decode_layer(const FfnDims &d, const nslm_seed_matrix *gate,
                             const nslm_seed_matrix *up, const nslm_seed_matrix *down,
                             const SlotPlan *plan, const uint16_t *x_bf16, const float *y_prev,
-                            int T, int k, const FfnWorkspace &w, float *y, cudaStream_t s,
-                            int &launches) {
+                            int T, int k, const FfnWorkspace &w, float *y, bool plan_early,
+                            cudaStream_t s, int &launches) {
+  if (T == 1 && decode1_supported(d, k))
+    return launch_decode1(d, gate, up, down, plan, x_bf16, y_prev, k, w.h, y, plan_early, s, launches);
   if (d.P == 4) {
     return T == 1 ? launch_decode_layer_t<4, 1>(d, gate, up, down, plan, x_bf16, y_prev, T, k, w, y, s, launches)
                   : launch_decode_layer_t<4, 8>(d, gate, up, down, plan, x_bf16, y_prev, T, k, w, y, s, launches);

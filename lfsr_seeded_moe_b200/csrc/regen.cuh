@@ -86,15 +86,27 @@ __device__ __forceinline__ void build_stream_tables_x32(StreamTablesX32 *tab) {
   for (int i = threadIdx.x; i < 512 * 32; i += blockDim.x) tab->t[i] = kStreamTab.t[i >> 5];
 }
 
-// W = seed | next32 << 16 from the replicated tables; lane4 = 4 * (lane id).
-__device__ __forceinline__ void stream_word_x32(const StreamTablesX32 *tab, uint32_t lane4, uint32_t seed,
-                                                uint32_t &lo, uint32_t &hi) {
+// (v, nxt) of a seed from the replicated tables; lane4 = 4 * (lane id).
+__device__ __forceinline__ void stream_pair_x32(const StreamTablesX32 *tab, uint32_t lane4, uint32_t seed,
+                                                uint32_t &v, uint32_t &nxt) {
   const char *base = reinterpret_cast<const char *>(tab->t) + lane4;
   const uint32_t a = *reinterpret_cast<const uint32_t *>(base + ((seed & 0xFFu) << 7));
   const uint32_t b = *reinterpret_cast<const uint32_t *>(base + (((seed >> 8) & 0xFFu) << 7) + 256 * 128);
-  const uint32_t nxt = a ^ b;
-  lo = __byte_perm(seed, nxt, 0x5410);
-  hi = nxt >> 16;
+  nxt = a ^ b;
+  v = seed << 16;
+}
+
+// The stream of seed `HALF` (0: bits 0..15, 1: bits 16..31) of a packed word
+// of two seeds, as v = seed << 16 and nxt = the 32 bits that follow the seed:
+// then W >> t = funnelshift_r(v, nxt, 16 + t) for 1 <= t < 16, and
+// W >> 16 = nxt.
+template <int HALF>
+__device__ __forceinline__ void stream_pair_of(const StreamTables *tab, uint32_t sw, uint32_t &v,
+                                               uint32_t &nxt) {
+  const uint32_t b0 = HALF ? ((sw >> 16) & 0xFFu) : (sw & 0xFFu);
+  const uint32_t b1 = HALF ? (sw >> 24) : ((sw >> 8) & 0xFFu);
+  nxt = tab->t[b0] ^ tab->t[256u + b1];
+  v = HALF ? (sw & 0xFFFF0000u) : (sw << 16);
 }
 
 // W = seed | next32 << 16, returned as (lo = bits 0..31, hi = bits 32..47).
@@ -126,6 +138,19 @@ __device__ __forceinline__ int32_t dp4a_us(uint32_t a_u8x4, uint32_t b_s8x4, int
 __device__ __forceinline__ int32_t dp4a_ss(uint32_t a_s8x4, uint32_t b_s8x4, int32_t acc) {
   int32_t d;
   asm("dp4a.s32.s32 %0, %1, %2, %3;" : "=r"(d) : "r"(a_s8x4), "r"(b_s8x4), "r"(acc));
+  return d;
+}
+
+// Two-way dot products of two unsigned 16-bit halves of a with the signed
+// bytes 0,1 (lo) or 2,3 (hi) of b, accumulated into acc.
+__device__ __forceinline__ int32_t dp2a_lo_us(uint32_t a_u16x2, uint32_t b_s8x4, int32_t acc) {
+  int32_t d;
+  asm("dp2a.lo.u32.s32 %0, %1, %2, %3;" : "=r"(d) : "r"(a_u16x2), "r"(b_s8x4), "r"(acc));
+  return d;
+}
+__device__ __forceinline__ int32_t dp2a_hi_us(uint32_t a_u16x2, uint32_t b_s8x4, int32_t acc) {
+  int32_t d;
+  asm("dp2a.hi.u32.s32 %0, %1, %2, %3;" : "=r"(d) : "r"(a_u16x2), "r"(b_s8x4), "r"(acc));
   return d;
 }
 

@@ -78,7 +78,7 @@ extern "C" int32_t nslm_moe_seed_ffn_static(const nslm_seed_matrix *gate, const 
                               d.hidden, s)))
     return st;
   int launches = 1;
-  st = launch_decode_layer(d, gate, up, down, fw.plans, x_bf16, nullptr, T, k, fw, y, s, launches);
+  st = launch_decode_layer(d, gate, up, down, fw.plans, x_bf16, nullptr, T, k, fw, y, false, s, launches);
   if (st == NSLM_OK) g_launches = launches;
   return st;
 }

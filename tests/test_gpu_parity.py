@@ -161,6 +161,55 @@ def _ffn_case(nslm, E, hidden, inter, P, T, k, tag, zipf=None):
     return y.cpu().numpy(), ref
 
 
+def _ffn_with_ids(nslm, L, E, hidden, inter, x, rid, w32, k):
+    T = rid.shape[0]
+    y = _out(T, hidden)
+    wsb = nslm.nslm_workspace_bytes(nslm.NSLM_OP_MOE_FFN, T, E, hidden, inter, k)
+    ws = torch.empty(wsb, dtype=torch.uint8, device="cuda")
+    nslm.nslm_moe_seed_ffn(_dev(L.gate), _dev(L.up), _dev(L.down), E, x, torch.from_numpy(rid).cuda(),
+                           torch.from_numpy(w32).cuda(), T, k, y, ws, wsb)
+    torch.cuda.synchronize()
+    return y.cpu().numpy()
+
+
+@pytest.mark.parametrize("E,hidden,inter,P,k", [
+    (16, 256, 128, 3, 4),      # whole 64-weight chunks
+    (12, 272, 120, 3, 8),      # ragged rows in both projections
+    (8, 4160, 208, 4, 2),      # 65 chunks per gate row (two rounds per lane), ragged down rows
+    (4, 64, 64, 4, 1),         # one chunk per row, one expert per token
+])
+def test_ffn_one_token_shapes(nslm, E, hidden, inter, P, k):
+    tag = 920 + hidden
+    y, ref = _ffn_case(nslm, E, hidden, inter, P, 1, k, tag)
+    assert O.normwise_rel_err(y, ref) <= TIGHT
+
+
+def test_ffn_one_token_duplicate_and_dropped_ids(nslm):
+    # a token that lists one expert twice gets both contributions; pairs whose
+    # expert id is outside [0, E) contribute nothing
+    E, hidden, inter, P, k = 10, 512, 256, 4, 6
+    L = synth.moe_layer(0, E, hidden, inter, P, config=930)
+    x, xh = _x((930, 1), 1, hidden)
+    rid = np.array([[3, 3, 7, -1, 12, 0]], dtype=np.int32)
+    w32 = np.array([[0.3, 0.2, 0.25, 0.1, 0.05, 0.1]], dtype=np.float32)
+    y = _ffn_with_ids(nslm, L, E, hidden, inter, x, rid, w32, k)
+    keep = (rid >= 0) & (rid < E)
+    oid = np.where(keep, rid, 0).astype(np.int32)
+    ow = np.where(keep, w32.astype(np.float64), 0.0)
+    g, u, d = (getattr(L, n).numpy() for n in ("gate", "up", "down"))
+    ref = O.moe_ffn(g, u, d, E, hidden, inter, xh, oid, ow, mode=0)
+    assert O.normwise_rel_err(y, ref) <= TIGHT
+
+
+def test_ffn_one_token_all_ids_dropped_gives_zero(nslm):
+    E, hidden, inter, P, k = 6, 256, 128, 3, 2
+    L = synth.moe_layer(0, E, hidden, inter, P, config=931)
+    x, _ = _x((931, 1), 1, hidden)
+    y = _ffn_with_ids(nslm, L, E, hidden, inter, x, np.array([[-1, 6]], dtype=np.int32),
+                      np.array([[0.5, 0.5]], dtype=np.float32), k)
+    assert np.array_equal(y, np.zeros_like(y))
+
+
 def test_ffn_decode_one_token_full_layer(nslm):
     # one MoE layer decode: 100 experts, hidden 2048, intermediate 1408, P=4, top-8
     y, ref = _ffn_case(nslm, 100, 2048, 1408, 4, 1, 8, 906)
