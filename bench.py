@@ -279,6 +279,40 @@ def batched_sweep(torch, nslm, synth, dev, hbm, bf16_peak):
     return out
 
 
+def profile_workload(kind: str, reps: int):
+    """A small fixed workload for ncu captures (no timing, no JSON): `reps`
+    calls of one decode layer (T=1, P=4), of one batched layer (T=512, P=3)
+    or of one seed GEMV (2048 x 4096, P=4)."""
+    import torch
+
+    from lfsr_seeded_moe_b200 import nslm, synth
+
+    dev = torch.device("cuda", 0)
+    if kind == "gemv":
+        m = synth.seed_matrix(2048, 4096, 4, (11, 2048, 4096, 4), device=dev)
+        x = synth.activations((11,), 1, 4096).to(dev)
+        y = torch.empty(1, 2048, device=dev)
+        for _ in range(reps):
+            nslm.nslm_seed_gemv(nslm.matrix(m), x, 1, y)
+        torch.cuda.synchronize()
+        return
+    T, Pv, cfg = (1, 4, 2) if kind == "layer" else (512, 3, 3)
+    L = synth.moe_layer(0, E, HIDDEN, INTER, Pv, device=dev, config=cfg)
+    logits = synth.router_logits((cfg, T), T, E).to(dev)
+    ids = torch.empty(T, K_TOP, dtype=torch.int32, device=dev)
+    w = torch.empty(T, K_TOP, device=dev)
+    nslm.nslm_moe_route_topk(logits, T, E, K_TOP, ids, w)
+    x = synth.activations((cfg, T), T, HIDDEN).to(dev)
+    y = torch.empty(T, HIDDEN, device=dev)
+    wsb = nslm.nslm_workspace_bytes(nslm.NSLM_OP_MOE_FFN, T, E, HIDDEN, INTER, K_TOP)
+    ws = torch.zeros(wsb, dtype=torch.uint8, device=dev)
+    for _ in range(reps):
+        nslm.nslm_moe_seed_ffn(L.gate, L.up, L.down, E, x, ids, w, T, K_TOP, y, ws, wsb)
+    torch.cuda.synchronize()
+    if int(ws[:4].view(torch.int32).item()) != 0 and T > 8:
+        raise SystemExit("batched layer reported a non-zero status")
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -289,7 +323,11 @@ def main():
     ap.add_argument("--no-gemv", action="store_true")
     ap.add_argument("--no-batched", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--profile", choices=["layer", "batched", "gemv"],
+                    help="run a small fixed workload for an ncu capture and exit")
     args = ap.parse_args()
+    if args.profile:
+        return profile_workload(args.profile, args.steps)
     if args.impl == "reference":
         return run_reference(args)
 
