@@ -236,6 +236,23 @@ __device__ __forceinline__ float regen_chunk_block(const StreamTables *tab, cons
   return block_scale(code, rowk);
 }
 
+// The same from R interleaved copies of the stream tables (entry e of copy c
+// at word R * e + c); tl points at this lane's copy (lane mod R), so lanes
+// that share a copy are R-fold fewer and bank conflicts fall accordingly.
+template <int P, int R>
+__device__ __forceinline__ float regen_chunk_block_r(const uint32_t *tl, const ChunkFields &f, int i,
+                                                     uint32_t rowk, float (&G)[8]) {
+  const uint32_t sw = f.s[i >> 1], qw = f.q[i >> 1];
+  const uint32_t q = (i & 1) ? (qw >> 16) : (qw & 0xFFFFu);
+  const uint32_t b0 = (i & 1) ? ((sw >> 16) & 0xFFu) : (sw & 0xFFu);
+  const uint32_t b1 = (i & 1) ? (sw >> 24) : ((sw >> 8) & 0xFFu);
+  const uint32_t nxt = tl[R * b0] ^ tl[R * (256u + b1)];
+  const uint32_t v = (i & 1) ? (sw & 0xFFFF0000u) : (sw << 16);
+  block_magic(v, nxt, coef_pairs2<P>(q), G);
+  const uint32_t code = (P == 4) ? ((f.codes >> (4 * i)) & 0xFu) : (q >> 12);
+  return block_scale(code, rowk);
+}
+
 // <G, x> - Mg * sum(x) for one staged vector, as a packed pair sum.
 __device__ __forceinline__ float block_dot(const float (&G)[8], const float4 &xa, const float4 &xb,
                                            const float2 &xn) {
@@ -368,22 +385,23 @@ __device__ __forceinline__ void block_fma(const float (&G)[8], float s, const fl
 }
 
 // One chunk against the staged slot at xa (16 float4) / xn (8 float2) of the
-// chunk-major layout: acc += sum_b scale_b * <w_b, x_b>.
-template <int P, bool VEC>
-__device__ __forceinline__ void chunk_dot_cm(const StreamTables *tab, const ChunkFields &f, int nvalid,
+// chunk-major layout: acc += sum_b scale_b * <w_b, x_b>.  tl: this lane's
+// copy of R interleaved stream tables.
+template <int P, bool VEC, int R>
+__device__ __forceinline__ void chunk_dot_cm(const uint32_t *tl, const ChunkFields &f, int nvalid,
                                              uint32_t rowk, const float4 *xa, const float2 *xn, float2 &acc) {
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
     if (!VEC && i >= nvalid) break;
     float G[8];
-    const float s = regen_chunk_block<P>(tab, f, i, rowk, G);
+    const float s = regen_chunk_block_r<P, R>(tl, f, i, rowk, G);
     block_fma(G, s, xa[2 * i], xa[2 * i + 1], xn[i], acc);
   }
 }
 
 // The gate and up chunks of one row against the same staged slot.
-template <int P, bool VEC>
-__device__ __forceinline__ void chunk_dot2_cm(const StreamTables *tab, const ChunkFields &fa,
+template <int P, bool VEC, int R>
+__device__ __forceinline__ void chunk_dot2_cm(const uint32_t *tl, const ChunkFields &fa,
                                               const ChunkFields &fb, int nvalid, uint32_t rowka,
                                               uint32_t rowkb, const float4 *xa, const float2 *xn,
                                               float2 &acca, float2 &accb) {
@@ -391,8 +409,8 @@ __device__ __forceinline__ void chunk_dot2_cm(const StreamTables *tab, const Chu
   for (int i = 0; i < 8; ++i) {
     if (!VEC && i >= nvalid) break;
     float Ga[8], Gb[8];
-    const float sa = regen_chunk_block<P>(tab, fa, i, rowka, Ga);
-    const float sb = regen_chunk_block<P>(tab, fb, i, rowkb, Gb);
+    const float sa = regen_chunk_block_r<P, R>(tl, fa, i, rowka, Ga);
+    const float sb = regen_chunk_block_r<P, R>(tl, fb, i, rowkb, Gb);
     const float4 x0 = xa[2 * i], x1 = xa[2 * i + 1];
     const float2 x2 = xn[i];
     block_fma(Ga, sa, x0, x1, x2, acca);

@@ -161,7 +161,7 @@ __global__ void __launch_bounds__(kGateUp1Threads) gate_up1_kernel(const GateUp1
     }
     if (c < p.C) {
       const int nvalid = VEC ? 8 : min(8, nb - 8 * c);
-      chunk_dot2_cm<P, VEC>(tab, fg, fu, nvalid, kg, ku, xs4 + kCmX4 * c, xn2 + kCmXn * c, ag, au);
+      chunk_dot2_cm<P, VEC, 1>(tab->t, fg, fu, nvalid, kg, ku, xs4 + kCmX4 * c, xn2 + kCmXn * c, ag, au);
     }
     if (p.J == 1 || c + 32 >= 32 * p.J) {  // last chunk round of the task
       const float g = warp_sum(ag.x + ag.y), u = warp_sum(au.x + au.y);
@@ -275,7 +275,7 @@ __global__ void __launch_bounds__(kDown1Threads) down1_kernel(const Down1Params 
     }
     float2 acc = make_float2(0.f, 0.f);
     const int nvalid = VEC ? 8 : min(8, nb - 8 * c);
-    chunk_dot_cm<P, VEC>(tab, f, nvalid, rowk, hs4 + kCmX4 * q, hn2 + kCmXn * q, acc);
+    chunk_dot_cm<P, VEC, 1>(tab->t, f, nvalid, rowk, hs4 + kCmX4 * q, hn2 + kCmXn * q, acc);
     red[t] = s_w[s] * (acc.x + acc.y);
     if (!(VEC && kAsyncFields)) {
       f = fn;

@@ -77,10 +77,12 @@ __global__ void __launch_bounds__(256) route_plan_kernel(const float *__restrict
                                                          const float *__restrict__ w_in, int T,
                                                          int E, int k, SlotPlan *plans,
                                                          int32_t *ids_out, float *w_out,
-                                                         int32_t *counters, int n_counters) {
+                                                         int32_t *counters, int n_counters,
+                                                         int32_t *sync) {
   const int layer = blockIdx.x;
   if (counters && layer == 0)
     for (int i = threadIdx.x; i < n_counters; i += blockDim.x) counters[i] = 0;
+  if (sync && layer == 0 && threadIdx.x < kSyncWords) sync[threadIdx.x] = 0;
   __shared__ int32_t s_ids[kMaxPairs];
   __shared__ float s_w[kMaxPairs];
   const int warp = threadIdx.x >> 5;
@@ -425,6 +427,10 @@ int32_t check_ffn_shapes(const nslm_seed_matrix *gate, const nslm_seed_matrix *u
 FfnWorkspace ffn_workspace(char *base, int T, int k, int hidden, int inter, int L) {
   FfnWorkspace w{};
   size_t off = 0;
+  w.sync = reinterpret_cast<int32_t *>(base ? base + off : nullptr);
+  off += 256;
+  w.rms_part = reinterpret_cast<float *>(base ? base + off : nullptr);
+  off += round256(kMaxNormParts * sizeof(float));
   w.plans = reinterpret_cast<SlotPlan *>(base ? base + off : nullptr);
   off += round256((size_t)std::max(L, 1) * kPlanBytes);
   w.counters = reinterpret_cast<int32_t *>(base ? base + off : nullptr);
@@ -516,9 +522,9 @@ int32_t launch_decode_layer(const FfnDims &d, const nslm_seed_matrix *gate,
 
 int32_t launch_route_plan(const float *logits, const int32_t *ids, const float *w, int T, int E,
                           int k, int L, SlotPlan *plans, int32_t *ids_out, float *w_out,
-                          int32_t *counters, int n_counters, cudaStream_t s) {
+                          int32_t *counters, int n_counters, int32_t *sync, cudaStream_t s) {
   route_plan_kernel<<<L, 256, 0, s>>>(logits, ids, w, T, E, k, plans, ids_out, w_out, counters,
-                                      n_counters);
+                                      n_counters, sync);
   return launch_status();
 }
 

@@ -36,7 +36,16 @@ int32_t check_ffn_shapes(const nslm_seed_matrix *gate, const nslm_seed_matrix *u
 // Workspace of the decode path, carved from the caller's buffer (base may be
 // null to size it).  counters must be zero before the first down kernel; the
 // routing kernel zeroes them and the down kernel leaves them zero.
+// Device status words at the head of the decode workspace: [0] status (0 ok,
+// 1 a grid barrier wait gave up), [1] barrier arrivals, [2] abort flag; the
+// routing kernel zeroes them at the start of every call.
+constexpr int kSyncWords = 4;
+
+constexpr int kMaxNormParts = 1024;
+
 struct FfnWorkspace {
+  int32_t *sync;       // [kSyncWords], at offset 0
+  float *rms_part;     // [kMaxNormParts] per-CTA sums of y^2 between fused layers
   SlotPlan *plans;     // [L]
   int32_t *counters;   // [hidden]
   float *h;            // [T*k][inter]
@@ -48,7 +57,7 @@ FfnWorkspace ffn_workspace(char *base, int T, int k, int hidden, int inter, int 
 
 int32_t launch_route_plan(const float *logits, const int32_t *ids, const float *w, int T, int E,
                           int k, int L, SlotPlan *plans, int32_t *ids_out, float *w_out,
-                          int32_t *counters, int n_counters, cudaStream_t s);
+                          int32_t *counters, int n_counters, int32_t *sync, cudaStream_t s);
 int32_t launch_decode_layer(const FfnDims &d, const nslm_seed_matrix *gate,
                             const nslm_seed_matrix *up, const nslm_seed_matrix *down,
                             const SlotPlan *plan, const uint16_t *x_bf16, const float *y_prev,

@@ -75,6 +75,12 @@ __device__ __forceinline__ void build_stream_tables(StreamTables *tab) {
   for (int i = threadIdx.x; i < 512; i += blockDim.x) tab->t[i] = kStreamTab.t[i];
 }
 
+// R interleaved copies of the tables: entry e of copy c at word R * e + c.
+template <int R>
+__device__ __forceinline__ void build_stream_tables_rep(uint32_t *t) {
+  for (int i = threadIdx.x; i < 512 * R; i += blockDim.x) t[i] = kStreamTab.t[i / R];
+}
+
 // The same tables replicated 32 times and interleaved by lane: entry i of copy
 // c at word i * 32 + c.  Lane l reads copy l, so the 32 lanes of a warp never
 // hit the same bank whatever seeds they hold (64 KB of shared memory).

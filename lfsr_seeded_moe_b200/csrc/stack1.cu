@@ -1,0 +1,486 @@
+// stack1.cu -- the one-token decode stack as one persistent cooperative kernel.
+//
+// "NanoSeedLM: LLM inference using pseudo-random numbers", "Why K2-Horizon-MoVA":
+// for one token every layer reads 8 of its 100 experts: gate and up
+// projections, SiLU, a down projection, and the routing-weighted sum.  The
+// weights are regenerated in registers ("What I changed: September 2026").
+//
+// One launch runs all layers.  Each CTA (one per SM, 26 warps) keeps its
+// stream tables for the whole stack and alternates two phases, separated by
+// grid barriers (the launch is cooperative, so every CTA is resident):
+//
+//   A (gate/up)  every CTA stages the layer input x (layer 0: the bf16 token;
+//                later layers: bf16(y / rms(y)) of the previous layer's fp32
+//                output); warp tasks are routed rows: the lanes take the
+//                64-weight chunks of the gate and up rows, a shuffle tree sums
+//                them, lane 0 writes h = SiLU(g) * u.
+//   B (down)     every CTA stages the routed h vectors back to back and owns
+//                a range of output rows: threads take (row, expert, chunk)
+//                tasks, partials go to shared memory and one warp per row adds
+//                them in a fixed order (deterministic, no atomics on data).
+//
+// Weight fields are copied with cp.async into per-thread shared-memory slots
+// one task ahead, and the first task of the next phase is fetched before the
+// barrier, so barrier latency overlaps the first loads.  Every barrier wait
+// is bounded: a CTA that gives up raises the abort flag (all others stop at
+// their next wait) and records status 1 in the workspace.
+#include <algorithm>
+
+#include "chunk.cuh"
+#include "common.cuh"
+#include "stack1.cuh"
+
+namespace nslm {
+
+namespace {
+
+// n / d for n < 2^22 and 0 < d < 2^16: m = ceil(2^40 / d), q = (n * m) >> 40
+// (exact, since n * (m * d - 2^40) < 2^38 < 2^40).
+struct FastDiv {
+  uint64_t m;
+};
+FastDiv make_fastdiv(uint32_t d) { return FastDiv{((1ull << 40) + d - 1) / d}; }
+__device__ __forceinline__ uint32_t fdiv(uint32_t n, FastDiv f) {
+  return (uint32_t)(((uint64_t)n * f.m) >> 40);
+}
+
+constexpr long long kBarrierWaitCycles = 2000000000ll;  // ~1 s at 1.9 GHz
+constexpr int kTabCopies = 1;  // interleaved stream-table copies (bank conflicts / kTabCopies)
+
+struct LayerMats {
+  nslm_seed_matrix gate, up, down;
+};
+
+struct Stack1Params {
+  const SlotPlan *plans;  // [n] this launch's layers
+  const uint16_t *x0;     // bf16 [hidden]: input of the first layer, or null
+  const float *y_in;      // fp32 [hidden]: the previous layer's output when x0 is null
+  float *h;               // [k][inter] by pair
+  float *y_mid;           // [hidden] fp32 between layers
+  float *y_out;           // [hidden] output of the last layer
+  int32_t *sync;          // status, barrier arrivals, abort
+  float *rms_part;        // [grid] sums of y^2 over each CTA's rows, written with y
+  uint32_t barrier_base;  // arrivals recorded by earlier launches of the same call
+  int32_t n, hidden, inter;
+  int32_t Ch, Ci;         // 64-weight chunks per row of gate/up (hidden) and down (inter)
+  int32_t J;              // chunk rounds per lane in phase A: ceil(Ch / 32)
+  int32_t rpc;            // output rows per CTA in phase B
+  int32_t stage_slots;    // chunk slots of the staging area
+  FastDiv div_inter, div_J, div_Ci, div_nbi;
+  FastDiv div_SC[kMaxK + 1];  // by S * Ci for S routed experts
+  LayerMats layer[kMaxFusedLayers];
+};
+
+__device__ __forceinline__ uint32_t ld_acquire(const int32_t *p) {
+  uint32_t v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+
+// Grid-wide barrier number e of this call, in two halves so that work which
+// does not depend on other CTAs (the next phase's weight prefetch) runs
+// between them.  Arrival: block barrier, then a release reduction by thread 0
+// (it orders the CTA's writes, gathered by the block barrier, before it).
+// Wait: thread 0 polls with acquire loads, bounded; false when aborting.
+__device__ __forceinline__ void grid_arrive(const Stack1Params &p) {
+  __syncthreads();
+  if (threadIdx.x == 0) asm volatile("red.release.gpu.global.add.u32 [%0], 1;" ::"l"(p.sync + 1) : "memory");
+}
+
+__device__ bool grid_wait(const Stack1Params &p, uint32_t e, int *s_ok) {
+  if (threadIdx.x == 0) {
+    int ok = 1;
+    const uint32_t target = p.barrier_base + (e + 1) * gridDim.x;
+    if (ld_acquire(p.sync + 1) < target) {
+      const long long t0 = clock64();
+      for (uint32_t it = 1; ld_acquire(p.sync + 1) < target; ++it) {
+        if ((it & 63) == 0) {
+          if (ld_acquire(p.sync + 2) != 0) {
+            ok = 0;
+            break;
+          }
+          if (clock64() - t0 > kBarrierWaitCycles) {
+            atomicExch(p.sync + 2, 1);
+            atomicCAS(p.sync, 0, 1);
+            ok = 0;
+            break;
+          }
+        }
+      }
+    }
+    *s_ok = ok;
+  }
+  __syncthreads();
+  return *s_ok != 0;
+}
+
+// Stage x = bf16(y / sqrt(mean(y^2) + 1e-6)) chunk-major.  The sum of squares
+// is the fixed-order sum of the per-CTA partials that were written with y.
+__device__ void stage_norm_y(float4 *xs4, float2 *xn2, const float *y, const float *part, int G, int K,
+                             float *scratch) {
+  const int tid = threadIdx.x, nthr = blockDim.x, nb = K >> 3;
+  const float4 *row = reinterpret_cast<const float4 *>(y);
+  float4 lo = make_float4(0.f, 0.f, 0.f, 0.f), hi = lo;
+  if (tid < nb) {  // the first block of this thread, in flight during the sum
+    lo = __ldcg(row + 2 * tid);
+    hi = __ldcg(row + 2 * tid + 1);
+  }
+  if (tid < 32) {
+    float ss = 0.f;
+    for (int i = tid; i < G; i += 32) ss += __ldcg(part + i);
+    ss = warp_sum(ss);
+    if (tid == 0) scratch[32] = sqrtf(ss / (float)K + 1e-6f);
+  }
+  __syncthreads();
+  const float r = scratch[32];
+  for (int b = tid; b < nb; b += nthr) {
+    if (b != tid) {
+      lo = __ldcg(row + 2 * b);
+      hi = __ldcg(row + 2 * b + 1);
+    }
+#define NSLM_NORM(v) __bfloat162float(__float2bfloat16_rn(__fdiv_rn((v), r)))
+    const float4 a = make_float4(NSLM_NORM(lo.x), NSLM_NORM(lo.y), NSLM_NORM(lo.z), NSLM_NORM(lo.w));
+    const float4 c = make_float4(NSLM_NORM(hi.x), NSLM_NORM(hi.y), NSLM_NORM(hi.z), NSLM_NORM(hi.w));
+#undef NSLM_NORM
+    cm_store_block(xs4, xn2, b, a, c);
+  }
+}
+
+template <int P, bool VEC>
+__global__ void __launch_bounds__(kStack1MaxThreads, 1) stack1_kernel(const __grid_constant__ Stack1Params p) {
+  extern __shared__ float4 smem4[];
+  const int tid = threadIdx.x, nthr = blockDim.x, lane = tid & 31, warp = tid >> 5;
+  const int nwarps = nthr >> 5;
+  uint32_t *tab = reinterpret_cast<uint32_t *>(smem4);  // kTabCopies interleaved copies
+  const uint32_t *tl = tab + (tid & (kTabCopies - 1));
+  // staging: chunk-major slots (x in phase A, the routed h vectors in phase B)
+  float4 *xs4 = smem4 + kTabCopies * sizeof(StreamTables) / 16;
+  float2 *xn2 = reinterpret_cast<float2 *>(xs4 + (size_t)kCmX4 * p.stage_slots);
+  // field slots: phase A [2 buffers][gate, up][threads], phase B [2 buffers][threads]
+  const FieldSlots fs(xn2 + (size_t)kCmXn * p.stage_slots + (p.stage_slots & 1), 4 * nthr);
+  float *red = reinterpret_cast<float *>(fs.b + 4 * nthr);  // phase B partials
+  __shared__ float scratch[33];
+  __shared__ int s_row0, s_ok, s_nslots;
+  __shared__ int s_expert[kMaxK], s_pair[kMaxK];
+  __shared__ float s_w[kMaxK];
+  __shared__ int s_next_expert[kMaxK], s_next_nslots;  // the next layer's plan, for its prefetch
+
+  build_stream_tables_rep<kTabCopies>(tab);
+  if (tid == 0) s_row0 = 0;
+
+  const int nbh = p.hidden >> 3, nbi = p.inter >> 3;
+  const int gw = blockIdx.x * nwarps + warp, W = gridDim.x * nwarps;
+  const int n0 = blockIdx.x * p.rpc;
+  const int nrows = max(0, min(p.rpc, p.hidden - n0));
+
+  // ---- phase A task geometry (a step = one chunk round of one routed row)
+  auto a_steps = [&](int nslots) {
+    const int ntask = nslots * p.inter;
+    return (gw < ntask ? (ntask - 1 - gw) / W + 1 : 0) * p.J;
+  };
+  auto a_locate = [&](int step, int &slot, int &row, int &c) {
+    const int i = p.J == 1 ? step : (int)fdiv(step, p.div_J);
+    const int t = gw + i * W;
+    slot = (int)fdiv(t, p.div_inter);
+    row = t - slot * p.inter;
+    c = lane + 32 * (step - i * p.J);
+  };
+  auto a_fetch = [&](const LayerMats &Lm, const int32_t *expert, int step, int buf, ChunkFields &fg,
+                     ChunkFields &fu, uint32_t &kg, uint32_t &ku) {
+    int slot, row, c;
+    a_locate(step, slot, row, c);
+    if (c >= p.Ch) return;
+    const size_t grow = (size_t)expert[slot] * p.inter + row;
+    if (VEC) {
+      fetch_chunk<P>(Lm.gate, grow, nbh, c, fs, (2 * buf) * nthr + tid);
+      fetch_chunk<P>(Lm.up, grow, nbh, c, fs, (2 * buf + 1) * nthr + tid);
+    } else {
+      load_chunk<P, false>(Lm.gate.seeds + grow * nbh, Lm.gate.coefs + grow * nbh,
+                           P == 4 ? Lm.gate.codes + grow * (nbh / 2) : nullptr, nbh, c, fg);
+      load_chunk<P, false>(Lm.up.seeds + grow * nbh, Lm.up.coefs + grow * nbh,
+                           P == 4 ? Lm.up.codes + grow * (nbh / 2) : nullptr, nbh, c, fu);
+      kg = row_scale_key(__ldg(Lm.gate.exp_bias + grow));
+      ku = row_scale_key(__ldg(Lm.up.exp_bias + grow));
+    }
+  };
+  // ---- phase B task geometry (row, routed expert, chunk) of this CTA's rows
+  auto b_locate = [&](int t, FastDiv dSC, int SC, int &r, int &s, int &c, int &q) {
+    r = (int)fdiv(t, dSC);
+    q = t - r * SC;
+    s = (int)fdiv(q, p.div_Ci);
+    c = q - s * p.Ci;
+  };
+  auto b_fetch = [&](const LayerMats &Lm, FastDiv dSC, int SC, int t, int buf, ChunkFields &f,
+                     uint32_t &k) {
+    int r, s, c, q;
+    b_locate(t, dSC, SC, r, s, c, q);
+    const size_t grow = (size_t)s_expert[s] * p.hidden + n0 + r;
+    if (VEC) {
+      fetch_chunk<P>(Lm.down, grow, nbi, c, fs, buf * nthr + tid);
+    } else {
+      load_chunk<P, false>(Lm.down.seeds + grow * nbi, Lm.down.coefs + grow * nbi,
+                           P == 4 ? Lm.down.codes + grow * (nbi / 2) : nullptr, nbi, c, f);
+      k = row_scale_key(__ldg(Lm.down.exp_bias + grow));
+    }
+  };
+
+  // register copies of the next fields on the ragged path (unused when VEC)
+  ChunkFields fg, fu, fd;
+  uint32_t kg = 0, ku = 0, kd = 0;
+  uint32_t nbar = 0;  // barriers passed in this launch
+
+  // first fields of layer 0, phase A
+  if (a_steps(min(p.plans->n_slots, kMaxK)) > 0) a_fetch(p.layer[0], p.plans->expert, 0, 0, fg, fu, kg, ku);
+  if (VEC) cp_async_commit();
+  __syncthreads();  // tables
+
+  for (int l = 0; l < p.n; ++l) {
+    const LayerMats &Lm = p.layer[l];
+    const SlotPlan *pl = p.plans + l;
+    __syncthreads();  // smem plan and staging reuse
+    if (tid < kMaxK && tid < pl->n_slots) {
+      const int pr = pl->pair[pl->start[tid]];
+      s_expert[tid] = pl->expert[tid];
+      s_pair[tid] = pr;
+      s_w[tid] = pl->w[pr];
+    }
+    if (tid == 0) s_nslots = min(pl->n_slots, kMaxK);
+    if (l + 1 < p.n) {
+      if (tid < kMaxK && tid < pl[1].n_slots) s_next_expert[tid] = pl[1].expert[tid];
+      if (tid == 0) s_next_nslots = min(pl[1].n_slots, kMaxK);
+    }
+
+    // =========================== phase A: gate/up + SiLU
+    if (l == 0 && p.x0)
+      stage_activations<true>(xs4, xn2, p.x0, nullptr, &s_row0, 1, p.hidden, p.Ch, scratch);
+    else
+      stage_norm_y(xs4, xn2, l == 0 ? p.y_in : p.y_mid, p.rms_part, gridDim.x, p.hidden, scratch);
+    __syncthreads();
+    {
+      const int nsteps = a_steps(s_nslots);
+      float2 ag = make_float2(0.f, 0.f), au = make_float2(0.f, 0.f);
+      for (int step = 0; step < nsteps; ++step) {
+        int slot, row, c;
+        a_locate(step, slot, row, c);
+        ChunkFields cg = fg, cu = fu;
+        uint32_t ckg = kg, cku = ku;
+        if (VEC) {
+          if (step + 1 < nsteps) a_fetch(Lm, s_expert, step + 1, (step + 1) & 1, fg, fu, kg, ku);
+          cp_async_commit();
+          cp_async_wait<1>();
+          read_chunk<P>(fs, (2 * (step & 1)) * nthr + tid, cg, ckg);
+          read_chunk<P>(fs, (2 * (step & 1) + 1) * nthr + tid, cu, cku);
+        } else if (step + 1 < nsteps) {
+          a_fetch(Lm, s_expert, step + 1, 0, fg, fu, kg, ku);
+        }
+        if (c < p.Ch) {
+          const int nvalid = VEC ? 8 : min(8, nbh - 8 * c);
+          chunk_dot2_cm<P, VEC, kTabCopies>(tl, cg, cu, nvalid, ckg, cku, xs4 + kCmX4 * c, xn2 + kCmXn * c, ag, au);
+        }
+        if (p.J == 1 || c + 32 >= 32 * p.J) {
+          const float g = warp_sum(ag.x + ag.y), u = warp_sum(au.x + au.y);
+          if (lane == 0) __stcg(p.h + (size_t)s_pair[slot] * p.inter + row, g / (1.f + expf(-g)) * u);
+          ag = au = make_float2(0.f, 0.f);
+        }
+      }
+    }
+    // arrive; fetch phase B's first fields (weights only) while the others arrive
+    const int SC = s_nslots * p.Ci;
+    const int bt = nrows * SC;
+    grid_arrive(p);
+    if (VEC) cp_async_wait<0>();
+    if (tid < bt) b_fetch(Lm, p.div_SC[s_nslots], SC, tid, 0, fd, kd);
+    if (VEC) cp_async_commit();
+    if (!grid_wait(p, nbar++, &s_ok)) break;
+
+    // =========================== phase B: down + weighted combine
+    {
+      const FastDiv dSC = p.div_SC[s_nslots];
+      // all routed h blocks, two per thread per round with both loads in flight
+      const int nhb = s_nslots * nbi;
+      for (int i = tid; i < nhb; i += 2 * nthr) {
+        const int i2 = i + nthr;
+        const int s = (int)fdiv(i, p.div_nbi), b = i - s * nbi;
+        const float4 *src = reinterpret_cast<const float4 *>(p.h + (size_t)s_pair[s] * p.inter) + 2 * b;
+        const float4 a0 = __ldcg(src), a1 = __ldcg(src + 1);
+        float4 c0, c1;
+        int s2 = 0, b2 = 0;
+        if (i2 < nhb) {
+          s2 = (int)fdiv(i2, p.div_nbi);
+          b2 = i2 - s2 * nbi;
+          const float4 *src2 = reinterpret_cast<const float4 *>(p.h + (size_t)s_pair[s2] * p.inter) + 2 * b2;
+          c0 = __ldcg(src2);
+          c1 = __ldcg(src2 + 1);
+        }
+        cm_store_block(xs4, xn2, s * p.Ci * 8 + b, a0, a1);
+        if (i2 < nhb) cm_store_block(xs4, xn2, s2 * p.Ci * 8 + b2, c0, c1);
+      }
+      __syncthreads();
+      for (int t = tid, it = 0; t < bt; t += nthr, ++it) {
+        int r, s, c, q;
+        b_locate(t, dSC, SC, r, s, c, q);
+        ChunkFields cf = fd;
+        uint32_t ck = kd;
+        if (VEC) {
+          if (t + nthr < bt) b_fetch(Lm, dSC, SC, t + nthr, (it + 1) & 1, fd, kd);
+          cp_async_commit();
+          cp_async_wait<1>();
+          read_chunk<P>(fs, (it & 1) * nthr + tid, cf, ck);
+        } else if (t + nthr < bt) {
+          b_fetch(Lm, dSC, SC, t + nthr, 0, fd, kd);
+        }
+        float2 acc = make_float2(0.f, 0.f);
+        const int nvalid = VEC ? 8 : min(8, nbi - 8 * c);
+        chunk_dot_cm<P, VEC, kTabCopies>(tl, cf, nvalid, ck, xs4 + kCmX4 * q, xn2 + kCmXn * q, acc);
+        red[t] = s_w[s] * (acc.x + acc.y);
+      }
+      __syncthreads();
+      float *yl = (l == p.n - 1) ? p.y_out : p.y_mid;
+      float *rowy = red + p.rpc * p.stage_slots;  // this CTA's outputs, for the norm partial
+      for (int r = warp; r < nrows; r += nwarps) {
+        float sum = 0.f;
+        for (int q = lane; q < SC; q += 32) sum += red[r * SC + q];
+        sum = warp_sum(sum);
+        if (lane == 0) {
+          __stcg(yl + n0 + r, sum);
+          rowy[r] = sum;
+        }
+      }
+      __syncthreads();
+      if (warp == 0) {  // sum of squares of this CTA's rows, fixed order
+        float ss = 0.f;
+        for (int r = lane; r < nrows; r += 32) ss = fmaf(rowy[r], rowy[r], ss);
+        ss = warp_sum(ss);
+        if (lane == 0) __stcg(p.rms_part + blockIdx.x, ss);
+      }
+    }
+    if (l + 1 == p.n) break;
+    // arrive; fetch the next layer's first phase A fields while the others arrive
+    grid_arrive(p);
+    if (VEC) cp_async_wait<0>();
+    if (a_steps(s_next_nslots) > 0) a_fetch(p.layer[l + 1], s_next_expert, 0, 0, fg, fu, kg, ku);
+    if (VEC) cp_async_commit();
+    if (!grid_wait(p, nbar++, &s_ok)) break;
+  }
+  if (VEC) cp_async_wait<0>();
+}
+
+}  // namespace
+
+// ---------------------------------------------------------------------- host
+
+static int stack1_rows_per_cta(const FfnDims &d) { return std::max(1, ceil_div(d.hidden, num_sms())); }
+
+// Threads per CTA: the whole warps, at most kStack1MaxThreads, that leave the
+// fewest idle task slots in both phases (a phase A task is 16 blocks per
+// lane, a phase B task 8); on a tie the most warps.  Few warps with many
+// registers each beat many warps here: the unrolled block loop needs the
+// registers to overlap its table lookups and dot products.
+static int stack1_threads(const FfnDims &d, int k) {
+  const int sms = num_sms();
+  const int Ch = ceil_div(d.hidden / 8, 8), Ci = ceil_div(d.inter / 8, 8);
+  const int J = ceil_div(Ch, 32);
+  const long long a_tasks = (long long)k * d.inter * J;
+  const long long b_tasks = (long long)stack1_rows_per_cta(d) * k * Ci;
+  int best = 8;
+  long long best_cost = -1;
+  for (int nw = kStack1MaxThreads / 32; nw >= 8; --nw) {
+    const long long ra = (a_tasks + (long long)sms * nw - 1) / ((long long)sms * nw);
+    const long long rb = (b_tasks + 32ll * nw - 1) / (32ll * nw);
+    const long long cost = (16 * ra + 8 * rb) * nw;
+    if (best_cost < 0 || cost < best_cost) {
+      best_cost = cost;
+      best = nw;
+    }
+  }
+  return 32 * best;
+}
+
+static size_t stack1_smem(const FfnDims &d, int k, int threads) {
+  const int Ch = ceil_div(d.hidden / 8, 8), Ci = ceil_div(d.inter / 8, 8);
+  const int slots = std::max(Ch, k * Ci);
+  return kTabCopies * sizeof(StreamTables) + cm_bytes(slots) + 16 + FieldSlots::bytes(4 * threads) +
+         (size_t)stack1_rows_per_cta(d) * (slots + 1) * sizeof(float);
+}
+
+bool stack1_supported(const FfnDims &d, int k) {
+  if (k < 1 || k > kMaxK) return false;
+  // fast divisions: divisors below 2^16, dividends below 2^22
+  if (d.inter >= (1 << 16) || d.hidden >= (1 << 16)) return false;
+  if ((int64_t)k * ceil_div(d.inter / 8, 8) >= (1 << 16)) return false;
+  if ((int64_t)k * d.inter * ceil_div(d.hidden / 64, 32) >= (1 << 22)) return false;
+  return stack1_smem(d, k, stack1_threads(d, k)) <= 224 * 1024;
+}
+
+template <int P, bool VEC>
+static int32_t launch_stack1_t(const FfnDims &d, const nslm_moe_layer *layers, int n,
+                               const SlotPlan *plans, const uint16_t *x0, const float *y_in, int k,
+                               float *h, float *y_mid, float *y_out, int32_t *sync, float *rms_part,
+                               cudaStream_t s, int &launches) {
+  const int threads = stack1_threads(d, k);
+  const size_t smem = stack1_smem(d, k, threads);
+  auto kern = stack1_kernel<P, VEC>;
+  int32_t st = ensure_smem((const void *)kern, smem);
+  if (st) return st;
+  const int per_sm = max_active_ctas((const void *)kern, threads, smem);
+  const int grid = num_sms() * per_sm;
+  Stack1Params p{};
+  p.h = h;
+  p.y_mid = y_mid;
+  p.sync = sync;
+  p.rms_part = rms_part;
+  p.hidden = d.hidden;
+  p.inter = d.inter;
+  p.Ch = ceil_div(d.hidden / 8, 8);
+  p.Ci = ceil_div(d.inter / 8, 8);
+  p.J = ceil_div(p.Ch, 32);
+  p.rpc = ceil_div(d.hidden, grid);
+  p.stage_slots = std::max(p.Ch, k * p.Ci);
+  p.div_inter = make_fastdiv((uint32_t)d.inter);
+  p.div_J = make_fastdiv((uint32_t)p.J);
+  p.div_Ci = make_fastdiv((uint32_t)p.Ci);
+  p.div_nbi = make_fastdiv((uint32_t)(d.inter / 8));
+  for (int S = 1; S <= kMaxK; ++S) p.div_SC[S] = make_fastdiv((uint32_t)(S * p.Ci));
+  p.div_SC[0] = p.div_SC[1];
+  if (p.rpc > stack1_rows_per_cta(d) || grid > kMaxStack1Ctas) return NSLM_ERR_SHAPE;
+  // chunks of kMaxFusedLayers layers; barrier arrivals keep counting across them
+  uint32_t base = 0;
+  for (int l0 = 0; l0 < n; l0 += kMaxFusedLayers) {
+    const int m = std::min(kMaxFusedLayers, n - l0);
+    p.plans = plans + l0;
+    p.x0 = l0 == 0 ? x0 : nullptr;
+    p.y_in = l0 == 0 ? y_in : y_mid;
+    p.y_out = (l0 + m == n) ? y_out : y_mid;
+    p.n = m;
+    p.barrier_base = base;
+    for (int i = 0; i < m; ++i)
+      p.layer[i] = LayerMats{layers[l0 + i].gate, layers[l0 + i].up, layers[l0 + i].down};
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = dim3((unsigned)grid);
+    cfg.blockDim = dim3((unsigned)threads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeCooperative;
+    attr[0].val.cooperative = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if ((st = cuda_status(cudaLaunchKernelEx(&cfg, kern, p)))) return st;
+    ++launches;
+    base += (uint32_t)(2 * m - 1) * (uint32_t)grid;
+  }
+  return NSLM_OK;
+}
+
+int32_t launch_stack1(const FfnDims &d, const nslm_moe_layer *layers, int n, const SlotPlan *plans,
+                      const uint16_t *x0, const float *y_in, int k, float *h, float *y_mid,
+                      float *y_out, int32_t *sync, float *rms_part, cudaStream_t s, int &launches) {
+  const bool vec = d.hidden % 64 == 0 && d.inter % 64 == 0;
+  if (d.P == 4)
+    return vec ? launch_stack1_t<4, true>(d, layers, n, plans, x0, y_in, k, h, y_mid, y_out, sync, rms_part, s, launches)
+               : launch_stack1_t<4, false>(d, layers, n, plans, x0, y_in, k, h, y_mid, y_out, sync, rms_part, s, launches);
+  return vec ? launch_stack1_t<3, true>(d, layers, n, plans, x0, y_in, k, h, y_mid, y_out, sync, rms_part, s, launches)
+             : launch_stack1_t<3, false>(d, layers, n, plans, x0, y_in, k, h, y_mid, y_out, sync, rms_part, s, launches);
+}
+
+}  // namespace nslm
