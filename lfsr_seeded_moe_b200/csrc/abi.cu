@@ -295,7 +295,7 @@ int32_t nslm_moe_seed_ffn(const nslm_seed_matrix *gate, const nslm_seed_matrix *
     const nslm_moe_layer layer{*gate, *up, *down};
     st = launch_stack1(d, &layer, 1, fw.plans, x_bf16, nullptr, k, fw.h, fw.y_mid, y, fw.sync, fw.rms_part, s, launches);
   } else {
-    st = launch_decode_layer(d, gate, up, down, fw.plans, x_bf16, nullptr, T, k, fw, y, false, s, launches);
+    st = launch_decode_layer(d, gate, up, down, fw.plans, x_bf16, nullptr, T, k, fw, y, s, launches);
   }
   if (st == NSLM_OK) g_launches = launches;
   return st;
@@ -335,9 +335,8 @@ int32_t nslm_moe_stack_decode(const nslm_moe_layer *layers, int32_t L, int32_t E
     const uint16_t *xin = (l == 0) ? x0_bf16 : nullptr;
     const float *yprev = (l == 0) ? nullptr : fw.y_mid;
     float *yout = (l == L - 1) ? y : fw.y_mid;
-    // layer l > 0: the routing kernel ran at least two kernels back
     st = launch_decode_layer(d, &layers[l].gate, &layers[l].up, &layers[l].down, fw.plans + l, xin,
-                             yprev, T, k, fw, yout, l > 0, s, launches);
+                             yprev, T, k, fw, yout, s, launches);
     if (st) return st;
   }
   g_launches = launches;

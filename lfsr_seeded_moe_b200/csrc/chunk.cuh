@@ -187,6 +187,17 @@ __device__ __forceinline__ void fetch_chunk(const nslm_seed_matrix &W, size_t gr
   cp_async4(fs.b + i, W.exp_bias + grow);
 }
 
+// The same for a row whose chunk starts at element `off` of the seeds/coefs
+// streams (off = row * nb + 8 * chunk, 32-bit: a matrix holds < 2^31 blocks).
+template <int P>
+__device__ __forceinline__ void fetch_chunk_off(const nslm_seed_matrix &W, uint32_t off, uint32_t row,
+                                                const FieldSlots &fs, int i) {
+  cp_async16(fs.s + i, W.seeds + off);
+  cp_async16(fs.q + i, W.coefs + off);
+  if (P == 4) cp_async4(fs.c + i, W.codes + (off >> 1));
+  cp_async4(fs.b + i, W.exp_bias + row);
+}
+
 // Read slot i back (after the copies have completed).
 template <int P>
 __device__ __forceinline__ void read_chunk(const FieldSlots &fs, int i, ChunkFields &f, uint32_t &rowk) {
@@ -325,63 +336,10 @@ __device__ __forceinline__ float2 block_dot2(const float (&G)[8], const float4 &
   return __ffma2_rn(make_float2(G[6], G[7]), make_float2(xb.z, xb.w), p);
 }
 
-// One chunk against one staged vector whose chunk slot is at xa (float4 pair
-// stride `stride` between the 16 half-blocks) and xn (stride `stride` between
-// the 8 block offsets): acc += sum_b scale_b * <w_b, x_b> as a packed pair.
-// nvalid: blocks of the chunk inside the row (8 unless the row is ragged).
-template <int P, bool VEC>
-__device__ __forceinline__ void chunk_dot_at(const StreamTables *tab, const ChunkFields &f, int nvalid,
-                                             uint32_t rowk, const float4 *xa, const float2 *xn,
-                                             int stride, float2 &acc) {
-#pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    if (!VEC && i >= nvalid) break;
-    float G[8];
-    const float s = regen_chunk_block<P>(tab, f, i, rowk, G);
-    const float2 d = block_dot2(G, xa[(2 * i) * stride], xa[(2 * i + 1) * stride], xn[i * stride]);
-    acc = __ffma2_rn(make_float2(s, s), d, acc);
-  }
-}
-
-// Two chunks (the gate and up rows of one expert) against the same staged
-// vector, interleaved block by block.
-template <int P, bool VEC>
-__device__ __forceinline__ void chunk_dot2_at(const StreamTables *tab, const ChunkFields &fa,
-                                              const ChunkFields &fb, int nvalid, uint32_t rowka,
-                                              uint32_t rowkb, const float4 *xa, const float2 *xn,
-                                              int stride, float2 &acca, float2 &accb) {
-#pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    if (!VEC && i >= nvalid) break;
-    float Ga[8], Gb[8];
-    const float sa = regen_chunk_block<P>(tab, fa, i, rowka, Ga);
-    const float sb = regen_chunk_block<P>(tab, fb, i, rowkb, Gb);
-    const float4 x0 = xa[(2 * i) * stride], x1 = xa[(2 * i + 1) * stride];
-    const float2 x2 = xn[i * stride];
-    acca = __ffma2_rn(make_float2(sa, sa), block_dot2(Ga, x0, x1, x2), acca);
-    accb = __ffma2_rn(make_float2(sb, sb), block_dot2(Gb, x0, x1, x2), accb);
-  }
-}
-
-// Packed fp32x2 products (FFMA2) or scalar FFMA chains in the chunk-major dots.
-constexpr bool kPackedDot = true;
-
 // scale * (<G, x> - Mg * sum(x)) added to acc, for one staged block.
 __device__ __forceinline__ void block_fma(const float (&G)[8], float s, const float4 &xa, const float4 &xb,
                                           const float2 &xn, float2 &acc) {
-  if (kPackedDot) {
-    acc = __ffma2_rn(make_float2(s, s), block_dot2(G, xa, xb, xn), acc);
-  } else {
-    float a = fmaf(G[0], xa.x, xn.x);
-    a = fmaf(G[1], xa.y, a);
-    a = fmaf(G[2], xa.z, a);
-    a = fmaf(G[3], xa.w, a);
-    a = fmaf(G[4], xb.x, a);
-    a = fmaf(G[5], xb.y, a);
-    a = fmaf(G[6], xb.z, a);
-    a = fmaf(G[7], xb.w, a);
-    acc.x = fmaf(s, a, acc.x);
-  }
+  acc = __ffma2_rn(make_float2(s, s), block_dot2(G, xa, xb, xn), acc);
 }
 
 // One chunk against the staged slot at xa (16 float4) / xn (8 float2) of the

@@ -36,33 +36,6 @@ int32_t max_active_ctas(const void *kernel, int threads, size_t smem);
 
 int32_t check_matrix(const nslm_seed_matrix *W);
 
-// Launch with programmatic stream serialisation: the kernel may begin while
-// the kernel ahead of it in the stream drains.  The kernel must call
-// grid_dependency_wait() before it reads what that kernel writes or writes
-// what it reads.
-template <typename Params>
-int32_t launch_after_previous(void (*kern)(Params), int grid, int threads, size_t smem,
-                              cudaStream_t s, const Params &p) {
-  cudaLaunchConfig_t cfg{};
-  cfg.gridDim = dim3((unsigned)grid);
-  cfg.blockDim = dim3((unsigned)threads);
-  cfg.dynamicSmemBytes = smem;
-  cfg.stream = s;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  return cuda_status(cudaLaunchKernelEx(&cfg, kern, p));
-}
-
-// Device side: wait until the grid ahead in the stream has completed and its
-// writes are visible; allow the grid behind to begin launching.
-__device__ __forceinline__ void grid_dependency_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
-__device__ __forceinline__ void grid_dependents_launch() {
-  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-}
-
 // Work layout of one seed matrix product: a CTA covers R rows x C chunks of
 // 8 blocks (64 weights); C = ceil(nb / 8).
 struct ChunkLayout {

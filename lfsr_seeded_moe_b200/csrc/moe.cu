@@ -25,7 +25,6 @@
 
 #include "chunk.cuh"
 #include "common.cuh"
-#include "decode1.cuh"
 #include "moe.cuh"
 
 namespace nslm {
@@ -508,10 +507,8 @@ static int32_t launch_decode_layer_t(const FfnDims &d, const nslm_seed_matrix *g
 int32_t launch_decode_layer(const FfnDims &d, const nslm_seed_matrix *gate,
                             const nslm_seed_matrix *up, const nslm_seed_matrix *down,
                             const SlotPlan *plan, const uint16_t *x_bf16, const float *y_prev,
-                            int T, int k, const FfnWorkspace &w, float *y, bool plan_early,
-                            cudaStream_t s, int &launches) {
-  if (T == 1 && decode1_supported(d, k))
-    return launch_decode1(d, gate, up, down, plan, x_bf16, y_prev, k, w.h, y, plan_early, s, launches);
+                            int T, int k, const FfnWorkspace &w, float *y, cudaStream_t s,
+                            int &launches) {
   if (d.P == 4) {
     return T == 1 ? launch_decode_layer_t<4, 1>(d, gate, up, down, plan, x_bf16, y_prev, T, k, w, y, s, launches)
                   : launch_decode_layer_t<4, 8>(d, gate, up, down, plan, x_bf16, y_prev, T, k, w, y, s, launches);

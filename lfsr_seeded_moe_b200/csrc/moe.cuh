@@ -61,7 +61,7 @@ int32_t launch_route_plan(const float *logits, const int32_t *ids, const float *
 int32_t launch_decode_layer(const FfnDims &d, const nslm_seed_matrix *gate,
                             const nslm_seed_matrix *up, const nslm_seed_matrix *down,
                             const SlotPlan *plan, const uint16_t *x_bf16, const float *y_prev,
-                            int T, int k, const FfnWorkspace &w, float *y, bool plan_early,
-                            cudaStream_t s, int &launches);
+                            int T, int k, const FfnWorkspace &w, float *y, cudaStream_t s,
+                            int &launches);
 
 }  // namespace nslm

@@ -192,8 +192,9 @@ __global__ void __launch_bounds__(kStack1MaxThreads, 1) stack1_kernel(const __gr
     if (c >= p.Ch) return;
     const size_t grow = (size_t)expert[slot] * p.inter + row;
     if (VEC) {
-      fetch_chunk<P>(Lm.gate, grow, nbh, c, fs, (2 * buf) * nthr + tid);
-      fetch_chunk<P>(Lm.up, grow, nbh, c, fs, (2 * buf + 1) * nthr + tid);
+      const uint32_t r32 = (uint32_t)grow, off = r32 * (uint32_t)nbh + 8u * (uint32_t)c;
+      fetch_chunk_off<P>(Lm.gate, off, r32, fs, (2 * buf) * nthr + tid);
+      fetch_chunk_off<P>(Lm.up, off, r32, fs, (2 * buf + 1) * nthr + tid);
     } else {
       load_chunk<P, false>(Lm.gate.seeds + grow * nbh, Lm.gate.coefs + grow * nbh,
                            P == 4 ? Lm.gate.codes + grow * (nbh / 2) : nullptr, nbh, c, fg);
@@ -216,7 +217,8 @@ __global__ void __launch_bounds__(kStack1MaxThreads, 1) stack1_kernel(const __gr
     b_locate(t, dSC, SC, r, s, c, q);
     const size_t grow = (size_t)s_expert[s] * p.hidden + n0 + r;
     if (VEC) {
-      fetch_chunk<P>(Lm.down, grow, nbi, c, fs, buf * nthr + tid);
+      const uint32_t r32 = (uint32_t)grow;
+      fetch_chunk_off<P>(Lm.down, r32 * (uint32_t)nbi + 8u * (uint32_t)c, r32, fs, buf * nthr + tid);
     } else {
       load_chunk<P, false>(Lm.down.seeds + grow * nbi, Lm.down.coefs + grow * nbi,
                            P == 4 ? Lm.down.codes + grow * (nbi / 2) : nullptr, nbi, c, f);
@@ -279,7 +281,9 @@ __global__ void __launch_bounds__(kStack1MaxThreads, 1) stack1_kernel(const __gr
         }
         if (p.J == 1 || c + 32 >= 32 * p.J) {
           const float g = warp_sum(ag.x + ag.y), u = warp_sum(au.x + au.y);
-          if (lane == 0) __stcg(p.h + (size_t)s_pair[slot] * p.inter + row, g / (1.f + expf(-g)) * u);
+          // SiLU with the fast exp and divide (relative error ~1e-6; an exp
+          // that overflows gives the limit 0)
+          if (lane == 0) __stcg(p.h + (size_t)s_pair[slot] * p.inter + row, __fdividef(g, 1.f + __expf(-g)) * u);
           ag = au = make_float2(0.f, 0.f);
         }
       }
@@ -405,6 +409,9 @@ static size_t stack1_smem(const FfnDims &d, int k, int threads) {
 
 bool stack1_supported(const FfnDims &d, int k) {
   if (k < 1 || k > kMaxK) return false;
+  // 32-bit element offsets into the field streams
+  if ((int64_t)d.E * d.inter * (d.hidden / 8) >= (1ll << 31) || (int64_t)d.E * d.hidden * (d.inter / 8) >= (1ll << 31))
+    return false;
   // fast divisions: divisors below 2^16, dividends below 2^22
   if (d.inter >= (1 << 16) || d.hidden >= (1 << 16)) return false;
   if ((int64_t)k * ceil_div(d.inter / 8, 8) >= (1 << 16)) return false;

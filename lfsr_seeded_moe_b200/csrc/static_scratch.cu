@@ -83,7 +83,7 @@ extern "C" int32_t nslm_moe_seed_ffn_static(const nslm_seed_matrix *gate, const 
     const nslm_moe_layer layer{*gate, *up, *down};
     st = launch_stack1(d, &layer, 1, fw.plans, x_bf16, nullptr, k, fw.h, fw.y_mid, y, fw.sync, fw.rms_part, s, launches);
   } else {
-    st = launch_decode_layer(d, gate, up, down, fw.plans, x_bf16, nullptr, T, k, fw, y, false, s, launches);
+    st = launch_decode_layer(d, gate, up, down, fw.plans, x_bf16, nullptr, T, k, fw, y, s, launches);
   }
   if (st == NSLM_OK) g_launches = launches;
   return st;
