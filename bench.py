@@ -458,7 +458,7 @@ def main():
                     traffic = int(ln.split(":")[1].split()[0])
                 except ValueError:
                     traffic = None
-    roofline = {"bound": "hbm", "kernel": "decode FFN layer (route-plan + gate/up + down)",
+    roofline = {"bound": "hbm", "kernel": "decode FFN layer: routing plan + one fused gate/up + down launch (stack1_kernel)",
                 "achieved": round(achieved, 1), "peak": hbm, "unit": "GB/s",
                 "frac": round(achieved / hbm, 4), "traffic": traffic,
                 "algorithmic_bytes_per_launch": layer_bytes, "us_per_launch": round(layer_s * 1e6, 3),

@@ -375,20 +375,22 @@ __global__ void __launch_bounds__(kStack1MaxThreads, 1) stack1_kernel(const __gr
 
 static int stack1_rows_per_cta(const FfnDims &d) { return std::max(1, ceil_div(d.hidden, num_sms())); }
 
-// Threads per CTA: the whole warps, at most kStack1MaxThreads, that leave the
+// Threads per CTA: whole warps in [16, kStack1MaxThreads / 32] that leave the
 // fewest idle task slots in both phases (a phase A task is 16 blocks per
-// lane, a phase B task 8); on a tie the most warps.  Few warps with many
-// registers each beat many warps here: the unrolled block loop needs the
-// registers to overlap its table lookups and dot products.
+// lane, a phase B task 8); on a tie the most warps.  Measured on B200 for the
+// 100-expert 2048/1408 layer: 20 warps 33.6 us, 16 warps 33.8, 14 warps 36.6,
+// 11 warps 35.7, 26 warps (72 registers) 37.0 per layer: the unrolled block
+// loop needs ~96 registers to overlap its table lookups and dot products, and
+// fewer than 16 warps cannot hide the remaining latency.
 static int stack1_threads(const FfnDims &d, int k) {
   const int sms = num_sms();
   const int Ch = ceil_div(d.hidden / 8, 8), Ci = ceil_div(d.inter / 8, 8);
   const int J = ceil_div(Ch, 32);
   const long long a_tasks = (long long)k * d.inter * J;
   const long long b_tasks = (long long)stack1_rows_per_cta(d) * k * Ci;
-  int best = 8;
+  int best = 16;
   long long best_cost = -1;
-  for (int nw = kStack1MaxThreads / 32; nw >= 8; --nw) {
+  for (int nw = kStack1MaxThreads / 32; nw >= 16; --nw) {
     const long long ra = (a_tasks + (long long)sms * nw - 1) / ((long long)sms * nw);
     const long long rb = (b_tasks + 32ll * nw - 1) / (32ll * nw);
     const long long cost = (16 * ra + 8 * rb) * nw;
