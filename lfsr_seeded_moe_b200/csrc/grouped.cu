@@ -11,9 +11,10 @@
 // bf16 (round to nearest even of the exact fp32 weight) straight into shared
 // memory (512 threads, each owning two blocks of two rows per slice), copy the
 // matching token rows, and one thread issues tcgen05.mma
-// (bf16 x bf16 -> fp32 in tensor memory).  Two shared-memory stages let the
-// tensor core work on one slice while the threads regenerate the next.  The
-// weights are never written to global memory.
+// (bf16 x bf16 -> fp32 in tensor memory).  Three shared-memory stages let the
+// tensor core work on one slice while the threads regenerate the next and
+// the token rows of the one after are in flight.  The weights are never
+// written to global memory.
 //
 // Shared-memory layout of both operands is the K-major, no-swizzle canonical
 // layout: one 8-weight block of a row is one 16-byte row of an 8 x 16-byte
@@ -29,9 +30,13 @@ namespace nslm {
 
 constexpr int kBM = 128;        // weight rows per tile (MMA M)
 constexpr int kBK = 64;         // K per stage: 8 blocks, 128 bytes of bf16 per row
-constexpr int kGThreads = 512;                 // producer threads
-constexpr int kCtaThreads = kGThreads + 32;    // + one warp that issues the MMAs
-constexpr int kStages = 2;
+constexpr int kGThreads = 512;                  // producer threads (warps 0-15)
+constexpr int kEpiWarp0 = kGThreads / 32;       // warps 16-19: the epilogue warpgroup
+constexpr int kMmaWarp = kEpiWarp0 + 4;         // warp 20: issues the MMAs
+constexpr int kCtaThreads = 32 * (kMmaWarp + 1);
+constexpr int kStages = 3;  // slice i uses stage i % 3: the token rows of slice i+1 are
+                             // copied while slice i is regenerated, into the stage that
+                             // the MMAs of slice i-2 have released
 constexpr long long kWaitCycles = 4000000000LL;  // ~2 s: a wait longer than this is an error
 
 enum GMode { GMODE_GEMM = 0, GMODE_GATEUP = 1, GMODE_DOWN = 2 };
@@ -53,19 +58,26 @@ struct GroupedParams {
   const float *pair_w;      // DOWN: pair -> routing weight
 };
 
+// Stream tables: kTabCopies interleaved copies (entry e of copy c at word
+// kTabCopies * e + c), lane l reading copy l % kTabCopies.  Measured on B200
+// (100-expert batched layer, P=3): one copy 727 / 890 us at T = 64 / 512,
+// eight copies 727 / 1252 us -- the larger shared footprint costs more than
+// the bank conflicts it removes.
+constexpr int kTabCopies = 1;
+
 // Regenerate blocks (b, b+1) of one row as bf16 and store them as two 16-byte
 // core-matrix rows.  seeds2/coefs2 hold the two blocks' 16-bit fields, code2
-// their two exponent nibbles.
+// their two exponent nibbles; tl is this lane's table copy.
 template <int P>
-__device__ __forceinline__ void regen_pair_bf16(const StreamTablesX32 *tab, uint32_t lane4, uint32_t seeds2,
-                                                uint32_t coefs2, uint32_t code2, uint32_t rowk, uint4 *dst0,
-                                                uint4 *dst1) {
+__device__ __forceinline__ void regen_pair_bf16(const uint32_t *tl, uint32_t seeds2, uint32_t coefs2,
+                                                uint32_t code2, uint32_t rowk, uint4 *dst0, uint4 *dst1) {
 #pragma unroll
   for (int h = 0; h < 2; ++h) {
-    const uint32_t seed = h ? (seeds2 >> 16) : (seeds2 & 0xFFFFu);
     const uint32_t q = h ? (coefs2 >> 16) : (coefs2 & 0xFFFFu);
-    uint32_t v, nxt;
-    stream_pair_x32(tab, lane4, seed, v, nxt);
+    const uint32_t b0 = h ? ((seeds2 >> 16) & 0xFFu) : (seeds2 & 0xFFu);
+    const uint32_t b1 = h ? (seeds2 >> 24) : ((seeds2 >> 8) & 0xFFu);
+    const uint32_t nxt = tl[kTabCopies * b0] ^ tl[kTabCopies * (256u + b1)];
+    const uint32_t v = h ? (seeds2 & 0xFFFF0000u) : (seeds2 << 16);
     float G[8];
     block_magic(v, nxt, coef_pairs2<P>(q), G);
     const uint32_t code = (P == 4) ? ((code2 >> (4 * h)) & 0xFu) : (q >> 12);
@@ -75,8 +87,8 @@ __device__ __forceinline__ void regen_pair_bf16(const StreamTablesX32 *tab, uint
 #pragma unroll
     for (int r = 0; r < 8; r += 2) {
       // (Mg + A) * s - Mg * s = A * s exactly (power-of-two scale)
-      const __nv_bfloat162 b = __floats2bfloat162_rn(fmaf(G[r], s, off), fmaf(G[r + 1], s, off));
-      packed[r >> 1] = *reinterpret_cast<const uint32_t *>(&b);
+      const __nv_bfloat162 bb = __floats2bfloat162_rn(fmaf(G[r], s, off), fmaf(G[r + 1], s, off));
+      packed[r >> 1] = *reinterpret_cast<const uint32_t *>(&bb);
     }
     *(h ? dst1 : dst0) = make_uint4(packed[0], packed[1], packed[2], packed[3]);
   }
@@ -90,16 +102,19 @@ template <int MODE> struct TileShape {
   static constexpr int kRows = (MODE == GMODE_GATEUP) ? kBM : 2 * kBM;
 };
 
-// Pipeline (no CTA-wide barrier in the main loop):
-//   each of the 512 producer threads, per K slice: wait empty[stage] -> start async copies of its
-//     token-row chunks -> regenerate its two tasks' blocks (weight fields were
-//     prefetched two slices earlier) -> wait for its copies -> proxy fence ->
-//     arrive full[stage]
-//   the MMA warp (lane 0), per K slice: wait full[stage] -> (first slice of a tile: wait
-//     acc_empty) -> issue the MMAs -> commit empty[stage] (and acc_full after
-//     the tile's last slice)
-//   warps 0-3, per tile: wait acc_full -> read D from tensor memory -> store
-//     -> arrive acc_empty
+// Pipeline (no CTA-wide barrier in the main loop; slice i uses stage i % 3),
+// three roles:
+//   producers (warps 0-15), per K slice i: start the async copies of their
+//     token-row chunks of slice i+1 (after waiting empty[(i+1) % 3], i.e. for
+//     the MMAs of slice i-2) -> regenerate their two tasks' blocks of slice i
+//     (weight fields were loaded three slices earlier) -> wait for their
+//     copies of slice i -> proxy fence -> arrive full[i % 3]
+//   the MMA warp (warp 20, lane 0), per K slice: wait full[stage] -> (first
+//     slice of a tile: wait acc_empty) -> issue the MMAs -> commit
+//     empty[stage] (and acc_full after the tile's last slice)
+//   the epilogue warpgroup (warps 16-19), per tile: wait acc_full -> read D
+//     from tensor memory -> store -> arrive acc_empty; the producers never
+//     stop for it
 // Every wait is bounded; a thread that gives up raises a shared abort flag
 // that all threads check before each slice.
 struct SliceFields {  // packed fields of one thread's two tasks for one K slice
@@ -119,12 +134,34 @@ __device__ __forceinline__ void load_slice(const uint32_t *const (&sp)[2], const
 }
 
 
+// The tile the CTA's n-th tile index t covers.
+struct TileInfo {
+  int e, m0, r_begin, n_valid, N;
+};
+template <int MODE>
+__device__ __forceinline__ TileInfo tile_info(const GroupedParams &p, int t) {
+  int lo_e = 0, hi_e = p.E - 1;  // the last e with tile_start[e] <= t
+  while (lo_e < hi_e) {
+    const int mid = (lo_e + hi_e + 1) >> 1;
+    if (p.tile_start[mid] <= t) lo_e = mid; else hi_e = mid - 1;
+  }
+  TileInfo ti;
+  ti.e = lo_e;
+  const int local = t - p.tile_start[ti.e];
+  const int mt = local % p.mtiles, nt = local / p.mtiles;
+  const int seg_begin = max(0, p.offsets[ti.e]), seg_end = min(p.R, p.offsets[ti.e + 1]);
+  ti.r_begin = seg_begin + nt * p.bn;
+  ti.n_valid = max(0, min(p.bn, seg_end - ti.r_begin));
+  ti.N = max(16, (ti.n_valid + 15) & ~15);
+  ti.m0 = mt * TileShape<MODE>::kRows;
+  return ti;
+}
+
 template <int P, int MODE>
 __global__ void __launch_bounds__(kCtaThreads, 1) grouped_seed_gemm_kernel(const GroupedParams p) {
-  constexpr int kRows = TileShape<MODE>::kRows;
   extern __shared__ __align__(1024) uint8_t gsm[];
-  StreamTablesX32 *tab = reinterpret_cast<StreamTablesX32 *>(gsm);
-  uint8_t *a_base = gsm + sizeof(StreamTablesX32);               // [stage][sub 0..1][128 rows x 128 B]
+  uint32_t *tab = reinterpret_cast<uint32_t *>(gsm);             // kTabCopies interleaved copies
+  uint8_t *a_base = gsm + kTabCopies * 2048;                     // [stage][sub 0..1][128 rows x 128 B]
   uint8_t *b_base = a_base + (size_t)kStages * 2 * kBM * 128;    // [stage][bn rows x 128 B]
   __shared__ __align__(8) uint64_t full_bar[kStages];
   __shared__ __align__(8) uint64_t empty_bar[kStages];
@@ -133,12 +170,11 @@ __global__ void __launch_bounds__(kCtaThreads, 1) grouped_seed_gemm_kernel(const
   __shared__ volatile int s_abort;
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const bool issuer_warp = tid >= kGThreads;
   // a producer's tasks: row trow, block pair bp, of sub-tiles 0 and 1
   const int trow = tid & (kBM - 1), bp = (tid >> 7) & 3;
-  build_stream_tables_x32(tab);
+  build_stream_tables_rep<kTabCopies>(tab);
+  const uint32_t *tl = tab + (lane & (kTabCopies - 1));
   if (warp == 0) umma::tmem_alloc(umma::smem_u32(&tmem_base_s), (uint32_t)p.tmem_cols);
-  const uint32_t lane4 = 4u * (uint32_t)lane;
   if (tid == 0) {
     for (int s = 0; s < kStages; ++s) {
       umma::mbar_init(umma::smem_u32(&full_bar[s]), kGThreads);
@@ -156,25 +192,17 @@ __global__ void __launch_bounds__(kCtaThreads, 1) grouped_seed_gemm_kernel(const
 
   const int total_tiles = p.tile_start[p.E];
   const int ksteps = p.K / kBK;
-  uint32_t it = 0;      // K slices produced (or consumed) by this CTA
-  uint32_t ntile = 0;   // tiles finished by this CTA
+  uint32_t it = 0;      // K slices produced (or consumed) by this thread's role
+  uint32_t ntile = 0;   // tiles finished
 
-  if (issuer_warp) {  // ---- the MMA warp: lane 0 waits for each slice and issues it
+  if (warp == kMmaWarp) {  // ---- lane 0 waits for each slice and issues its MMAs
     if (lane == 0) {
       for (int t = blockIdx.x; t < total_tiles && !s_abort; t += gridDim.x, ++ntile) {
-        int lo_e = 0, hi_e = p.E - 1;
-        while (lo_e < hi_e) {
-          const int mid = (lo_e + hi_e + 1) >> 1;
-          if (p.tile_start[mid] <= t) lo_e = mid; else hi_e = mid - 1;
-        }
-        const int e = lo_e;
-        const int nt = (t - p.tile_start[e]) / p.mtiles;
-        const int r_begin = max(0, p.offsets[e]) + nt * p.bn;
-        const int n_valid = max(0, min(p.bn, min(p.R, p.offsets[e + 1]) - r_begin));
-        const uint32_t idesc = umma::idesc_bf16_f32(kBM, max(16, (n_valid + 15) & ~15));
+        const TileInfo ti = tile_info<MODE>(p, t);
+        const uint32_t idesc = umma::idesc_bf16_f32(kBM, max(16, (ti.n_valid + 15) & ~15));
         for (int kt = 0; kt < ksteps; ++kt, ++it) {
-          const int stage = it & 1;
-          bool go = umma::mbar_wait_bounded(umma::smem_u32(&full_bar[stage]), (it >> 1) & 1, kWaitCycles);
+          const int stage = it % kStages;
+          bool go = umma::mbar_wait_bounded(umma::smem_u32(&full_bar[stage]), (it / kStages) & 1, kWaitCycles);
           if (go && kt == 0 && ntile > 0)  // the epilogue has drained the last tile's accumulators
             go = umma::mbar_wait_bounded(umma::smem_u32(&acc_empty_bar), (ntile - 1) & 1, kWaitCycles);
           if (!go) { s_abort = 1; break; }
@@ -196,143 +224,148 @@ __global__ void __launch_bounds__(kCtaThreads, 1) grouped_seed_gemm_kernel(const
       }
     }
     __syncwarp();
-  } else
-  for (int t = blockIdx.x; t < total_tiles; t += gridDim.x, ++ntile) {
-    if (s_abort) break;
-    int lo_e = 0, hi_e = p.E - 1;  // the last e with tile_start[e] <= t
-    while (lo_e < hi_e) {
-      const int mid = (lo_e + hi_e + 1) >> 1;
-      if (p.tile_start[mid] <= t) lo_e = mid; else hi_e = mid - 1;
-    }
-    const int e = lo_e;
-    const int local = t - p.tile_start[e];
-    const int mt = local % p.mtiles, nt = local / p.mtiles;
-    const int seg_begin = max(0, p.offsets[e]), seg_end = min(p.R, p.offsets[e + 1]);
-    const int r_begin = seg_begin + nt * p.bn;
-    const int n_valid = max(0, min(p.bn, seg_end - r_begin));
-    const int N = max(16, (n_valid + 15) & ~15);
-    const int m0 = mt * kRows;
-
-    // the two tasks' weight rows for the whole tile
-    const uint32_t *sp[2];
-    const uint32_t *qp[2];
-    const uint8_t *cpp[2];
-    bool ok[2];
-    uint32_t rowk[2];
-#pragma unroll
-    for (int j = 0; j < 2; ++j) {
-      const nslm_seed_matrix &W = (MODE == GMODE_GATEUP && j) ? p.A1 : p.A0;
-      const int grow = m0 + (MODE == GMODE_GATEUP ? 0 : j * kBM) + trow;
-      ok[j] = grow < p.rows;
-      const size_t wr = (size_t)e * p.rows + (ok[j] ? grow : 0);
-      sp[j] = reinterpret_cast<const uint32_t *>(W.seeds + wr * p.nb) + bp;
-      qp[j] = reinterpret_cast<const uint32_t *>(W.coefs + wr * p.nb) + bp;
-      cpp[j] = (P == 4) ? W.codes + wr * (p.nb / 2) + bp : nullptr;
-      rowk[j] = row_scale_key(__ldg(W.exp_bias + wr));
-    }
-    const size_t a_off = ((trow >> 3) * 8 + 2 * bp) * 128 + (trow & 7) * 16;
-    // token rows this thread copies: chunks (n, kc) for n = trow, trow + 128 and kc = bp, bp + 4
-    const uint16_t *brow[2];
-    uint32_t bbytes[2], bdst[2][2];
-#pragma unroll
-    for (int i = 0; i < 2; ++i) {
-      const int n = trow + 128 * i;
-#pragma unroll
-      for (int h = 0; h < 2; ++h) bdst[i][h] = ((n >> 3) * 8 + bp + 4 * h) * 128 + (n & 7) * 16;
-      const bool v = n < n_valid;
-      const int xr = v ? (p.row_of ? p.row_of[r_begin + n] : r_begin + n) : 0;
-      brow[i] = p.x + (size_t)xr * p.K;
-      bbytes[i] = v ? 16u : 0u;  // zero-fill rows past n_valid
-    }
-
-    SliceFields f0, f1;
-    load_slice<P>(sp, qp, cpp, ok, 0, f0);
-    if (ksteps > 1) load_slice<P>(sp, qp, cpp, ok, 1, f1);
-    for (int kt = 0; kt < ksteps; ++kt, ++it) {
-      const int stage = it & 1;
-      if (it >= 2 && !umma::mbar_wait_bounded(umma::smem_u32(&empty_bar[stage]), ((it >> 1) - 1) & 1, kWaitCycles))
-        s_abort = 1;
+  } else if (warp >= kEpiWarp0) {  // ---- epilogue warpgroup: tensor memory -> outputs
+    const int ew = warp - kEpiWarp0;  // tensor-memory lanes 32 ew .. 32 ew + 31
+    for (int t = blockIdx.x; t < total_tiles; t += gridDim.x, ++ntile) {
       if (s_abort) break;
-      uint8_t *atile = a_base + (size_t)stage * 2 * kBM * 128;
-      uint8_t *btile = b_base + (size_t)stage * p.bn * 128;
-      // token rows for this slice: asynchronous copies, overlapped with the regeneration
-      const uint32_t bsa = umma::smem_u32(btile);
-#pragma unroll
-      for (int i = 0; i < 2; ++i) {
-        if (trow + 128 * i < N) {
-#pragma unroll
-          for (int h = 0; h < 2; ++h)
-            cp_async16(bsa + bdst[i][h], brow[i] + kt * kBK + (bp + 4 * h) * 8, bbytes[i]);
-        }
-      }
-      const SliceFields cur = f0;
-      f0 = f1;
-      if (kt + 2 < ksteps) load_slice<P>(sp, qp, cpp, ok, kt + 2, f1);
-      // rows past the matrix carry zero coefficient fields, which regenerate
-      // to exactly zero weights: no branch
-#pragma unroll
-      for (int j = 0; j < 2; ++j) {
-        uint4 *dst0 = reinterpret_cast<uint4 *>(atile + j * kBM * 128 + a_off);
-        uint4 *dst1 = reinterpret_cast<uint4 *>(atile + j * kBM * 128 + a_off + 128);
-        regen_pair_bf16<P>(tab, lane4, cur.s2[j], cur.q2[j], cur.c2[j], rowk[j], dst0, dst1);
-      }
-      cp_async_wait_all();
-      umma::fence_proxy_async();
-      umma::mbar_arrive(umma::smem_u32(&full_bar[stage]));
-
-    }
-    if (s_abort) break;
-
-    // ---- epilogue (warps 0-3): read D from tensor memory once the tile's MMAs are done
-    if (warp < 4) {
+      const TileInfo ti = tile_info<MODE>(p, t);
       __syncwarp();
       const bool acc_ok = umma::mbar_wait_bounded(umma::smem_u32(&acc_full_bar), ntile & 1, kWaitCycles);
       if (!acc_ok) s_abort = 1;
       // tcgen05.ld is warp-collective: the whole warp takes one decision
-      if (__all_sync(0xffffffffu, acc_ok && !s_abort)) {
-        umma::fence_after_sync();
-        const uint32_t lane_addr = tmem + ((uint32_t)(32 * warp) << 16);
-        if (MODE == GMODE_GATEUP) {
-          const int row = m0 + 32 * warp + lane;
+      if (!__all_sync(0xffffffffu, acc_ok && !s_abort)) break;
+      umma::fence_after_sync();
+      const uint32_t lane_addr = tmem + ((uint32_t)(32 * ew) << 16);
+      if (MODE == GMODE_GATEUP) {
+        const int row = ti.m0 + 32 * ew + lane;
+        const bool rok = row < p.rows;
+        for (int c = 0; c * 8 < ti.N; ++c) {
+          float g[8], up[8];
+          umma::tmem_ld8(lane_addr + (uint32_t)(c * 8), g);
+          umma::tmem_ld8(lane_addr + (uint32_t)(p.bn + c * 8), up);
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            const int n = c * 8 + j;
+            if (!rok || n >= ti.n_valid) continue;
+            const size_t sr = (size_t)(ti.r_begin + n);
+            const float hv = __fdividef(g[j], 1.f + __expf(-g[j])) * up[j];
+            p.h[sr * p.rows + row] = __bfloat16_as_ushort(__float2bfloat16_rn(hv));
+          }
+        }
+      } else {
+#pragma unroll
+        for (int mh = 0; mh < 2; ++mh) {
+          const int row = ti.m0 + mh * kBM + 32 * ew + lane;
           const bool rok = row < p.rows;
-          for (int c = 0; c * 8 < N; ++c) {
-            float g[8], up[8];
-            umma::tmem_ld8(lane_addr + (uint32_t)(c * 8), g);
-            umma::tmem_ld8(lane_addr + (uint32_t)(p.bn + c * 8), up);
+          for (int c = 0; c * 8 < ti.N; ++c) {
+            float v[8];
+            umma::tmem_ld8(lane_addr + (uint32_t)(mh * p.bn + c * 8), v);
 #pragma unroll
             for (int j = 0; j < 8; ++j) {
               const int n = c * 8 + j;
-              if (!rok || n >= n_valid) continue;
-              const size_t sr = (size_t)(r_begin + n);
-              p.h[sr * p.rows + row] = __bfloat16_as_ushort(__float2bfloat16_rn(g[j] / (1.f + expf(-g[j])) * up[j]));
-            }
-          }
-        } else {
-#pragma unroll
-          for (int mh = 0; mh < 2; ++mh) {
-            const int row = m0 + mh * kBM + 32 * warp + lane;
-            const bool rok = row < p.rows;
-            for (int c = 0; c * 8 < N; ++c) {
-              float v[8];
-              umma::tmem_ld8(lane_addr + (uint32_t)(mh * p.bn + c * 8), v);
-#pragma unroll
-              for (int j = 0; j < 8; ++j) {
-                const int n = c * 8 + j;
-                if (!rok || n >= n_valid) continue;
-                const size_t sr = (size_t)(r_begin + n);
-                if (MODE == GMODE_GEMM) {
-                  p.y[sr * p.rows + row] = v[j];
-                } else {
-                  const int pr = p.pair_of[sr];
-                  p.part[(size_t)pr * p.rows + row] = p.pair_w[pr] * v[j];
-                }
+              if (!rok || n >= ti.n_valid) continue;
+              const size_t sr = (size_t)(ti.r_begin + n);
+              if (MODE == GMODE_GEMM) {
+                p.y[sr * p.rows + row] = v[j];
+              } else {
+                const int pr = p.pair_of[sr];
+                p.part[(size_t)pr * p.rows + row] = p.pair_w[pr] * v[j];
               }
             }
           }
         }
-        umma::fence_before_sync();
-        umma::mbar_arrive(umma::smem_u32(&acc_empty_bar));
       }
+      umma::fence_before_sync();
+      umma::mbar_arrive(umma::smem_u32(&acc_empty_bar));
+    }
+  } else {  // ---- producers (warps 0-15)
+    for (int t = blockIdx.x; t < total_tiles; t += gridDim.x) {
+      if (s_abort) break;
+      const TileInfo ti = tile_info<MODE>(p, t);
+      const int N = ti.N;
+      // the two tasks' weight rows for the whole tile
+      const uint32_t *sp[2];
+      const uint32_t *qp[2];
+      const uint8_t *cpp[2];
+      bool ok[2];
+      uint32_t rowk[2];
+#pragma unroll
+      for (int j = 0; j < 2; ++j) {
+        const nslm_seed_matrix &W = (MODE == GMODE_GATEUP && j) ? p.A1 : p.A0;
+        const int grow = ti.m0 + (MODE == GMODE_GATEUP ? 0 : j * kBM) + trow;
+        ok[j] = grow < p.rows;
+        const size_t wr = (size_t)ti.e * p.rows + (ok[j] ? grow : 0);
+        sp[j] = reinterpret_cast<const uint32_t *>(W.seeds + wr * p.nb) + bp;
+        qp[j] = reinterpret_cast<const uint32_t *>(W.coefs + wr * p.nb) + bp;
+        cpp[j] = (P == 4) ? W.codes + wr * (p.nb / 2) + bp : nullptr;
+        rowk[j] = row_scale_key(__ldg(W.exp_bias + wr));
+      }
+      const size_t a_off = ((trow >> 3) * 8 + 2 * bp) * 128 + (trow & 7) * 16;
+      // token rows this thread copies: chunks (n, kc) for n = trow, trow + 128 and kc = bp, bp + 4
+      const uint16_t *brow[2];
+      uint32_t bbytes[2], bdst[2][2];
+#pragma unroll
+      for (int i = 0; i < 2; ++i) {
+        const int n = trow + 128 * i;
+#pragma unroll
+        for (int h = 0; h < 2; ++h) bdst[i][h] = ((n >> 3) * 8 + bp + 4 * h) * 128 + (n & 7) * 16;
+        const bool v = n < ti.n_valid;
+        const int xr = v ? (p.row_of ? p.row_of[ti.r_begin + n] : ti.r_begin + n) : 0;
+        brow[i] = p.x + (size_t)xr * p.K;
+        bbytes[i] = v ? 16u : 0u;  // zero-fill rows past n_valid
+      }
+
+      // Token rows of slice kt+1 are copied while slice kt is regenerated; the
+      // stage they land in is free once the MMAs of slice (it+1) - kStages are done.
+      const uint32_t b_stage0 = umma::smem_u32(b_base);
+      auto copy_b = [&](int kt_b, uint32_t it_b) -> bool {
+        if (it_b >= (uint32_t)kStages &&
+            !umma::mbar_wait_bounded(umma::smem_u32(&empty_bar[it_b % kStages]), (it_b / kStages - 1) & 1,
+                                     kWaitCycles))
+          return false;
+        const uint32_t bsa = b_stage0 + (uint32_t)((it_b % kStages) * p.bn * 128);
+#pragma unroll
+        for (int i = 0; i < 2; ++i) {
+          if (trow + 128 * i < N) {
+#pragma unroll
+            for (int h = 0; h < 2; ++h)
+              cp_async16(bsa + bdst[i][h], brow[i] + kt_b * kBK + (bp + 4 * h) * 8, bbytes[i]);
+          }
+        }
+        return true;
+      };
+      if (!copy_b(0, it)) s_abort = 1;
+      cp_async_commit();
+
+      // weight fields three slices ahead
+      SliceFields f0, f1, f2;
+      load_slice<P>(sp, qp, cpp, ok, 0, f0);
+      if (ksteps > 1) load_slice<P>(sp, qp, cpp, ok, 1, f1);
+      if (ksteps > 2) load_slice<P>(sp, qp, cpp, ok, 2, f2);
+      for (int kt = 0; kt < ksteps; ++kt, ++it) {
+        const int stage = it % kStages;
+        if (s_abort) break;
+        // the stage of slice it was claimed when its token rows were copied
+        if (kt + 1 < ksteps && !copy_b(kt + 1, it + 1)) s_abort = 1;
+        cp_async_commit();
+        uint8_t *atile = a_base + (size_t)stage * 2 * kBM * 128;
+        const SliceFields cur = f0;
+        f0 = f1;
+        f1 = f2;
+        if (kt + 3 < ksteps) load_slice<P>(sp, qp, cpp, ok, kt + 3, f2);
+        // rows past the matrix carry zero coefficient fields, which regenerate
+        // to exactly zero weights: no branch
+#pragma unroll
+        for (int j = 0; j < 2; ++j) {
+          uint4 *dst0 = reinterpret_cast<uint4 *>(atile + j * kBM * 128 + a_off);
+          uint4 *dst1 = reinterpret_cast<uint4 *>(atile + j * kBM * 128 + a_off + 128);
+          regen_pair_bf16<P>(tl, cur.s2[j], cur.q2[j], cur.c2[j], rowk[j], dst0, dst1);
+        }
+        cp_async_wait<1>();  // this slice's token rows (the next slice's may still be in flight)
+        umma::fence_proxy_async();
+        umma::mbar_arrive(umma::smem_u32(&full_bar[stage]));
+      }
+      cp_async_wait_all();
     }
   }
 
@@ -341,9 +374,9 @@ __global__ void __launch_bounds__(kCtaThreads, 1) grouped_seed_gemm_kernel(const
   if (s_abort) {
     if (tid == 0) atomicExch(p.status, 1);
     // let MMAs still in flight finish (bounded) before the tensor memory is freed
-    if (tid == kGThreads && it > 0) {
+    if (warp == kMmaWarp && lane == 0 && it > 0) {
       const uint32_t last = it - 1;
-      umma::mbar_wait_bounded(umma::smem_u32(&empty_bar[last & 1]), (last >> 1) & 1, kWaitCycles);
+      umma::mbar_wait_bounded(umma::smem_u32(&empty_bar[last % kStages]), (last / kStages) & 1, kWaitCycles);
     }
   }
   umma::fence_before_sync();
@@ -453,7 +486,7 @@ static int tmem_cols_for(int ncols) {
 }
 
 static size_t grouped_smem(int bn) {
-  return sizeof(StreamTablesX32) + (size_t)kStages * 2 * kBM * 128 + (size_t)kStages * bn * 128;
+  return kTabCopies * 2048 + (size_t)kStages * 2 * kBM * 128 + (size_t)kStages * bn * 128;
 }
 
 template <int P, int MODE>
