@@ -141,8 +141,9 @@ int32_t nslm_moe_route_topk(const float *logits, int32_t T, int32_t E, int32_t k
  * ids: int32 [T][k] in [0, E); w: fp32 [T][k]; y: fp32 [T][hidden].
  * T <= 8 runs the decode path (fp32 weights and hidden activations);
  * larger T runs the tensor-core path (bf16 weights, bf16 hidden activation;
- * hidden and inter multiples of 64, E <= 1024; the first int32 of the
- * workspace is set to 1 if a tensor-core wait timed out).
+ * hidden and inter multiples of 64, E <= 1024).  The first int32 of the
+ * workspace is set nonzero if a device-side wait (the tensor-core pipeline,
+ * or the grid barrier of the one-token kernel) gave up.
  * Workspace: nslm_workspace_bytes(NSLM_OP_MOE_FFN, T, E, hidden, inter, k, 0). */
 int32_t nslm_moe_seed_ffn(const nslm_seed_matrix *gate, const nslm_seed_matrix *up,
                           const nslm_seed_matrix *down, int32_t E, const uint16_t *x_bf16,
@@ -186,6 +187,26 @@ int32_t nslm_moe_seed_ffn_static(const nslm_seed_matrix *gate, const nslm_seed_m
 int32_t nslm_moe_stack_decode(const nslm_moe_layer *layers, int32_t L, int32_t E, int32_t k,
                               const float *logits, const uint16_t *x0_bf16, int32_t T,
                               float *y, void *ws, size_t ws_bytes, nslm_stream_t stream);
+
+/* Seed search, the encoder ("NanoSeedLM: LLM inference using pseudo-random
+ * numbers", "What I changed: September 2026": every block walks all 65,535
+ * seeds; "'GPU search == CPU search'": the GPU search gives the C reference's
+ * answer bit for bit).  For each block of 8 weights of w (fp32 [N][K], row
+ * major, device) and every seed in [seed_lo, seed_hi] (1 <= seed_lo <=
+ * seed_hi <= 65535) and code in 0..15:
+ *   c = round_half_even(pinv(U(seed)) w_block / 2^(code + exp_bias[row])),
+ *       clamped to [-8, 7];  pinv(U) = (U^T U)^-1 U^T by Gauss-Jordan
+ *       elimination with partial pivoting, fp64, no fused multiply-add
+ *   err = sum_r (w_r - 2^(code + exp_bias[row]) (U c)_r)^2, fp64
+ * The smallest err wins; ties go to the larger code, then the lower seed.
+ * out: the packed matrix to fill (N, K, P give the shape; K % 8 == 0, P=4
+ * needs K % 16 == 0): seeds, coefs (and codes for P = 4) are WRITTEN;
+ * exp_bias [N] is READ (the row biases to encode with).  err: fp64 [N][K/8]
+ * of the winning errors, or null.  A block whose every seed is singular gets
+ * seed 0, zero coefficients and err = +inf.  All pointers are device
+ * pointers; the seed streams of out must not overlap w. */
+int32_t nslm_seed_search(const float *w, const nslm_seed_matrix *out, int32_t seed_lo,
+                         int32_t seed_hi, double *err, nslm_stream_t stream);
 
 /* Test exports: the regenerated weights themselves, written out densely.
  * w_out: fp32 [N][K] (exact) or bf16 bit patterns [N][K] (round to nearest

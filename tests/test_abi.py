@@ -90,3 +90,15 @@ def test_workspace_sizes_are_monotone():
     b = nslm.nslm_workspace_bytes(nslm.NSLM_OP_MOE_STACK, 8, 100, 2048, 1408, 8, 45)
     assert 0 < a < b
     assert nslm.nslm_workspace_bytes(nslm.NSLM_OP_GEMV, 1, 1, 1, 1, 1) == 0
+
+
+def test_search_argument_checks():
+    f = nslm.raw().nslm_seed_search
+    W = _mat(N=4, K=32, P=4)
+    w = 0x9000000
+    assert f(w, ctypes.byref(W), 0, 10, 0, 0) == nslm.NSLM_ERR_ARG        # seeds start at 1
+    assert f(w, ctypes.byref(W), 10, 65536, 0, 0) == nslm.NSLM_ERR_ARG    # 16-bit seeds
+    assert f(w, ctypes.byref(W), 20, 10, 0, 0) == nslm.NSLM_ERR_ARG       # empty range
+    assert f(0, ctypes.byref(W), 1, 10, 0, 0) == nslm.NSLM_ERR_ARG        # no weights
+    assert f(w, ctypes.byref(_mat(N=4, K=24, P=4)), 1, 10, 0, 0) == nslm.NSLM_ERR_SHAPE
+    assert f(w, None, 1, 10, 0, 0) == nslm.NSLM_ERR_ARG
