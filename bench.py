@@ -279,6 +279,50 @@ def batched_sweep(torch, nslm, synth, dev, hbm, bf16_peak):
     return out
 
 
+class _Encoded:
+    """Device streams of an N x K packed matrix for the seed search to fill."""
+
+    def __init__(self, torch, dev, N, K, P, bias):
+        nb = K // 8
+        self.N, self.K, self.P = N, K, P
+        self.seeds = torch.empty(N, nb, dtype=torch.int16, device=dev)
+        self.coefs = torch.empty(N, nb, dtype=torch.int16, device=dev)
+        self.codes = torch.empty(N, nb // 2, dtype=torch.uint8, device=dev) if P == 4 else None
+        self.exp_bias = torch.full((N,), bias, dtype=torch.int32, device=dev)
+
+
+def search_leg(torch, nslm, dev, with_cpu: bool):
+    """Seed search (the encoder) over all 65,535 seeds x 16 codes: GPU blocks/s
+    on a 64 x 2048 fp32 matrix (16,384 blocks, P=4), and the oracle's time per
+    block on two of them (one host core)."""
+    N, K, Pv = 64, 2048, 4
+    g = torch.Generator().manual_seed(0x5EED)
+    w = (torch.randn(N, K, generator=g) * 4.0).to(dev)
+    nslm.nslm_seed_search(w[:2], _Encoded(torch, dev, 2, K, Pv, -12), 1, 65535)  # warm-up
+    out = _Encoded(torch, dev, N, K, Pv, -12)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    nslm.nslm_seed_search(w, out, 1, 65535)
+    e1.record()
+    torch.cuda.synchronize()
+    t = e0.elapsed_time(e1) * 1e-3
+    nblk = N * (K // 8)
+    res = {"workload": "seed search of a 64 x 2048 fp32 matrix (16,384 blocks, P=4) over all 65,535 seeds x 16 codes",
+           "gpu_blocks_per_s": round(nblk / t, 1), "gpu_s": round(t, 4),
+           "candidates_per_s": nblk * 65535 * 16 / t}
+    if with_cpu:
+        from oracle import oracle as O
+        wh = w[:1, :16].double().cpu().numpy()
+        t0 = time.time()
+        for b in range(2):
+            O.search_block(wh[0, 8 * b:8 * b + 8], Pv, -12, 1, 65535)
+        cpu = (time.time() - t0) / 2
+        res["oracle_s_per_block_one_core"] = round(cpu, 4)
+        res["gpu_vs_one_core"] = round(cpu * nblk / t, 1)
+    return res
+
+
 def profile_workload(kind: str, reps: int):
     """A small fixed workload for ncu captures (no timing, no JSON): `reps`
     calls of one decode layer (T=1, P=4), of one batched layer (T=512, P=3)
@@ -323,6 +367,7 @@ def main():
     ap.add_argument("--no-gemv", action="store_true")
     ap.add_argument("--no-batched", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--no-search", action="store_true")
     ap.add_argument("--profile", choices=["layer", "batched", "gemv"],
                     help="run a small fixed workload for an ncu capture and exit")
     args = ap.parse_args()
@@ -481,6 +526,10 @@ def main():
         gemv = {"metric": GEMV_METRIC, "shapes": gemv_sweep(torch, nslm, synth, dev, hbm),
                 "note": "batch 1, each shape timed over rotating copies (> 4x L2) in a CUDA graph"}
 
+    search = None
+    if not args.no_search:
+        search = search_leg(torch, nslm, dev, with_cpu=(rank == 0 and not args.no_cpu))
+
     line = {
         "metric": METRIC, "value": round(value, 2), "unit": "tokens/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(elapsed / args.steps * 1e3, 4),
@@ -501,6 +550,8 @@ def main():
         line["gemv"] = gemv
     if batched is not None:
         line["batched"] = batched
+    if search is not None:
+        line["seed_search"] = search
     if rank == 0 and world == 1 and not args.no_cpu:
         line["cpu_baseline"] = cpu_baseline()
     if rank == 0:

@@ -10,9 +10,10 @@
 // pivoting, in fp64.  The smallest error wins; ties go to the larger code,
 // then to the lower seed.
 //
-// A CTA takes two consecutive blocks of a row (they share the P = 4 codes
-// byte); its threads split the seed range, each keeps its best candidate,
-// and a shared-memory tree picks the CTA's best.  The order (error, larger
+// A CTA takes four consecutive blocks of a row (pairs share a P = 4 codes
+// byte) and forms pinv(U) once per seed for all four; its threads split the
+// seed range, each keeps its best candidate per block, and a shared-memory
+// tree picks the CTA's best.  The order (error, larger
 // code, lower seed) is total, so the tree gives the sequential scan's answer
 // whatever the split.  Every fp64 operation of the reference is issued as the
 // same correctly rounded operation (__dmul_rn / __dadd_rn / __dsub_rn,
@@ -112,43 +113,48 @@ struct SearchParams {
   int32_t nb;                // blocks per row
 };
 
+// Blocks searched together by one CTA: pinv(U) depends only on the seed, so
+// it is formed once per seed for all of them (an even count keeps the P = 4
+// code bytes inside one CTA).
+constexpr int kSearchGroup = 4;
+
 template <int P>
 __global__ void __launch_bounds__(kSearchThreads) seed_search_kernel(const SearchParams p) {
   __shared__ StreamTables tab;
   __shared__ Cand s_c[kSearchThreads];
-  __shared__ double s_w[8];
+  __shared__ double s_w[kSearchGroup][8];
   build_stream_tables(&tab);
   const int tid = threadIdx.x;
-  const int64_t pair = blockIdx.x;
-  const int npairs_row = (p.nb + 1) / 2;
-  const int64_t row = pair / npairs_row;
-  const int b0 = (int)(pair - row * npairs_row) * 2;
+  const int groups_row = (p.nb + kSearchGroup - 1) / kSearchGroup;
+  const int64_t row = blockIdx.x / groups_row;
+  const int b0 = (int)(blockIdx.x - row * groups_row) * kSearchGroup;
+  const int nblk = min(kSearchGroup, p.nb - b0);
   const int32_t bias = p.out.exp_bias[row];
-  uint32_t code_byte = 0;
+  if (tid < 8 * nblk) s_w[tid >> 3][tid & 7] = (double)p.w[row * (int64_t)p.nb * 8 + 8 * b0 + tid];
+  __syncthreads();
 
-  for (int h = 0; h < 2 && b0 + h < p.nb; ++h) {
-    const int b = b0 + h;
-    __syncthreads();  // tables; s_w and s_c of the previous block are consumed
-    if (tid < 8) s_w[tid] = (double)p.w[row * (int64_t)p.nb * 8 + 8 * b + tid];
-    __syncthreads();
-    double w[8];
+  Cand best[kSearchGroup];
 #pragma unroll
-    for (int r = 0; r < 8; ++r) w[r] = s_w[r];
-
-    Cand best{INFINITY, -1, -1, 0u};
-    for (int seed = p.seed_lo + tid; seed <= p.seed_hi; seed += kSearchThreads) {
-      // states s_1 .. s_{8P} as windows of the stream word (offsets up to 32:
-      // the clamping funnel shift, which gives hi itself at 32)
-      uint32_t lo, hi;
-      stream_word(&tab, (uint32_t)seed, lo, hi);
-      int32_t u[8][4];
+  for (int g = 0; g < kSearchGroup; ++g) best[g] = Cand{INFINITY, -1, -1, 0u};
+  for (int seed = p.seed_lo + tid; seed <= p.seed_hi; seed += kSearchThreads) {
+    // states s_1 .. s_{8P} as windows of the stream word (offsets up to 32:
+    // the clamping funnel shift, which gives hi itself at 32)
+    uint32_t lo, hi;
+    stream_word(&tab, (uint32_t)seed, lo, hi);
+    int32_t u[8][4];
 #pragma unroll
-      for (int r = 0; r < 8; ++r)
+    for (int r = 0; r < 8; ++r)
 #pragma unroll
-        for (int j = 0; j < 4; ++j)
-          u[r][j] = (j < P) ? (int32_t)(__funnelshift_rc(lo, hi, 1 + 8 * j + r) & 0xFFFFu) - 32768 : 0;
-      double B[4][8];
-      if (!pinv_of<P>(u, B)) continue;
+      for (int j = 0; j < 4; ++j)
+        u[r][j] = (j < P) ? (int32_t)(__funnelshift_rc(lo, hi, 1 + 8 * j + r) & 0xFFFFu) - 32768 : 0;
+    double B[4][8];
+    if (!pinv_of<P>(u, B)) continue;
+#pragma unroll
+    for (int g = 0; g < kSearchGroup; ++g) {
+      if (g >= nblk) break;
+      double w[8];
+#pragma unroll
+      for (int r = 0; r < 8; ++r) w[r] = s_w[g][r];
       double proj[4];
 #pragma unroll
       for (int a = 0; a < P; ++a) {
@@ -157,6 +163,7 @@ __global__ void __launch_bounds__(kSearchThreads) seed_search_kernel(const Searc
         for (int r = 0; r < 8; ++r) s = __dadd_rn(s, __dmul_rn(B[a][r], w[r]));
         proj[a] = s;
       }
+      bool zero_seen = false;
       for (int code = 15; code >= 0; --code) {
         const double inv = pow2(-(code + bias));  // proj / 2^(code+bias), exact
         int32_t c[4];
@@ -167,6 +174,12 @@ __global__ void __launch_bounds__(kSearchThreads) seed_search_kernel(const Searc
           v = fmin(fmax(v, -8.0), 7.0);
           c[a] = (int32_t)v;
           cp |= ((uint32_t)c[a] & 0xFu) << (4 * a);
+        }
+        // all-zero coefficients give the same error for every code; the
+        // first (largest) such code is the only one that can win
+        if (cp == 0u) {
+          if (zero_seen) continue;
+          zero_seen = true;
         }
         // 2^(code+bias) (U c)_r = A_r 2^(code+bias-15), A_r = sum_j u_rj c_j (exact)
         const double sc = pow2(code + bias - 15);
@@ -180,10 +193,17 @@ __global__ void __launch_bounds__(kSearchThreads) seed_search_kernel(const Searc
           err = __dadd_rn(err, __dmul_rn(d, d));
         }
         const Cand cand{err, code, seed, cp};
-        if (better(cand, best)) best = cand;
+        if (better(cand, best[g])) best[g] = cand;
       }
     }
-    s_c[tid] = best;
+  }
+
+  uint32_t code_byte = 0;
+#pragma unroll
+  for (int g = 0; g < kSearchGroup; ++g) {
+    if (g >= nblk) break;
+    __syncthreads();  // s_c of the previous block is consumed
+    s_c[tid] = best[g];
     __syncthreads();
     for (int off = kSearchThreads / 2; off > 0; off >>= 1) {
       if (tid < off && better(s_c[tid + off], s_c[tid])) s_c[tid] = s_c[tid + off];
@@ -191,17 +211,19 @@ __global__ void __launch_bounds__(kSearchThreads) seed_search_kernel(const Searc
     }
     if (tid == 0) {
       const Cand c = s_c[0];
-      const int64_t idx = row * (int64_t)p.nb + b;
+      const int64_t idx = row * (int64_t)p.nb + b0 + g;
       const bool found = c.seed > 0;
       const uint32_t code = found ? (uint32_t)c.code : 0u;
       const_cast<uint16_t *>(p.out.seeds)[idx] = found ? (uint16_t)c.seed : (uint16_t)0;
       const uint32_t q = (found ? c.cpack : 0u) | (P == 3 ? code << 12 : 0u);
       const_cast<uint16_t *>(p.out.coefs)[idx] = (uint16_t)q;
-      code_byte |= code << (4 * h);
+      code_byte |= code << (4 * (g & 1));
       if (p.err) p.err[idx] = found ? c.err : INFINITY;
+      if (P == 4 && (g & 1))
+        const_cast<uint8_t *>(p.out.codes)[row * (int64_t)(p.nb / 2) + (b0 + g) / 2] = (uint8_t)code_byte;
+      if (g & 1) code_byte = 0;
     }
   }
-  if (P == 4 && tid == 0) const_cast<uint8_t *>(p.out.codes)[row * (int64_t)(p.nb / 2) + b0 / 2] = (uint8_t)code_byte;
 }
 
 }  // namespace
@@ -226,7 +248,7 @@ extern "C" int32_t nslm_seed_search(const float *w, const nslm_seed_matrix *out,
   p.seed_lo = seed_lo;
   p.seed_hi = seed_hi;
   p.nb = out->K / 8;
-  const int64_t grid = (int64_t)out->N * ((p.nb + 1) / 2);
+  const int64_t grid = (int64_t)out->N * ((p.nb + kSearchGroup - 1) / kSearchGroup);
   if (grid > 0x7FFFFFFF) return NSLM_ERR_SHAPE;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   if (out->P == 4) seed_search_kernel<4><<<(unsigned)grid, kSearchThreads, 0, s>>>(p);
