@@ -325,13 +325,22 @@ def search_leg(torch, nslm, dev, with_cpu: bool):
 
 def profile_workload(kind: str, reps: int):
     """A small fixed workload for ncu captures (no timing, no JSON): `reps`
-    calls of one decode layer (T=1, P=4), of one batched layer (T=512, P=3)
-    or of one seed GEMV (2048 x 4096, P=4)."""
+    calls of one decode layer (T=1, P=4), of one batched layer (T=512, P=3),
+    of one seed GEMV (2048 x 4096, P=4) or of the seed search of a 16 x 256
+    fp32 matrix over all seeds."""
     import torch
 
     from lfsr_seeded_moe_b200 import nslm, synth
 
     dev = torch.device("cuda", 0)
+    if kind == "search":
+        g = torch.Generator().manual_seed(0x5EED)
+        w = (torch.randn(16, 256, generator=g) * 4.0).to(dev)
+        out = _Encoded(torch, dev, 16, 256, 4, -12)
+        for _ in range(reps):
+            nslm.nslm_seed_search(w, out, 1, 65535)
+        torch.cuda.synchronize()
+        return
     if kind == "gemv":
         m = synth.seed_matrix(2048, 4096, 4, (11, 2048, 4096, 4), device=dev)
         x = synth.activations((11,), 1, 4096).to(dev)
@@ -368,7 +377,7 @@ def main():
     ap.add_argument("--no-batched", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--no-search", action="store_true")
-    ap.add_argument("--profile", choices=["layer", "batched", "gemv"],
+    ap.add_argument("--profile", choices=["layer", "batched", "gemv", "search"],
                     help="run a small fixed workload for an ncu capture and exit")
     args = ap.parse_args()
     if args.profile:
