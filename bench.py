@@ -192,6 +192,23 @@ def run_reference(args):
     return 0
 
 
+def slowest_rank_time(elapsed_s: float, world: int, device) -> float:
+    """The timed region's duration as the maximum over the ranks of the job
+    (one process per GPU; every rank calls this at the same point)."""
+    if world <= 1:
+        return elapsed_s
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([elapsed_s], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(world: int, steps: int, tokens_per_step: int, elapsed_s: float) -> float:
+    """Whole-job tokens/s: every rank decodes its own tokens (replicas)."""
+    return world * steps * tokens_per_step / elapsed_s
+
+
 # ------------------------------------------------------------------- GPU leg
 
 def gemv_sweep(torch, nslm, synth, dev, hbm):
@@ -439,12 +456,8 @@ def main():
         torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
-    elapsed = e0.elapsed_time(e1) * 1e-3
-    if world > 1:
-        t = torch.tensor([elapsed], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        elapsed = float(t.item())
-    value = world * args.steps * T / elapsed
+    elapsed = slowest_rank_time(e0.elapsed_time(e1) * 1e-3, world, dev)
+    value = job_throughput(world, args.steps, T, elapsed)
 
     # --- end to end through the C ABI: pinned host inputs in, result out, every step
     hx = [x.cpu().pin_memory() for x in xs]
@@ -469,12 +482,8 @@ def main():
         hy.copy_(y, non_blocking=True)
     f1.record()
     torch.cuda.synchronize()
-    e2e_t = f0.elapsed_time(f1) * 1e-3
-    if world > 1:
-        t = torch.tensor([e2e_t], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_t = float(t.item())
-    e2e = {"value": world * args.steps * T / e2e_t, "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+    e2e_t = slowest_rank_time(f0.elapsed_time(f1) * 1e-3, world, dev)
+    e2e = {"value": job_throughput(world, args.steps, T, e2e_t), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
            "d2h_bytes_per_step": d2h}
 
     # --- roofline: the per-layer decode FFN (route-plan + gate/up + down launches)

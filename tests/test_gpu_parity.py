@@ -243,3 +243,35 @@ def test_stack_decode_matches_oracle(nslm, T):
     hl = [tuple(getattr(m, n).numpy() for n in ("gate", "up", "down")) for m in layers]
     ref, _ = O.layer_stack(hl, logits.numpy(), xh, hidden, inter, E, k, mode=0)
     assert O.normwise_rel_err(y.cpu().numpy(), ref) <= TOL
+
+
+def test_stack_decode_past_one_launch_per_layer(nslm):
+    # 70 one-token layers run as two persistent launches (64 + 6).  A long
+    # stack is chaotic (one bf16 ulp of a layer input changes everything
+    # downstream), so each checked layer is fed the GPU's own input: the
+    # prefix of l layers gives y_{l-1}, and layer l's output from the prefix
+    # of l+1 layers must match the oracle applied to bf16(y_{l-1} / rms).
+    Lyr, E, hidden, inter, P, k, T = 70, 4, 64, 64, 4, 2, 1
+    layers = [synth.moe_layer(l, E, hidden, inter, P, config=950) for l in range(Lyr)]
+    logits = torch.stack([synth.router_logits((950, l), T, E) for l in range(Lyr)])
+    x, _ = _x((950, T), T, hidden)
+    dl = [(_dev(m.gate), _dev(m.up), _dev(m.down)) for m in layers]
+
+    def prefix(n):
+        y = _out(T, hidden)
+        wsb = nslm.nslm_workspace_bytes(nslm.NSLM_OP_MOE_STACK, T, E, hidden, inter, k, n)
+        ws = torch.zeros(wsb, dtype=torch.uint8, device="cuda")
+        nslm.nslm_moe_stack_decode(dl[:n], n, E, k, logits[:n].cuda().contiguous(), x, T, y, ws, wsb)
+        torch.cuda.synchronize()
+        assert int(ws[:4].view(torch.int32).item()) == 0
+        return y.cpu().numpy().astype(np.float64)
+
+    for l in (63, 64, 69):  # the last layer of launch 1, the first and last of launch 2
+        y_prev, y_l = prefix(l), prefix(l + 1)
+        g, u, d = (getattr(layers[l], n).numpy() for n in ("gate", "up", "down"))
+        xl = O.rms_chain(y_prev)
+        ids, w = O.route_topk(logits[l].numpy(), k)
+        ref = O.moe_ffn(g, u, d, E, hidden, inter, xl, ids, w, mode=0)
+        assert O.normwise_rel_err(y_l, ref) <= TOL, l
+    y70 = prefix(Lyr)
+    assert np.array_equal(y70, prefix(Lyr))  # deterministic run to run
