@@ -108,6 +108,95 @@ static int32_t dispatch_gemv(const GemvParams &p, bool vec, int grid, int thread
   }
 }
 
+// ------------------------------------------------------------- M = 1, whole chunks
+//
+// The single-vector product is latency-bound at expert sizes (1-5 MB of
+// fields, a few microseconds), so this kernel issues its first weight copies
+// before anything else, keeps the next task's fields in flight (cp.async into
+// per-thread shared-memory slots) and has no barrier between tasks.  A CTA
+// owns a range of rows; its threads take (row, chunk) tasks, partial sums go
+// to shared memory and one warp per row adds them in a fixed order.
+
+constexpr int kGemv1Threads = 1024;  // at most; a CTA's (row, chunk) tasks in as few rounds as fit
+
+// n / d for n < 2^22 and 0 < d < 2^16 (m = ceil(2^40 / d); exact, see stack1.cu)
+struct Gemv1Div {
+  uint64_t m;
+};
+__device__ __forceinline__ uint32_t gdiv(uint32_t n, Gemv1Div f) { return (uint32_t)(((uint64_t)n * f.m) >> 40); }
+
+struct Gemv1Params {
+  nslm_seed_matrix W;
+  const uint16_t *x;
+  float *y;
+  int32_t C;     // chunks per row (K / 64)
+  int32_t rpc;   // rows per CTA
+  Gemv1Div div_C;
+};
+
+template <int P>
+__global__ void __launch_bounds__(kGemv1Threads) gemv1_kernel(const Gemv1Params p) {
+  extern __shared__ float4 smem4[];
+  const int tid = threadIdx.x, nthr = blockDim.x, warp = tid >> 5, lane = tid & 31;
+  StreamTables *tab = reinterpret_cast<StreamTables *>(smem4);
+  const FieldSlots fs(smem4 + sizeof(StreamTables) / 16, 2 * nthr);  // [2 buffers][threads]
+  float4 *xs4 = reinterpret_cast<float4 *>(fs.b + 2 * nthr);
+  float2 *xn2 = reinterpret_cast<float2 *>(xs4 + (size_t)kCmX4 * p.C);
+  float *red = reinterpret_cast<float *>(xn2 + (size_t)kCmXn * p.C + (p.C & 1));
+  const int n0 = blockIdx.x * p.rpc;
+  const int nrows = max(0, min(p.rpc, p.W.N - n0));
+  const int ntask = nrows * p.C;
+  const int nb = p.W.K >> 3;
+
+  auto fetch = [&](int t, int buf) {
+    const uint32_t r = gdiv((uint32_t)t, p.div_C), c = (uint32_t)t - r * (uint32_t)p.C;
+    const uint32_t row = (uint32_t)n0 + r;
+    fetch_chunk_off<P>(p.W, row * (uint32_t)nb + 8u * c, row, fs, buf * nthr + tid);
+  };
+  if (tid < ntask) fetch(tid, 0);
+  cp_async_commit();
+  // stream tables and activations: every load in flight before the first store
+  {
+    const uint4 *xrow = reinterpret_cast<const uint4 *>(p.x);
+    uint4 xv = make_uint4(0, 0, 0, 0);
+    if (tid < nb) xv = __ldg(xrow + tid);
+    for (int i = tid; i < 512; i += nthr) tab->t[i] = kStreamTab.t[i];
+    for (int b = tid; b < nb; b += nthr) {
+      if (b != tid) xv = __ldg(xrow + b);
+      float4 lo, hi;
+      bf16x8_to_f32(xv, lo, hi);
+      cm_store_block(xs4, xn2, b, lo, hi);
+    }
+  }
+  __syncthreads();
+
+  for (int t = tid, it = 0; t < ntask; t += nthr, ++it) {
+    const uint32_t c = (uint32_t)t - gdiv((uint32_t)t, p.div_C) * (uint32_t)p.C;
+    if (t + nthr < ntask) fetch(t + nthr, (it + 1) & 1);
+    cp_async_commit();
+    cp_async_wait<1>();
+    ChunkFields f;
+    uint32_t rowk;
+    read_chunk<P>(fs, (it & 1) * nthr + tid, f, rowk);
+    float2 acc = make_float2(0.f, 0.f);
+    chunk_dot_cm<P, true, 1>(tab->t, f, 8, rowk, xs4 + kCmX4 * c, xn2 + kCmXn * c, acc);
+    red[t] = acc.x + acc.y;
+  }
+  cp_async_wait<0>();
+  __syncthreads();
+  for (int r = warp; r < nrows; r += nthr >> 5) {
+    float sum = 0.f;
+    for (int q = lane; q < p.C; q += 32) sum += red[r * p.C + q];
+    sum = warp_sum(sum);
+    if (lane == 0) p.y[n0 + r] = sum;
+  }
+}
+
+static size_t gemv1_smem(int C, int rpc, int threads) {
+  return sizeof(StreamTables) + FieldSlots::bytes(2 * threads) + cm_bytes(C) + 16 +
+         (size_t)rpc * C * sizeof(float);
+}
+
 }  // namespace nslm
 
 using namespace nslm;
@@ -126,6 +215,31 @@ extern "C" int32_t nslm_seed_gemv(const nslm_seed_matrix *W, const uint16_t *x_b
   if ((st = check_device())) return st;
   if (W->N == 0) return NSLM_OK;
 
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  // one vector, whole 64-weight chunks: the latency-oriented kernel
+  if (M == 1 && W->K % 64 == 0 && (int64_t)W->N * (W->K / 8) < (1ll << 31) && W->K / 64 < (1 << 16)) {
+    const int sms = num_sms();
+    Gemv1Params q{};
+    q.W = *W;
+    q.x = x_bf16;
+    q.y = y;
+    q.C = W->K / 64;
+    q.rpc = std::max(1, ceil_div(W->N, sms));
+    q.div_C = Gemv1Div{((1ull << 40) + (uint64_t)q.C - 1) / (uint64_t)q.C};
+    const int tasks = q.rpc * q.C;
+    const int rounds = ceil_div(tasks, kGemv1Threads);
+    const int threads = std::max(64, 32 * ceil_div(ceil_div(tasks, rounds), 32));
+    const size_t smem = gemv1_smem(q.C, q.rpc, threads);
+    if (smem <= 200 * 1024 && (int64_t)q.rpc * q.C < (1 << 22)) {
+      auto k = (W->P == 4) ? gemv1_kernel<4> : gemv1_kernel<3>;
+      if ((st = ensure_smem((const void *)k, smem))) return st;
+      k<<<ceil_div(W->N, q.rpc), threads, smem, s>>>(q);
+      st = launch_status();
+      if (st == NSLM_OK) g_launches = 1;
+      return st;
+    }
+  }
+
   GemvParams p{};
   p.seeds = W->seeds; p.coefs = W->coefs; p.codes = W->codes; p.exp_bias = W->exp_bias;
   p.x = x_bf16; p.y = y; p.N = W->N; p.K = W->K; p.nb = W->K / 8; p.M = M;
@@ -138,7 +252,6 @@ extern "C" int32_t nslm_seed_gemv(const nslm_seed_matrix *W, const uint16_t *x_b
   if (smem > 227 * 1024) return NSLM_ERR_SHAPE;
   const int per_sm = std::max(1, std::min(2048 / L.threads, (int)((227 * 1024) / smem)));
   const int grid = std::min(p.groups, per_sm * sms);
-  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   st = (W->P == 4) ? dispatch_gemv<4>(p, vec, grid, L.threads, smem, s)
                    : dispatch_gemv<3>(p, vec, grid, L.threads, smem, s);
   if (st == NSLM_OK) g_launches = 1;

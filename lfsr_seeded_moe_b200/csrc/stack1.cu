@@ -169,7 +169,9 @@ __global__ void __launch_bounds__(kStack1MaxThreads, 1) stack1_kernel(const __gr
   if (tid == 0) s_row0 = 0;
 
   const int nbh = p.hidden >> 3, nbi = p.inter >> 3;
-  const int gw = blockIdx.x * nwarps + warp, W = gridDim.x * nwarps;
+  // phase A warp number: consecutive tasks go to different CTAs, so every SM
+  // receives the same number of routed rows (to within one)
+  const int gw = warp * gridDim.x + blockIdx.x, W = gridDim.x * nwarps;
   const int n0 = blockIdx.x * p.rpc;
   const int nrows = max(0, min(p.rpc, p.hidden - n0));
 
