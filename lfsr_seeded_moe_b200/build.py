@@ -1,9 +1,14 @@
 """Build libnslm.so (the CUDA library) in-tree for sm_100a with nvcc.
 
-    python -m lfsr_seeded_moe_b200.build [--force]
+    python -m lfsr_seeded_moe_b200.build [--force] [--stream-source l2next|l2basis]
 
 The shared library lands in lfsr_seeded_moe_b200/_build/libnslm.so; it is
 rebuilt when any source under csrc/ or include/ is newer than it.
+--stream-source builds an ablation library instead, in _build/<source>/, whose
+decode kernels take a block's stream bits from an L2-resident 65,536-entry
+table (l2next: the 32 bits after each seed; l2basis: the 16 shifted words of
+each seed) in place of the shared-memory GF(2) tables; the binding loads it
+when NSLM_STREAM_SOURCE names it.
 """
 from __future__ import annotations
 
@@ -33,21 +38,33 @@ def _inputs():
     return sources() + glob.glob(os.path.join(CSRC, "*.cuh")) + glob.glob(os.path.join(ROOT, "include", "*.h"))
 
 
-def up_to_date() -> bool:
-    if not os.path.exists(LIB):
+STREAM_SOURCES = {"l2next": 1, "l2basis": 2}
+
+
+def lib_path(stream_source: str | None = None) -> str:
+    return os.path.join(OUT_DIR, stream_source, "libnslm.so") if stream_source else LIB
+
+
+def up_to_date(stream_source: str | None = None) -> bool:
+    lib = lib_path(stream_source)
+    if not os.path.exists(lib):
         return False
-    t = os.path.getmtime(LIB)
+    t = os.path.getmtime(lib)
     return all(os.path.getmtime(p) <= t for p in _inputs())
 
 
-def build(force: bool = False, verbose: bool = False, extra_flags=None) -> str:
-    if not force and up_to_date():
-        return LIB
-    os.makedirs(OUT_DIR, exist_ok=True)
+def build(force: bool = False, verbose: bool = False, extra_flags=None,
+          stream_source: str | None = None) -> str:
+    lib = lib_path(stream_source)
+    if not force and up_to_date(stream_source):
+        return lib
+    out_dir = os.path.dirname(lib)
+    os.makedirs(out_dir, exist_ok=True)
+    defs = [f"-DNSLM_STREAM_SOURCE={STREAM_SOURCES[stream_source]}"] if stream_source else []
     jobs = []
     for src in sources():
-        obj = os.path.join(OUT_DIR, os.path.basename(src)[:-3] + ".o")
-        cmd = [NVCC, *ARCH, *FLAGS, *(extra_flags or []), "-I", os.path.join(ROOT, "include"),
+        obj = os.path.join(out_dir, os.path.basename(src)[:-3] + ".o")
+        cmd = [NVCC, *ARCH, *FLAGS, *defs, *(extra_flags or []), "-I", os.path.join(ROOT, "include"),
                "-c", src, "-o", obj]
         if verbose:
             print(" ".join(cmd), file=sys.stderr)
@@ -59,15 +76,18 @@ def build(force: bool = False, verbose: bool = False, extra_flags=None) -> str:
                 print(r.stdout + r.stderr, file=sys.stderr, end="")
             r.check_returncode()
     objs = [o for _, o in jobs]
-    tmp = LIB + f".tmp{os.getpid()}"
+    tmp = lib + f".tmp{os.getpid()}"
     cmd = [NVCC, *ARCH, "-shared", "-o", tmp, *objs]  # static cudart (nvcc default)
     if verbose:
         print(" ".join(cmd), file=sys.stderr)
     subprocess.run(cmd, check=True)
-    os.replace(tmp, LIB)
-    return LIB
+    os.replace(tmp, lib)
+    return lib
 
 
 if __name__ == "__main__":
-    print(build(force="--force" in sys.argv, verbose=True,
+    src = sys.argv[sys.argv.index("--stream-source") + 1] if "--stream-source" in sys.argv else None
+    if src is not None and src not in STREAM_SOURCES:
+        raise SystemExit(f"--stream-source must be one of {sorted(STREAM_SOURCES)}")
+    print(build(force="--force" in sys.argv, verbose=True, stream_source=src,
                 extra_flags=["-Xptxas", "-v"] if "--ptxas-v" in sys.argv else None))

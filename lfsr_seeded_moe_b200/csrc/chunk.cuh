@@ -232,6 +232,28 @@ __device__ __forceinline__ void block_magic(uint32_t v, uint32_t nxt, uint32_t c
   }
 }
 
+#if NSLM_STREAM_SOURCE != 0
+// block_magic from the L2-resident table of the ablation builds.
+__device__ __forceinline__ void block_magic_src(uint32_t seed, uint32_t cp2, float (&G)[8]) {
+  const int32_t base = (int32_t)kMagic2Bits - 32768 * dp4a_ss(cp2, 0x01010101u, 0);
+#if NSLM_STREAM_SOURCE == 1
+  const uint32_t nxt = __ldg(reinterpret_cast<const uint32_t *>(g_stream_src) + seed);
+  const uint32_t v = seed << 16;
+#pragma unroll
+  for (int r = 0; r < 8; ++r) {
+    const uint32_t z = (r == 7) ? nxt : __funnelshift_r(v, nxt, 25 + r);
+    G[r] = __int_as_float(dp2a_hi_us(z, cp2, dp2a_lo_us(__funnelshift_r(v, nxt, 17 + r), cp2, base)));
+  }
+#else
+  const uint4 *e = g_stream_src + 4 * seed;  // W >> 1 .. W >> 16
+  const uint4 a = __ldg(e), b = __ldg(e + 1), c = __ldg(e + 2), d = __ldg(e + 3);
+  const uint32_t z[16] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w, c.x, c.y, c.z, c.w, d.x, d.y, d.z, d.w};
+#pragma unroll
+  for (int r = 0; r < 8; ++r) G[r] = __int_as_float(dp2a_hi_us(z[8 + r], cp2, dp2a_lo_us(z[r], cp2, base)));
+#endif
+}
+#endif
+
 // Regenerate block i (0..7) of a loaded chunk: G[r] = Mg + A_r (exact fp32);
 // returns the block's power-of-two scale 2^(code + bias - 15).
 template <int P>
@@ -239,10 +261,14 @@ __device__ __forceinline__ float regen_chunk_block(const StreamTables *tab, cons
                                                    int i, uint32_t rowk, float (&G)[8]) {
   const uint32_t sw = f.s[i >> 1], qw = f.q[i >> 1];
   const uint32_t q = (i & 1) ? (qw >> 16) : (qw & 0xFFFFu);
+#if NSLM_STREAM_SOURCE == 0
   uint32_t v, nxt;
   if (i & 1) stream_pair_of<1>(tab, sw, v, nxt);
   else stream_pair_of<0>(tab, sw, v, nxt);
   block_magic(v, nxt, coef_pairs2<P>(q), G);
+#else
+  block_magic_src((i & 1) ? (sw >> 16) : (sw & 0xFFFFu), coef_pairs2<P>(q), G);
+#endif
   const uint32_t code = (P == 4) ? ((f.codes >> (4 * i)) & 0xFu) : (q >> 12);
   return block_scale(code, rowk);
 }
@@ -255,11 +281,15 @@ __device__ __forceinline__ float regen_chunk_block_r(const uint32_t *tl, const C
                                                      uint32_t rowk, float (&G)[8]) {
   const uint32_t sw = f.s[i >> 1], qw = f.q[i >> 1];
   const uint32_t q = (i & 1) ? (qw >> 16) : (qw & 0xFFFFu);
+#if NSLM_STREAM_SOURCE == 0
   const uint32_t b0 = (i & 1) ? ((sw >> 16) & 0xFFu) : (sw & 0xFFu);
   const uint32_t b1 = (i & 1) ? (sw >> 24) : ((sw >> 8) & 0xFFu);
   const uint32_t nxt = tl[R * b0] ^ tl[R * (256u + b1)];
   const uint32_t v = (i & 1) ? (sw & 0xFFFF0000u) : (sw << 16);
   block_magic(v, nxt, coef_pairs2<P>(q), G);
+#else
+  block_magic_src((i & 1) ? (sw >> 16) : (sw & 0xFFFFu), coef_pairs2<P>(q), G);
+#endif
   const uint32_t code = (P == 4) ? ((f.codes >> (4 * i)) & 0xFu) : (q >> 12);
   return block_scale(code, rowk);
 }

@@ -73,6 +73,7 @@ static int32_t launch_gemv(const GemvParams &p, int grid, int threads, size_t sm
                            cudaStream_t s) {
   auto k = seed_gemv_kernel<P, M, VEC, CPAD>;
   if (int32_t st = ensure_smem((const void *)k, smem)) return st;
+  ensure_stream_source(s);
   k<<<grid, threads, smem, s>>>(p);
   return launch_status();
 }
@@ -233,6 +234,7 @@ extern "C" int32_t nslm_seed_gemv(const nslm_seed_matrix *W, const uint16_t *x_b
     if (smem <= 200 * 1024 && (int64_t)q.rpc * q.C < (1 << 22)) {
       auto k = (W->P == 4) ? gemv1_kernel<4> : gemv1_kernel<3>;
       if ((st = ensure_smem((const void *)k, smem))) return st;
+      ensure_stream_source(s);
       k<<<ceil_div(W->N, q.rpc), threads, smem, s>>>(q);
       st = launch_status();
       if (st == NSLM_OK) g_launches = 1;

@@ -448,6 +448,7 @@ template <typename Kern, typename Params>
 static int32_t launch_k(Kern kern, const Params &p, int grid, int threads, size_t smem,
                         cudaStream_t s) {
   if (int32_t st = ensure_smem((const void *)kern, smem)) return st;
+  ensure_stream_source(s);
   kern<<<grid, threads, smem, s>>>(p);
   return launch_status();
 }

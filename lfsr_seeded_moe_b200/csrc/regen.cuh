@@ -69,6 +69,52 @@ struct StreamTableInit {
 };
 static __device__ const StreamTableInit kStreamTab{};
 
+// ------------------------------------------------- stream source (ablation)
+//
+// NSLM_STREAM_SOURCE selects where the chunk regenerators of the decode
+// kernels take a block's stream bits from:
+//   0 (the library): the two 256-entry GF(2) tables above, in shared memory;
+//   1: one 32-bit word per seed, the bits that follow it (65,536 entries,
+//      256 KB, L2-resident), one 4-byte global load per block -- the table
+//      of "NanoSeedLM: LLM inference using pseudo-random numbers", "'LFSR is
+//      free'";
+//   2: a 65,536-entry basis table holding per seed the 16 words W >> t,
+//      t = 1..16, that the two-way dot products consume (64 B per seed, 4 MB,
+//      L2-resident): four 16-byte global loads per block and no shifts.
+// 1 and 2 are built only as separate libraries, to measure those designs
+// against the tables kept here; results are identical in all three.
+#ifndef NSLM_STREAM_SOURCE
+#define NSLM_STREAM_SOURCE 0
+#endif
+
+#if NSLM_STREAM_SOURCE != 0
+static __device__ uint4 g_stream_src[NSLM_STREAM_SOURCE == 1 ? 65536 / 4 : 65536 * 4];
+
+static __global__ void fill_stream_src_kernel() {
+  const uint32_t s = blockIdx.x * blockDim.x + threadIdx.x;  // seed 0..65535
+  const uint32_t nxt = kStreamTab.t[s & 0xFFu] ^ kStreamTab.t[256u + (s >> 8)];
+  if (NSLM_STREAM_SOURCE == 1) {
+    reinterpret_cast<uint32_t *>(g_stream_src)[s] = nxt;
+  } else {
+    uint32_t z[16];
+    for (int t = 1; t < 16; ++t) z[t - 1] = __funnelshift_r(s << 16, nxt, 16 + t);
+    z[15] = nxt;
+    for (int k = 0; k < 4; ++k) g_stream_src[4 * s + k] = make_uint4(z[4 * k], z[4 * k + 1], z[4 * k + 2], z[4 * k + 3]);
+  }
+}
+
+// Fill this translation unit's table before its first launch.
+static inline void ensure_stream_source(cudaStream_t s) {
+  static bool done = false;
+  if (!done) {
+    fill_stream_src_kernel<<<256, 256, 0, s>>>();
+    done = true;
+  }
+}
+#else
+static inline void ensure_stream_source(cudaStream_t) {}
+#endif
+
 // Copy the tables into shared memory with all threads of the CTA (the caller
 // synchronises afterwards).
 __device__ __forceinline__ void build_stream_tables(StreamTables *tab) {

@@ -476,6 +476,7 @@ static int32_t launch_stack1_t(const FfnDims &d, const nslm_moe_layer *layers, i
     attr[0].val.cooperative = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
+    ensure_stream_source(s);
     if ((st = cuda_status(cudaLaunchKernelEx(&cfg, kern, p)))) return st;
     ++launches;
     base += (uint32_t)(2 * m - 1) * (uint32_t)grid;

@@ -13,7 +13,11 @@ import os
 import re
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_HERE, "_build", "libnslm.so")
+# NSLM_STREAM_SOURCE=l2next or l2basis loads an ablation build of the library
+# (`python -m lfsr_seeded_moe_b200.build --stream-source l2next`), whose
+# decode kernels read the stream bits from an L2-resident 65,536-entry table
+_SOURCE = os.environ.get("NSLM_STREAM_SOURCE", "")
+LIB_PATH = os.path.join(_HERE, "_build", *([_SOURCE] if _SOURCE else []), "libnslm.so")
 HEADER_PATH = os.path.join(os.path.dirname(_HERE), "include", "nslm.h")
 
 NSLM_OK = 0
