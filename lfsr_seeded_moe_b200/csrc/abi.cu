@@ -9,6 +9,7 @@
 #include "grouped.cuh"
 #include "moe.cuh"
 #include "stack1.cuh"
+#include "stackb.cuh"
 
 namespace nslm {
 
@@ -255,7 +256,7 @@ int32_t nslm_moe_route_topk(const float *logits, int32_t T, int32_t E, int32_t k
   for (int t0 = 0; t0 < T; t0 += kMaxT) {
     const int tn = std::min(kMaxT, T - t0);
     st = launch_route_plan(logits + (size_t)t0 * E, nullptr, nullptr, tn, E, k, 1, nullptr,
-                           ids + (size_t)t0 * k, w + (size_t)t0 * k, nullptr, 0, nullptr, s);
+                           ids + (size_t)t0 * k, w + (size_t)t0 * k, nullptr, 0, nullptr, tn, s);
     if (st) return st;
     ++g_launches;
   }
@@ -288,15 +289,11 @@ int32_t nslm_moe_seed_ffn(const nslm_seed_matrix *gate, const nslm_seed_matrix *
   }
   const FfnWorkspace fw = ffn_workspace(reinterpret_cast<char *>(ws), T, k, d.hidden, d.inter, 1);
   if ((st = launch_route_plan(nullptr, ids, w, T, E, k, 1, fw.plans, nullptr, nullptr, fw.counters,
-                              d.hidden, fw.sync, s)))
+                              d.hidden, fw.sync, decode_slot_cap(d, T, k), s)))
     return st;
   int launches = 1;
-  if (T == 1 && stack1_supported(d, k)) {
-    const nslm_moe_layer layer{*gate, *up, *down};
-    st = launch_stack1(d, &layer, 1, fw.plans, x_bf16, nullptr, k, fw.h, fw.y_mid, y, fw.sync, fw.rms_part, s, launches);
-  } else {
-    st = launch_decode_layer(d, gate, up, down, fw.plans, x_bf16, nullptr, T, k, fw, y, s, launches);
-  }
+  const nslm_moe_layer layer{*gate, *up, *down};
+  st = launch_decode_stack(d, &layer, 1, x_bf16, T, k, fw, y, s, launches);
   if (st == NSLM_OK) g_launches = launches;
   return st;
 }
@@ -323,24 +320,12 @@ int32_t nslm_moe_stack_decode(const nslm_moe_layer *layers, int32_t L, int32_t E
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   const FfnWorkspace fw = ffn_workspace(reinterpret_cast<char *>(ws), T, k, d.hidden, d.inter, L);
   if ((st = launch_route_plan(logits, nullptr, nullptr, T, E, k, L, fw.plans, nullptr, nullptr,
-                              fw.counters, d.hidden, fw.sync, s)))
+                              fw.counters, d.hidden, fw.sync, decode_slot_cap(d, T, k), s)))
     return st;
   int launches = 1;
-  if (T == 1 && stack1_supported(d, k)) {
-    st = launch_stack1(d, layers, L, fw.plans, x0_bf16, nullptr, k, fw.h, fw.y_mid, y, fw.sync, fw.rms_part, s, launches);
-    if (st == NSLM_OK) g_launches = launches;
-    return st;
-  }
-  for (int l = 0; l < L; ++l) {
-    const uint16_t *xin = (l == 0) ? x0_bf16 : nullptr;
-    const float *yprev = (l == 0) ? nullptr : fw.y_mid;
-    float *yout = (l == L - 1) ? y : fw.y_mid;
-    st = launch_decode_layer(d, &layers[l].gate, &layers[l].up, &layers[l].down, fw.plans + l, xin,
-                             yprev, T, k, fw, yout, s, launches);
-    if (st) return st;
-  }
-  g_launches = launches;
-  return NSLM_OK;
+  st = launch_decode_stack(d, layers, L, x0_bf16, T, k, fw, y, s, launches);
+  if (st == NSLM_OK) g_launches = launches;
+  return st;
 }
 
 }  // extern "C"

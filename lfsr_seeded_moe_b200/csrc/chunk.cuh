@@ -406,6 +406,54 @@ __device__ __forceinline__ void chunk_dot2_cm(const uint32_t *tl, const ChunkFie
   }
 }
 
+// The same for up to MT vectors that share the regenerated weights: vector m
+// (m < M) has its chunk slot at xa + kCmX4 * off[m], xn + kCmXn * off[m].
+// A vector past M is skipped (M is the same for all lanes of a warp in the
+// gate/up phase, and nearly always so in the down phase).
+template <int P, bool VEC, int R, int MT>
+__device__ __forceinline__ void chunk_dot_cm_multi(const uint32_t *tl, const ChunkFields &f, int nvalid,
+                                                   uint32_t rowk, const float4 *xa, const float2 *xn,
+                                                   const int (&off)[MT], int M, float2 (&acc)[MT]) {
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    if (!VEC && i >= nvalid) break;
+    float G[8];
+    const float s = regen_chunk_block_r<P, R>(tl, f, i, rowk, G);
+#pragma unroll
+    for (int m = 0; m < MT; ++m) {
+      if (m < M) {
+        const float4 *x = xa + kCmX4 * off[m];
+        block_fma(G, s, x[2 * i], x[2 * i + 1], xn[kCmXn * off[m] + i], acc[m]);
+      }
+    }
+  }
+}
+
+template <int P, bool VEC, int R, int MT>
+__device__ __forceinline__ void chunk_dot2_cm_multi(const uint32_t *tl, const ChunkFields &fa,
+                                                    const ChunkFields &fb, int nvalid, uint32_t rowka,
+                                                    uint32_t rowkb, const float4 *xa, const float2 *xn,
+                                                    const int (&off)[MT], int M, float2 (&acca)[MT],
+                                                    float2 (&accb)[MT]) {
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    if (!VEC && i >= nvalid) break;
+    float Ga[8], Gb[8];
+    const float sa = regen_chunk_block_r<P, R>(tl, fa, i, rowka, Ga);
+    const float sb = regen_chunk_block_r<P, R>(tl, fb, i, rowkb, Gb);
+#pragma unroll
+    for (int m = 0; m < MT; ++m) {
+      if (m < M) {
+        const float4 *x = xa + kCmX4 * off[m];
+        const float4 x0 = x[2 * i], x1 = x[2 * i + 1];
+        const float2 x2 = xn[kCmXn * off[m] + i];
+        block_fma(Ga, sa, x0, x1, x2, acca[m]);
+        block_fma(Gb, sb, x0, x1, x2, accb[m]);
+      }
+    }
+  }
+}
+
 // Sum of a float over the 32 lanes of a warp (fixed order: deterministic).
 __device__ __forceinline__ float warp_sum(float v) {
 #pragma unroll

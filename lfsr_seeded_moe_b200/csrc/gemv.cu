@@ -11,6 +11,7 @@
 
 #include "chunk.cuh"
 #include "common.cuh"
+#include "persist.cuh"
 
 namespace nslm {
 
@@ -120,19 +121,13 @@ static int32_t dispatch_gemv(const GemvParams &p, bool vec, int grid, int thread
 
 constexpr int kGemv1Threads = 1024;  // at most; a CTA's (row, chunk) tasks in as few rounds as fit
 
-// n / d for n < 2^22 and 0 < d < 2^16 (m = ceil(2^40 / d); exact, see stack1.cu)
-struct Gemv1Div {
-  uint64_t m;
-};
-__device__ __forceinline__ uint32_t gdiv(uint32_t n, Gemv1Div f) { return (uint32_t)(((uint64_t)n * f.m) >> 40); }
-
 struct Gemv1Params {
   nslm_seed_matrix W;
   const uint16_t *x;
   float *y;
   int32_t C;     // chunks per row (K / 64)
   int32_t rpc;   // rows per CTA
-  Gemv1Div div_C;
+  FastDiv div_C;
 };
 
 template <int P>
@@ -150,7 +145,7 @@ __global__ void __launch_bounds__(kGemv1Threads) gemv1_kernel(const Gemv1Params 
   const int nb = p.W.K >> 3;
 
   auto fetch = [&](int t, int buf) {
-    const uint32_t r = gdiv((uint32_t)t, p.div_C), c = (uint32_t)t - r * (uint32_t)p.C;
+    const uint32_t r = fdiv((uint32_t)t, p.div_C), c = (uint32_t)t - r * (uint32_t)p.C;
     const uint32_t row = (uint32_t)n0 + r;
     fetch_chunk_off<P>(p.W, row * (uint32_t)nb + 8u * c, row, fs, buf * nthr + tid);
   };
@@ -172,7 +167,7 @@ __global__ void __launch_bounds__(kGemv1Threads) gemv1_kernel(const Gemv1Params 
   __syncthreads();
 
   for (int t = tid, it = 0; t < ntask; t += nthr, ++it) {
-    const uint32_t c = (uint32_t)t - gdiv((uint32_t)t, p.div_C) * (uint32_t)p.C;
+    const uint32_t c = (uint32_t)t - fdiv((uint32_t)t, p.div_C) * (uint32_t)p.C;
     if (t + nthr < ntask) fetch(t + nthr, (it + 1) & 1);
     cp_async_commit();
     cp_async_wait<1>();
@@ -226,7 +221,7 @@ extern "C" int32_t nslm_seed_gemv(const nslm_seed_matrix *W, const uint16_t *x_b
     q.y = y;
     q.C = W->K / 64;
     q.rpc = std::max(1, ceil_div(W->N, sms));
-    q.div_C = Gemv1Div{((1ull << 40) + (uint64_t)q.C - 1) / (uint64_t)q.C};
+    q.div_C = make_fastdiv((uint32_t)q.C);
     const int tasks = q.rpc * q.C;
     const int rounds = ceil_div(tasks, kGemv1Threads);
     const int threads = std::max(64, 32 * ceil_div(ceil_div(tasks, rounds), 32));

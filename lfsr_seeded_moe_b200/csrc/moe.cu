@@ -77,7 +77,7 @@ __global__ void __launch_bounds__(256) route_plan_kernel(const float *__restrict
                                                          int E, int k, SlotPlan *plans,
                                                          int32_t *ids_out, float *w_out,
                                                          int32_t *counters, int n_counters,
-                                                         int32_t *sync) {
+                                                         int32_t *sync, int slot_cap) {
   const int layer = blockIdx.x;
   if (counters && layer == 0)
     for (int i = threadIdx.x; i < n_counters; i += blockDim.x) counters[i] = 0;
@@ -116,11 +116,11 @@ __global__ void __launch_bounds__(256) route_plan_kernel(const float *__restrict
       while (j > 0 && s_ids[order[j - 1]] > s_ids[i]) { order[j] = order[j - 1]; --j; }
       order[j] = i;
     }
-    // a new slot starts at a new expert, or after T pairs of the same expert
-    // (only possible if a token lists an expert twice)
+    // a new slot starts at a new expert, or after slot_cap pairs of the same
+    // expert (slot_cap <= T: more only if a token lists an expert twice)
     int ns = 0, in_slot = 0;
     for (int i = 0; i < cnt; ++i) {
-      if (i == 0 || s_ids[order[i]] != s_ids[order[i - 1]] || in_slot == T) {
+      if (i == 0 || s_ids[order[i]] != s_ids[order[i - 1]] || in_slot == slot_cap) {
         pl.expert[ns] = s_ids[order[i]];
         pl.start[ns] = i;
         ++ns;
@@ -429,7 +429,7 @@ FfnWorkspace ffn_workspace(char *base, int T, int k, int hidden, int inter, int 
   w.sync = reinterpret_cast<int32_t *>(base ? base + off : nullptr);
   off += 256;
   w.rms_part = reinterpret_cast<float *>(base ? base + off : nullptr);
-  off += round256(kMaxNormParts * sizeof(float));
+  off += round256((size_t)T * kMaxNormParts * sizeof(float));
   w.plans = reinterpret_cast<SlotPlan *>(base ? base + off : nullptr);
   off += round256((size_t)std::max(L, 1) * kPlanBytes);
   w.counters = reinterpret_cast<int32_t *>(base ? base + off : nullptr);
@@ -520,9 +520,9 @@ int32_t launch_decode_layer(const FfnDims &d, const nslm_seed_matrix *gate,
 
 int32_t launch_route_plan(const float *logits, const int32_t *ids, const float *w, int T, int E,
                           int k, int L, SlotPlan *plans, int32_t *ids_out, float *w_out,
-                          int32_t *counters, int n_counters, int32_t *sync, cudaStream_t s) {
+                          int32_t *counters, int n_counters, int32_t *sync, int slot_cap, cudaStream_t s) {
   route_plan_kernel<<<L, 256, 0, s>>>(logits, ids, w, T, E, k, plans, ids_out, w_out, counters,
-                                      n_counters, sync);
+                                      n_counters, sync, std::max(1, std::min(slot_cap, T)));
   return launch_status();
 }
 

@@ -14,7 +14,8 @@ constexpr int kMaxK = 8;                 // at most 8 experts per token
 constexpr int kMaxPairs = kMaxT * kMaxK;
 
 // One layer's routing grouped by expert.  A slot is one expert together with
-// the (token, slot-in-token) pairs routed to it, at most T pairs per slot.
+// the (token, slot-in-token) pairs routed to it, at most slot_cap <= T pairs
+// per slot (an expert with more pairs takes several slots).
 struct SlotPlan {
   int32_t n_slots;
   int32_t n_pairs;
@@ -45,7 +46,7 @@ constexpr int kMaxNormParts = 1024;
 
 struct FfnWorkspace {
   int32_t *sync;       // [kSyncWords], at offset 0
-  float *rms_part;     // [kMaxNormParts] per-CTA sums of y^2 between fused layers
+  float *rms_part;     // [T][kMaxNormParts] per-token, per-CTA sums of y^2 between fused layers
   SlotPlan *plans;     // [L]
   int32_t *counters;   // [hidden]
   float *h;            // [T*k][inter]
@@ -57,7 +58,7 @@ FfnWorkspace ffn_workspace(char *base, int T, int k, int hidden, int inter, int 
 
 int32_t launch_route_plan(const float *logits, const int32_t *ids, const float *w, int T, int E,
                           int k, int L, SlotPlan *plans, int32_t *ids_out, float *w_out,
-                          int32_t *counters, int n_counters, int32_t *sync, cudaStream_t s);
+                          int32_t *counters, int n_counters, int32_t *sync, int slot_cap, cudaStream_t s);
 int32_t launch_decode_layer(const FfnDims &d, const nslm_seed_matrix *gate,
                             const nslm_seed_matrix *up, const nslm_seed_matrix *down,
                             const SlotPlan *plan, const uint16_t *x_bf16, const float *y_prev,

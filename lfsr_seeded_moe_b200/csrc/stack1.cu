@@ -28,23 +28,13 @@
 
 #include "chunk.cuh"
 #include "common.cuh"
+#include "persist.cuh"
 #include "stack1.cuh"
 
 namespace nslm {
 
 namespace {
 
-// n / d for n < 2^22 and 0 < d < 2^16: m = ceil(2^40 / d), q = (n * m) >> 40
-// (exact, since n * (m * d - 2^40) < 2^38 < 2^40).
-struct FastDiv {
-  uint64_t m;
-};
-FastDiv make_fastdiv(uint32_t d) { return FastDiv{((1ull << 40) + d - 1) / d}; }
-__device__ __forceinline__ uint32_t fdiv(uint32_t n, FastDiv f) {
-  return (uint32_t)(((uint64_t)n * f.m) >> 40);
-}
-
-constexpr long long kBarrierWaitCycles = 2000000000ll;  // ~1 s at 1.9 GHz
 constexpr int kTabCopies = 1;  // interleaved stream-table copies (bank conflicts / kTabCopies)
 
 struct LayerMats {
@@ -71,47 +61,8 @@ struct Stack1Params {
   LayerMats layer[kMaxFusedLayers];
 };
 
-__device__ __forceinline__ uint32_t ld_acquire(const int32_t *p) {
-  uint32_t v;
-  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
-  return v;
-}
-
-// Grid-wide barrier number e of this call, in two halves so that work which
-// does not depend on other CTAs (the next phase's weight prefetch) runs
-// between them.  Arrival: block barrier, then a release reduction by thread 0
-// (it orders the CTA's writes, gathered by the block barrier, before it).
-// Wait: thread 0 polls with acquire loads, bounded; false when aborting.
-__device__ __forceinline__ void grid_arrive(const Stack1Params &p) {
-  __syncthreads();
-  if (threadIdx.x == 0) asm volatile("red.release.gpu.global.add.u32 [%0], 1;" ::"l"(p.sync + 1) : "memory");
-}
-
-__device__ bool grid_wait(const Stack1Params &p, uint32_t e, int *s_ok) {
-  if (threadIdx.x == 0) {
-    int ok = 1;
-    const uint32_t target = p.barrier_base + (e + 1) * gridDim.x;
-    if (ld_acquire(p.sync + 1) < target) {
-      const long long t0 = clock64();
-      for (uint32_t it = 1; ld_acquire(p.sync + 1) < target; ++it) {
-        if ((it & 63) == 0) {
-          if (ld_acquire(p.sync + 2) != 0) {
-            ok = 0;
-            break;
-          }
-          if (clock64() - t0 > kBarrierWaitCycles) {
-            atomicExch(p.sync + 2, 1);
-            atomicCAS(p.sync, 0, 1);
-            ok = 0;
-            break;
-          }
-        }
-      }
-    }
-    *s_ok = ok;
-  }
-  __syncthreads();
-  return *s_ok != 0;
+__device__ __forceinline__ bool stack_wait(const Stack1Params &p, uint32_t e, int *s_ok) {
+  return grid_wait(p.sync, p.barrier_base + (e + 1) * gridDim.x, s_ok);
 }
 
 // Stage x = bf16(y / sqrt(mean(y^2) + 1e-6)) chunk-major.  The sum of squares
@@ -293,11 +244,11 @@ __global__ void __launch_bounds__(kStack1MaxThreads, 1) stack1_kernel(const __gr
     // arrive; fetch phase B's first fields (weights only) while the others arrive
     const int SC = s_nslots * p.Ci;
     const int bt = nrows * SC;
-    grid_arrive(p);
+    grid_arrive(p.sync);
     if (VEC) cp_async_wait<0>();
     if (tid < bt) b_fetch(Lm, p.div_SC[s_nslots], SC, tid, 0, fd, kd);
     if (VEC) cp_async_commit();
-    if (!grid_wait(p, nbar++, &s_ok)) break;
+    if (!stack_wait(p, nbar++, &s_ok)) break;
 
     // =========================== phase B: down + weighted combine
     {
@@ -362,11 +313,11 @@ __global__ void __launch_bounds__(kStack1MaxThreads, 1) stack1_kernel(const __gr
     }
     if (l + 1 == p.n) break;
     // arrive; fetch the next layer's first phase A fields while the others arrive
-    grid_arrive(p);
+    grid_arrive(p.sync);
     if (VEC) cp_async_wait<0>();
     if (a_steps(s_next_nslots) > 0) a_fetch(p.layer[l + 1], s_next_expert, 0, 0, fg, fu, kg, ku);
     if (VEC) cp_async_commit();
-    if (!grid_wait(p, nbar++, &s_ok)) break;
+    if (!stack_wait(p, nbar++, &s_ok)) break;
   }
   if (VEC) cp_async_wait<0>();
 }

@@ -17,7 +17,7 @@
 
 #include "common.cuh"
 #include "moe.cuh"
-#include "stack1.cuh"
+#include "stackb.cuh"
 
 namespace nslm {
 namespace {
@@ -76,15 +76,11 @@ extern "C" int32_t nslm_moe_seed_ffn_static(const nslm_seed_matrix *gate, const 
   // counters on every call, so whatever an earlier call left in the array is
   // harmless; h and the partial sums are written before they are read.
   if ((st = launch_route_plan(nullptr, ids, w, T, E, k, 1, fw.plans, nullptr, nullptr, fw.counters,
-                              d.hidden, fw.sync, s)))
+                              d.hidden, fw.sync, decode_slot_cap(d, T, k), s)))
     return st;
   int launches = 1;
-  if (T == 1 && stack1_supported(d, k)) {
-    const nslm_moe_layer layer{*gate, *up, *down};
-    st = launch_stack1(d, &layer, 1, fw.plans, x_bf16, nullptr, k, fw.h, fw.y_mid, y, fw.sync, fw.rms_part, s, launches);
-  } else {
-    st = launch_decode_layer(d, gate, up, down, fw.plans, x_bf16, nullptr, T, k, fw, y, s, launches);
-  }
+  const nslm_moe_layer layer{*gate, *up, *down};
+  st = launch_decode_stack(d, &layer, 1, x_bf16, T, k, fw, y, s, launches);
   if (st == NSLM_OK) g_launches = launches;
   return st;
 }

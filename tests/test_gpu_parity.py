@@ -223,6 +223,44 @@ def test_ffn_decode_batch(nslm, T, P):
     assert O.normwise_rel_err(y, ref) <= TIGHT
 
 
+def test_ffn_decode_batch8_full_layer(nslm):
+    # 8 tokens on the 100-expert 2048/1408 P=4 layer: about 49 distinct
+    # experts, and the 64 routed h vectors are staged for the down projection
+    # in several groups
+    y, ref = _ffn_case(nslm, 100, 2048, 1408, 4, 8, 8, 940)
+    assert O.normwise_rel_err(y, ref) <= TIGHT
+
+
+@pytest.mark.parametrize("P", [3, 4])
+def test_ffn_decode_batch_shared_experts_split_slots(nslm, P):
+    # all 8 tokens pick the same experts, so an expert carries up to 9 pairs
+    # and the plan splits it into slots of at most 4; one token lists an
+    # expert twice, and two pairs name experts outside [0, E)
+    E, hidden, inter, k, T = 12, 512, 256, 8, 8
+    L = synth.moe_layer(0, E, hidden, inter, P, config=941)
+    x, xh = _x((941, T), T, hidden)
+    rid = np.tile(np.array([5, 1, 9, 0, 11, 3, 7, 2], dtype=np.int32), (T, 1))
+    rid[2, 3] = 5
+    rid[6, 0] = -1
+    rid[7, 7] = E
+    w32 = np.random.default_rng(941).uniform(0.05, 0.3, size=(T, k)).astype(np.float32)
+    y = _ffn_with_ids(nslm, L, E, hidden, inter, x, rid, w32, k)
+    keep = (rid >= 0) & (rid < E)
+    g, u, d = (getattr(L, n).numpy() for n in ("gate", "up", "down"))
+    ref = O.moe_ffn(g, u, d, E, hidden, inter, xh, np.where(keep, rid, 0).astype(np.int32),
+                    np.where(keep, w32.astype(np.float64), 0.0), mode=0)
+    assert O.normwise_rel_err(y, ref) <= TIGHT
+
+
+def test_ffn_decode_batch_all_ids_dropped_gives_zero(nslm):
+    E, hidden, inter, P, k, T = 6, 256, 128, 4, 2, 3
+    L = synth.moe_layer(0, E, hidden, inter, P, config=942)
+    x, _ = _x((942, T), T, hidden)
+    y = _ffn_with_ids(nslm, L, E, hidden, inter, x, np.full((T, k), -1, dtype=np.int32),
+                      np.full((T, k), 0.5, dtype=np.float32), k)
+    assert np.array_equal(y, np.zeros_like(y))
+
+
 def test_ffn_decode_ragged_and_zipf(nslm):
     y, ref = _ffn_case(nslm, 12, 272, 120, 3, 3, 8, 908, zipf=1.1)
     assert O.normwise_rel_err(y, ref) <= TIGHT
@@ -245,26 +283,50 @@ def test_stack_decode_matches_oracle(nslm, T):
     assert O.normwise_rel_err(y.cpu().numpy(), ref) <= TOL
 
 
-def test_stack_decode_past_one_launch_per_layer(nslm):
-    # 70 one-token layers run as two persistent launches (64 + 6).  A long
+def _stack_prefix(nslm, dl, logits, x, T, E, hidden, inter, k, n):
+    """Output of the first n layers of a stack (status word checked)."""
+    y = _out(T, hidden)
+    wsb = nslm.nslm_workspace_bytes(nslm.NSLM_OP_MOE_STACK, T, E, hidden, inter, k, n)
+    ws = torch.zeros(wsb, dtype=torch.uint8, device="cuda")
+    nslm.nslm_moe_stack_decode(dl[:n], n, E, k, logits[:n].cuda().contiguous(), x, T, y, ws, wsb)
+    torch.cuda.synchronize()
+    assert int(ws[:4].view(torch.int32).item()) == 0
+    return y.cpu().numpy().astype(np.float64)
+
+
+def test_stack_decode_batch8_full_layers_pinned(nslm):
+    # 8 tokens through two layers of the 100-expert 2048/1408 P=4 stack, each
+    # layer checked against the oracle on the GPU's own input
+    Lyr, E, hidden, inter, P, k, T = 2, 100, 2048, 1408, 4, 8, 8
+    layers = [synth.moe_layer(l, E, hidden, inter, P, config=943) for l in range(Lyr)]
+    logits = torch.stack([synth.router_logits((943, l), T, E) for l in range(Lyr)])
+    x, xh = _x((943, T), T, hidden)
+    dl = [(_dev(m.gate), _dev(m.up), _dev(m.down)) for m in layers]
+    ys = [_stack_prefix(nslm, dl, logits, x, T, E, hidden, inter, k, n) for n in (1, 2)]
+    for l in range(Lyr):
+        g, u, d = (getattr(layers[l], n).numpy() for n in ("gate", "up", "down"))
+        xl = xh if l == 0 else O.rms_chain(ys[l - 1])
+        ids, w = O.route_topk(logits[l].numpy(), k)
+        ref = O.moe_ffn(g, u, d, E, hidden, inter, xl, ids, w, mode=0)
+        assert O.normwise_rel_err(ys[l], ref) <= TOL, l
+    assert np.array_equal(ys[1], _stack_prefix(nslm, dl, logits, x, T, E, hidden, inter, k, 2))
+
+
+@pytest.mark.parametrize("T", [1, 2])
+def test_stack_decode_past_one_launch_per_layer(nslm, T):
+    # 70 layers run as two persistent launches (64 + 6).  A long
     # stack is chaotic (one bf16 ulp of a layer input changes everything
     # downstream), so each checked layer is fed the GPU's own input: the
     # prefix of l layers gives y_{l-1}, and layer l's output from the prefix
     # of l+1 layers must match the oracle applied to bf16(y_{l-1} / rms).
-    Lyr, E, hidden, inter, P, k, T = 70, 4, 64, 64, 4, 2, 1
+    Lyr, E, hidden, inter, P, k = 70, 4, 64, 64, 4, 2
     layers = [synth.moe_layer(l, E, hidden, inter, P, config=950) for l in range(Lyr)]
-    logits = torch.stack([synth.router_logits((950, l), T, E) for l in range(Lyr)])
+    logits = torch.stack([synth.router_logits((950, l, T), T, E) for l in range(Lyr)])
     x, _ = _x((950, T), T, hidden)
     dl = [(_dev(m.gate), _dev(m.up), _dev(m.down)) for m in layers]
 
     def prefix(n):
-        y = _out(T, hidden)
-        wsb = nslm.nslm_workspace_bytes(nslm.NSLM_OP_MOE_STACK, T, E, hidden, inter, k, n)
-        ws = torch.zeros(wsb, dtype=torch.uint8, device="cuda")
-        nslm.nslm_moe_stack_decode(dl[:n], n, E, k, logits[:n].cuda().contiguous(), x, T, y, ws, wsb)
-        torch.cuda.synchronize()
-        assert int(ws[:4].view(torch.int32).item()) == 0
-        return y.cpu().numpy().astype(np.float64)
+        return _stack_prefix(nslm, dl, logits, x, T, E, hidden, inter, k, n)
 
     for l in (63, 64, 69):  # the last layer of launch 1, the first and last of launch 2
         y_prev, y_l = prefix(l), prefix(l + 1)
