@@ -342,7 +342,7 @@ def search_leg(torch, nslm, dev, with_cpu: bool):
 
 def profile_workload(kind: str, reps: int):
     """A small fixed workload for ncu captures (no timing, no JSON): `reps`
-    calls of one decode layer (T=1, P=4), of one batched layer (T=512, P=3),
+    calls of one decode layer (T=1 or T=8, P=4), of one batched layer (T=512, P=3),
     of one seed GEMV (2048 x 4096, P=4) or of the seed search of a 16 x 256
     fp32 matrix over all seeds."""
     import torch
@@ -366,7 +366,7 @@ def profile_workload(kind: str, reps: int):
             nslm.nslm_seed_gemv(nslm.matrix(m), x, 1, y)
         torch.cuda.synchronize()
         return
-    T, Pv, cfg = (1, 4, 2) if kind == "layer" else (512, 3, 3)
+    T, Pv, cfg = {"layer": (1, 4, 2), "layer8": (8, 4, 2)}.get(kind, (512, 3, 3))
     L = synth.moe_layer(0, E, HIDDEN, INTER, Pv, device=dev, config=cfg)
     logits = synth.router_logits((cfg, T), T, E).to(dev)
     ids = torch.empty(T, K_TOP, dtype=torch.int32, device=dev)
@@ -394,7 +394,7 @@ def main():
     ap.add_argument("--no-batched", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--no-search", action="store_true")
-    ap.add_argument("--profile", choices=["layer", "batched", "gemv", "search"],
+    ap.add_argument("--profile", choices=["layer", "layer8", "batched", "gemv", "search"],
                     help="run a small fixed workload for an ncu capture and exit")
     args = ap.parse_args()
     if args.profile:

@@ -16,14 +16,16 @@
 //                of squares added in a fixed order from per-CTA partials);
 //                warp tasks are (slot, row): the lanes take the 64-weight
 //                chunks of the gate and up rows and dot every regenerated
-//                block with the slot's token vectors; lane 0 writes
+//                block with the slot's token vectors (a one-token slot, the
+//                common case, takes the one-token inner loop); lane 0 writes
 //                h = SiLU(g) * u for each pair.
 //   B (down)     a CTA owns a range of output rows.  The T * k routed h
 //                vectors do not fit in shared memory together, so the slots
 //                are taken in groups whose pairs do: the CTA stages a group's
-//                h vectors, then threads take (row, slot, chunk pair) tasks
-//                (chunks q and q + Cq, one per step) and dot every regenerated
-//                down chunk with the slot's pairs.  Partial sums per (pair,
+//                h vectors, then threads take (slot, row, chunk pair) tasks
+//                (chunks q and q + Cq, one per step; slot-major, so the lanes
+//                of a warp nearly always share a slot) and dot every
+//                regenerated down chunk with the slot's pairs.  Partial sums per (pair,
 //                row, chunk pair) stay in shared memory; after the last group
 //                one warp per row adds them per token, pairs in plan order
 //                (deterministic, no atomics on data).
@@ -44,6 +46,10 @@ namespace nslm {
 namespace {
 
 constexpr int MT = kSlotTokens;
+// Staged blocks per thread with their loads in flight together.  Measured at
+// 8 tokens per layer: 1 -> 227 us, 2 -> 256 us, 4 -> 293 us (more live
+// registers push the inner loops past 128 registers and into spills).
+constexpr int kStageBatch = 1;
 
 struct LayerMatsB {
   nslm_seed_matrix gate, up, down;
@@ -89,7 +95,6 @@ __global__ void __launch_bounds__(kStackBThreads, 1) stackb_kernel(const __grid_
   __shared__ int s_pid[kMaxPairs], s_tok[kMaxPairs];  // by plan position: pair id, token
   __shared__ float s_w[kMaxPairs];
   __shared__ int s_gslot[kMaxPairs + 1];               // group g: slots s_gslot[g] .. s_gslot[g+1]
-  __shared__ unsigned long long s_gdiv[kMaxPairs];     // FastDiv by (slots of group g) * Cq
   __shared__ int s_next_expert[kMaxPairs];
   __shared__ float s_rms[kMaxT];
 
@@ -99,6 +104,10 @@ __global__ void __launch_bounds__(kStackBThreads, 1) stackb_kernel(const __grid_
   const int gw = warp * gridDim.x + blockIdx.x, W = gridDim.x * nwarps;
   const int n0 = blockIdx.x * p.rpc;
   const int nrows = max(0, min(p.rpc, p.hidden - n0));
+  // phase B tasks per slot, padded to whole warps so that a warp never
+  // straddles two slots (its token count then decides a uniform branch)
+  const int RC = nrows * p.Cq, RCp = (RC + 31) & ~31;
+  const FastDiv div_RCp = make_fastdiv((uint32_t)max(1, RCp));
 
   // one layer's plan into shared memory, and the slot groups of phase B
   // (called between block barriers)
@@ -118,16 +127,9 @@ __global__ void __launch_bounds__(kStackBThreads, 1) stackb_kernel(const __grid_
       // greedy groups of whole slots with at most hcap pairs each
       int g = 0, gs = 0;
       s_gslot[0] = 0;
-      for (int s = 1; s < ns; ++s) {
-        if (pl->start[s + 1] - pl->start[gs] > p.hcap) {
-          s_gdiv[g] = make_fastdiv((uint32_t)((s - gs) * p.Cq)).m;
-          s_gslot[++g] = gs = s;
-        }
-      }
-      if (ns > 0) {
-        s_gdiv[g] = make_fastdiv((uint32_t)((ns - gs) * p.Cq)).m;
-        s_gslot[++g] = ns;
-      }
+      for (int s = 1; s < ns; ++s)
+        if (pl->start[s + 1] - pl->start[gs] > p.hcap) s_gslot[++g] = gs = s;
+      if (ns > 0) s_gslot[++g] = ns;
       s_ngroups = g;
     }
   };
@@ -153,26 +155,27 @@ __global__ void __launch_bounds__(kStackBThreads, 1) stackb_kernel(const __grid_
     fetch_chunk_off<P>(Lm.gate, off, r32, fsA, (2 * buf) * nthr + tid);
     fetch_chunk_off<P>(Lm.up, off, r32, fsA, (2 * buf + 1) * nthr + tid);
   };
-  // ---- phase B task geometry: task t of group g = (row r, slot s, chunk pair q);
+  // ---- phase B task geometry: task t of group g = (slot s, row r, chunk pair q);
   // its step 0 takes chunk q, step 1 chunk q + Cq
   auto b_nsteps = [&](int g) {
-    const int nt = nrows * (s_gslot[g + 1] - s_gslot[g]) * p.Cq;
+    const int nt = (s_gslot[g + 1] - s_gslot[g]) * RCp;
     return tid < nt ? 2 * ((nt - 1 - tid) / nthr + 1) : 0;
   };
+  // r < 0 marks a padding task; c >= Ci the missing second chunk of an odd Ci
   auto b_locate = [&](int g, int step, int &r, int &s, int &q, int &c) {
     const int t = tid + (step >> 1) * nthr;
-    const int SC = (s_gslot[g + 1] - s_gslot[g]) * p.Cq;
-    r = (int)fdiv((uint32_t)t, FastDiv{s_gdiv[g]});
-    const int rem = t - r * SC;
-    const int sr = (int)fdiv((uint32_t)rem, p.div_Cq);
-    q = rem - sr * p.Cq;
+    const int sr = (int)fdiv((uint32_t)t, div_RCp);
+    const int rem = t - sr * RCp;
+    r = (int)fdiv((uint32_t)rem, p.div_Cq);
+    q = rem - r * p.Cq;
     s = s_gslot[g] + sr;
     c = q + (step & 1) * p.Cq;
+    if (rem >= RC) r = -1;
   };
   auto b_fetch = [&](const LayerMatsB &Lm, int g, int step, int buf) {
     int r, s, q, c;
     b_locate(g, step, r, s, q, c);
-    if (c >= p.Ci) return;
+    if (r < 0 || c >= p.Ci) return;
     const uint32_t r32 = (uint32_t)s_expert[s] * (uint32_t)p.hidden + (uint32_t)(n0 + r);
     fetch_chunk_off<P>(Lm.down, r32 * (uint32_t)nbi + 8u * (uint32_t)c, r32, fsB, buf * nthr + tid);
   };
@@ -196,15 +199,40 @@ __global__ void __launch_bounds__(kStackBThreads, 1) stackb_kernel(const __grid_
     }
 
     // =========================== phase A: gate/up + SiLU
+    // (token t's block b is staged as block t * Ch * 8 + b; blocks are taken
+    // kStageBatch per thread at a time, all loads in flight before the stores)
+    const int nxb = p.T * nbh;
     if (l == 0 && p.x0) {
-      for (int i = tid; i < p.T * nbh; i += nthr) {
-        const int t = i / nbh, b = i - t * nbh;
-        float4 lo, hi;
-        bf16x8_to_f32(__ldg(reinterpret_cast<const uint4 *>(p.x0 + (size_t)t * p.hidden) + b), lo, hi);
-        cm_store_block(xs4, xn2, t * p.Ch * 8 + b, lo, hi);
+      for (int i0 = tid; i0 < nxb; i0 += kStageBatch * nthr) {
+        uint4 v[kStageBatch];
+#pragma unroll
+        for (int u = 0; u < kStageBatch; ++u) {
+          const int i = i0 + u * nthr;
+          if (i < nxb) v[u] = __ldg(reinterpret_cast<const uint4 *>(p.x0) + i);  // [T][hidden] bf16
+        }
+#pragma unroll
+        for (int u = 0; u < kStageBatch; ++u) {
+          const int i = i0 + u * nthr;
+          if (i < nxb) {
+            const int t = i / nbh;
+            float4 lo, hi;
+            bf16x8_to_f32(v[u], lo, hi);
+            cm_store_block(xs4, xn2, t * p.Ch * 8 + (i - t * nbh), lo, hi);
+          }
+        }
       }
     } else {
-      const float *y = l == 0 ? p.y_in : p.y_mid;
+      const float4 *y4 = reinterpret_cast<const float4 *>(l == 0 ? p.y_in : p.y_mid);  // [T][hidden]
+      float4 v[kStageBatch][2];
+      // the first batch of loads is in flight during the sums of squares
+#pragma unroll
+      for (int u = 0; u < kStageBatch; ++u) {
+        const int i = tid + u * nthr;
+        if (i < nxb) {
+          v[u][0] = __ldcg(y4 + 2 * i);
+          v[u][1] = __ldcg(y4 + 2 * i + 1);
+        }
+      }
       if (warp < p.T) {  // rms of token `warp`: per-CTA partials in a fixed order
         float ss = 0.f;
         for (int i = lane; i < (int)gridDim.x; i += 32) ss += __ldcg(p.rms_part + warp * gridDim.x + i);
@@ -212,16 +240,31 @@ __global__ void __launch_bounds__(kStackBThreads, 1) stackb_kernel(const __grid_
         if (lane == 0) s_rms[warp] = sqrtf(ss / (float)p.hidden + 1e-6f);
       }
       __syncthreads();
-      for (int i = tid; i < p.T * nbh; i += nthr) {
-        const int t = i / nbh, b = i - t * nbh;
-        const float4 *row = reinterpret_cast<const float4 *>(y + (size_t)t * p.hidden);
-        const float4 lo = __ldcg(row + 2 * b), hi = __ldcg(row + 2 * b + 1);
-        const float r = s_rms[t];
-#define NSLM_NORM(v) __bfloat162float(__float2bfloat16_rn(__fdiv_rn((v), r)))
-        cm_store_block(xs4, xn2, t * p.Ch * 8 + b,
-                       make_float4(NSLM_NORM(lo.x), NSLM_NORM(lo.y), NSLM_NORM(lo.z), NSLM_NORM(lo.w)),
-                       make_float4(NSLM_NORM(hi.x), NSLM_NORM(hi.y), NSLM_NORM(hi.z), NSLM_NORM(hi.w)));
+      for (int i0 = tid; i0 < nxb; i0 += kStageBatch * nthr) {
+        if (i0 != tid) {
+#pragma unroll
+          for (int u = 0; u < kStageBatch; ++u) {
+            const int i = i0 + u * nthr;
+            if (i < nxb) {
+              v[u][0] = __ldcg(y4 + 2 * i);
+              v[u][1] = __ldcg(y4 + 2 * i + 1);
+            }
+          }
+        }
+#pragma unroll
+        for (int u = 0; u < kStageBatch; ++u) {
+          const int i = i0 + u * nthr;
+          if (i < nxb) {
+            const int t = i / nbh;
+            const float r = s_rms[t];
+            const float4 lo = v[u][0], hi = v[u][1];
+#define NSLM_NORM(x) __bfloat162float(__float2bfloat16_rn(__fdiv_rn((x), r)))
+            cm_store_block(xs4, xn2, t * p.Ch * 8 + (i - t * nbh),
+                           make_float4(NSLM_NORM(lo.x), NSLM_NORM(lo.y), NSLM_NORM(lo.z), NSLM_NORM(lo.w)),
+                           make_float4(NSLM_NORM(hi.x), NSLM_NORM(hi.y), NSLM_NORM(hi.z), NSLM_NORM(hi.w)));
 #undef NSLM_NORM
+          }
+        }
       }
     }
     __syncthreads();
@@ -244,9 +287,18 @@ __global__ void __launch_bounds__(kStackBThreads, 1) stackb_kernel(const __grid_
         int off[MT];
 #pragma unroll
         for (int m = 0; m < MT; ++m) off[m] = (m < M ? s_tok[q0 + m] : 0) * p.Ch;
-        if (c < p.Ch)
-          chunk_dot2_cm_multi<P, true, 1, MT>(tab, cg, cu, 8, ckg, cku, xs4 + kCmX4 * c, xn2 + kCmXn * c, off,
-                                              M, ag, au);
+        if (c < p.Ch) {
+          // M is warp-uniform; the literal 2 folds the token guards away
+          if (M == 1)
+            chunk_dot2_cm<P, true, 1>(tab, cg, cu, 8, ckg, cku, xs4 + kCmX4 * (c + off[0]),
+                                      xn2 + kCmXn * (c + off[0]), ag[0], au[0]);
+          else if (M == 2)
+            chunk_dot2_cm_multi<P, true, 1, MT>(tab, cg, cu, 8, ckg, cku, xs4 + kCmX4 * c, xn2 + kCmXn * c,
+                                                off, 2, ag, au);
+          else
+            chunk_dot2_cm_multi<P, true, 1, MT>(tab, cg, cu, 8, ckg, cku, xs4 + kCmX4 * c, xn2 + kCmXn * c,
+                                                off, M, ag, au);
+        }
         if (p.J == 1 || c + 32 >= 32 * p.J) {
 #pragma unroll
           for (int m = 0; m < MT; ++m) {
@@ -279,11 +331,27 @@ __global__ void __launch_bounds__(kStackBThreads, 1) stackb_kernel(const __grid_
         // staging in bounds regardless)
         const int qa = s_start[s_gslot[g]], np = min(p.hcap, s_start[s_gslot[g + 1]] - qa);
         // the group's h vectors, chunk-major, pair j at chunk slot j * Ci
-        for (int i = tid; i < np * nbi; i += nthr) {
-          const int j = (int)fdiv((uint32_t)i, p.div_nbi), b = i - j * nbi;
-          const float4 *src = reinterpret_cast<const float4 *>(p.h + (size_t)s_pid[qa + j] * p.inter) + 2 * b;
-          const float4 lo = __ldcg(src), hi = __ldcg(src + 1);
-          cm_store_block(xs4, xn2, j * p.Ci * 8 + b, lo, hi);
+        const int nhb = np * nbi;
+        for (int i0 = tid; i0 < nhb; i0 += kStageBatch * nthr) {
+          float4 v[kStageBatch][2];
+#pragma unroll
+          for (int u = 0; u < kStageBatch; ++u) {
+            const int i = i0 + u * nthr;
+            if (i < nhb) {
+              const int j = (int)fdiv((uint32_t)i, p.div_nbi), b = i - j * nbi;
+              const float4 *src = reinterpret_cast<const float4 *>(p.h + (size_t)s_pid[qa + j] * p.inter) + 2 * b;
+              v[u][0] = __ldcg(src);
+              v[u][1] = __ldcg(src + 1);
+            }
+          }
+#pragma unroll
+          for (int u = 0; u < kStageBatch; ++u) {
+            const int i = i0 + u * nthr;
+            if (i < nhb) {
+              const int j = (int)fdiv((uint32_t)i, p.div_nbi);
+              cm_store_block(xs4, xn2, j * p.Ci * 8 + (i - j * nbi), v[u][0], v[u][1]);
+            }
+          }
         }
         __syncthreads();
         const int n = b_nsteps(g);
@@ -312,13 +380,20 @@ __global__ void __launch_bounds__(kStackBThreads, 1) stackb_kernel(const __grid_
 #pragma unroll
             for (int m = 0; m < MT; ++m) acc[m] = make_float2(0.f, 0.f);
           }
-          if (c < p.Ci) {
+          if (r >= 0 && c < p.Ci) {
             int off[MT];
 #pragma unroll
             for (int m = 0; m < MT; ++m) off[m] = (q0 - qa + m) * p.Ci;
-            chunk_dot_cm_multi<P, true, 1, MT>(tab, cf, 8, ck, xs4 + kCmX4 * c, xn2 + kCmXn * c, off, M, acc);
+            // M is warp-uniform (slots are padded to whole warps)
+            if (M == 1)
+              chunk_dot_cm<P, true, 1>(tab, cf, 8, ck, xs4 + kCmX4 * (c + off[0]), xn2 + kCmXn * (c + off[0]),
+                                       acc[0]);
+            else if (M == 2)
+              chunk_dot_cm_multi<P, true, 1, MT>(tab, cf, 8, ck, xs4 + kCmX4 * c, xn2 + kCmXn * c, off, 2, acc);
+            else
+              chunk_dot_cm_multi<P, true, 1, MT>(tab, cf, 8, ck, xs4 + kCmX4 * c, xn2 + kCmXn * c, off, M, acc);
           }
-          if (k & 1) {
+          if ((k & 1) && r >= 0) {
 #pragma unroll
             for (int m = 0; m < MT; ++m)
               if (m < M) red[((q0 + m) * p.rpc + r) * p.Cq + q] = acc[m].x + acc[m].y;
@@ -429,6 +504,7 @@ bool stackb_supported(const FfnDims &d, int T, int k) {
   if ((int64_t)kMaxPairs * sh.Cq >= (1 << 16)) return false;
   if ((int64_t)T * k * d.inter * ceil_div(sh.Ch, 32) >= (1 << 22)) return false;
   if ((int64_t)sh.rpc * T * k * sh.Cq >= (1 << 22) || (int64_t)sh.hcap * (d.inter / 8) >= (1 << 22)) return false;
+  if ((int64_t)sh.rpc * sh.Cq >= (1 << 16)) return false;
   return true;
 }
 
