@@ -143,7 +143,7 @@ int32_t nslm_moe_route_topk(const float *logits, int32_t T, int32_t E, int32_t k
  * larger T runs the tensor-core path (bf16 weights, bf16 hidden activation;
  * hidden and inter multiples of 64, E <= 1024).  The first int32 of the
  * workspace is set nonzero if a device-side wait (the tensor-core pipeline,
- * or the grid barrier of the one-token kernel) gave up.
+ * or the grid barrier of a persistent decode kernel) gave up.
  * Workspace: nslm_workspace_bytes(NSLM_OP_MOE_FFN, T, E, hidden, inter, k, 0). */
 int32_t nslm_moe_seed_ffn(const nslm_seed_matrix *gate, const nslm_seed_matrix *up,
                           const nslm_seed_matrix *down, int32_t E, const uint16_t *x_bf16,
@@ -182,7 +182,11 @@ int32_t nslm_moe_seed_ffn_static(const nslm_seed_matrix *gate, const nslm_seed_m
  * put attention between MoE layers; this normalisation stands in for it).
  * layers: HOST array of L layers (device pointers inside), all with the same
  * E, hidden, inter and P.  x0: bf16 [T][hidden]; y: fp32 [T][hidden], the
- * last layer's output.
+ * last layer's output.  Where the shape allows (T = 1, or T >= 2 with
+ * hidden and inter multiples of 64) all layers run in one cooperative launch
+ * per 64 layers after one routing launch; otherwise each layer takes two
+ * launches.  The first int32 of the workspace is set nonzero if a grid
+ * barrier wait of the persistent kernel gave up (about 1 s).
  * Workspace: nslm_workspace_bytes(NSLM_OP_MOE_STACK, T, E, hidden, inter, k, L). */
 int32_t nslm_moe_stack_decode(const nslm_moe_layer *layers, int32_t L, int32_t E, int32_t k,
                               const float *logits, const uint16_t *x0_bf16, int32_t T,
