@@ -465,13 +465,25 @@ static int32_t round_clamp_int4(double v)
  * For every seed in [seed_lo, seed_hi] and every code in 0..15: the
  * least-squares coefficients c = pinv(U) w / 2^(code + bias), rounded half to
  * even and clamped to [-8, 7]; the error |w - 2^(code+bias) U c|^2.  Keeps
- * the smallest error; ties go to the larger code, then the lower seed. */
-int32_t nslmo_search_block(const double *w8, int32_t P, int32_t bias, int32_t seed_lo,
-                           int32_t seed_hi, int32_t *best_seed, int32_t *best_c,
-                           int32_t *best_code, double *best_err)
+ * the smallest error; ties go to the larger code, then the lower seed.
+ *
+ * d8 (may be NULL): per-weight importances, the mean square of each weight's
+ * input activation ([QWEN] "How it works": the search weighted the error of
+ * each weight that way).  Then err = sum_r d_r (w_r - 2^(code+bias) (U c)_r)^2
+ * and, reading the pages' weighted error as the objective, the coefficients
+ * are its least-squares minimiser: c = (U^T D U)^-1 U^T D w / 2^(code+bias),
+ * D = diag(d), rounded and clamped as above.  d = NULL is d_r = 1, which gives
+ * the unweighted search bit for bit (every product with 1.0 is exact).  The
+ * operation order, fixed here, is A[a][b] = sum_r ((U_ra U_rb) d_r),
+ * B[a][r] = U_ra d_r, err = sum_r d_r (e_r e_r). */
+int32_t nslmo_search_block_w(const double *w8, const double *d8, int32_t P, int32_t bias,
+                             int32_t seed_lo, int32_t seed_hi, int32_t *best_seed, int32_t *best_c,
+                             int32_t *best_code, double *best_err)
 {
     if ((P != 3 && P != 4) || seed_lo < 1 || seed_hi > 65535 || seed_lo > seed_hi)
         return NSLMO_ERR_ARG;
+    double d[8];
+    for (int r = 0; r < 8; ++r) d[r] = d8 ? d8[r] : 1.0;
     double err_min = INFINITY;
     int32_t s_best = -1, code_best = -1, c_best[4] = {0, 0, 0, 0};
     for (int32_t seed = seed_lo; seed <= seed_hi; ++seed) {
@@ -482,11 +494,11 @@ int32_t nslmo_search_block(const double *w8, int32_t P, int32_t bias, int32_t se
         for (int a = 0; a < P; ++a)
             for (int b = 0; b < P; ++b) {
                 double s = 0.0;
-                for (int r = 0; r < 8; ++r) s += U[r * P + a] * U[r * P + b];
+                for (int r = 0; r < 8; ++r) s += (U[r * P + a] * U[r * P + b]) * d[r];
                 A[a * P + b] = s;
             }
         for (int a = 0; a < P; ++a)
-            for (int r = 0; r < 8; ++r) B[a * 8 + r] = U[r * P + a];
+            for (int r = 0; r < 8; ++r) B[a * 8 + r] = U[r * P + a] * d[r];
         if (!solve_small(A, B, P, 8)) continue;
         double proj[4];
         for (int a = 0; a < P; ++a) {
@@ -502,8 +514,8 @@ int32_t nslmo_search_block(const double *w8, int32_t P, int32_t bias, int32_t se
             for (int r = 0; r < 8; ++r) {
                 double v = 0.0;
                 for (int a = 0; a < P; ++a) v += U[r * P + a] * (double)c[a];
-                double d = w8[r] - scale * v;
-                err += d * d;
+                double e = w8[r] - scale * v;
+                err += d[r] * (e * e);
             }
             /* strict '<': the first hit wins, and codes run from 15 down and
                seeds from low to high, so ties keep the larger code, then the
@@ -525,4 +537,12 @@ int32_t nslmo_search_block(const double *w8, int32_t P, int32_t bias, int32_t se
     for (int a = 0; a < P; ++a) best_c[a] = c_best[a];
     *best_err = err_min;
     return NSLMO_OK;
+}
+
+int32_t nslmo_search_block(const double *w8, int32_t P, int32_t bias, int32_t seed_lo,
+                           int32_t seed_hi, int32_t *best_seed, int32_t *best_c,
+                           int32_t *best_code, double *best_err)
+{
+    return nslmo_search_block_w(w8, NULL, P, bias, seed_lo, seed_hi, best_seed, best_c, best_code,
+                                best_err);
 }

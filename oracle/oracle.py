@@ -97,6 +97,10 @@ def lib():
         L.nslmo_search_block.argtypes = [
             _f64p, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32,
             _i32p, _i32p, _i32p, _f64p]
+        L.nslmo_search_block_w.restype = ctypes.c_int32
+        L.nslmo_search_block_w.argtypes = [
+            _f64p, ctypes.c_void_p, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32,
+            _i32p, _i32p, _i32p, _f64p]
         _lib = L
     return _lib
 
@@ -301,14 +305,22 @@ def layer_stack(layers, logits, x0_bf16, hidden: int, inter: int, E: int, k: int
 
 # ------------------------------------------------------------ seed search
 
-def search_block(w8, P: int, bias: int, seed_lo: int = 1, seed_hi: int = 65535):
-    """Brute-force search of one block: best (seed, c, code, err)."""
+def search_block(w8, P: int, bias: int, seed_lo: int = 1, seed_hi: int = 65535, d8=None):
+    """Brute-force search of one block: best (seed, c, code, err).
+
+    d8: optional per-weight importances (the mean square of each weight's
+    input activation); the error and the least-squares fit are then weighted."""
     w8 = np.ascontiguousarray(w8, np.float64)
     s = np.zeros(1, np.int32)
     c = np.zeros(4, np.int32)
     code = np.zeros(1, np.int32)
     err = np.zeros(1, np.float64)
-    rc = lib().nslmo_search_block(w8, P, bias, seed_lo, seed_hi, s, c, code, err)
+    if d8 is None:
+        rc = lib().nslmo_search_block(w8, P, bias, seed_lo, seed_hi, s, c, code, err)
+    else:
+        d8 = np.ascontiguousarray(d8, np.float64)
+        assert d8.shape == (8,)
+        rc = lib().nslmo_search_block_w(w8, d8.ctypes.data, P, bias, seed_lo, seed_hi, s, c, code, err)
     assert rc == 0, rc
     return int(s[0]), c[:P].copy(), int(code[0]), float(err[0])
 

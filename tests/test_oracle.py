@@ -309,3 +309,87 @@ def test_search_matches_brute_force_on_a_tiny_range():
     # on random blocks rounding the LS solution is close to optimal
     assert err >= best - 1e-18
     assert err <= 4.0 * best
+
+
+# ---- activation-weighted search ([QWEN] "How it works": the error of each
+# weight weighted by the mean square of its input activation)
+
+def _weighted_search_numpy(w, d, P, bias, lo, hi):
+    """The weighted search restated with numpy's least squares: for every seed
+    and code, c = clamp(rint(argmin_c |D^1/2 (w - 2^e U c)|)), err weighted;
+    smallest error, then larger code, then lower seed."""
+    sq = np.sqrt(d)
+    best = (np.inf, 0, 0, 0, None)
+    for seed in range(lo, hi + 1):
+        U = O.basis(seed, P)
+        proj = np.linalg.lstsq(sq[:, None] * U, sq * w, rcond=None)[0]
+        for code in range(15, -1, -1):
+            sc = 2.0 ** (code + bias)
+            c = np.clip(np.rint(proj / sc), -8, 7).astype(np.int64)
+            err = float(np.sum(d * (w - sc * (U @ c)) ** 2))
+            key = (err, -code, seed)
+            if key < best[:3]:
+                best = (err, -code, seed, code, c)
+    return best[2], best[4], best[3], best[0]
+
+
+@pytest.mark.parametrize("P", [3, 4])
+def test_weighted_search_matches_a_numpy_least_squares_restatement(P):
+    rng = np.random.default_rng(70 + P)
+    bias = -12
+    for _ in range(3):
+        w = rng.standard_normal(8) * 2.0 ** (bias + 14)
+        d = rng.uniform(0.05, 4.0, 8)
+        s, c, code, err = O.search_block(w, P, bias, 500, 531, d8=d)
+        rs, rc, rcode, rerr = _weighted_search_numpy(w, d, P, bias, 500, 531)
+        assert (s, code) == (rs, rcode)
+        assert np.array_equal(c, rc)
+        assert abs(err - rerr) <= 1e-12 * rerr
+
+
+def test_weighted_search_with_unit_importances_is_the_plain_search():
+    rng = np.random.default_rng(80)
+    w = rng.standard_normal(8) * 2.0 ** 3
+    s, c, code, err = O.search_block(w, 4, -12, 1, 2000, d8=np.ones(8))
+    s0, c0, code0, err0 = O.search_block(w, 4, -12, 1, 2000)
+    assert (s, code, err) == (s0, code0, err0) and np.array_equal(c, c0)
+
+
+@pytest.mark.parametrize("P", [3, 4])
+def test_weighted_search_scales_with_the_importances(P):
+    # importances times a power of two: same choice, error times that power
+    # exactly (d enters the fit and the error consistently)
+    rng = np.random.default_rng(90 + P)
+    w = rng.standard_normal(8) * 2.0 ** 2
+    d = rng.uniform(0.1, 3.0, 8)
+    s, c, code, err = O.search_block(w, P, -12, 1, 3000, d8=d)
+    s2, c2, code2, err2 = O.search_block(w, P, -12, 1, 3000, d8=d * 8.0)
+    assert (s, code) == (s2, code2) and np.array_equal(c, c2)
+    assert err2 == 8.0 * err
+
+
+@pytest.mark.parametrize("P", [3, 4])
+def test_weighted_search_recovers_a_planted_block(P):
+    rng = np.random.default_rng(100 + P)
+    seed = int(rng.integers(1, 65536))
+    c = rng.integers(-8, 8, P)
+    c[0] |= 1
+    code = int(rng.integers(0, 16))
+    w = O.regen_block(seed, c, code, -12)
+    s, cc, cd, err = O.search_block(w, P, -12, d8=rng.uniform(0.01, 10.0, 8))
+    assert (s, cd, err) == (seed, code, 0.0)
+    assert np.array_equal(cc, c)
+
+
+def test_weighting_changes_the_choice():
+    # a block with a large weight at one position: the weighted search fits
+    # that position better than the plain one does
+    rng = np.random.default_rng(110)
+    w = rng.standard_normal(8) * 2.0 ** 2
+    d = np.full(8, 1e-3)
+    d[5] = 1.0
+    s, c, code, _ = O.search_block(w, 4, -12, 1, 4000)
+    sw, cw, codew, _ = O.search_block(w, 4, -12, 1, 4000, d8=d)
+    fit = lambda s_, c_, code_: abs(w[5] - O.regen_block(s_, c_, code_, -12)[5])
+    assert (s, code) != (sw, codew)
+    assert fit(sw, cw, codew) < fit(s, c, code)
