@@ -369,9 +369,17 @@ def search_leg(torch, nslm, dev, with_cpu: bool):
     torch.cuda.synchronize()
     t = e0.elapsed_time(e1) * 1e-3
     nblk = N * (K // 8)
+    # activation-weighted search: importances = mean squares of N(0,1)-like activations
+    imp = (torch.rand(K, generator=g) * 2.0).to(dev)
+    e0.record()
+    nslm.nslm_seed_search(w, out, 1, 65535, imp=imp)
+    e1.record()
+    torch.cuda.synchronize()
+    tw = e0.elapsed_time(e1) * 1e-3
     res = {"workload": "seed search of a 64 x 2048 fp32 matrix (16,384 blocks, P=4) over all 65,535 seeds x 16 codes",
            "gpu_blocks_per_s": round(nblk / t, 1), "gpu_s": round(t, 4),
-           "candidates_per_s": nblk * 65535 * 16 / t}
+           "candidates_per_s": nblk * 65535 * 16 / t,
+           "gpu_blocks_per_s_weighted": round(nblk / tw, 1)}
     if with_cpu:
         from oracle import oracle as O
         wh = w[:1, :16].double().cpu().numpy()

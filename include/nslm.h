@@ -203,14 +203,22 @@ int32_t nslm_moe_stack_decode(const nslm_moe_layer *layers, int32_t L, int32_t E
  *       elimination with partial pivoting, fp64, no fused multiply-add
  *   err = sum_r (w_r - 2^(code + exp_bias[row]) (U c)_r)^2, fp64
  * The smallest err wins; ties go to the larger code, then the lower seed.
+ * imp: fp32 [K] per-column importances (the mean square of each column's
+ * input activation, "Qwen3.8-Flash-Next-NanoSeedLM-P4", "How it works"), or
+ * null.  With imp, d_r = imp[8 b + r] weights each term of err, and the fit is
+ * the weighted least-squares one: pinv = (U^T D U)^-1 U^T D with
+ * A[a][b] = sum_r ((U_ra U_rb) d_r) and B[a][r] = U_ra d_r, then
+ * err = sum_r d_r ((w_r - ...)^2); unit importances give the unweighted
+ * answer.  Importances should be finite and >= 0 (they are not checked);
+ * a block whose importances make every seed singular is unencodable.
  * out: the packed matrix to fill (N, K, P give the shape; K % 8 == 0, P=4
  * needs K % 16 == 0): seeds, coefs (and codes for P = 4) are WRITTEN;
  * exp_bias [N] is READ (the row biases to encode with).  err: fp64 [N][K/8]
  * of the winning errors, or null.  A block whose every seed is singular gets
  * seed 0, zero coefficients and err = +inf.  All pointers are device
  * pointers; the seed streams of out must not overlap w. */
-int32_t nslm_seed_search(const float *w, const nslm_seed_matrix *out, int32_t seed_lo,
-                         int32_t seed_hi, double *err, nslm_stream_t stream);
+int32_t nslm_seed_search(const float *w, const float *imp, const nslm_seed_matrix *out,
+                         int32_t seed_lo, int32_t seed_hi, double *err, nslm_stream_t stream);
 
 /* Test exports: the regenerated weights themselves, written out densely.
  * w_out: fp32 [N][K] (exact) or bf16 bit patterns [N][K] (round to nearest

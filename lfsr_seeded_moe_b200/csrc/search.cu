@@ -10,6 +10,12 @@
 // pivoting, in fp64.  The smallest error wins; ties go to the larger code,
 // then to the lower seed.
 //
+// With per-column importances d ("Qwen3.8-Flash-Next-NanoSeedLM-P4", "How it
+// works": the search weighted each weight's error by the mean square of its
+// input activation) the error is sum_r d_r (w_r - 2^(code+bias) (U c)_r)^2 and
+// the fit its least-squares minimiser, (U^T D U)^-1 U^T D w; the weighted
+// pinv then differs per block and is formed for each (seed, block).
+//
 // A CTA takes four consecutive blocks of a row (pairs share a P = 4 codes
 // byte) and forms pinv(U) once per seed for all four; its threads split the
 // seed range, each keeps its best candidate per block, and a shared-memory
@@ -47,25 +53,10 @@ __device__ __forceinline__ bool better(const Cand &a, const Cand &b) {
   return a.seed < b.seed;
 }
 
-// pinv(U) for one seed: returns false when U^T U is singular (the seed is
-// skipped).  u[r][j] = s_{1+8j+r} - 32768, so U = u / 32768.
+// A^-1 B in place by Gauss-Jordan elimination with partial pivoting, exactly
+// the reference's steps; false when A is singular.
 template <int P>
-__device__ bool pinv_of(const int32_t (&u)[8][4], double (&B)[4][8]) {
-  double A[4][4];
-#pragma unroll
-  for (int a = 0; a < P; ++a)
-#pragma unroll
-    for (int b = 0; b < P; ++b) {
-      long long s = 0;
-#pragma unroll
-      for (int r = 0; r < 8; ++r) s += (long long)u[r][a] * u[r][b];
-      A[a][b] = (double)s * pow2(-30);  // exact: |s| < 2^33
-    }
-#pragma unroll
-  for (int a = 0; a < P; ++a)
-#pragma unroll
-    for (int r = 0; r < 8; ++r) B[a][r] = (double)u[r][a] * pow2(-15);
-  // Gauss-Jordan with partial pivoting, exactly the reference's steps
+__device__ __forceinline__ bool gauss_jordan(double (&A)[4][4], double (&B)[4][8]) {
 #pragma unroll
   for (int col = 0; col < P; ++col) {
     int piv = col;
@@ -105,8 +96,52 @@ __device__ bool pinv_of(const int32_t (&u)[8][4], double (&B)[4][8]) {
   return true;
 }
 
+// pinv(U) for one seed: returns false when U^T U is singular (the seed is
+// skipped).  u[r][j] = s_{1+8j+r} - 32768, so U = u / 32768.
+template <int P>
+__device__ bool pinv_of(const int32_t (&u)[8][4], double (&B)[4][8]) {
+  double A[4][4];
+#pragma unroll
+  for (int a = 0; a < P; ++a)
+#pragma unroll
+    for (int b = 0; b < P; ++b) {
+      long long s = 0;
+#pragma unroll
+      for (int r = 0; r < 8; ++r) s += (long long)u[r][a] * u[r][b];
+      A[a][b] = (double)s * pow2(-30);  // exact: |s| < 2^33
+    }
+#pragma unroll
+  for (int a = 0; a < P; ++a)
+#pragma unroll
+    for (int r = 0; r < 8; ++r) B[a][r] = (double)u[r][a] * pow2(-15);
+  return gauss_jordan<P>(A, B);
+}
+
+// The weighted pinv (U^T D U)^-1 U^T D, in the reference's operation order:
+// A[a][b] = sum_r ((U_ra U_rb) d_r), B[a][r] = U_ra d_r (U_ra U_rb is exact).
+template <int P>
+__device__ bool pinv_weighted(const int32_t (&u)[8][4], const double *d, double (&B)[4][8]) {
+  double A[4][4];
+#pragma unroll
+  for (int a = 0; a < P; ++a)
+#pragma unroll
+    for (int b = 0; b < P; ++b) {
+      double s = 0.0;
+#pragma unroll
+      for (int r = 0; r < 8; ++r)
+        s = __dadd_rn(s, __dmul_rn((double)((long long)u[r][a] * u[r][b]) * pow2(-30), d[r]));
+      A[a][b] = s;
+    }
+#pragma unroll
+  for (int a = 0; a < P; ++a)
+#pragma unroll
+    for (int r = 0; r < 8; ++r) B[a][r] = __dmul_rn((double)u[r][a] * pow2(-15), d[r]);
+  return gauss_jordan<P>(A, B);
+}
+
 struct SearchParams {
   const float *w;            // [N][K]
+  const float *imp;          // [K] importances, or null (unweighted)
   nslm_seed_matrix out;      // seeds, coefs, codes written; exp_bias read
   double *err;               // [N][K/8] or null
   int32_t seed_lo, seed_hi;
@@ -118,11 +153,12 @@ struct SearchParams {
 // code bytes inside one CTA).
 constexpr int kSearchGroup = 4;
 
-template <int P>
+template <int P, bool WEIGHTED>
 __global__ void __launch_bounds__(kSearchThreads) seed_search_kernel(const SearchParams p) {
   __shared__ StreamTables tab;
   __shared__ Cand s_c[kSearchThreads];
   __shared__ double s_w[kSearchGroup][8];
+  __shared__ double s_d[kSearchGroup][8];
   build_stream_tables(&tab);
   const int tid = threadIdx.x;
   const int groups_row = (p.nb + kSearchGroup - 1) / kSearchGroup;
@@ -130,7 +166,10 @@ __global__ void __launch_bounds__(kSearchThreads) seed_search_kernel(const Searc
   const int b0 = (int)(blockIdx.x - row * groups_row) * kSearchGroup;
   const int nblk = min(kSearchGroup, p.nb - b0);
   const int32_t bias = p.out.exp_bias[row];
-  if (tid < 8 * nblk) s_w[tid >> 3][tid & 7] = (double)p.w[row * (int64_t)p.nb * 8 + 8 * b0 + tid];
+  if (tid < 8 * nblk) {
+    s_w[tid >> 3][tid & 7] = (double)p.w[row * (int64_t)p.nb * 8 + 8 * b0 + tid];
+    s_d[tid >> 3][tid & 7] = WEIGHTED ? (double)p.imp[8 * b0 + tid] : 1.0;
+  }
   __syncthreads();
 
   Cand best[kSearchGroup];
@@ -148,10 +187,11 @@ __global__ void __launch_bounds__(kSearchThreads) seed_search_kernel(const Searc
       for (int j = 0; j < 4; ++j)
         u[r][j] = (j < P) ? (int32_t)(__funnelshift_rc(lo, hi, 1 + 8 * j + r) & 0xFFFFu) - 32768 : 0;
     double B[4][8];
-    if (!pinv_of<P>(u, B)) continue;
+    if (!WEIGHTED && !pinv_of<P>(u, B)) continue;
 #pragma unroll
     for (int g = 0; g < kSearchGroup; ++g) {
       if (g >= nblk) break;
+      if (WEIGHTED && !pinv_weighted<P>(u, s_d[g], B)) continue;
       double w[8];
 #pragma unroll
       for (int r = 0; r < 8; ++r) w[r] = s_w[g][r];
@@ -189,8 +229,8 @@ __global__ void __launch_bounds__(kSearchThreads) seed_search_kernel(const Searc
           int32_t A = 0;
 #pragma unroll
           for (int a = 0; a < P; ++a) A += u[r][a] * c[a];
-          const double d = __dsub_rn(w[r], (double)A * sc);
-          err = __dadd_rn(err, __dmul_rn(d, d));
+          const double e = __dsub_rn(w[r], (double)A * sc);
+          err = WEIGHTED ? __dadd_rn(err, __dmul_rn(s_d[g][r], __dmul_rn(e, e))) : __dadd_rn(err, __dmul_rn(e, e));
         }
         const Cand cand{err, code, seed, cp};
         if (better(cand, best[g])) best[g] = cand;
@@ -232,8 +272,8 @@ __global__ void __launch_bounds__(kSearchThreads) seed_search_kernel(const Searc
 
 using namespace nslm;
 
-extern "C" int32_t nslm_seed_search(const float *w, const nslm_seed_matrix *out, int32_t seed_lo,
-                                    int32_t seed_hi, double *err, nslm_stream_t stream) {
+extern "C" int32_t nslm_seed_search(const float *w, const float *imp, const nslm_seed_matrix *out,
+                                    int32_t seed_lo, int32_t seed_hi, double *err, nslm_stream_t stream) {
   g_launches = 0;
   int32_t st = check_matrix(out);
   if (st) return st;
@@ -243,6 +283,7 @@ extern "C" int32_t nslm_seed_search(const float *w, const nslm_seed_matrix *out,
   if ((st = check_device())) return st;
   SearchParams p{};
   p.w = w;
+  p.imp = imp;
   p.out = *out;
   p.err = err;
   p.seed_lo = seed_lo;
@@ -251,8 +292,13 @@ extern "C" int32_t nslm_seed_search(const float *w, const nslm_seed_matrix *out,
   const int64_t grid = (int64_t)out->N * ((p.nb + kSearchGroup - 1) / kSearchGroup);
   if (grid > 0x7FFFFFFF) return NSLM_ERR_SHAPE;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  if (out->P == 4) seed_search_kernel<4><<<(unsigned)grid, kSearchThreads, 0, s>>>(p);
-  else seed_search_kernel<3><<<(unsigned)grid, kSearchThreads, 0, s>>>(p);
+  if (out->P == 4) {
+    if (imp) seed_search_kernel<4, true><<<(unsigned)grid, kSearchThreads, 0, s>>>(p);
+    else seed_search_kernel<4, false><<<(unsigned)grid, kSearchThreads, 0, s>>>(p);
+  } else {
+    if (imp) seed_search_kernel<3, true><<<(unsigned)grid, kSearchThreads, 0, s>>>(p);
+    else seed_search_kernel<3, false><<<(unsigned)grid, kSearchThreads, 0, s>>>(p);
+  }
   st = launch_status();
   if (st == NSLM_OK) g_launches = 1;
   return st;

@@ -72,7 +72,7 @@ def _load():
         "nslm_moe_seed_ffn_static": (i32, [mp, mp, mp, i32, vp, vp, vp, i32, i32, vp, vp]),
         "nslm_moe_stack_decode": (i32, [ctypes.POINTER(nslm_moe_layer), i32, i32, i32, vp, vp, i32,
                                         vp, vp, sz, vp]),
-        "nslm_seed_search": (i32, [vp, mp, i32, i32, vp, vp]),
+        "nslm_seed_search": (i32, [vp, vp, mp, i32, i32, vp, vp]),
         "nslm_debug_decompress": (i32, [mp, vp, vp]),
         "nslm_debug_decompress_bf16": (i32, [mp, vp, vp]),
         "nslm_status_string": (ctypes.c_char_p, [i32]),
@@ -195,10 +195,11 @@ def nslm_moe_stack_decode(layers, L: int, E: int, k: int, logits, x0_bf16, T: in
                                       ws_bytes, _s(stream)))
 
 
-def nslm_seed_search(w, out, seed_lo: int = 1, seed_hi: int = 65535, err=None, stream=None) -> None:
-    """Encode fp32 weights w [N][K] into `out` (seeds/coefs/codes written, exp_bias read)."""
-    _check("nslm_seed_search", _lib.nslm_seed_search(_p(w), ctypes.byref(_mat(out)), seed_lo, seed_hi,
-                                                      _p(err), _s(stream)))
+def nslm_seed_search(w, out, seed_lo: int = 1, seed_hi: int = 65535, err=None, stream=None, imp=None) -> None:
+    """Encode fp32 weights w [N][K] into `out` (seeds/coefs/codes written, exp_bias read);
+    imp: optional fp32 [K] importances weighting the error (None: unweighted)."""
+    _check("nslm_seed_search", _lib.nslm_seed_search(_p(w), _p(imp), ctypes.byref(_mat(out)), seed_lo,
+                                                      seed_hi, _p(err), _s(stream)))
 
 
 def nslm_debug_decompress(W, w_out, stream=None) -> None:

@@ -96,9 +96,9 @@ def test_search_argument_checks():
     f = nslm.raw().nslm_seed_search
     W = _mat(N=4, K=32, P=4)
     w = 0x9000000
-    assert f(w, ctypes.byref(W), 0, 10, 0, 0) == nslm.NSLM_ERR_ARG        # seeds start at 1
-    assert f(w, ctypes.byref(W), 10, 65536, 0, 0) == nslm.NSLM_ERR_ARG    # 16-bit seeds
-    assert f(w, ctypes.byref(W), 20, 10, 0, 0) == nslm.NSLM_ERR_ARG       # empty range
-    assert f(0, ctypes.byref(W), 1, 10, 0, 0) == nslm.NSLM_ERR_ARG        # no weights
-    assert f(w, ctypes.byref(_mat(N=4, K=24, P=4)), 1, 10, 0, 0) == nslm.NSLM_ERR_SHAPE
-    assert f(w, None, 1, 10, 0, 0) == nslm.NSLM_ERR_ARG
+    assert f(w, 0, ctypes.byref(W), 0, 10, 0, 0) == nslm.NSLM_ERR_ARG        # seeds start at 1
+    assert f(w, 0, ctypes.byref(W), 10, 65536, 0, 0) == nslm.NSLM_ERR_ARG    # 16-bit seeds
+    assert f(w, 0, ctypes.byref(W), 20, 10, 0, 0) == nslm.NSLM_ERR_ARG       # empty range
+    assert f(0, 0, ctypes.byref(W), 1, 10, 0, 0) == nslm.NSLM_ERR_ARG        # no weights
+    assert f(w, 0, ctypes.byref(_mat(N=4, K=24, P=4)), 1, 10, 0, 0) == nslm.NSLM_ERR_SHAPE
+    assert f(w, 0, None, 1, 10, 0, 0) == nslm.NSLM_ERR_ARG

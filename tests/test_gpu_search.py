@@ -47,21 +47,24 @@ class _Out:
         return s, c, code
 
 
-def _run(nslm, w, P, bias, lo, hi):
+def _run(nslm, w, P, bias, lo, hi, imp=None):
     N, K = w.shape
     out = _Out(N, K, P, bias)
     err = torch.full((N, K // 8), float("nan"), dtype=torch.float64, device="cuda")
-    nslm.nslm_seed_search(torch.as_tensor(w, dtype=torch.float32).cuda(), out, lo, hi, err)
+    dimp = None if imp is None else torch.as_tensor(imp, dtype=torch.float32).cuda()
+    nslm.nslm_seed_search(torch.as_tensor(w, dtype=torch.float32).cuda(), out, lo, hi, err, imp=dimp)
     torch.cuda.synchronize()
     s, c, code = out.fields()
     return s, c, code, err.cpu().numpy()
 
 
-def _compare_with_oracle(w, P, bias, lo, hi, s, c, code, err):
+def _compare_with_oracle(w, P, bias, lo, hi, s, c, code, err, imp=None):
     N, K = w.shape
     for i in range(N):
         for b in range(K // 8):
-            rs, rc, rcode, rerr = O.search_block(w[i, 8 * b:8 * b + 8].astype(np.float64), P, int(bias[i]), lo, hi)
+            d8 = None if imp is None else np.asarray(imp[8 * b:8 * b + 8], np.float32).astype(np.float64)
+            rs, rc, rcode, rerr = O.search_block(w[i, 8 * b:8 * b + 8].astype(np.float64), P, int(bias[i]), lo, hi,
+                                                 d8=d8)
             assert (s[i, b], code[i, b]) == (rs, rcode), (i, b, s[i, b], code[i, b], rs, rcode)
             assert np.array_equal(c[i, b], rc), (i, b)
             assert err[i, b] == rerr, (i, b, err[i, b], rerr)  # bit-identical fp64
@@ -103,6 +106,42 @@ def test_search_matches_oracle_on_gaussian_weights(nslm, P, bias):
     lo, hi = 1000, 2999
     s, c, code, err = _run(nslm, w, P, bias, lo, hi)
     _compare_with_oracle(w, P, bias, lo, hi, s, c, code, err)
+
+
+@pytest.mark.parametrize("P,bias", [(3, [-12, -40]), (4, [-12, 60])])
+def test_weighted_search_matches_oracle(nslm, P, bias):
+    # per-column importances (mean square activations): the weighted fit and
+    # error, bit for bit
+    rng = np.random.default_rng(150 + P)
+    N, K = 2, 32
+    w = np.zeros((N, K), np.float32)
+    for i in range(N):
+        w[i] = (rng.standard_normal(K) * 2.0 ** (bias[i] + 14)).astype(np.float32)
+    imp = rng.uniform(0.01, 5.0, K).astype(np.float32)
+    imp[3] = 0.0  # a column that does not count
+    lo, hi = 2000, 3999
+    s, c, code, err = _run(nslm, w, P, bias, lo, hi, imp)
+    _compare_with_oracle(w, P, bias, lo, hi, s, c, code, err, imp)
+
+
+@pytest.mark.parametrize("P", [3, 4])
+def test_weighted_search_recovers_planted_blocks(nslm, P):
+    rng = np.random.default_rng(160 + P)
+    N, K = 1, 32
+    w = np.zeros((N, K), np.float32)
+    planted = []
+    for b in range(K // 8):
+        seed = int(rng.integers(1, 65536))
+        c = rng.integers(-8, 8, size=P).astype(np.int32)
+        c[0] = 2 * int(rng.integers(-4, 4)) + 1
+        code = int(rng.integers(0, 16))
+        w[0, 8 * b:8 * b + 8] = O.regen_block(seed, c, code, -12)
+        planted.append((b, seed, c, code))
+    s, c, code, err = _run(nslm, w, P, [-12], 1, 65535, rng.uniform(0.1, 8.0, K))
+    for b, seed, cc, cd in planted:
+        assert (s[0, b], code[0, b]) == (seed, cd)
+        assert np.array_equal(c[0, b], cc)
+        assert err[0, b] == 0.0
 
 
 def test_search_full_range_matches_oracle(nslm):
