@@ -347,3 +347,61 @@ def elementwise_rel_err(y, y_ref, floor: float = 1e-3) -> float:
 
 __all__ = [n for n in dir() if not n.startswith("_")
            and n not in ("np", "math", "ctypes", "os", "annotations")]
+
+
+# ------------------------------------------------------- the nibbles layout
+
+def blocks_from_streams(m):
+    """Per-block fields (c [N][nb][P] signed, code [N][nb]) of a packed matrix in
+    this library's streams: c_j in bits 4j..4j+3 of the coefs word; P=4 codes
+    in the codes stream (block 2m low nibble, 2m+1 high), P=3 in coefs bits 12..15."""
+    seeds, coefs, codes, eb, N, K, P = _fields(m)
+    nb = K // 8
+    c = np.zeros((N, nb, P), np.int64)
+    code = np.zeros((N, nb), np.int64)
+    for i in range(N):
+        for b in range(nb):
+            q = int(coefs[i, b])
+            for j in range(P):
+                c[i, b, j] = (((q >> (4 * j)) & 0xF) ^ 8) - 8
+            if P == 4:
+                code[i, b] = (int(codes[i, b // 2]) >> (4 * (b % 2))) & 0xF
+            else:
+                code[i, b] = (q >> 12) & 0xF
+    return c, code
+
+
+def nibbles_from_blocks(c, code, P: int) -> np.ndarray:
+    """The "nibbles" stream of packed rows ([QWEN] "Files": the routed experts are
+    NAME.seeds, NAME.nibbles and NAME.exp_bias).  Reading: block b of a row holds
+    nibbles (P+1)b .. (P+1)b+P, namely c_0 .. c_{P-1} as two's-complement
+    nibbles and then the exponent code; nibble n of a row is in byte n // 2,
+    the low half for even n.  That is 2.5 bytes per block for P=4 and 2 for
+    P=3, the pages' 4.5 and 4.0 bits per weight with the 16-bit seed."""
+    code = np.asarray(code)
+    N, nb = code.shape
+    out = np.zeros((N, (P + 1) * nb // 2), np.uint8)
+    for i in range(N):
+        for b in range(nb):
+            vals = [int(c[i][b][j]) & 0xF for j in range(P)] + [int(code[i][b])]
+            for j, v in enumerate(vals):
+                n = (P + 1) * b + j
+                out[i, n // 2] |= v << (4 * (n % 2))
+    return out
+
+
+def blocks_from_nibbles(nib, N: int, K: int, P: int):
+    """Inverse of nibbles_from_blocks: (c [N][nb][P], code [N][nb])."""
+    nib = np.asarray(nib, np.uint8).reshape(N, -1)
+    nb = K // 8
+    c = np.zeros((N, nb, P), np.int64)
+    code = np.zeros((N, nb), np.int64)
+    for i in range(N):
+        for b in range(nb):
+            vals = []
+            for j in range(P + 1):
+                n = (P + 1) * b + j
+                vals.append((int(nib[i, n // 2]) >> (4 * (n % 2))) & 0xF)
+            c[i, b] = [(v ^ 8) - 8 for v in vals[:P]]
+            code[i, b] = vals[P]
+    return c, code

@@ -393,3 +393,35 @@ def test_weighting_changes_the_choice():
     fit = lambda s_, c_, code_: abs(w[5] - O.regen_block(s_, c_, code_, -12)[5])
     assert (s, code) != (sw, codew)
     assert fit(sw, cw, codew) < fit(s, c, code)
+
+
+# ---- the nibbles layout (seeds, nibbles, exp_bias)
+
+def test_nibbles_layout_matches_hand_encoded_rows():
+    n = 0
+    for line in _read_rows("nibbles_examples.txt"):
+        P, blocks, hexs = [t.strip() for t in line.split("|")]
+        P = int(P)
+        cs, cds = [], []
+        for blk in blocks.split():
+            cc, cd = blk.split(":")
+            cs.append([int(v) for v in cc.split(",")])
+            cds.append(int(cd))
+        nib = O.nibbles_from_blocks([cs], [cds], P)
+        assert [int(v, 16) for v in hexs.split()] == nib[0].tolist()
+        c, code = O.blocks_from_nibbles(nib, 1, 8 * len(cs), P)
+        assert c[0].tolist() == cs and code[0].tolist() == cds
+        n += 1
+    assert n == 4
+
+
+@pytest.mark.parametrize("P", [3, 4])
+def test_nibbles_round_trip_and_p3_identity(P):
+    m = synth.seed_matrix(5, 64, P, (700, P))
+    c, code = O.blocks_from_streams(m)
+    nib = O.nibbles_from_blocks(c, code, P)
+    assert nib.shape == (5, (P + 1) * 8 // 2)
+    c2, code2 = O.blocks_from_nibbles(nib, 5, 64, P)
+    assert np.array_equal(c, c2) and np.array_equal(code, code2)
+    if P == 3:  # 4 nibbles per block in the same order as the coefs word
+        assert np.array_equal(nib, m.coefs.numpy().view(np.uint16).astype("<u2").view(np.uint8).reshape(5, -1))
