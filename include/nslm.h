@@ -220,6 +220,21 @@ int32_t nslm_moe_stack_decode(const nslm_moe_layer *layers, int32_t L, int32_t E
 int32_t nslm_seed_search(const float *w, const float *imp, const nslm_seed_matrix *out,
                          int32_t seed_lo, int32_t seed_hi, double *err, nslm_stream_t stream);
 
+/* The "nibbles" layout of seed packs ("Qwen3.8-Flash-Next-NanoSeedLM-P4",
+ * "Files": routed experts as NAME.seeds, NAME.nibbles and NAME.exp_bias).
+ * nibbles: u8 [N][(P+1) * K / 16], device; block b of a row holds nibbles
+ * (P+1)b .. (P+1)b+P, namely c_0 .. c_{P-1} (two's complement) and then the
+ * exponent code, nibble n in byte n / 2 (low half for even n).  Seeds and
+ * exp_bias are the same streams in both layouts.
+ * nslm_unpack_nibbles WRITES out->coefs (and out->codes for P = 4) from the
+ * nibbles (out->seeds and out->exp_bias are not touched);
+ * nslm_pack_nibbles READS in->coefs (and in->codes) and WRITES nibbles.
+ * For P = 3 the two layouts are the same bytes.  Shapes as for any matrix
+ * (K % 8 == 0; P = 4: K % 16 == 0 and codes present).  One launch; buffers
+ * must not overlap. */
+int32_t nslm_unpack_nibbles(const uint8_t *nibbles, const nslm_seed_matrix *out, nslm_stream_t stream);
+int32_t nslm_pack_nibbles(const nslm_seed_matrix *in, uint8_t *nibbles, nslm_stream_t stream);
+
 /* Test exports: the regenerated weights themselves, written out densely.
  * w_out: fp32 [N][K] (exact) or bf16 bit patterns [N][K] (round to nearest
  * even of the exact value).  Not on the hot path. */

@@ -73,6 +73,8 @@ def _load():
         "nslm_moe_stack_decode": (i32, [ctypes.POINTER(nslm_moe_layer), i32, i32, i32, vp, vp, i32,
                                         vp, vp, sz, vp]),
         "nslm_seed_search": (i32, [vp, vp, mp, i32, i32, vp, vp]),
+        "nslm_unpack_nibbles": (i32, [vp, mp, vp]),
+        "nslm_pack_nibbles": (i32, [mp, vp, vp]),
         "nslm_debug_decompress": (i32, [mp, vp, vp]),
         "nslm_debug_decompress_bf16": (i32, [mp, vp, vp]),
         "nslm_status_string": (ctypes.c_char_p, [i32]),
@@ -200,6 +202,16 @@ def nslm_seed_search(w, out, seed_lo: int = 1, seed_hi: int = 65535, err=None, s
     imp: optional fp32 [K] importances weighting the error (None: unweighted)."""
     _check("nslm_seed_search", _lib.nslm_seed_search(_p(w), _p(imp), ctypes.byref(_mat(out)), seed_lo,
                                                       seed_hi, _p(err), _s(stream)))
+
+
+def nslm_unpack_nibbles(nibbles, out, stream=None) -> None:
+    """Write out's coefs (and codes) from a nibbles stream u8 [N][(P+1)*K/16]."""
+    _check("nslm_unpack_nibbles", _lib.nslm_unpack_nibbles(_p(nibbles), ctypes.byref(_mat(out)), _s(stream)))
+
+
+def nslm_pack_nibbles(W, nibbles, stream=None) -> None:
+    """Write the nibbles stream u8 [N][(P+1)*K/16] of W's coefs (and codes)."""
+    _check("nslm_pack_nibbles", _lib.nslm_pack_nibbles(ctypes.byref(_mat(W)), _p(nibbles), _s(stream)))
 
 
 def nslm_debug_decompress(W, w_out, stream=None) -> None:

@@ -102,3 +102,15 @@ def test_search_argument_checks():
     assert f(0, 0, ctypes.byref(W), 1, 10, 0, 0) == nslm.NSLM_ERR_ARG        # no weights
     assert f(w, 0, ctypes.byref(_mat(N=4, K=24, P=4)), 1, 10, 0, 0) == nslm.NSLM_ERR_SHAPE
     assert f(w, 0, None, 1, 10, 0, 0) == nslm.NSLM_ERR_ARG
+
+
+def test_nibbles_argument_checks():
+    up, pk = nslm.raw().nslm_unpack_nibbles, nslm.raw().nslm_pack_nibbles
+    nib = 0x9000000
+    assert up(0, ctypes.byref(_mat(N=4, K=32, P=4)), 0) == nslm.NSLM_ERR_ARG
+    assert up(nib, None, 0) == nslm.NSLM_ERR_ARG
+    assert up(nib, ctypes.byref(_mat(N=4, K=32, P=4, codes=False)), 0) == nslm.NSLM_ERR_ARG
+    assert up(nib, ctypes.byref(_mat(N=4, K=24, P=4)), 0) == nslm.NSLM_ERR_SHAPE
+    assert pk(ctypes.byref(_mat(N=4, K=32, P=5)), nib, 0) == nslm.NSLM_ERR_SHAPE
+    assert pk(ctypes.byref(_mat(N=0, K=32, P=4)), nib, 0) == nslm.NSLM_OK    # empty: nothing to do
+
