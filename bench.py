@@ -352,6 +352,65 @@ def stack_batch_leg(torch, nslm, synth, dev, arr, hbm, T: int, steps: int, rank:
             "note": "one cooperative launch for all 45 layers (plus the routing launch); inputs > L2"}
 
 
+def host_experts_leg(torch, nslm, synth, dev, n_layers: int = 8, slots: int = 400, tokens: int = 32):
+    """One-token decode with the routed experts in pinned host memory behind the
+    VRAM expert cache (LRU, copies by the device from host memory): per token and
+    layer, routing + cache fetch + the FFN on the cache.  8 layers x 100 experts
+    (3.9 GB pinned) behind 400 slots, so about half the experts fit."""
+    def pinned(m):
+        return synth.SeedMatrix(m.seeds.pin_memory(), m.coefs.pin_memory(), m.codes.pin_memory(),
+                                m.exp_bias.pin_memory(), m.rows, m.K, m.P, m.n_experts)
+
+    def empty(rows, K):
+        nb = K // 8
+        return synth.SeedMatrix(torch.zeros(slots * rows, nb, dtype=torch.int16, device=dev),
+                                torch.zeros(slots * rows, nb, dtype=torch.int16, device=dev),
+                                torch.zeros(slots * rows, nb // 2, dtype=torch.uint8, device=dev),
+                                torch.zeros(slots * rows, dtype=torch.int32, device=dev), rows, K, P, slots)
+
+    host = []
+    for l in range(n_layers):
+        m = synth.moe_layer(l, E, HIDDEN, INTER, P, config=4)
+        host.append(tuple(pinned(getattr(m, n)) for n in ("gate", "up", "down")))
+    cache = (empty(INTER, HIDDEN), empty(INTER, HIDDEN), empty(HIDDEN, INTER))
+    state = torch.zeros(nslm.nslm_expert_cache_state_bytes(slots), dtype=torch.uint8, device=dev)
+    wsb = nslm.nslm_workspace_bytes(nslm.NSLM_OP_MOE_FFN, 1, slots, HIDDEN, INTER, K_TOP)
+    ws = torch.empty(wsb, dtype=torch.uint8, device=dev)
+    warm = 16
+    logits = [[synth.router_logits((4, l, 0, t), 1, E).to(dev) for l in range(n_layers)] for t in range(warm + tokens)]
+    x = synth.activations((4, 0, 0), 1, HIDDEN).to(dev)
+    ids = torch.empty(1, K_TOP, dtype=torch.int32, device=dev)
+    w = torch.empty(1, K_TOP, device=dev)
+    sl = torch.empty(1, K_TOP, dtype=torch.int32, device=dev)
+    y = torch.empty(1, HIDDEN, device=dev)
+
+    def token(t):
+        for l in range(n_layers):
+            nslm.nslm_moe_route_topk(logits[t][l], 1, E, K_TOP, ids, w)
+            nslm.nslm_expert_cache_fetch(host[l], E, l, cache, slots, state, ids, 1, K_TOP, sl)
+            nslm.nslm_moe_seed_ffn(cache[0], cache[1], cache[2], slots, x, sl, w, 1, K_TOP, y, ws, wsb)
+
+    for t in range(warm):
+        token(t)
+    torch.cuda.synchronize()
+    st0 = state[:16].view(torch.int32).cpu().tolist()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for t in range(warm, warm + tokens):
+        token(t)
+    e1.record()
+    torch.cuda.synchronize()
+    st1 = state[:16].view(torch.int32).cpu().tolist()
+    dt = e0.elapsed_time(e1) * 1e-3
+    hits, miss = st1[2] - st0[2], st1[3] - st0[3]
+    per_expert = layer_packed_bytes_per_token() / K_TOP
+    return {"workload": f"{n_layers} layers x {E} experts (P=4, 2048/1408) in pinned host memory, "
+                        f"{slots}-slot VRAM expert cache, one token per step",
+            "tokens_per_s": round(tokens / dt, 1), "ms_per_token": round(dt / tokens * 1e3, 3),
+            "hit_rate": round(hits / max(1, hits + miss), 3), "misses_per_token": round(miss / tokens, 2),
+            "copy_GB_per_s": round(miss * per_expert / dt / 1e9, 1)}
+
+
 def search_leg(torch, nslm, dev, with_cpu: bool):
     """Seed search (the encoder) over all 65,535 seeds x 16 codes: GPU blocks/s
     on a 64 x 2048 fp32 matrix (16,384 blocks, P=4), and the oracle's time per
@@ -447,6 +506,7 @@ def main():
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--no-search", action="store_true")
     ap.add_argument("--no-batch8", action="store_true", help="skip the 8-token stack leg")
+    ap.add_argument("--no-host-experts", action="store_true", help="skip the host-memory expert cache leg")
     ap.add_argument("--profile", choices=["layer", "layer8", "batched", "gemv", "search"],
                     help="run a small fixed workload for an ncu capture and exit")
     args = ap.parse_args()
@@ -601,6 +661,10 @@ def main():
     if T == 1 and not args.no_batch8:
         batch8 = stack_batch_leg(torch, nslm, synth, dev, arr, hbm, 8, max(10, args.steps // 4), rank)
 
+    host_experts = None
+    if T == 1 and not args.no_host_experts:
+        host_experts = host_experts_leg(torch, nslm, synth, dev)
+
     search = None
     if not args.no_search:
         search = search_leg(torch, nslm, dev, with_cpu=(rank == 0 and not args.no_cpu))
@@ -627,6 +691,8 @@ def main():
         line["batched"] = batched
     if batch8 is not None:
         line["stack_batch8"] = batch8
+    if host_experts is not None:
+        line["host_experts"] = host_experts
     if search is not None:
         line["seed_search"] = search
     if rank == 0 and world == 1 and not args.no_cpu:

@@ -220,6 +220,37 @@ int32_t nslm_moe_stack_decode(const nslm_moe_layer *layers, int32_t L, int32_t E
 int32_t nslm_seed_search(const float *w, const float *imp, const nslm_seed_matrix *out,
                          int32_t seed_lo, int32_t seed_hi, double *err, nslm_stream_t stream);
 
+/* Routed experts in host memory behind a VRAM cache of recently used experts
+ * ("NanoSeedLM" README, "Highlights": the CUDA engine can keep the routed
+ * experts in RAM while a VRAM cache holds the recently used ones; LRU was the
+ * pages' best policy).  One call prepares one layer's decode step:
+ *   - a one-CTA kernel runs LRU over the routed pairs ids [T][k] (device, in
+ *     order): a hit refreshes the slot; a miss takes the least recently used
+ *     slot not used in this step (empty slots first, then the oldest, ties to
+ *     the lower slot) and schedules a copy; slot_ids [T][k] (device) gets the
+ *     slot of every pair (-1 for ids outside [0, E));
+ *   - a copy kernel moves each missed expert's gate, up and down fields from
+ *     the source stacks into its slot.
+ * Then nslm_moe_seed_ffn(gate_cache, up_cache, down_cache, S, x, slot_ids, w,
+ * ...) computes the layer.  No host synchronisation; graph-capturable.
+ * *_src: the layer's E experts stacked as for nslm_moe_seed_ffn, in memory the
+ * device can read: device memory, or pinned host memory (cudaHostAlloc /
+ * cudaHostRegister) under unified addressing.  *_cache: S expert slots
+ * stacked the same way, device memory, same hidden / inter / P.  Cache keys
+ * are (layer, expert), so one cache can serve every layer of a stack.
+ * state: device, nslm_expert_cache_state_bytes(S) bytes, zero-filled before
+ * first use (an empty cache); int32 [0] calls so far, [1] copies of the last
+ * call, [2] total hits, [3] total misses.  Needs T * k <= S <= 4096,
+ * T * k <= 64, hidden and inter multiples of 64, 16-byte aligned streams.
+ * Two launches. */
+size_t nslm_expert_cache_state_bytes(int32_t slots);
+int32_t nslm_expert_cache_fetch(const nslm_seed_matrix *gate_src, const nslm_seed_matrix *up_src,
+                                const nslm_seed_matrix *down_src, int32_t E, int32_t layer,
+                                const nslm_seed_matrix *gate_cache, const nslm_seed_matrix *up_cache,
+                                const nslm_seed_matrix *down_cache, int32_t S, void *state,
+                                const int32_t *ids, int32_t T, int32_t k, int32_t *slot_ids,
+                                nslm_stream_t stream);
+
 /* The "nibbles" layout of seed packs ("Qwen3.8-Flash-Next-NanoSeedLM-P4",
  * "Files": routed experts as NAME.seeds, NAME.nibbles and NAME.exp_bias).
  * nibbles: u8 [N][(P+1) * K / 16], device; block b of a row holds nibbles

@@ -73,6 +73,8 @@ def _load():
         "nslm_moe_stack_decode": (i32, [ctypes.POINTER(nslm_moe_layer), i32, i32, i32, vp, vp, i32,
                                         vp, vp, sz, vp]),
         "nslm_seed_search": (i32, [vp, vp, mp, i32, i32, vp, vp]),
+        "nslm_expert_cache_state_bytes": (sz, [i32]),
+        "nslm_expert_cache_fetch": (i32, [mp, mp, mp, i32, i32, mp, mp, mp, i32, vp, vp, i32, i32, vp, vp]),
         "nslm_unpack_nibbles": (i32, [vp, mp, vp]),
         "nslm_pack_nibbles": (i32, [mp, vp, vp]),
         "nslm_debug_decompress": (i32, [mp, vp, vp]),
@@ -202,6 +204,19 @@ def nslm_seed_search(w, out, seed_lo: int = 1, seed_hi: int = 65535, err=None, s
     imp: optional fp32 [K] importances weighting the error (None: unweighted)."""
     _check("nslm_seed_search", _lib.nslm_seed_search(_p(w), _p(imp), ctypes.byref(_mat(out)), seed_lo,
                                                       seed_hi, _p(err), _s(stream)))
+
+
+def nslm_expert_cache_state_bytes(slots: int) -> int:
+    return int(_lib.nslm_expert_cache_state_bytes(int(slots)))
+
+
+def nslm_expert_cache_fetch(src, E: int, layer: int, cache, S: int, state, ids, T: int, k: int, slot_ids,
+                            stream=None) -> None:
+    """src / cache: (gate, up, down) matrices (host-resident source, device slots)."""
+    g, u, d = (ctypes.byref(_mat(m)) for m in src)
+    gc, uc, dc = (ctypes.byref(_mat(m)) for m in cache)
+    _check("nslm_expert_cache_fetch", _lib.nslm_expert_cache_fetch(g, u, d, E, layer, gc, uc, dc, S, _p(state),
+                                                                    _p(ids), T, k, _p(slot_ids), _s(stream)))
 
 
 def nslm_unpack_nibbles(nibbles, out, stream=None) -> None:

@@ -114,3 +114,27 @@ def test_nibbles_argument_checks():
     assert pk(ctypes.byref(_mat(N=4, K=32, P=5)), nib, 0) == nslm.NSLM_ERR_SHAPE
     assert pk(ctypes.byref(_mat(N=0, K=32, P=4)), nib, 0) == nslm.NSLM_OK    # empty: nothing to do
 
+
+def test_expert_cache_argument_checks():
+    f = nslm.raw().nslm_expert_cache_fetch
+    E, hidden, inter, S = 4, 256, 128, 8
+    src = [_mat(E * inter, hidden), _mat(E * inter, hidden), _mat(E * hidden, inter)]
+    cac = [_mat(S * inter, hidden, base=0x2000000), _mat(S * inter, hidden, base=0x2000000),
+           _mat(S * hidden, inter, base=0x2000000)]
+    st, ids, out = 0x9000000, 0x9100000, 0x9200000
+
+    def call(src=src, cac=cac, E_=E, S_=S, T=1, k=4, state=st, layer=0):
+        a = [ctypes.byref(m) for m in src]
+        c = [ctypes.byref(m) for m in cac]
+        return f(*a, E_, layer, *c, S_, state, ids, T, k, out, 0)
+
+    assert nslm.nslm_expert_cache_state_bytes(0) == 0
+    assert nslm.nslm_expert_cache_state_bytes(8) > 8 * 8
+    assert call(state=0) == nslm.NSLM_ERR_ARG
+    assert call(T=3) == nslm.NSLM_ERR_SHAPE                # T * k > S slots
+    assert call(S_=4097) == nslm.NSLM_ERR_SHAPE
+    assert call(layer=-1) == nslm.NSLM_ERR_SHAPE
+    assert call(E_=3) == nslm.NSLM_ERR_SHAPE               # source rows not divisible by E
+    assert call(cac=[_mat(S * inter, 512), cac[1], cac[2]]) == nslm.NSLM_ERR_SHAPE   # cache shape differs
+    assert call(state=0x9000004) == nslm.NSLM_ERR_ALIGN
+
