@@ -185,9 +185,13 @@ def _seed_stream(key: int, n: int, device) -> torch.Tensor:
 
 def seed_matrix(rows: int, K: int, P: int, tag=(0,), n_experts: int = 1,
                 exp_bias: int = -12, device="cpu") -> SeedMatrix:
-    """Uniform random packed fields for a (stack of) rows x K seed matrix."""
-    if K % (16 if P == 4 else 8) != 0:
-        raise ValueError("K must be a multiple of 16 (P=4) or 8 (P=3)")
+    """Uniform random packed fields for a (stack of) rows x K seed matrix.
+
+    P = 35 is P = 3 with 5-bit coefficients: a uniform coefs word is three
+    uniform 5-bit fields and one uniform code bit, and the codes stream holds
+    3 uniform code bits per block (3K/64 bytes per row)."""
+    if K % {4: 16, 3: 8, 35: 64}[P] != 0:
+        raise ValueError("K must be a multiple of 16 (P=4), 8 (P=3) or 64 (P=35)")
     R = rows * n_experts
     nb = K // 8
     seeds = _seed_stream(stream_key(*tag, FIELD_SEEDS), R * nb, device).reshape(R, nb)
@@ -195,6 +199,8 @@ def seed_matrix(rows: int, K: int, P: int, tag=(0,), n_experts: int = 1,
     codes = None
     if P == 4:
         codes = _u8_stream(stream_key(*tag, FIELD_CODES), R * nb // 2, device).reshape(R, nb // 2)
+    elif P == 35:
+        codes = _u8_stream(stream_key(*tag, FIELD_CODES), R * 3 * nb // 8, device).reshape(R, 3 * nb // 8)
     eb = torch.full((R,), exp_bias, dtype=torch.int32, device=device)
     return SeedMatrix(seeds.contiguous(), coefs.contiguous(),
                       None if codes is None else codes.contiguous(), eb, rows, K, P, n_experts)

@@ -126,6 +126,22 @@ void nslmo_regen_block(uint16_t seed, const int32_t *c, int32_t P, int32_t code,
 
 /* ----------------------------------------------------- the packed streams */
 
+/* P = 35 denotes P = 3 with 5-bit coefficients ([BLOG] "'Four bits is four
+ * bits'": "Seeds, P=3, 5-bit coefficients", 4.375 bits per weight).  Reading
+ * for its 35 bits per block: the seed stream as usual; the coefs word holds
+ * c_0, c_1, c_2 as 5-bit two's complement in bits 0-4, 5-9, 10-14 and bit 0 of
+ * the exponent code in bit 15; a codes stream u8 [N][3 K / 64] holds code bits
+ * 1..3 of block b of a row at bits 3b .. 3b+2 of the row's bit string (byte
+ * 3b / 8 .. , least significant bit first).  K must be a multiple of 64. */
+#define NSLMO_P3C5 35
+
+static int32_t basis_count(int32_t P) { return P == NSLMO_P3C5 ? 3 : P; }
+
+static int fivebit_to_int(unsigned q)
+{
+    return (int)((q & 0x1Fu) ^ 16u) - 16;
+}
+
 /* Unpack block (i, b) of a packed matrix (reading R7, [K2] "This upload"). */
 static void unpack_block(const uint16_t *seeds, const uint16_t *coefs,
                          const uint8_t *codes, int32_t nb, int32_t P, int64_t i,
@@ -133,6 +149,17 @@ static void unpack_block(const uint16_t *seeds, const uint16_t *coefs,
 {
     *seed = seeds[i * nb + b];
     unsigned q = coefs[i * nb + b];
+    if (P == NSLMO_P3C5) {
+        for (int j = 0; j < 3; ++j) c[j] = fivebit_to_int(q >> (5 * j));
+        const uint8_t *row = codes + i * (3 * nb / 8);
+        unsigned hi = 0;
+        for (int t = 0; t < 3; ++t) {
+            int64_t bit = 3 * b + t;
+            hi |= ((row[bit / 8] >> (bit % 8)) & 1u) << t;
+        }
+        *code = (int32_t)(((q >> 15) & 1u) | (hi << 1));
+        return;
+    }
     for (int j = 0; j < P; ++j) c[j] = nibble_to_int(q >> (4 * j));
     if (P == 4) {
         unsigned byte = codes[i * (nb / 2) + b / 2];
@@ -144,9 +171,10 @@ static void unpack_block(const uint16_t *seeds, const uint16_t *coefs,
 
 static int check_shape(int32_t N, int32_t K, int32_t P)
 {
-    if (N < 0 || K < 0 || (P != 3 && P != 4)) return NSLMO_ERR_ARG;
+    if (N < 0 || K < 0 || (P != 3 && P != 4 && P != NSLMO_P3C5)) return NSLMO_ERR_ARG;
     if (K % 8 != 0) return NSLMO_ERR_ARG;
     if (P == 4 && K % 16 != 0) return NSLMO_ERR_ARG;
+    if (P == NSLMO_P3C5 && K % 64 != 0) return NSLMO_ERR_ARG;
     return NSLMO_OK;
 }
 
@@ -163,7 +191,7 @@ int32_t nslmo_decompress_f64(const uint16_t *seeds, const uint16_t *coefs,
             uint16_t seed;
             int32_t c[4], code;
             unpack_block(seeds, coefs, codes, nb, P, i, b, &seed, c, &code);
-            nslmo_regen_block(seed, c, P, code, exp_bias[i], &w_out[i * K + 8 * b]);
+            nslmo_regen_block(seed, c, basis_count(P), code, exp_bias[i], &w_out[i * K + 8 * b]);
         }
     }
     return NSLMO_OK;
@@ -185,7 +213,7 @@ int32_t nslmo_decompress_f32(const uint16_t *seeds, const uint16_t *coefs,
             int32_t c[4], code;
             double w8[8];
             unpack_block(seeds, coefs, codes, nb, P, i, b, &seed, c, &code);
-            nslmo_regen_block(seed, c, P, code, exp_bias[i], w8);
+            nslmo_regen_block(seed, c, basis_count(P), code, exp_bias[i], w8);
             for (int r = 0; r < 8; ++r) {
                 float f = (float)w8[r];
                 if ((double)f != w8[r]) inexact = 1;
@@ -258,7 +286,7 @@ int32_t nslmo_seed_matvec(const uint16_t *seeds, const uint16_t *coefs,
                 int32_t c[4], code;
                 double w8[8];
                 unpack_block(seeds, coefs, codes, nb, P, i, b, &seed, c, &code);
-                nslmo_regen_block(seed, c, P, code, exp_bias[i], w8);
+                nslmo_regen_block(seed, c, basis_count(P), code, exp_bias[i], w8);
                 for (int r = 0; r < 8; ++r)
                     acc += w8[r] * nslmo_bf16_to_f64(x_bf16[(int64_t)m * K + 8 * b + r]);
             }
@@ -286,7 +314,7 @@ int32_t nslmo_seed_matvec_bf16w(const uint16_t *seeds, const uint16_t *coefs,
                 int32_t c[4], code;
                 double w8[8];
                 unpack_block(seeds, coefs, codes, nb, P, i, b, &seed, c, &code);
-                nslmo_regen_block(seed, c, P, code, exp_bias[i], w8);
+                nslmo_regen_block(seed, c, basis_count(P), code, exp_bias[i], w8);
                 for (int r = 0; r < 8; ++r)
                     acc += nslmo_bf16_to_f64(nslmo_f64_to_bf16(w8[r])) *
                            x[(int64_t)m * K + 8 * b + r];
@@ -346,10 +374,10 @@ static void expert_matvec(const nslmo_stack *S, int32_t rows, int32_t K, int32_t
                           int32_t e, const double *x, int bf16_weights, double *y)
 {
     int32_t nb = K / 8;
-    int64_t ncodes = (P == 4) ? (int64_t)rows * (nb / 2) : 0;
+    int64_t ncodes = (P == 4) ? (int64_t)rows * (nb / 2) : (P == NSLMO_P3C5 ? (int64_t)rows * (3 * nb / 8) : 0);
     const uint16_t *sd = S->seeds + (int64_t)e * rows * nb;
     const uint16_t *cf = S->coefs + (int64_t)e * rows * nb;
-    const uint8_t *cd = (P == 4) ? S->codes + (int64_t)e * ncodes : NULL;
+    const uint8_t *cd = (P == 4 || P == NSLMO_P3C5) ? S->codes + (int64_t)e * ncodes : NULL;
     const int32_t *eb = S->exp_bias + (int64_t)e * rows;
 #pragma omp parallel for schedule(static)
     for (int64_t i = 0; i < rows; ++i) {
@@ -359,7 +387,7 @@ static void expert_matvec(const nslmo_stack *S, int32_t rows, int32_t K, int32_t
             int32_t c[4], code;
             double w8[8];
             unpack_block(sd, cf, cd, nb, P, i, b, &seed, c, &code);
-            nslmo_regen_block(seed, c, P, code, eb[i], w8);
+            nslmo_regen_block(seed, c, basis_count(P), code, eb[i], w8);
             for (int r = 0; r < 8; ++r) {
                 double wr = bf16_weights ? nslmo_bf16_to_f64(nslmo_f64_to_bf16(w8[r])) : w8[r];
                 acc += wr * x[8 * b + r];

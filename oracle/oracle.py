@@ -149,10 +149,13 @@ def regen_block(seed: int, c, code: int, bias: int) -> np.ndarray:
 
 # ------------------------------------------------------------------ packing
 
+P3C5 = 35  # P = 3 with 5-bit coefficients (see the C oracle for its layout)
+
+
 def packed_bytes(N: int, K: int, P: int) -> int:
     """Packed bytes of one matrix: streams plus the per-row int32 bias."""
     nb = K // 8
-    per_block = 4.5 if P == 4 else 4.0
+    per_block = {4: 4.5, 3: 4.0, P3C5: 4.375}[P]
     return int(N * nb * per_block) + 4 * N
 
 
@@ -160,7 +163,7 @@ def _fields(m):
     P = int(m.P)
     seeds = np.ascontiguousarray(m.seeds, np.uint16)
     coefs = np.ascontiguousarray(m.coefs, np.uint16)
-    codes = None if P == 3 else np.ascontiguousarray(m.codes, np.uint8)
+    codes = None if P == 3 else np.ascontiguousarray(m.codes, np.uint8)  # P=4: [N][K/16]; P3C5: [N][3K/64]
     eb = np.ascontiguousarray(m.exp_bias, np.int32)
     N = seeds.shape[0]
     K = seeds.shape[1] * 8

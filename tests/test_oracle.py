@@ -425,3 +425,37 @@ def test_nibbles_round_trip_and_p3_identity(P):
     assert np.array_equal(c, c2) and np.array_equal(code, code2)
     if P == 3:  # 4 nibbles per block in the same order as the coefs word
         assert np.array_equal(nib, m.coefs.numpy().view(np.uint16).astype("<u2").view(np.uint8).reshape(5, -1))
+
+
+# ---- P = 3 with 5-bit coefficients (P = 35)
+
+def test_p3c5_layout_matches_hand_encoded_blocks():
+    n = 0
+    for line in _read_rows("p3c5_examples.txt"):
+        q, row, b, bias, fields, weight = [t.strip() for t in line.split("|")]
+        b, bias = int(b), int(bias)
+        m = synth.seed_matrix(1, 64, 35, (720,))
+        m.seeds.zero_()
+        m.coefs.zero_()
+        m.coefs[0, b] = int(np.array(int(q, 16), np.uint16).view(np.int16))
+        m.codes[0] = torch.tensor([int(v, 16) for v in row.split()], dtype=torch.uint8)
+        m.exp_bias.fill_(bias)
+        w = O.decompress(m, np.float64)[0].reshape(8, 8)
+        assert np.all(w[b] == float(weight)), (line, w[b])
+        c0, c1, c2, code = (int(v) for v in fields.split())
+        assert float(weight) == -2.0 ** (code + bias) * (c0 + c1 + c2)
+        others = [i for i in range(8) if i != b]
+        assert np.all(w[others] == 0.0)  # zero coefficients, whatever their codes
+        n += 1
+    assert n == 3
+
+
+def test_p3c5_matvec_equals_dense_product_and_reaches_5bit_values():
+    m = synth.seed_matrix(16, 128, 35, (721,))
+    x = synth.activations((721,), 2, 128)
+    xb = synth.bf16_bits(x).numpy().view(np.uint16)
+    w = O.decompress(m, np.float64)
+    assert O.normwise_rel_err(O.seed_matvec(m, xb), O.dense_matvec(w, O.bf16_to_f64(xb))) <= 1e-14
+    # coefficients beyond the int4 range occur: |sum_j c_j U| reaches 3 * 16
+    assert np.max(np.abs(w)) * 2.0 ** 12 > 24.0
+
