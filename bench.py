@@ -213,7 +213,7 @@ def job_throughput(world: int, steps: int, tokens_per_step: int, elapsed_s: floa
 
 def gemv_sweep(torch, nslm, synth, dev, hbm):
     out = []
-    for Pv in (4, 3):
+    for Pv in (4, 3, 35):  # 35: P = 3 with 5-bit coefficients
         for (N, K) in GEMV_SHAPES:
             m0 = synth.seed_matrix(N, K, Pv, (11, N, K, Pv), device=dev)
             nbytes = m0.packed_bytes()

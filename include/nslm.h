@@ -69,6 +69,17 @@ typedef struct CUstream_st *nslm_stream_t;
 #define NSLM_ERR_CUDA (-5)        /* a CUDA call or launch failed */
 #define NSLM_ERR_UNSUPPORTED (-7) /* the current device is not sm_100 */
 
+/* P = NSLM_P3C5: three coefficients of 5 bits ("NanoSeedLM: LLM inference
+ * using pseudo-random numbers", "'Four bits is four bits'": P=3 with 5-bit
+ * coefficients, 4.375 bits per weight).  Its 35 bits per block: the seeds
+ * stream as usual; the coefs word holds c_0, c_1, c_2 as 5-bit two's
+ * complement in bits 0-4, 5-9, 10-14 and bit 0 of the exponent code in bit 15;
+ * codes: u8 [N][3 K / 64] holds code bits 1..3 of block b of a row at bits
+ * 3b .. 3b+2 of the row's bit string, least significant bit first.  K must be
+ * a multiple of 64.  Taken by nslm_seed_gemv and the debug decompression; the
+ * FFN, grouped GEMM and search entry points return NSLM_ERR_SHAPE for it. */
+#define NSLM_P3C5 35
+
 /* One packed seed matrix (see the layout above).  For a stack of E experts,
  * N = E * rows and expert e owns rows [e * rows, (e + 1) * rows). */
 typedef struct {
@@ -78,7 +89,7 @@ typedef struct {
     const int32_t *exp_bias;
     int32_t N;
     int32_t K;
-    int32_t P;               /* 3 or 4 */
+    int32_t P;               /* 3, 4 or NSLM_P3C5 */
 } nslm_seed_matrix;
 
 /* One MoE layer: gate and up are [E * inter][hidden], down is [E * hidden][inter]. */

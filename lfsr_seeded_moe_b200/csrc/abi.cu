@@ -101,14 +101,14 @@ int32_t max_active_ctas(const void *kernel, int threads, size_t smem) {
 
 int32_t check_matrix(const nslm_seed_matrix *W) {
   if (!W) return NSLM_ERR_ARG;
-  if (W->P != 3 && W->P != 4) return NSLM_ERR_SHAPE;
+  if (W->P != 3 && W->P != 4 && W->P != kP3C5) return NSLM_ERR_SHAPE;
   if (W->N < 0 || W->K <= 0) return NSLM_ERR_SHAPE;
-  if (W->K % (W->P == 4 ? 16 : 8) != 0) return NSLM_ERR_SHAPE;
+  if (W->K % (W->P == 4 ? 16 : (W->P == kP3C5 ? 64 : 8)) != 0) return NSLM_ERR_SHAPE;
   if (W->N > 0) {
     if (!W->seeds || !W->coefs || !W->exp_bias) return NSLM_ERR_ARG;
-    if (W->P == 4 && !W->codes) return NSLM_ERR_ARG;
+    if (W->P != 3 && !W->codes) return NSLM_ERR_ARG;
     if (!aligned16(W->seeds) || !aligned16(W->coefs) || !aligned16(W->exp_bias)) return NSLM_ERR_ALIGN;
-    if (W->P == 4 && !aligned16(W->codes)) return NSLM_ERR_ALIGN;
+    if (W->P != 3 && !aligned16(W->codes)) return NSLM_ERR_ALIGN;
   }
   return NSLM_OK;
 }
@@ -160,8 +160,17 @@ __global__ void decompress_kernel(const nslm_seed_matrix W, float *w32, uint16_t
     float F[8];
     block_ints(lo, hi, coef_bytes<P>(q), F);
     uint32_t code;
-    if (P == 4) code = (W.codes[row * (nb / 2) + col / 2] >> (4 * (col & 1))) & 0xFu;
-    else code = q >> 12;
+    if (P == 4) {
+      code = (W.codes[row * (nb / 2) + col / 2] >> (4 * (col & 1))) & 0xFu;
+    } else if (P == kP3C5) {  // code bits 1..3 at bits 3col.. of the row's codes
+      const uint8_t *cr = W.codes + row * (3 * (size_t)nb / 8);
+      const size_t bit = 3 * col;
+      uint32_t two = cr[bit >> 3];
+      if ((bit & 7) > 5) two |= (uint32_t)cr[(bit >> 3) + 1] << 8;
+      code = ((q >> 15) & 1u) | (((two >> (bit & 7)) & 7u) << 1);
+    } else {
+      code = q >> 12;
+    }
     const float scale = block_scale(code, row_scale_key(W.exp_bias[row]));
     const size_t base = row * (size_t)W.K + col * 8;
 #pragma unroll
@@ -185,6 +194,7 @@ static int32_t decompress(const nslm_seed_matrix *W, float *w32, uint16_t *wbf, 
   const int grid = (int)std::min<size_t>((nblk + threads - 1) / threads, (size_t)num_sms() * 8);
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   if (W->P == 4) decompress_kernel<4><<<grid, threads, 0, s>>>(*W, w32, wbf);
+  else if (W->P == kP3C5) decompress_kernel<kP3C5><<<grid, threads, 0, s>>>(*W, w32, wbf);
   else decompress_kernel<3><<<grid, threads, 0, s>>>(*W, w32, wbf);
   st = launch_status();
   if (st == NSLM_OK) g_launches = 1;

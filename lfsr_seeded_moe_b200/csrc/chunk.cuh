@@ -142,6 +142,9 @@ __device__ __forceinline__ void load_chunk(const uint16_t *__restrict__ seeds_ro
     f.s[0] = s.x; f.s[1] = s.y; f.s[2] = s.z; f.s[3] = s.w;
     f.q[0] = q.x; f.q[1] = q.y; f.q[2] = q.z; f.q[3] = q.w;
     f.codes = (P == 4) ? __ldcs(reinterpret_cast<const uint32_t *>(codes_row + b0 / 2)) : 0u;
+    if (P == 35)  // code bits 1..3 of the chunk's 8 blocks: bytes 3ch .. 3ch+2
+      f.codes = (uint32_t)__ldcs(codes_row + 3 * ch) | ((uint32_t)__ldcs(codes_row + 3 * ch + 1) << 8) |
+                ((uint32_t)__ldcs(codes_row + 3 * ch + 2) << 16);
   } else {
 #pragma unroll
     for (int w = 0; w < 4; ++w) {
@@ -213,6 +216,10 @@ __device__ __forceinline__ void read_chunk(const FieldSlots &fs, int i, ChunkFie
 // (P = 3: byte 3 is 0; the top nibble there is the exponent code).
 template <int P>
 __device__ __forceinline__ uint32_t coef_pairs2(uint32_t q16) {
+  if (P == 35) {  // [2c0, 2c2, 2c1, 0] from three 5-bit fields: 2c mod 256
+    const uint32_t v = (q16 & 0x1Fu) | ((q16 >> 2) & 0x1F00u) | ((q16 << 11) & 0x1F0000u);
+    return (v << 1) + (v & 0x101010u) * 12u;
+  }
   const uint32_t v = (q16 | (q16 << 12)) & (P == 4 ? 0x0F0F0F0Fu : 0x000F0F0Fu);
   // 2c mod 256 per byte: 2q, plus 224 where bit 3 is set (no carry out)
   return (v << 1) + (v & 0x08080808u) * 28u;
@@ -269,7 +276,9 @@ __device__ __forceinline__ float regen_chunk_block(const StreamTables *tab, cons
 #else
   block_magic_src((i & 1) ? (sw >> 16) : (sw & 0xFFFFu), coef_pairs2<P>(q), G);
 #endif
-  const uint32_t code = (P == 4) ? ((f.codes >> (4 * i)) & 0xFu) : (q >> 12);
+  const uint32_t code = (P == 4) ? ((f.codes >> (4 * i)) & 0xFu)
+                      : (P == 35) ? (((q >> 15) & 1u) | (((f.codes >> (3 * i)) & 7u) << 1))
+                                  : (q >> 12);
   return block_scale(code, rowk);
 }
 
@@ -290,7 +299,9 @@ __device__ __forceinline__ float regen_chunk_block_r(const uint32_t *tl, const C
 #else
   block_magic_src((i & 1) ? (sw >> 16) : (sw & 0xFFFFu), coef_pairs2<P>(q), G);
 #endif
-  const uint32_t code = (P == 4) ? ((f.codes >> (4 * i)) & 0xFu) : (q >> 12);
+  const uint32_t code = (P == 4) ? ((f.codes >> (4 * i)) & 0xFu)
+                      : (P == 35) ? (((q >> 15) & 1u) | (((f.codes >> (3 * i)) & 7u) << 1))
+                                  : (q >> 12);
   return block_scale(code, rowk);
 }
 

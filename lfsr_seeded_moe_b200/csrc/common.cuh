@@ -8,6 +8,9 @@
 
 namespace nslm {
 
+// P value of the P = 3, 5-bit-coefficient format (NSLM_P3C5 in the header).
+constexpr int kP3C5 = 35;
+
 // Launch accounting for benchmarks: kernels enqueued by the last call made on
 // this host thread.
 extern thread_local int32_t g_launches;

@@ -50,7 +50,10 @@ __global__ void __launch_bounds__(512) seed_gemv_kernel(const GemvParams p) {
     if (row < p.N && ch < p.C) {
       ChunkFields f;
       load_chunk<P, VEC>(p.seeds + (size_t)row * p.nb, p.coefs + (size_t)row * p.nb,
-                         P == 4 ? p.codes + (size_t)row * (p.nb / 2) : nullptr, p.nb, ch, f);
+                         P == 4    ? p.codes + (size_t)row * (p.nb / 2)
+                         : P == 35 ? p.codes + (size_t)row * (3 * p.nb / 8)
+                                   : nullptr,
+                         p.nb, ch, f);
       const uint32_t rowk = row_scale_key(__ldg(p.exp_bias + row));
       chunk_dot<P, M, VEC, CPAD>(tab, f, p.nb, ch, rowk, xs4, xn2, cpad, 0, acc);
     }
@@ -213,7 +216,10 @@ extern "C" int32_t nslm_seed_gemv(const nslm_seed_matrix *W, const uint16_t *x_b
 
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   // one vector, whole 64-weight chunks: the latency-oriented kernel
-  if (M == 1 && W->K % 64 == 0 && (int64_t)W->N * (W->K / 8) < (1ll << 31) && W->K / 64 < (1 << 16)) {
+  // (the P = 3 5-bit format keeps its code bits in 3-byte groups, which the
+  // kernel's 4-byte cp.async copies do not take; it uses the kernel below)
+  if (M == 1 && W->P != kP3C5 && W->K % 64 == 0 && (int64_t)W->N * (W->K / 8) < (1ll << 31) &&
+      W->K / 64 < (1 << 16)) {
     const int sms = num_sms();
     Gemv1Params q{};
     q.W = *W;
@@ -249,8 +255,9 @@ extern "C" int32_t nslm_seed_gemv(const nslm_seed_matrix *W, const uint16_t *x_b
   if (smem > 227 * 1024) return NSLM_ERR_SHAPE;
   const int per_sm = std::max(1, std::min(2048 / L.threads, (int)((227 * 1024) / smem)));
   const int grid = std::min(p.groups, per_sm * sms);
-  st = (W->P == 4) ? dispatch_gemv<4>(p, vec, grid, L.threads, smem, s)
-                   : dispatch_gemv<3>(p, vec, grid, L.threads, smem, s);
+  st = (W->P == 4)       ? dispatch_gemv<4>(p, vec, grid, L.threads, smem, s)
+       : (W->P == kP3C5) ? dispatch_gemv<kP3C5>(p, vec, grid, L.threads, smem, s)
+                         : dispatch_gemv<3>(p, vec, grid, L.threads, smem, s);
   if (st == NSLM_OK) g_launches = 1;
   return st;
 }

@@ -587,6 +587,7 @@ extern "C" int32_t nslm_seed_grouped_gemm(const nslm_seed_matrix *W, int32_t E,
   g_launches = 0;
   int32_t st = check_matrix(W);
   if (st) return st;
+  if (W->P == kP3C5) return NSLM_ERR_SHAPE;  // the tensor-core path takes P = 3 and P = 4
   if (!x_bf16 || !offsets || !y) return NSLM_ERR_ARG;
   if (E < 1 || E > 1024 || R < 0) return NSLM_ERR_SHAPE;
   if (W->N % E != 0) return NSLM_ERR_SHAPE;

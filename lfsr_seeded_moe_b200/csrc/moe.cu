@@ -411,6 +411,8 @@ int32_t check_ffn_shapes(const nslm_seed_matrix *gate, const nslm_seed_matrix *u
                          const nslm_seed_matrix *down, int32_t E, FfnDims &d) {
   int32_t st;
   if ((st = check_matrix(gate)) || (st = check_matrix(up)) || (st = check_matrix(down))) return st;
+  // the FFN kernels take P = 3 and P = 4 (the 5-bit format runs in the GEMV)
+  if (gate->P == kP3C5 || up->P == kP3C5 || down->P == kP3C5) return NSLM_ERR_SHAPE;
   if (E <= 0) return NSLM_ERR_ARG;
   if (gate->N % E != 0) return NSLM_ERR_SHAPE;
   d.E = E;

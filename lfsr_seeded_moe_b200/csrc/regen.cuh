@@ -175,6 +175,10 @@ __device__ __forceinline__ void stream_word(const StreamTables *tab, uint32_t se
 // (P = 3: byte 3 is 0; the top nibble there is the exponent code).
 template <int P>
 __device__ __forceinline__ uint32_t coef_bytes(uint32_t q16) {
+  if (P == 35) {  // three 5-bit fields: a set bit 4 adds 0xE0
+    const uint32_t v = (q16 & 0x1Fu) | ((q16 << 3) & 0x1F00u) | ((q16 << 6) & 0x1F0000u);
+    return v + (v & 0x101010u) * 14u;
+  }
   uint32_t v = (q16 | (q16 << 12)) & 0x0F0F0F0Fu;            // [c0, c2, c1, c3]
   v = __byte_perm(v, 0u, P == 4 ? 0x3120 : 0x4120);          // [c0, c1, c2, c3|0]
   // two's-complement nibble -> byte: a set bit 3 adds 0xF0 (no carry out)

@@ -277,6 +277,7 @@ extern "C" int32_t nslm_seed_search(const float *w, const float *imp, const nslm
   g_launches = 0;
   int32_t st = check_matrix(out);
   if (st) return st;
+  if (out->P == kP3C5) return NSLM_ERR_SHAPE;  // the search encodes P = 3 and P = 4
   if (!w) return NSLM_ERR_ARG;
   if (seed_lo < 1 || seed_hi > 65535 || seed_lo > seed_hi) return NSLM_ERR_ARG;
   if (out->N == 0) return NSLM_OK;

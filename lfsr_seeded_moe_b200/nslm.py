@@ -28,6 +28,8 @@ NSLM_ERR_WORKSPACE = -4
 NSLM_ERR_CUDA = -5
 NSLM_ERR_UNSUPPORTED = -7
 
+NSLM_P3C5 = 35  # P = 3 with 5-bit coefficients
+
 NSLM_OP_GEMV = 0
 NSLM_OP_GROUPED_GEMM = 1
 NSLM_OP_MOE_FFN = 2

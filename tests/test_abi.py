@@ -138,3 +138,19 @@ def test_expert_cache_argument_checks():
     assert call(cac=[_mat(S * inter, 512), cac[1], cac[2]]) == nslm.NSLM_ERR_SHAPE   # cache shape differs
     assert call(state=0x9000004) == nslm.NSLM_ERR_ALIGN
 
+
+def test_p3c5_format_checks():
+    # P = 35 (three 5-bit coefficients): K a multiple of 64 and a codes stream;
+    # taken by the GEMV and decompression, refused by the FFN, grouped GEMM
+    # and search entry points
+    assert _gemv(_mat(K=96, P=35)) == nslm.NSLM_ERR_SHAPE
+    assert _gemv(_mat(K=128, P=35, codes=False)) == nslm.NSLM_ERR_ARG
+    E, hidden, inter = 4, 256, 128
+    f = nslm.raw().nslm_moe_seed_ffn
+    g, u, d = _mat(E * inter, hidden, P=35), _mat(E * inter, hidden, P=35), _mat(E * hidden, inter, P=35)
+    ws = nslm.nslm_workspace_bytes(nslm.NSLM_OP_MOE_FFN, 1, E, hidden, inter, 2)
+    assert f(ctypes.byref(g), ctypes.byref(u), ctypes.byref(d), E, 0x7000000, 0x7100000, 0x7200000, 1, 2,
+             0x7300000, 0x7400000, ws, 0) == nslm.NSLM_ERR_SHAPE
+    srch = nslm.raw().nslm_seed_search
+    assert srch(0x9000000, 0, ctypes.byref(_mat(N=4, K=64, P=35)), 1, 10, 0, 0) == nslm.NSLM_ERR_SHAPE
+

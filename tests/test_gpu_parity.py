@@ -47,7 +47,7 @@ def _all_seed_matrix(P, bias_lo=-100, bias_hi=100):
     return m
 
 
-@pytest.mark.parametrize("P", [3, 4])
+@pytest.mark.parametrize("P", [3, 4, 35])
 def test_decompress_fp32_bit_exact_all_seeds(nslm, P):
     m = _all_seed_matrix(P)
     md = _dev(m)
@@ -59,7 +59,7 @@ def test_decompress_fp32_bit_exact_all_seeds(nslm, P):
     assert np.array_equal(got.view(np.uint32), ref.view(np.uint32))
 
 
-@pytest.mark.parametrize("P", [3, 4])
+@pytest.mark.parametrize("P", [3, 4, 35])
 def test_decompress_bf16_bit_exact_all_seeds(nslm, P):
     m = _all_seed_matrix(P, -20, 10)
     md = _dev(m)
@@ -73,7 +73,7 @@ def test_decompress_bf16_bit_exact_all_seeds(nslm, P):
 GEMV_SHAPES = [(512, 1024), (2048, 4096), (4096, 2048), (1408, 2048), (2048, 1408)]
 
 
-@pytest.mark.parametrize("P", [3, 4])
+@pytest.mark.parametrize("P", [3, 4, 35])
 @pytest.mark.parametrize("N,K", GEMV_SHAPES)
 def test_gemv_matches_oracle(nslm, P, N, K):
     m = synth.seed_matrix(N, K, P, (901, N, K, P))
@@ -87,7 +87,7 @@ def test_gemv_matches_oracle(nslm, P, N, K):
 
 
 @pytest.mark.parametrize("M", [2, 3, 8])
-@pytest.mark.parametrize("P", [3, 4])
+@pytest.mark.parametrize("P", [3, 4, 35])
 def test_gemv_multi_token(nslm, M, P):
     N, K = 704, 2048
     m = synth.seed_matrix(N, K, P, (902, M, P))
