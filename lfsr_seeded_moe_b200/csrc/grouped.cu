@@ -170,8 +170,11 @@ __global__ void __launch_bounds__(kCtaThreads, 1) grouped_seed_gemm_kernel(const
   __shared__ volatile int s_abort;
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  // a producer's tasks: row trow, block pair bp, of sub-tiles 0 and 1
-  const int trow = tid & (kBM - 1), bp = (tid >> 7) & 3;
+  // a producer's tasks: row trow, block pair bp, of sub-tiles 0 and 1.  A
+  // warp covers 8 rows x the 4 block pairs: a field load touches 8 sectors
+  // (4 lanes per 16-byte row piece), and each 8-lane wavefront of the tile
+  // stores writes 8 consecutive rows (128 contiguous bytes)
+  const int trow = ((tid >> 5) << 3) | (tid & 7), bp = (tid >> 3) & 3;
   build_stream_tables_rep<kTabCopies>(tab);
   const uint32_t *tl = tab + (lane & (kTabCopies - 1));
   if (warp == 0) umma::tmem_alloc(umma::smem_u32(&tmem_base_s), (uint32_t)p.tmem_cols);
@@ -337,33 +340,40 @@ __global__ void __launch_bounds__(kCtaThreads, 1) grouped_seed_gemm_kernel(const
       if (!copy_b(0, it)) s_abort = 1;
       cp_async_commit();
 
-      // weight fields three slices ahead
+      // weight fields three slices ahead, in three register sets: slice kt
+      // uses set kt % 3 and reloads it for slice kt + 3 (the loop is unrolled
+      // by three, so no set is ever copied while its loads are in flight)
       SliceFields f0, f1, f2;
       load_slice<P>(sp, qp, cpp, ok, 0, f0);
       if (ksteps > 1) load_slice<P>(sp, qp, cpp, ok, 1, f1);
       if (ksteps > 2) load_slice<P>(sp, qp, cpp, ok, 2, f2);
-      for (int kt = 0; kt < ksteps; ++kt, ++it) {
+      auto slice = [&](SliceFields &f, int kt) {
         const int stage = it % kStages;
-        if (s_abort) break;
         // the stage of slice it was claimed when its token rows were copied
         if (kt + 1 < ksteps && !copy_b(kt + 1, it + 1)) s_abort = 1;
         cp_async_commit();
         uint8_t *atile = a_base + (size_t)stage * 2 * kBM * 128;
-        const SliceFields cur = f0;
-        f0 = f1;
-        f1 = f2;
-        if (kt + 3 < ksteps) load_slice<P>(sp, qp, cpp, ok, kt + 3, f2);
         // rows past the matrix carry zero coefficient fields, which regenerate
         // to exactly zero weights: no branch
 #pragma unroll
         for (int j = 0; j < 2; ++j) {
           uint4 *dst0 = reinterpret_cast<uint4 *>(atile + j * kBM * 128 + a_off);
           uint4 *dst1 = reinterpret_cast<uint4 *>(atile + j * kBM * 128 + a_off + 128);
-          regen_pair_bf16<P>(tl, cur.s2[j], cur.q2[j], cur.c2[j], rowk[j], dst0, dst1);
+          regen_pair_bf16<P>(tl, f.s2[j], f.q2[j], f.c2[j], rowk[j], dst0, dst1);
         }
+        if (kt + 3 < ksteps) load_slice<P>(sp, qp, cpp, ok, kt + 3, f);
         cp_async_wait<1>();  // this slice's token rows (the next slice's may still be in flight)
         umma::fence_proxy_async();
         umma::mbar_arrive(umma::smem_u32(&full_bar[stage]));
+        ++it;
+      };
+      for (int kt = 0; kt < ksteps; kt += 3) {
+        if (s_abort) break;
+        slice(f0, kt);
+        if (kt + 1 >= ksteps || s_abort) break;
+        slice(f1, kt + 1);
+        if (kt + 2 >= ksteps || s_abort) break;
+        slice(f2, kt + 2);
       }
       cp_async_wait_all();
     }
