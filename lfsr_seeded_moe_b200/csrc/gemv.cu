@@ -146,6 +146,10 @@ __global__ void __launch_bounds__(kGemv1Threads) gemv1_kernel(const Gemv1Params 
   const int nrows = max(0, min(p.rpc, p.W.N - n0));
   const int ntask = nrows * p.C;
   const int nb = p.W.K >> 3;
+  // launched with programmatic stream serialization: wait here for the
+  // preceding kernel (its writes of W or x), then let the next one launch
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  asm volatile("griddepcontrol.launch_dependents;");
 
   auto fetch = [&](int t, int buf) {
     const uint32_t r = fdiv((uint32_t)t, p.div_C), c = (uint32_t)t - r * (uint32_t)p.C;
@@ -236,8 +240,18 @@ extern "C" int32_t nslm_seed_gemv(const nslm_seed_matrix *W, const uint16_t *x_b
       auto k = (W->P == 4) ? gemv1_kernel<4> : gemv1_kernel<3>;
       if ((st = ensure_smem((const void *)k, smem))) return st;
       ensure_stream_source(s);
-      k<<<ceil_div(W->N, q.rpc), threads, smem, s>>>(q);
-      st = launch_status();
+      cudaLaunchConfig_t cfg{};
+      cfg.gridDim = dim3((unsigned)ceil_div(W->N, q.rpc));
+      cfg.blockDim = dim3((unsigned)threads);
+      cfg.dynamicSmemBytes = smem;
+      cfg.stream = s;
+      cudaLaunchAttribute attr[1];
+      attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+      attr[0].val.programmaticStreamSerializationAllowed = 1;
+      cfg.attrs = attr;
+      cfg.numAttrs = 1;
+      st = cuda_status(cudaLaunchKernelEx(&cfg, k, q));
+      if (st == NSLM_OK) st = launch_status();
       if (st == NSLM_OK) g_launches = 1;
       return st;
     }
