@@ -30,6 +30,7 @@ namespace nslm {
 
 constexpr int kBM = 128;        // weight rows per tile (MMA M)
 constexpr int kBK = 64;         // K per stage: 8 blocks, 128 bytes of bf16 per row
+constexpr int kMaxBn = 256;     // token rows per tile at most (2 x bn tensor-memory columns)
 constexpr int kGThreads = 512;                  // producer threads (warps 0-15)
 constexpr int kEpiWarp0 = kGThreads / 32;       // warps 16-19: the epilogue warpgroup
 constexpr int kMmaWarp = kEpiWarp0 + 4;         // warp 20: issues the MMAs
@@ -168,6 +169,9 @@ __global__ void __launch_bounds__(kCtaThreads, 1) grouped_seed_gemm_kernel(const
   __shared__ __align__(8) uint64_t acc_full_bar, acc_empty_bar;
   __shared__ uint32_t tmem_base_s;
   __shared__ volatile int s_abort;
+  // DOWN epilogue: each epilogue warp's copy of the tile's pair ids and weights
+  __shared__ int s_epr[MODE == GMODE_DOWN ? 4 : 1][MODE == GMODE_DOWN ? kMaxBn : 1];
+  __shared__ float s_epw[MODE == GMODE_DOWN ? 4 : 1][MODE == GMODE_DOWN ? kMaxBn : 1];
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   // a producer's tasks: row trow, block pair bp, of sub-tiles 0 and 1.  A
@@ -233,6 +237,19 @@ __global__ void __launch_bounds__(kCtaThreads, 1) grouped_seed_gemm_kernel(const
       if (s_abort) break;
       const TileInfo ti = tile_info<MODE>(p, t);
       __syncwarp();
+      if (MODE == GMODE_DOWN) {
+        // the tile's pair ids and routing weights, loaded once per tile and
+        // warp before the accumulators are ready (loaded per element they
+        // were two dependent global loads on the tile's critical path)
+#pragma unroll 4
+        for (int n = lane; n < ti.N; n += 32) {
+          const bool v = n < ti.n_valid;
+          const int pr = v ? p.pair_of[ti.r_begin + n] : 0;
+          s_epr[ew][n] = pr;
+          s_epw[ew][n] = v ? p.pair_w[pr] : 0.f;
+        }
+        __syncwarp();
+      }
       const bool acc_ok = umma::mbar_wait_bounded(umma::smem_u32(&acc_full_bar), ntile & 1, kWaitCycles);
       if (!acc_ok) s_abort = 1;
       // tcgen05.ld is warp-collective: the whole warp takes one decision
@@ -271,8 +288,8 @@ __global__ void __launch_bounds__(kCtaThreads, 1) grouped_seed_gemm_kernel(const
               if (MODE == GMODE_GEMM) {
                 p.y[sr * p.rows + row] = v[j];
               } else {
-                const int pr = p.pair_of[sr];
-                p.part[(size_t)pr * p.rows + row] = p.pair_w[pr] * v[j];
+                p.part[(size_t)s_epr[MODE == GMODE_DOWN ? ew : 0][MODE == GMODE_DOWN ? n : 0] * p.rows + row] =
+                    s_epw[MODE == GMODE_DOWN ? ew : 0][MODE == GMODE_DOWN ? n : 0] * v[j];
               }
             }
           }
@@ -522,7 +539,7 @@ int32_t launch_grouped(const GroupedParams &p, int P, int mode, cudaStream_t s) 
 // Token rows per tile (up to 256: two accumulators of 256 fp32 columns fill the
 // 512 tensor-memory columns); experts with more rows take several tiles.
 static int choose_bn(int max_rows_per_expert) {
-  return std::max(16, (std::min(max_rows_per_expert, 256) + 15) & ~15);
+  return std::max(16, (std::min(max_rows_per_expert, kMaxBn) + 15) & ~15);
 }
 
 BatchedPlan batched_workspace(char *base, int T, int k, int E, int hidden, int inter) {
