@@ -37,6 +37,10 @@ __global__ void __launch_bounds__(512) seed_gemv_kernel(const GemvParams p) {
   const int tid = threadIdx.x, nthr = blockDim.x;
 
   build_stream_tables(tab);
+  // launched with programmatic stream serialization (as the one-vector
+  // kernel): wait for the preceding kernel before the first global read
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  asm volatile("griddepcontrol.launch_dependents;");
   stage_bf16(xs4, xn2, p.x, nullptr, M, p.K, cpad);
   __syncthreads();
 
@@ -78,7 +82,17 @@ static int32_t launch_gemv(const GemvParams &p, int grid, int threads, size_t sm
   auto k = seed_gemv_kernel<P, M, VEC, CPAD>;
   if (int32_t st = ensure_smem((const void *)k, smem)) return st;
   ensure_stream_source(s);
-  k<<<grid, threads, smem, s>>>(p);
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3((unsigned)grid);
+  cfg.blockDim = dim3((unsigned)threads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (int32_t st = cuda_status(cudaLaunchKernelEx(&cfg, k, p))) return st;
   return launch_status();
 }
 

@@ -261,6 +261,26 @@ def test_ffn_decode_batch_all_ids_dropped_gives_zero(nslm):
     assert np.array_equal(y, np.zeros_like(y))
 
 
+@pytest.mark.parametrize("P", [3, 4])
+def test_ffn_decode_batch_with_an_empty_token(nslm, P):
+    # token 2 of 4 has every id out of range: its row is exactly zero and the
+    # other tokens still match the oracle (persistent batched kernel)
+    E, hidden, inter, k, T = 20, 512, 256, 4, 4
+    L = synth.moe_layer(0, E, hidden, inter, P, config=944)
+    x, xh = _x((944, T), T, hidden)
+    rng = np.random.default_rng(944)
+    rid = np.stack([rng.choice(E, k, replace=False) for _ in range(T)]).astype(np.int32)
+    rid[2] = [-1, E, E + 3, -5]
+    w32 = rng.uniform(0.05, 0.3, size=(T, k)).astype(np.float32)
+    y = _ffn_with_ids(nslm, L, E, hidden, inter, x, rid, w32, k)
+    assert np.array_equal(y[2], np.zeros(hidden, np.float32))
+    keep = (rid >= 0) & (rid < E)
+    g, u, d = (getattr(L, n).numpy() for n in ("gate", "up", "down"))
+    ref = O.moe_ffn(g, u, d, E, hidden, inter, xh, np.where(keep, rid, 0).astype(np.int32),
+                    np.where(keep, w32.astype(np.float64), 0.0), mode=0)
+    assert O.normwise_rel_err(y, ref) <= TIGHT
+
+
 def test_ffn_decode_ragged_and_zipf(nslm):
     y, ref = _ffn_case(nslm, 12, 272, 120, 3, 3, 8, 908, zipf=1.1)
     assert O.normwise_rel_err(y, ref) <= TIGHT
