@@ -277,6 +277,18 @@ int32_t nslm_expert_cache_fetch(const nslm_seed_matrix *gate_src, const nslm_see
 int32_t nslm_unpack_nibbles(const uint8_t *nibbles, const nslm_seed_matrix *out, nslm_stream_t stream);
 int32_t nslm_pack_nibbles(const nslm_seed_matrix *in, uint8_t *nibbles, nslm_stream_t stream);
 
+/* Test export: the bounded device waits give up and report, they do not
+ * hang.  kind 0: the grid-barrier wait of the persistent decode kernels,
+ * waiting for one arrival on out[0..3] (status, arrivals, abort, as at the
+ * head of the decode workspace; the caller initialises them: arrivals 0 makes
+ * the wait run out, 1 lets it pass); on giving up it sets out[0] = 1 and
+ * out[2] = 1.  out[4] = 1 if the wait passed, 0 if it gave up.
+ * kind 1 / 2: the mbarrier wait of the tensor-core pipeline on a barrier
+ * whose phase nothing completes (1) or that one arrival completed first (2);
+ * out[0] = 1 if it passed, 0 if it gave up.  cycles: the wait limit in SM
+ * clocks (> 0).  out: device, 5 int32.  One launch of one CTA. */
+int32_t nslm_debug_wait_probe(int32_t kind, int32_t *out, int64_t cycles, nslm_stream_t stream);
+
 /* Test exports: the regenerated weights themselves, written out densely.
  * w_out: fp32 [N][K] (exact) or bf16 bit patterns [N][K] (round to nearest
  * even of the exact value).  Not on the hot path. */

@@ -40,7 +40,8 @@ __device__ __forceinline__ void grid_arrive(int32_t *sync) {
 // Wait until `target` arrivals: thread 0 polls with acquire loads, bounded by
 // kBarrierWaitCycles; a CTA that gives up raises the abort flag and records
 // status 1, and every CTA stops at its next wait.  False when aborting.
-static __device__ bool grid_wait(int32_t *sync, uint32_t target, int *s_ok) {
+static __device__ bool grid_wait(int32_t *sync, uint32_t target, int *s_ok,
+                                 long long max_cycles = kBarrierWaitCycles) {
   if (threadIdx.x == 0) {
     int ok = 1;
     if (ld_acquire(sync + 1) < target) {
@@ -51,7 +52,7 @@ static __device__ bool grid_wait(int32_t *sync, uint32_t target, int *s_ok) {
             ok = 0;
             break;
           }
-          if (clock64() - t0 > kBarrierWaitCycles) {
+          if (clock64() - t0 > max_cycles) {
             atomicExch(sync + 2, 1);
             atomicCAS(sync, 0, 1);
             ok = 0;

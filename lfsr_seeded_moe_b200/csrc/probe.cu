@@ -1,0 +1,52 @@
+// probe.cu -- test export: the bounded device waits of the persistent decode
+// kernels (grid barrier) and of the tensor-core pipeline (mbarrier) give up
+// after their limit and report it, instead of hanging.  One CTA waits for an
+// event that nothing produces (or, for the positive case, one that already
+// happened) with the kernels' own wait routines and a caller-chosen limit.
+#include "common.cuh"
+#include "persist.cuh"
+#include "umma.cuh"
+
+namespace nslm {
+namespace {
+
+// out[0..3]: the sync words the grid barrier uses (status, arrivals, abort),
+// initialised by the caller; out[4] = 1 if the wait succeeded, 0 if it gave up.
+__global__ void grid_wait_probe_kernel(int32_t *out, long long cycles) {
+  __shared__ int s_ok;
+  const bool ok = grid_wait(out, 1u, &s_ok, cycles);  // one arrival, which no CTA makes unless preset
+  if (threadIdx.x == 0) out[4] = ok ? 1 : 0;
+}
+
+// out[0] = 1 if the mbarrier wait succeeded, 0 if it gave up; `arrive` = 1
+// completes the barrier's phase before the wait.
+__global__ void mbar_wait_probe_kernel(int32_t *out, long long cycles, int arrive) {
+  __shared__ __align__(8) uint64_t bar;
+  if (threadIdx.x == 0) {
+    umma::mbar_init(umma::smem_u32(&bar), 1);
+    umma::mbar_init_fence();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    if (arrive) umma::mbar_arrive(umma::smem_u32(&bar));
+    out[0] = umma::mbar_wait_bounded(umma::smem_u32(&bar), 0, cycles) ? 1 : 0;
+  }
+}
+
+}  // namespace
+}  // namespace nslm
+
+using namespace nslm;
+
+extern "C" int32_t nslm_debug_wait_probe(int32_t kind, int32_t *out, int64_t cycles, nslm_stream_t stream) {
+  g_launches = 0;
+  if (!out || cycles <= 0 || (kind != 0 && kind != 1 && kind != 2)) return NSLM_ERR_ARG;
+  int32_t st = check_device();
+  if (st) return st;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (kind == 0) grid_wait_probe_kernel<<<1, 32, 0, s>>>(out, (long long)cycles);
+  else mbar_wait_probe_kernel<<<1, 32, 0, s>>>(out, (long long)cycles, kind == 2 ? 1 : 0);
+  st = launch_status();
+  if (st == NSLM_OK) g_launches = 1;
+  return st;
+}

@@ -79,6 +79,7 @@ def _load():
         "nslm_expert_cache_fetch": (i32, [mp, mp, mp, i32, i32, mp, mp, mp, i32, vp, vp, i32, i32, vp, vp]),
         "nslm_unpack_nibbles": (i32, [vp, mp, vp]),
         "nslm_pack_nibbles": (i32, [mp, vp, vp]),
+        "nslm_debug_wait_probe": (i32, [i32, vp, ctypes.c_int64, vp]),
         "nslm_debug_decompress": (i32, [mp, vp, vp]),
         "nslm_debug_decompress_bf16": (i32, [mp, vp, vp]),
         "nslm_status_string": (ctypes.c_char_p, [i32]),
@@ -229,6 +230,11 @@ def nslm_unpack_nibbles(nibbles, out, stream=None) -> None:
 def nslm_pack_nibbles(W, nibbles, stream=None) -> None:
     """Write the nibbles stream u8 [N][(P+1)*K/16] of W's coefs (and codes)."""
     _check("nslm_pack_nibbles", _lib.nslm_pack_nibbles(ctypes.byref(_mat(W)), _p(nibbles), _s(stream)))
+
+
+def nslm_debug_wait_probe(kind: int, out, cycles: int, stream=None) -> None:
+    """Run one bounded device wait (see include/nslm.h) with results in out (5 int32)."""
+    _check("nslm_debug_wait_probe", _lib.nslm_debug_wait_probe(int(kind), _p(out), int(cycles), _s(stream)))
 
 
 def nslm_debug_decompress(W, w_out, stream=None) -> None:

@@ -154,3 +154,10 @@ def test_p3c5_format_checks():
     srch = nslm.raw().nslm_seed_search
     assert srch(0x9000000, 0, ctypes.byref(_mat(N=4, K=64, P=35)), 1, 10, 0, 0) == nslm.NSLM_ERR_SHAPE
 
+
+def test_wait_probe_argument_checks():
+    f = nslm.raw().nslm_debug_wait_probe
+    assert f(0, 0, 1000, 0) == nslm.NSLM_ERR_ARG          # no output buffer
+    assert f(0, 0x9000000, 0, 0) == nslm.NSLM_ERR_ARG     # no limit
+    assert f(3, 0x9000000, 1000, 0) == nslm.NSLM_ERR_ARG  # unknown kind
+
