@@ -127,27 +127,6 @@ __device__ __forceinline__ void build_stream_tables_rep(uint32_t *t) {
   for (int i = threadIdx.x; i < 512 * R; i += blockDim.x) t[i] = kStreamTab.t[i / R];
 }
 
-// The same tables replicated 32 times and interleaved by lane: entry i of copy
-// c at word i * 32 + c.  Lane l reads copy l, so the 32 lanes of a warp never
-// hit the same bank whatever seeds they hold (64 KB of shared memory).
-struct StreamTablesX32 {
-  uint32_t t[512 * 32];
-};
-
-__device__ __forceinline__ void build_stream_tables_x32(StreamTablesX32 *tab) {
-  for (int i = threadIdx.x; i < 512 * 32; i += blockDim.x) tab->t[i] = kStreamTab.t[i >> 5];
-}
-
-// (v, nxt) of a seed from the replicated tables; lane4 = 4 * (lane id).
-__device__ __forceinline__ void stream_pair_x32(const StreamTablesX32 *tab, uint32_t lane4, uint32_t seed,
-                                                uint32_t &v, uint32_t &nxt) {
-  const char *base = reinterpret_cast<const char *>(tab->t) + lane4;
-  const uint32_t a = *reinterpret_cast<const uint32_t *>(base + ((seed & 0xFFu) << 7));
-  const uint32_t b = *reinterpret_cast<const uint32_t *>(base + (((seed >> 8) & 0xFFu) << 7) + 256 * 128);
-  nxt = a ^ b;
-  v = seed << 16;
-}
-
 // The stream of seed `HALF` (0: bits 0..15, 1: bits 16..31) of a packed word
 // of two seeds, as v = seed << 16 and nxt = the 32 bits that follow the seed:
 // then W >> t = funnelshift_r(v, nxt, 16 + t) for 1 <= t < 16, and
@@ -207,13 +186,6 @@ __device__ __forceinline__ int32_t dp2a_lo_us(uint32_t a_u16x2, uint32_t b_s8x4,
 __device__ __forceinline__ int32_t dp2a_hi_us(uint32_t a_u16x2, uint32_t b_s8x4, int32_t acc) {
   int32_t d;
   asm("dp2a.hi.u32.s32 %0, %1, %2, %3;" : "=r"(d) : "r"(a_u16x2), "r"(b_s8x4), "r"(acc));
-  return d;
-}
-
-// a * b + c in one integer multiply-add.
-__device__ __forceinline__ int32_t imad(int32_t a, int32_t b, int32_t c) {
-  int32_t d;
-  asm("mad.lo.s32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
   return d;
 }
 
