@@ -4,7 +4,8 @@
 // shared memory.
 //
 // Dot-product form.  For block b with weights w_r = scale * A_r (A_r an
-// integer, |A_r| <= 2^20) the regeneration yields G_r = Mg + A_r exactly as an
+// integer, |A_r| < 2^21 (4 * 8 * 32768 for int4, 3 * 16 * 32768 for the 5-bit
+// format)) the regeneration yields G_r = Mg + A_r exactly as an
 // fp32 value (Mg = 1.5 * 2^22, so G_r lies in [2^22, 2^23) where the fp32 step
 // is 0.5).  Then
 //     sum_r x_r A_r = sum_r x_r G_r - Mg * sum_r x_r,

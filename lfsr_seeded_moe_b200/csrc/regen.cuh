@@ -8,7 +8,8 @@
 //   w_r = 2^(code + bias) * sum_j c_j * (s_{1+8j+r} - 32768) / 32768
 //       = 2^(code + bias - 15) * A_r,   A_r = sum_j c_j * (s_{1+8j+r} - 32768),
 //
-// an integer A_r with |A_r| <= 2^20 times a power of two, so fp32 holds w_r
+// an integer A_r with |A_r| < 2^21 (at most 4 * 8 * 32768, or 3 * 16 * 32768 for
+// 5-bit coefficients) times a power of two, so fp32 holds w_r
 // exactly.  This file rebuilds A_r without stepping the register:
 //
 // 1. Stream word.  The register is a Fibonacci LFSR (x^16 + x^14 + x^13 +
