@@ -104,6 +104,7 @@ typedef struct {
 #define NSLM_OP_GROUPED_GEMM 1
 #define NSLM_OP_MOE_FFN 2
 #define NSLM_OP_MOE_STACK 3
+#define NSLM_OP_MOE_FFN_HYBRID 4  /* E = E3 + E4 */
 
 /* Bytes of workspace an operation needs (0 if none).  T = tokens, E =
  * experts, hidden/inter = FFN sizes, k = experts per token, L = layers (only
@@ -160,6 +161,23 @@ int32_t nslm_moe_seed_ffn(const nslm_seed_matrix *gate, const nslm_seed_matrix *
                           const nslm_seed_matrix *down, int32_t E, const uint16_t *x_bf16,
                           const int32_t *ids, const float *w, int32_t T, int32_t k, float *y,
                           void *ws, size_t ws_bytes, nslm_stream_t stream);
+
+/* A routed expert FFN whose experts are packed with different P ("NanoSeedLM:
+ * LLM inference using pseudo-random numbers", news list: hybrid P3 / P4 seed
+ * packs, ~4.17 bits per weight; reading: each expert is P = 3 or P = 4 as a
+ * whole).  p3: HOST pointer to the layer's E3 P = 3 experts (stacked as for
+ * nslm_moe_seed_ffn); p4: its E4 P = 4 experts, same hidden and inter.  Expert
+ * id e < E3 is p3's expert e, E3 <= e < E3 + E4 is p4's expert e - E3; other
+ * ids contribute nothing.  y = the layer's output, as nslm_moe_seed_ffn
+ * computes it over all E3 + E4 experts: the routed FFN runs per stack (the
+ * same kernels, the same T-dependent path) and the two partial outputs are
+ * added in a fixed order.  Workspace: nslm_workspace_bytes(
+ * NSLM_OP_MOE_FFN_HYBRID, T, E3 + E4, hidden, inter, k, 0).  Launches: the
+ * two FFNs' plus two. */
+int32_t nslm_moe_seed_ffn_hybrid(const nslm_moe_layer *p3, int32_t E3, const nslm_moe_layer *p4,
+                                 int32_t E4, const uint16_t *x_bf16, const int32_t *ids, const float *w,
+                                 int32_t T, int32_t k, float *y, void *ws, size_t ws_bytes,
+                                 nslm_stream_t stream);
 
 /* The decode path of nslm_moe_seed_ffn (T <= 8) for callers that may not
  * allocate device memory: the scratch it needs lives in a 1 MiB array built

@@ -235,6 +235,9 @@ size_t nslm_workspace_bytes(int32_t op, int32_t T, int32_t E, int32_t hidden, in
                              std::max(inter, 0), 1).bytes;
       return batched_workspace(nullptr, T, std::max(k, 1), std::max(E, 1), std::max(hidden, 0),
                                std::max(inter, 0)).bytes;
+    case NSLM_OP_MOE_FFN_HYBRID:
+      return nslm_workspace_bytes(NSLM_OP_MOE_FFN, T, E, hidden, inter, k, 0) +
+             hybrid_extra_bytes(std::max(T, 1), std::max(k, 1), std::max(hidden, 0));
     case NSLM_OP_MOE_STACK:
       return ffn_workspace(nullptr, std::max(T, 1), std::max(k, 1), std::max(hidden, 0),
                            std::max(inter, 0), std::max(L, 1)).bytes;

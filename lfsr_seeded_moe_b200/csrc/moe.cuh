@@ -56,6 +56,10 @@ struct FfnWorkspace {
 };
 FfnWorkspace ffn_workspace(char *base, int T, int k, int hidden, int inter, int L);
 
+// Workspace a hybrid P3/P4 layer needs beyond the FFN's: two id arrays and
+// the P = 3 stack's output.
+size_t hybrid_extra_bytes(int T, int k, int hidden);
+
 int32_t launch_route_plan(const float *logits, const int32_t *ids, const float *w, int T, int E,
                           int k, int L, SlotPlan *plans, int32_t *ids_out, float *w_out,
                           int32_t *counters, int n_counters, int32_t *sync, int slot_cap, cudaStream_t s);

@@ -34,6 +34,7 @@ NSLM_OP_GEMV = 0
 NSLM_OP_GROUPED_GEMM = 1
 NSLM_OP_MOE_FFN = 2
 NSLM_OP_MOE_STACK = 3
+NSLM_OP_MOE_FFN_HYBRID = 4
 
 
 class NslmError(RuntimeError):
@@ -71,6 +72,8 @@ def _load():
         "nslm_seed_grouped_gemm": (i32, [mp, i32, vp, vp, i32, vp, vp, sz, vp]),
         "nslm_moe_route_topk": (i32, [vp, i32, i32, i32, vp, vp, vp]),
         "nslm_moe_seed_ffn": (i32, [mp, mp, mp, i32, vp, vp, vp, i32, i32, vp, vp, sz, vp]),
+        "nslm_moe_seed_ffn_hybrid": (i32, [ctypes.POINTER(nslm_moe_layer), i32, ctypes.POINTER(nslm_moe_layer), i32,
+                                           vp, vp, vp, i32, i32, vp, vp, sz, vp]),
         "nslm_moe_seed_ffn_static": (i32, [mp, mp, mp, i32, vp, vp, vp, i32, i32, vp, vp]),
         "nslm_moe_stack_decode": (i32, [ctypes.POINTER(nslm_moe_layer), i32, i32, i32, vp, vp, i32,
                                         vp, vp, sz, vp]),
@@ -174,6 +177,16 @@ def nslm_moe_seed_ffn(gate, up, down, E: int, x_bf16, ids, w, T: int, k: int, y,
            _lib.nslm_moe_seed_ffn(ctypes.byref(_mat(gate)), ctypes.byref(_mat(up)),
                                   ctypes.byref(_mat(down)), E, _p(x_bf16), _p(ids), _p(w), T, k,
                                   _p(y), _p(ws), ws_bytes, _s(stream)))
+
+
+def nslm_moe_seed_ffn_hybrid(p3, E3: int, p4, E4: int, x_bf16, ids, w, T: int, k: int, y, ws=None,
+                             ws_bytes: int = 0, stream=None) -> None:
+    """p3 / p4: (gate, up, down) of the P=3 and P=4 expert stacks; ids index E3 + E4 experts."""
+    l3 = nslm_moe_layer(*(_mat(m) for m in p3))
+    l4 = nslm_moe_layer(*(_mat(m) for m in p4))
+    _check("nslm_moe_seed_ffn_hybrid",
+           _lib.nslm_moe_seed_ffn_hybrid(ctypes.byref(l3), E3, ctypes.byref(l4), E4, _p(x_bf16), _p(ids), _p(w),
+                                         T, k, _p(y), _p(ws), ws_bytes, _s(stream)))
 
 
 def nslm_moe_seed_ffn_static(gate, up, down, E: int, x_bf16, ids, w, T: int, k: int, y,

@@ -161,3 +161,26 @@ def test_wait_probe_argument_checks():
     assert f(0, 0x9000000, 0, 0) == nslm.NSLM_ERR_ARG     # no limit
     assert f(3, 0x9000000, 1000, 0) == nslm.NSLM_ERR_ARG  # unknown kind
 
+
+def test_hybrid_argument_checks():
+    f = nslm.raw().nslm_moe_seed_ffn_hybrid
+    E3, E4, hidden, inter = 3, 4, 256, 128
+
+    def layer(E, P, base):
+        return nslm.nslm_moe_layer(_mat(E * inter, hidden, P=P, base=base), _mat(E * inter, hidden, P=P, base=base),
+                                   _mat(E * hidden, inter, P=P, base=base))
+
+    l3, l4 = layer(E3, 3, 0x1000000), layer(E4, 4, 0x2000000)
+    wsb = nslm.nslm_workspace_bytes(nslm.NSLM_OP_MOE_FFN_HYBRID, 1, E3 + E4, hidden, inter, 2)
+    assert wsb > nslm.nslm_workspace_bytes(nslm.NSLM_OP_MOE_FFN, 1, E3 + E4, hidden, inter, 2)
+
+    def call(a=l3, b=l4, e3=E3, e4=E4, ws=0x7400000, n=wsb):
+        return f(ctypes.byref(a), e3, ctypes.byref(b), e4, 0x7000000, 0x7100000, 0x7200000, 1, 2, 0x7300000,
+                 ws, n, 0)
+
+    assert call(a=l4, b=l3, e3=E4, e4=E3) == nslm.NSLM_ERR_SHAPE   # stacks swapped: P must be 3 then 4
+    assert call(e3=0) == nslm.NSLM_ERR_SHAPE
+    assert call(n=wsb - 1) == nslm.NSLM_ERR_WORKSPACE
+    assert f(None, E3, ctypes.byref(l4), E4, 0x7000000, 0x7100000, 0x7200000, 1, 2, 0x7300000, 0x7400000, wsb,
+             0) == nslm.NSLM_ERR_ARG
+

@@ -281,6 +281,36 @@ def test_ffn_decode_batch_with_an_empty_token(nslm, P):
     assert O.normwise_rel_err(y, ref) <= TIGHT
 
 
+@pytest.mark.parametrize("T", [1, 3, 12])
+def test_ffn_hybrid_p3_p4_experts(nslm, T):
+    # experts 0..4 packed with P=3, 5..11 with P=4; one routed pair dropped
+    E3, E4, hidden, inter, k = 5, 7, 512, 256, 4
+    E = E3 + E4
+    L3 = synth.moe_layer(0, E3, hidden, inter, 3, config=945)
+    L4 = synth.moe_layer(0, E4, hidden, inter, 4, config=946)
+    x, xh = _x((945, T), T, hidden)
+    rng = np.random.default_rng(945 + T)
+    rid = np.stack([rng.choice(E, k, replace=False) for _ in range(T)]).astype(np.int32)
+    rid[0, 1] = E + 2
+    w32 = rng.uniform(0.05, 0.3, (T, k)).astype(np.float32)
+    y = _out(T, hidden)
+    wsb = nslm.nslm_workspace_bytes(nslm.NSLM_OP_MOE_FFN_HYBRID, T, E, hidden, inter, k)
+    ws = torch.empty(wsb, dtype=torch.uint8, device="cuda")
+    d3 = tuple(_dev(getattr(L3, n)) for n in ("gate", "up", "down"))
+    d4 = tuple(_dev(getattr(L4, n)) for n in ("gate", "up", "down"))
+    nslm.nslm_moe_seed_ffn_hybrid(d3, E3, d4, E4, x, torch.from_numpy(rid).cuda(), torch.from_numpy(w32).cuda(),
+                                  T, k, y, ws, wsb)
+    torch.cuda.synchronize()
+    mode = 0 if T <= 8 else 1  # T > 8: the tensor-core path (bf16 weights and h)
+    ref = 0.0
+    for L, lo, hi in ((L3, 0, E3), (L4, E3, E)):
+        keep = (rid >= lo) & (rid < hi)
+        g, u, d = (getattr(L, n).numpy() for n in ("gate", "up", "down"))
+        ref = ref + O.moe_ffn(g, u, d, hi - lo, hidden, inter, xh, np.where(keep, rid - lo, 0).astype(np.int32),
+                              np.where(keep, w32.astype(np.float64), 0.0), mode=mode)
+    assert O.normwise_rel_err(y.cpu().numpy(), ref) <= (TIGHT if T <= 8 else TOL)
+
+
 def test_ffn_decode_ragged_and_zipf(nslm):
     y, ref = _ffn_case(nslm, 12, 272, 120, 3, 3, 8, 908, zipf=1.1)
     assert O.normwise_rel_err(y, ref) <= TIGHT
