@@ -673,7 +673,7 @@ def main():
         batch8 = stack_batch_leg(torch, nslm, synth, dev, arr, hbm, 8, max(10, args.steps // 4), rank)
 
     host_experts = None
-    if T == 1 and not args.no_host_experts:
+    if T == 1 and world == 1 and not args.no_host_experts:  # pins 3.9 GB of host memory per process
         host_experts = host_experts_leg(torch, nslm, synth, dev)
 
     search = None
