@@ -2,6 +2,7 @@
 rejects bad arguments with the documented status codes before launching
 anything (these checks run on the host; no pointer is dereferenced)."""
 import ctypes
+import os
 
 import pytest
 
@@ -183,4 +184,19 @@ def test_hybrid_argument_checks():
     assert call(n=wsb - 1) == nslm.NSLM_ERR_WORKSPACE
     assert f(None, E3, ctypes.byref(l4), E4, 0x7000000, 0x7100000, 0x7200000, 1, 2, 0x7300000, 0x7400000, wsb,
              0) == nslm.NSLM_ERR_ARG
+
+
+def test_header_compiles_as_c99(tmp_path):
+    # the boundary is a C ABI: its header must be plain C99 (and C++)
+    import shutil
+    import subprocess
+    gcc = shutil.which("gcc")
+    if gcc is None:
+        pytest.skip("no C compiler")
+    src = tmp_path / "use.c"
+    src.write_text('#include "nslm.h"\nint main(void) { nslm_seed_matrix m = {0}; (void)m; return 0; }\n')
+    inc = os.path.dirname(nslm.HEADER_PATH)
+    for args in (["-std=c99", "-pedantic", "-Wall", "-Wextra", "-Werror"], ["-x", "c++", "-std=c++17", "-Wall", "-Werror"]):
+        r = subprocess.run([gcc, *args, "-I", inc, "-fsyntax-only", str(src)], capture_output=True, text=True)
+        assert r.returncode == 0, r.stderr
 
