@@ -165,10 +165,19 @@ __global__ void __launch_bounds__(kGemv1Threads) gemv1_kernel(const Gemv1Params 
   asm volatile("griddepcontrol.wait;" ::: "memory");
   asm volatile("griddepcontrol.launch_dependents;");
 
+  // the 5-bit format's code bits (3 bytes per chunk, not 4-byte aligned) come
+  // by plain loads into one register per buffer, one task ahead like the rest
+  uint32_t cq0 = 0, cq1 = 0;
   auto fetch = [&](int t, int buf) {
     const uint32_t r = fdiv((uint32_t)t, p.div_C), c = (uint32_t)t - r * (uint32_t)p.C;
     const uint32_t row = (uint32_t)n0 + r;
     fetch_chunk_off<P>(p.W, row * (uint32_t)nb + 8u * c, row, fs, buf * nthr + tid);
+    if (P == kP3C5) {
+      const uint8_t *cb = p.W.codes + (size_t)row * (3u * (uint32_t)nb / 8u) + 3u * c;
+      const uint32_t v = (uint32_t)__ldcs(cb) | ((uint32_t)__ldcs(cb + 1) << 8) | ((uint32_t)__ldcs(cb + 2) << 16);
+      if (buf) cq1 = v;
+      else cq0 = v;
+    }
   };
   if (tid < ntask) fetch(tid, 0);
   cp_async_commit();
@@ -195,6 +204,7 @@ __global__ void __launch_bounds__(kGemv1Threads) gemv1_kernel(const Gemv1Params 
     ChunkFields f;
     uint32_t rowk;
     read_chunk<P>(fs, (it & 1) * nthr + tid, f, rowk);
+    if (P == kP3C5) f.codes = (it & 1) ? cq1 : cq0;
     float2 acc = make_float2(0.f, 0.f);
     chunk_dot_cm<P, true, 1>(tab->t, f, 8, rowk, xs4 + kCmX4 * c, xn2 + kCmXn * c, acc);
     red[t] = acc.x + acc.y;
@@ -234,10 +244,7 @@ extern "C" int32_t nslm_seed_gemv(const nslm_seed_matrix *W, const uint16_t *x_b
 
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   // one vector, whole 64-weight chunks: the latency-oriented kernel
-  // (the P = 3 5-bit format keeps its code bits in 3-byte groups, which the
-  // kernel's 4-byte cp.async copies do not take; it uses the kernel below)
-  if (M == 1 && W->P != kP3C5 && W->K % 64 == 0 && (int64_t)W->N * (W->K / 8) < (1ll << 31) &&
-      W->K / 64 < (1 << 16)) {
+  if (M == 1 && W->K % 64 == 0 && (int64_t)W->N * (W->K / 8) < (1ll << 31) && W->K / 64 < (1 << 16)) {
     const int sms = num_sms();
     Gemv1Params q{};
     q.W = *W;
@@ -251,7 +258,7 @@ extern "C" int32_t nslm_seed_gemv(const nslm_seed_matrix *W, const uint16_t *x_b
     const int threads = std::max(64, 32 * ceil_div(ceil_div(tasks, rounds), 32));
     const size_t smem = gemv1_smem(q.C, q.rpc, threads);
     if (smem <= 200 * 1024 && (int64_t)q.rpc * q.C < (1 << 22)) {
-      auto k = (W->P == 4) ? gemv1_kernel<4> : gemv1_kernel<3>;
+      auto k = (W->P == 4) ? gemv1_kernel<4> : (W->P == kP3C5 ? gemv1_kernel<kP3C5> : gemv1_kernel<3>);
       if ((st = ensure_smem((const void *)k, smem))) return st;
       ensure_stream_source(s);
       cudaLaunchConfig_t cfg{};
