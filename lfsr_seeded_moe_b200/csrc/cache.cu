@@ -200,6 +200,7 @@ extern "C" int32_t nslm_expert_cache_fetch(const nslm_seed_matrix *gate_src, con
   if ((int64_t)layer * E + E >= INT_MAX) return NSLM_ERR_SHAPE;
   if ((st = check_ffn_shapes(gate_cache, up_cache, down_cache, S, dc))) return st;
   if (dc.hidden != d.hidden || dc.inter != d.inter || dc.P != d.P) return NSLM_ERR_SHAPE;
+  if (d.P == kP3C5) return NSLM_ERR_SHAPE;  // the copies know the P = 3 and P = 4 streams
   // whole 16-byte words per range: rows a multiple of 4 (biases), K a multiple of 64
   if (d.hidden % 64 || d.inter % 64) return NSLM_ERR_SHAPE;
   const nslm_seed_matrix *all[6] = {gate_src, up_src, down_src, gate_cache, up_cache, down_cache};

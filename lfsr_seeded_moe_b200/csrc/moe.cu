@@ -135,6 +135,14 @@ __global__ void __launch_bounds__(256) route_plan_kernel(const float *__restrict
   }
 }
 
+// The codes stream of row `grow`: P = 4 packs two 4-bit codes per byte, the
+// 5-bit P = 3 format 3 code bits per block (3 bytes per 8 blocks); P = 3 has
+// none.
+template <int P>
+__device__ __forceinline__ const uint8_t *codes_row(const uint8_t *codes, size_t grow, int nb) {
+  return P == 4 ? codes + grow * (nb / 2) : (P == kP3C5 ? codes + grow * (3 * (size_t)nb / 8) : nullptr);
+}
+
 // ------------------------------------------------------------- gate / up
 
 struct GateUpParams {
@@ -210,9 +218,9 @@ __global__ void __launch_bounds__(256) ffn_gate_up_kernel(const GateUpParams p) 
   if (active) {
     const size_t grow = (size_t)e * p.inter + row;
     load_chunk<P, VEC>(p.gate.seeds + grow * nb, p.gate.coefs + grow * nb,
-                       P == 4 ? p.gate.codes + grow * (nb / 2) : nullptr, nb, ch, fg);
+                       codes_row<P>(p.gate.codes, grow, nb), nb, ch, fg);
     load_chunk<P, VEC>(p.up.seeds + grow * nb, p.up.coefs + grow * nb,
-                       P == 4 ? p.up.codes + grow * (nb / 2) : nullptr, nb, ch, fu);
+                       codes_row<P>(p.up.codes, grow, nb), nb, ch, fu);
     rowkg = row_scale_key(__ldg(p.gate.exp_bias + grow));
     rowku = row_scale_key(__ldg(p.up.exp_bias + grow));
   }
@@ -321,7 +329,7 @@ __global__ void __launch_bounds__(512) ffn_down_kernel(const DownParams p) {
   if (active && s0 < s1) {
     const size_t grow = (size_t)pl->expert[s0] * p.hidden + row;
     load_chunk<P, VEC>(p.down.seeds + grow * nb, p.down.coefs + grow * nb,
-                       P == 4 ? p.down.codes + grow * (nb / 2) : nullptr, nb, ch, f);
+                       codes_row<P>(p.down.codes, grow, nb), nb, ch, f);
     rowk = row_scale_key(__ldg(p.down.exp_bias + grow));
   }
   build_stream_tables(tab);
@@ -345,7 +353,7 @@ __global__ void __launch_bounds__(512) ffn_down_kernel(const DownParams p) {
     if (active && s + 1 < s1) {
       const size_t grow = (size_t)pl->expert[s + 1] * p.hidden + row;
       load_chunk<P, VEC>(p.down.seeds + grow * nb, p.down.coefs + grow * nb,
-                         P == 4 ? p.down.codes + grow * (nb / 2) : nullptr, nb, ch, fn);
+                         codes_row<P>(p.down.codes, grow, nb), nb, ch, fn);
       rowkn = row_scale_key(__ldg(p.down.exp_bias + grow));
     }
     if (active) {
@@ -411,8 +419,8 @@ int32_t check_ffn_shapes(const nslm_seed_matrix *gate, const nslm_seed_matrix *u
                          const nslm_seed_matrix *down, int32_t E, FfnDims &d) {
   int32_t st;
   if ((st = check_matrix(gate)) || (st = check_matrix(up)) || (st = check_matrix(down))) return st;
-  // the FFN kernels take P = 3 and P = 4 (the 5-bit format runs in the GEMV)
-  if (gate->P == kP3C5 || up->P == kP3C5 || down->P == kP3C5) return NSLM_ERR_SHAPE;
+  // one format for the whole layer
+  if (gate->P != up->P || gate->P != down->P) return NSLM_ERR_SHAPE;
   if (E <= 0) return NSLM_ERR_ARG;
   if (gate->N % E != 0) return NSLM_ERR_SHAPE;
   d.E = E;
@@ -515,6 +523,10 @@ int32_t launch_decode_layer(const FfnDims &d, const nslm_seed_matrix *gate,
   if (d.P == 4) {
     return T == 1 ? launch_decode_layer_t<4, 1>(d, gate, up, down, plan, x_bf16, y_prev, T, k, w, y, s, launches)
                   : launch_decode_layer_t<4, 8>(d, gate, up, down, plan, x_bf16, y_prev, T, k, w, y, s, launches);
+  }
+  if (d.P == kP3C5) {
+    return T == 1 ? launch_decode_layer_t<kP3C5, 1>(d, gate, up, down, plan, x_bf16, y_prev, T, k, w, y, s, launches)
+                  : launch_decode_layer_t<kP3C5, 8>(d, gate, up, down, plan, x_bf16, y_prev, T, k, w, y, s, launches);
   }
   return T == 1 ? launch_decode_layer_t<3, 1>(d, gate, up, down, plan, x_bf16, y_prev, T, k, w, y, s, launches)
                 : launch_decode_layer_t<3, 8>(d, gate, up, down, plan, x_bf16, y_prev, T, k, w, y, s, launches);

@@ -364,6 +364,7 @@ static size_t stack1_smem(const FfnDims &d, int k, int threads) {
 
 bool stack1_supported(const FfnDims &d, int k) {
   if (k < 1 || k > kMaxK) return false;
+  if (d.P != 3 && d.P != 4) return false;  // the 5-bit format runs on the per-layer kernels
   // 32-bit element offsets into the field streams
   if ((int64_t)d.E * d.inter * (d.hidden / 8) >= (1ll << 31) || (int64_t)d.E * d.hidden * (d.inter / 8) >= (1ll << 31))
     return false;

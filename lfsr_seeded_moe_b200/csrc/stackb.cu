@@ -494,6 +494,7 @@ bool stackb_shape(const FfnDims &d, int T, int k, StackBShape &sh) {
 }  // namespace
 
 bool stackb_supported(const FfnDims &d, int T, int k) {
+  if (d.P != 3 && d.P != 4) return false;  // the 5-bit format runs on the per-layer kernels
   StackBShape sh{};
   if (!stackb_shape(d, T, k, sh)) return false;
   // 32-bit element offsets into the field streams

@@ -149,9 +149,17 @@ def test_p3c5_format_checks():
     E, hidden, inter = 4, 256, 128
     f = nslm.raw().nslm_moe_seed_ffn
     g, u, d = _mat(E * inter, hidden, P=35), _mat(E * inter, hidden, P=35), _mat(E * hidden, inter, P=35)
-    ws = nslm.nslm_workspace_bytes(nslm.NSLM_OP_MOE_FFN, 1, E, hidden, inter, 2)
-    assert f(ctypes.byref(g), ctypes.byref(u), ctypes.byref(d), E, 0x7000000, 0x7100000, 0x7200000, 1, 2,
+    ws = nslm.nslm_workspace_bytes(nslm.NSLM_OP_MOE_FFN, 16, E, hidden, inter, 2)
+    # T <= 8 runs the per-layer decode kernels: the arguments pass (without a
+    # device the call then stops at the device check); T > 8 is refused
+    st1 = f(ctypes.byref(g), ctypes.byref(u), ctypes.byref(d), E, 0x7000000, 0x7100000, 0x7200000, 1, 2,
+            0x7300000, 0x7400000, ws, 0)
+    assert st1 not in (nslm.NSLM_ERR_SHAPE, nslm.NSLM_ERR_ARG, nslm.NSLM_ERR_ALIGN, nslm.NSLM_ERR_WORKSPACE)
+    assert f(ctypes.byref(g), ctypes.byref(u), ctypes.byref(d), E, 0x7000000, 0x7100000, 0x7200000, 16, 2,
              0x7300000, 0x7400000, ws, 0) == nslm.NSLM_ERR_SHAPE
+    # a layer mixing formats is refused
+    assert f(ctypes.byref(g), ctypes.byref(_mat(E * inter, hidden, P=4)), ctypes.byref(d), E, 0x7000000, 0x7100000,
+             0x7200000, 1, 2, 0x7300000, 0x7400000, ws, 0) == nslm.NSLM_ERR_SHAPE
     srch = nslm.raw().nslm_seed_search
     assert srch(0x9000000, 0, ctypes.byref(_mat(N=4, K=64, P=35)), 1, 10, 0, 0) == nslm.NSLM_ERR_SHAPE
 

@@ -311,6 +311,28 @@ def test_ffn_hybrid_p3_p4_experts(nslm, T):
     assert O.normwise_rel_err(y.cpu().numpy(), ref) <= (TIGHT if T <= 8 else TOL)
 
 
+@pytest.mark.parametrize("T", [1, 3])
+def test_ffn_decode_p3c5_layer(nslm, T):
+    # the 5-bit P=3 format through the decode FFN (the per-layer kernels)
+    y, ref = _ffn_case(nslm, 10, 512, 256, 35, T, 4, 947 + T)
+    assert O.normwise_rel_err(y, ref) <= TIGHT
+
+
+def test_stack_decode_p3c5(nslm):
+    Lyr, E, hidden, inter, P, k, T = 4, 8, 256, 128, 35, 2, 2
+    layers = [synth.moe_layer(l, E, hidden, inter, P, config=948) for l in range(Lyr)]
+    logits = torch.stack([synth.router_logits((948, l), T, E) for l in range(Lyr)])
+    x, xh = _x((948, T), T, hidden)
+    dl = [(_dev(m.gate), _dev(m.up), _dev(m.down)) for m in layers]
+    ys = [_stack_prefix(nslm, dl, logits, x, T, E, hidden, inter, k, n) for n in range(1, Lyr + 1)]
+    for l in range(Lyr):  # each layer on the GPU's own input (a long stack is chaotic)
+        g, u, d = (getattr(layers[l], n).numpy() for n in ("gate", "up", "down"))
+        xl = xh if l == 0 else O.rms_chain(ys[l - 1])
+        ids, w = O.route_topk(logits[l].numpy(), k)
+        ref = O.moe_ffn(g, u, d, E, hidden, inter, xl, ids, w, mode=0)
+        assert O.normwise_rel_err(ys[l], ref) <= TOL, l
+
+
 def test_ffn_decode_ragged_and_zipf(nslm):
     y, ref = _ffn_case(nslm, 12, 272, 120, 3, 3, 8, 908, zipf=1.1)
     assert O.normwise_rel_err(y, ref) <= TIGHT
