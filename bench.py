@@ -37,7 +37,8 @@ E, HIDDEN, INTER, P, K_TOP, LAYERS = 100, 2048, 1408, 4, 8, 45
 WORKLOAD = "45-layer seed-expert MoE decode: 100 experts/layer, hidden 2048, inter 1408, P=4, top-8"
 METRIC = "MoE seed-FFN decode tokens/s"
 GEMV_METRIC = "seed-GEMV packed-byte HBM GB/s (% of peak)"
-GEMV_SHAPES = [(2048, 4096), (4096, 2048), (1408, 2048), (2048, 1408)]
+GEMV_SHAPES = [(2048, 4096), (4096, 2048), (1408, 2048), (2048, 1408)]  # the expert-sized sweep
+GEMV_SMALL = (512, 1024)  # the single small GEMV (P=4); L2-resident, so its % of HBM means little
 FALLBACK_HBM_GBS = 6650.0
 
 
@@ -212,38 +213,43 @@ def job_throughput(world: int, steps: int, tokens_per_step: int, elapsed_s: floa
 # ------------------------------------------------------------------- GPU leg
 
 def gemv_sweep(torch, nslm, synth, dev, hbm):
+    """The single small GEMV (512 x 1024, P=4) and the expert-sized sweep for
+    P=4, P=3 and the 5-bit P=3 format (35), batch 1.  Each shape is timed over
+    rotating weight copies in one CUDA graph (more than 4x L2 where 400 copies
+    reach it; the small GEMV's copies stay largely in L2)."""
     out = []
-    for Pv in (4, 3, 35):  # 35: P = 3 with 5-bit coefficients
-        for (N, K) in GEMV_SHAPES:
-            m0 = synth.seed_matrix(N, K, Pv, (11, N, K, Pv), device=dev)
-            nbytes = m0.packed_bytes()
-            ncopy = min(400, max(2, int(4 * 126e6 // nbytes) + 1))
-            mats = [synth.seed_matrix(N, K, Pv, (11, N, K, Pv, c), device=dev) for c in range(ncopy)]
-            structs = [nslm.matrix(m) for m in mats]
-            x = synth.activations((11,), 1, K).to(dev)
-            y = torch.empty(1, N, device=dev)
-            nslm.nslm_seed_gemv(structs[0], x, 1, y)
-            torch.cuda.synchronize()
-            g = torch.cuda.CUDAGraph()
-            with torch.cuda.graph(g):
-                for c in range(ncopy):
-                    nslm.nslm_seed_gemv(structs[c], x, 1, y)
-            for _ in range(3):
-                g.replay()
-            torch.cuda.synchronize()
-            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            reps = 5
-            e0.record()
-            for _ in range(reps):
-                g.replay()
-            e1.record()
-            torch.cuda.synchronize()
-            t = e0.elapsed_time(e1) * 1e-3 / (reps * ncopy)
-            gbs = nbytes / t / 1e9
-            out.append({"P": Pv, "N": N, "K": K, "us": round(t * 1e6, 3), "GB_s": round(gbs, 1),
-                        "pct_of_hbm": round(100 * gbs / hbm, 2), "weights_per_s": N * K / t})
-            del g, mats, structs
-            torch.cuda.empty_cache()
+    cases = [(4, GEMV_SMALL)] + [(Pv, nk) for Pv in (4, 3, 35) for nk in GEMV_SHAPES]
+    for Pv, (N, K) in cases:
+        m0 = synth.seed_matrix(N, K, Pv, (11, N, K, Pv), device=dev)
+        nbytes = m0.packed_bytes()
+        ncopy = min(400, max(2, int(4 * 126e6 // nbytes) + 1))
+        mats = [synth.seed_matrix(N, K, Pv, (11, N, K, Pv, c), device=dev) for c in range(ncopy)]
+        structs = [nslm.matrix(m) for m in mats]
+        x = synth.activations((11,), 1, K).to(dev)
+        y = torch.empty(1, N, device=dev)
+        nslm.nslm_seed_gemv(structs[0], x, 1, y)
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            for c in range(ncopy):
+                nslm.nslm_seed_gemv(structs[c], x, 1, y)
+        for _ in range(3):
+            g.replay()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        reps = 5
+        e0.record()
+        for _ in range(reps):
+            g.replay()
+        e1.record()
+        torch.cuda.synchronize()
+        t = e0.elapsed_time(e1) * 1e-3 / (reps * ncopy)
+        gbs = nbytes / t / 1e9
+        out.append({"P": Pv, "N": N, "K": K, "us": round(t * 1e6, 3), "GB_s": round(gbs, 1),
+                    "pct_of_hbm": round(100 * gbs / hbm, 2), "weights_per_s": N * K / t,
+                    "rotated_bytes": nbytes * ncopy, "rotation_below_4x_l2": nbytes * ncopy < 4 * 126e6})
+        del g, mats, structs
+        torch.cuda.empty_cache()
     return out
 
 
@@ -641,6 +647,12 @@ def main():
     r1.record()
     torch.cuda.synchronize()
     layer_s = r0.elapsed_time(r1) * 1e-3 / nreps
+    one_layer = {"workload": "one MoE layer decode: 100 experts, 2048/1408, P=4, top-8, one token "
+                             "(routing plan + the persistent kernel for one layer, per call)",
+                 "us": round(layer_s * 1e6, 3), "tokens_per_s": round(1.0 / layer_s, 1),
+                 "packed_GB_s": round(layer_packed_bytes_per_token() / layer_s / 1e9, 1),
+                 "hbm_frac": round(layer_packed_bytes_per_token() / layer_s / 1e9 / hbm, 4),
+                 "weights_per_s": round(K_TOP * 3 * HIDDEN * INTER / layer_s, 1)}
     roofline = {"bound": "hbm",
                 "kernel": f"{'stack1_kernel' if T == 1 else 'stackb_kernel'}: one cooperative launch running all "
                           f"{LAYERS} layers (with the routing launch, ~1% of the step)",
@@ -700,6 +712,7 @@ def main():
         line["gemv"] = gemv
     if batched is not None:
         line["batched"] = batched
+    line["one_layer_decode"] = one_layer
     if batch8 is not None:
         line["stack_batch8"] = batch8
     if host_experts is not None:
