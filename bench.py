@@ -14,6 +14,14 @@ The JSON line also carries the seed-GEMV sweep (packed-byte GB/s per expert
 shape, rotating copies to defeat L2), a roofline object for the per-layer
 decode FFN, the end-to-end number through the C ABI with host buffers, the
 clocks seen during the timed region and the CPU oracle's time on a sample.
+Extra objects, each skippable by its flag: one_layer_decode (one layer's
+latency and HBM fraction), stack_batch8 (the same stack at 8 tokens a step,
+--no-batch8), batched (the tcgen05 grouped GEMM layer at 64 and 512 tokens,
+--no-batched), host_experts (experts kept in pinned host memory behind the
+device expert cache, one GPU only, --no-host-experts) and seed_search (the
+seed/coefficient search, plain and importance-weighted, --no-search).
+--profile runs one small case of a single kernel family for ncu and prints
+no JSON line.
 
 --impl reference times the CPU oracle (the plain C definition of the method)
 on this host's cores on a bounded sample of the same workload.
