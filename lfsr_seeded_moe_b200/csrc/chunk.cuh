@@ -418,50 +418,86 @@ __device__ __forceinline__ void chunk_dot2_cm(const uint32_t *tl, const ChunkFie
   }
 }
 
+// Moves a chunk's fields down by N2 words (2 * N2 blocks): block 2 * N2
+// becomes block 0.  Lets a loop over the chunk run rolled, N2 words a trip,
+// with every field index still a compile-time constant (so in registers).
+template <int P, int N2>
+__device__ __forceinline__ void shift_chunk(ChunkFields &f) {
+  static_assert(N2 == 1 || N2 == 2, "a shift of one or two words");
+#pragma unroll
+  for (int w = 0; w + N2 < 4; ++w) {
+    f.s[w] = f.s[w + N2];
+    f.q[w] = f.q[w + N2];
+  }
+  // codes: 4 bits a block at P = 4, 3 at the 5-bit P = 3 format, none at P = 3
+  f.codes = (P == 4) ? (f.codes >> (8 * N2)) : (P == 35) ? (f.codes >> (6 * N2)) : 0u;
+}
+
 // The same for up to MT vectors that share the regenerated weights: vector m
 // (m < M) has its chunk slot at xa + kCmX4 * off[m], xn + kCmXn * off[m].
 // A vector past M is skipped (M is the same for all lanes of a warp in the
-// gate/up phase, and nearly always so in the down phase).
-template <int P, bool VEC, int R, int MT>
+// gate/up phase, and nearly always so in the down phase).  BPI blocks are
+// unrolled per loop trip (8: the whole chunk); a smaller BPI keeps the code
+// small when several of these loops are live on one SM at once, at the cost
+// of a few register moves per block.  The arithmetic, and its order, is the
+// same for every BPI.
+template <int P, bool VEC, int R, int MT, int BPI = 8>
 __device__ __forceinline__ void chunk_dot_cm_multi(const uint32_t *tl, const ChunkFields &f, int nvalid,
                                                    uint32_t rowk, const float4 *xa, const float2 *xn,
                                                    const int (&off)[MT], int M, float2 (&acc)[MT]) {
+  static_assert(BPI == 2 || BPI == 4 || BPI == 8, "blocks per trip");
+  ChunkFields g = f;
+#pragma unroll 1
+  for (int i0 = 0; i0 < 8; i0 += BPI) {
 #pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    if (!VEC && i >= nvalid) break;
-    float G[8];
-    const float s = regen_chunk_block_r<P, R>(tl, f, i, rowk, G);
+    for (int j = 0; j < BPI; ++j) {
+      const int i = i0 + j;
+      if (!VEC && i >= nvalid) break;
+      float G[8];
+      const float s = regen_chunk_block_r<P, R>(tl, g, j, rowk, G);
 #pragma unroll
-    for (int m = 0; m < MT; ++m) {
-      if (m < M) {
-        const float4 *x = xa + kCmX4 * off[m];
-        block_fma(G, s, x[2 * i], x[2 * i + 1], xn[kCmXn * off[m] + i], acc[m]);
+      for (int m = 0; m < MT; ++m) {
+        if (m < M) {
+          const float4 *x = xa + kCmX4 * off[m];
+          block_fma(G, s, x[2 * i], x[2 * i + 1], xn[kCmXn * off[m] + i], acc[m]);
+        }
       }
     }
+    if (BPI < 8) shift_chunk<P, (BPI < 8 ? BPI / 2 : 1)>(g);
   }
 }
 
-template <int P, bool VEC, int R, int MT>
+template <int P, bool VEC, int R, int MT, int BPI = 8>
 __device__ __forceinline__ void chunk_dot2_cm_multi(const uint32_t *tl, const ChunkFields &fa,
                                                     const ChunkFields &fb, int nvalid, uint32_t rowka,
                                                     uint32_t rowkb, const float4 *xa, const float2 *xn,
                                                     const int (&off)[MT], int M, float2 (&acca)[MT],
                                                     float2 (&accb)[MT]) {
+  static_assert(BPI == 2 || BPI == 4 || BPI == 8, "blocks per trip");
+  ChunkFields ga = fa, gb = fb;
+#pragma unroll 1
+  for (int i0 = 0; i0 < 8; i0 += BPI) {
 #pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    if (!VEC && i >= nvalid) break;
-    float Ga[8], Gb[8];
-    const float sa = regen_chunk_block_r<P, R>(tl, fa, i, rowka, Ga);
-    const float sb = regen_chunk_block_r<P, R>(tl, fb, i, rowkb, Gb);
+    for (int j = 0; j < BPI; ++j) {
+      const int i = i0 + j;
+      if (!VEC && i >= nvalid) break;
+      float Ga[8], Gb[8];
+      const float sa = regen_chunk_block_r<P, R>(tl, ga, j, rowka, Ga);
+      const float sb = regen_chunk_block_r<P, R>(tl, gb, j, rowkb, Gb);
 #pragma unroll
-    for (int m = 0; m < MT; ++m) {
-      if (m < M) {
-        const float4 *x = xa + kCmX4 * off[m];
-        const float4 x0 = x[2 * i], x1 = x[2 * i + 1];
-        const float2 x2 = xn[kCmXn * off[m] + i];
-        block_fma(Ga, sa, x0, x1, x2, acca[m]);
-        block_fma(Gb, sb, x0, x1, x2, accb[m]);
+      for (int m = 0; m < MT; ++m) {
+        if (m < M) {
+          const float4 *x = xa + kCmX4 * off[m];
+          const float4 x0 = x[2 * i], x1 = x[2 * i + 1];
+          const float2 x2 = xn[kCmXn * off[m] + i];
+          block_fma(Ga, sa, x0, x1, x2, acca[m]);
+          block_fma(Gb, sb, x0, x1, x2, accb[m]);
+        }
       }
+    }
+    if (BPI < 8) {
+      shift_chunk<P, (BPI < 8 ? BPI / 2 : 1)>(ga);
+      shift_chunk<P, (BPI < 8 ? BPI / 2 : 1)>(gb);
     }
   }
 }

@@ -50,6 +50,12 @@ constexpr int MT = kSlotTokens;
 // 8 tokens per layer: 1 -> 227 us, 2 -> 256 us, 4 -> 293 us (more live
 // registers push the inner loops past 128 registers and into spills).
 constexpr int kStageBatch = 1;
+// Blocks unrolled per loop trip in the inner loops of one-token slots
+// (kRollOne) and of slots shared by several tokens (kRollMulti).  Warps of
+// one SM run both kinds of slot at once; fully unrolled, the loops together
+// outgrow the instruction cache.
+constexpr int kRollOne = 8;
+constexpr int kRollMulti = 2;
 
 struct LayerMatsB {
   nslm_seed_matrix gate, up, down;
@@ -290,14 +296,14 @@ __global__ void __launch_bounds__(kStackBThreads, 1) stackb_kernel(const __grid_
         if (c < p.Ch) {
           // M is warp-uniform; the literal 2 folds the token guards away
           if (M == 1)
-            chunk_dot2_cm<P, true, 1>(tab, cg, cu, 8, ckg, cku, xs4 + kCmX4 * (c + off[0]),
-                                      xn2 + kCmXn * (c + off[0]), ag[0], au[0]);
+            chunk_dot2_cm_multi<P, true, 1, MT, kRollOne>(tab, cg, cu, 8, ckg, cku, xs4 + kCmX4 * c,
+                                                          xn2 + kCmXn * c, off, 1, ag, au);
           else if (M == 2)
-            chunk_dot2_cm_multi<P, true, 1, MT>(tab, cg, cu, 8, ckg, cku, xs4 + kCmX4 * c, xn2 + kCmXn * c,
-                                                off, 2, ag, au);
+            chunk_dot2_cm_multi<P, true, 1, MT, kRollMulti>(tab, cg, cu, 8, ckg, cku, xs4 + kCmX4 * c,
+                                                            xn2 + kCmXn * c, off, 2, ag, au);
           else
-            chunk_dot2_cm_multi<P, true, 1, MT>(tab, cg, cu, 8, ckg, cku, xs4 + kCmX4 * c, xn2 + kCmXn * c,
-                                                off, M, ag, au);
+            chunk_dot2_cm_multi<P, true, 1, MT, kRollMulti>(tab, cg, cu, 8, ckg, cku, xs4 + kCmX4 * c,
+                                                            xn2 + kCmXn * c, off, M, ag, au);
         }
         if (p.J == 1 || c + 32 >= 32 * p.J) {
 #pragma unroll
@@ -386,12 +392,14 @@ __global__ void __launch_bounds__(kStackBThreads, 1) stackb_kernel(const __grid_
             for (int m = 0; m < MT; ++m) off[m] = (q0 - qa + m) * p.Ci;
             // M is warp-uniform (slots are padded to whole warps)
             if (M == 1)
-              chunk_dot_cm<P, true, 1>(tab, cf, 8, ck, xs4 + kCmX4 * (c + off[0]), xn2 + kCmXn * (c + off[0]),
-                                       acc[0]);
+              chunk_dot_cm_multi<P, true, 1, MT, kRollOne>(tab, cf, 8, ck, xs4 + kCmX4 * c, xn2 + kCmXn * c, off,
+                                                           1, acc);
             else if (M == 2)
-              chunk_dot_cm_multi<P, true, 1, MT>(tab, cf, 8, ck, xs4 + kCmX4 * c, xn2 + kCmXn * c, off, 2, acc);
+              chunk_dot_cm_multi<P, true, 1, MT, kRollMulti>(tab, cf, 8, ck, xs4 + kCmX4 * c, xn2 + kCmXn * c,
+                                                             off, 2, acc);
             else
-              chunk_dot_cm_multi<P, true, 1, MT>(tab, cf, 8, ck, xs4 + kCmX4 * c, xn2 + kCmXn * c, off, M, acc);
+              chunk_dot_cm_multi<P, true, 1, MT, kRollMulti>(tab, cf, 8, ck, xs4 + kCmX4 * c, xn2 + kCmXn * c,
+                                                             off, M, acc);
           }
           if ((k & 1) && r >= 0) {
 #pragma unroll
