@@ -463,7 +463,7 @@ __device__ __forceinline__ void chunk_dot_cm_multi(const uint32_t *tl, const Chu
         }
       }
     }
-    if (BPI < 8) shift_chunk<P, (BPI < 8 ? BPI / 2 : 1)>(g);
+    if constexpr (BPI < 8) shift_chunk<P, BPI / 2>(g);
   }
 }
 
@@ -495,9 +495,9 @@ __device__ __forceinline__ void chunk_dot2_cm_multi(const uint32_t *tl, const Ch
         }
       }
     }
-    if (BPI < 8) {
-      shift_chunk<P, (BPI < 8 ? BPI / 2 : 1)>(ga);
-      shift_chunk<P, (BPI < 8 ? BPI / 2 : 1)>(gb);
+    if constexpr (BPI < 8) {
+      shift_chunk<P, BPI / 2>(ga);
+      shift_chunk<P, BPI / 2>(gb);
     }
   }
 }
