@@ -53,7 +53,10 @@ constexpr int kStageBatch = 1;
 // Blocks unrolled per loop trip in the inner loops of one-token slots
 // (kRollOne) and of slots shared by several tokens (kRollMulti).  Warps of
 // one SM run both kinds of slot at once; fully unrolled, the loops together
-// outgrow the instruction cache.
+// outgrow the instruction cache (15% of warp samples stalled for
+// instructions, 4% with these values).  Measured per layer at 8 tokens,
+// (kRollOne, kRollMulti): (8, 8) 215.4 us, (8, 4) 205.9, (4, 4) 205.6,
+// (2, 2) 208.1, (8, 2) 201.2.
 constexpr int kRollOne = 8;
 constexpr int kRollMulti = 2;
 
