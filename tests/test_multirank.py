@@ -56,3 +56,23 @@ def test_single_rank_needs_no_process_group():
     import bench
     assert bench.slowest_rank_time(0.25, 1, "cpu") == 0.25
     assert bench.job_throughput(1, 100, 1, 0.25) == 400.0
+
+
+def test_reference_arm_line_on_rank_zero(monkeypatch, capsys):
+    # rank 0 runs the oracle on a bounded sample and prints one JSON line with
+    # the arm's keys; its e2e moves no bytes between host and device
+    import json
+
+    import bench
+    monkeypatch.setenv("RANK", "0")
+    args = type("A", (), {"batch": 1, "warmup": 1, "steps": 1, "gpus": 1})()
+    assert bench.run_reference(args) == 0
+    lines = [l for l in capsys.readouterr().out.splitlines() if l.strip()]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    assert d["impl"] == "reference" and d["value"] > 0 and d["higher_is_better"] is True
+    assert d["metric"] == "MoE seed-FFN decode tokens/s" and d["unit"] == "tokens/s"
+    assert d["steps"] == 1 and d["n_gpus"] == 1 and "workload" in d["config"]
+    cb = d["cpu_baseline"]
+    assert cb["kind"] == "oracle" and cb["cores"] >= 1 and cb["sample"] and cb["value"] == d["value"]
+    assert d["e2e"] == {"value": d["value"], "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}
