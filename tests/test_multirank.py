@@ -1,5 +1,5 @@
 """The multi-process bench logic on the CPU: two gloo ranks (one process per
-GPU on the GPU machine; here plain processes), replicas only."""
+GPU in a real run; here plain processes), replicas only."""
 import os
 import socket
 
