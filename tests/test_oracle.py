@@ -268,6 +268,68 @@ def test_layer_stack_chaining_normalises():
         assert abs(np.sqrt(np.mean(xf * xf)) - 1.0) < 1e-2
 
 
+# Closed forms for the layer chaining x' = bf16(y / sqrt(mean(y^2) + 1e-6)),
+# worked by hand.  bf16 keeps 8 significant bits, so a value v in [2^e, 2^(e+1))
+# is a multiple of 2^(e-7) after rounding.
+#   * y = (3, 4, 0, 0): mean(y^2) = 25/4, r = 2.5 (the 1e-6 moves r by 2e-7):
+#     1.2 lies between 1.1953125 and 1.203125 (step 2^-7) and is nearer the
+#     upper; 1.6 lies between 1.59375 and 1.6015625, nearer the upper.  A sum
+#     in place of the mean would give r = 5 and (0.6, 0.8).
+#   * y = 1e-4 everywhere: mean(y^2) = 1e-8, r = sqrt(1.01e-6), so every
+#     entry is 1e-4 / sqrt(1.01e-6) = 1 / sqrt(101) = 0.0995037...; in
+#     [2^-4, 2^-3) the step is 2^-11, and 0.0995037 * 2048 = 203.78, so RNE
+#     gives 204 / 2048 = 0.099609375 where truncation gives 203 / 2048.  Without
+#     the epsilon every entry would be 1.0; with 1e-5 it would be 0.0316...
+_RMS_CASES = [
+    (np.array([3.0, 4.0, 0.0, 0.0]), np.array([1.203125, 1.6015625, 0.0, 0.0])),
+    (np.array([-3.0, 0.0, 4.0, 0.0]), np.array([-1.203125, 0.0, 1.6015625, 0.0])),
+    (np.full(8, 1e-4), np.full(8, 204.0 / 2048.0)),
+]
+
+
+@pytest.mark.parametrize("case", range(len(_RMS_CASES)))
+def test_rms_chain_closed_forms(case):
+    y, want = _RMS_CASES[case]
+    got = O.bf16_to_f64(O.rms_chain(y[None, :]))[0]
+    assert np.array_equal(got, want)
+
+
+def test_rms_chain_normalises_each_token_on_its_own():
+    # three tokens whose scales differ by 10^6: per-token normalisation maps
+    # each to the same closed form (3, 4, 0, 0) -> (1.203125, 1.6015625, 0, 0);
+    # one norm over the whole batch would shrink the small tokens to ~0
+    y = np.array([[3.0, 4.0, 0.0, 0.0], [3e3, 4e3, 0.0, 0.0], [-6.0, -8.0, 0.0, 0.0]])
+    got = O.bf16_to_f64(O.rms_chain(y))
+    assert np.array_equal(got[0], [1.203125, 1.6015625, 0.0, 0.0])
+    assert np.array_equal(got[1], [1.203125, 1.6015625, 0.0, 0.0])
+    assert np.array_equal(got[2], [-1.203125, -1.6015625, 0.0, 0.0])
+
+
+def test_layer_stack_feeds_each_layer_its_predecessors_normalised_output():
+    # layer l+1's input must be the normalised OUTPUT of layer l (not its input):
+    # run the layers one at a time with moe_ffn (pinned on its own above), then
+    # check the chained input is proportional to that output, at unit RMS, to
+    # bf16 precision
+    E, hidden, inter, P, L, k, T = 6, 64, 32, 4, 3, 2, 3
+    layers = []
+    for li in range(L):
+        m = synth.moe_layer(li, E, hidden, inter, P, config=106)
+        layers.append(tuple(getattr(m, n).numpy() for n in ("gate", "up", "down")))
+    logits = np.stack([synth.router_logits((106, li), T, E).numpy() for li in range(L)])
+    x0 = synth.bf16_bits(synth.activations((106,), T, hidden)).numpy().view(np.uint16)
+    _, xs = O.layer_stack(layers, logits, x0, hidden, inter, E, k)
+    for li in range(L - 1):
+        g, u, d = layers[li]
+        ids, w = O.route_topk(logits[li], k)
+        y = O.moe_ffn(g, u, d, E, hidden, inter, xs[li], ids, w, mode=0)
+        nxt = O.bf16_to_f64(xs[li + 1])
+        for t in range(T):
+            rms = np.sqrt(np.mean(y[t] ** 2))
+            # each entry within half a bf16 step (2^-8 relative) of y / rms
+            assert np.all(np.abs(nxt[t] - y[t] / rms) <= (2.0 ** -8 + 1e-4) * np.abs(y[t] / rms))
+            assert abs(np.sqrt(np.mean(nxt[t] ** 2)) - 1.0) < 4e-3
+
+
 # --------------------------------------------------------------- search
 
 @pytest.mark.parametrize("P", [3, 4])
