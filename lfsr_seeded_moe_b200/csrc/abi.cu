@@ -143,42 +143,84 @@ ChunkLayout chunk_layout(int32_t K, int32_t N, int32_t target_ctas, int32_t max_
 
 // --------------------------------------------------------- debug kernels
 
+// The debug dumps run the hot kernels' own regenerators, so that their
+// bit-exact comparison with the oracle covers the code that computes products.
+
+// The 5-bit format's exponent code of block `col` of a row: bit 0 in bit 15 of
+// the coefs word, bits 1..3 at bits 3 col .. 3 col + 2 of the row's codes bytes.
+__device__ __forceinline__ uint32_t p3c5_code(const uint8_t *codes_row, uint32_t q, int col) {
+  const int bit = 3 * col;
+  uint32_t two = codes_row[bit >> 3];
+  if ((bit & 7) > 5) two |= (uint32_t)codes_row[(bit >> 3) + 1] << 8;
+  return ((q >> 15) & 1u) | (((two >> (bit & 7)) & 7u) << 1);
+}
+
+__device__ __forceinline__ const uint8_t *codes_row_of(const nslm_seed_matrix &W, int P, size_t row, int nb) {
+  if (P == 4) return W.codes + row * (size_t)(nb / 2);
+  if (P == kP3C5) return W.codes + row * (size_t)(3 * nb / 8);
+  return nullptr;
+}
+
+// fp32: the decode kernels' chunk regenerator (regen_chunk_block_r, i.e.
+// block_magic on the shared-memory stream tables) gives G[r] = Mg + A_r and the
+// block's scale; the weight is (G[r] - Mg) * scale, both steps exact.  One
+// thread per 64-weight chunk of a row, loaded as the decode kernels load it.
 template <int P>
-__global__ void decompress_kernel(const nslm_seed_matrix W, float *w32, uint16_t *wbf) {
+__global__ void decompress_f32_kernel(const nslm_seed_matrix W, float *w32) {
   __shared__ StreamTables tab;
   build_stream_tables(&tab);
   __syncthreads();
-  const int nb = W.K / 8;
-  const size_t nblk = (size_t)W.N * nb;
-  for (size_t b = (size_t)blockIdx.x * blockDim.x + threadIdx.x; b < nblk;
-       b += (size_t)gridDim.x * blockDim.x) {
-    const size_t row = b / nb, col = b - row * nb;
-    const uint32_t seed = W.seeds[b];
-    const uint32_t q = W.coefs[b];
-    uint32_t lo, hi;
-    stream_word(&tab, seed, lo, hi);
-    float F[8];
-    block_ints(lo, hi, coef_bytes<P>(q), F);
-    uint32_t code;
-    if (P == 4) {
-      code = (W.codes[row * (nb / 2) + col / 2] >> (4 * (col & 1))) & 0xFu;
-    } else if (P == kP3C5) {  // code bits 1..3 at bits 3col.. of the row's codes
-      const uint8_t *cr = W.codes + row * (3 * (size_t)nb / 8);
-      const size_t bit = 3 * col;
-      uint32_t two = cr[bit >> 3];
-      if ((bit & 7) > 5) two |= (uint32_t)cr[(bit >> 3) + 1] << 8;
-      code = ((q >> 15) & 1u) | (((two >> (bit & 7)) & 7u) << 1);
-    } else {
-      code = q >> 12;
-    }
-    const float scale = block_scale(code, row_scale_key(W.exp_bias[row]));
-    const size_t base = row * (size_t)W.K + col * 8;
+  const int nb = W.K / 8, C = (nb + 7) / 8;
+  const size_t nchunk = (size_t)W.N * C;
+  for (size_t t = (size_t)blockIdx.x * blockDim.x + threadIdx.x; t < nchunk;
+       t += (size_t)gridDim.x * blockDim.x) {
+    const size_t row = t / C;
+    const int ch = (int)(t - row * C);
+    const uint16_t *sr = W.seeds + row * nb, *qr = W.coefs + row * nb;
+    const uint8_t *cr = codes_row_of(W, P, row, nb);
+    ChunkFields f;
+    if (nb % 8 == 0) load_chunk<P, true>(sr, qr, cr, nb, ch, f);
+    else load_chunk<P, false>(sr, qr, cr, nb, ch, f);
+    const uint32_t rowk = row_scale_key(W.exp_bias[row]);
+    const int nvalid = min(8, nb - 8 * ch);
+    float *dst = w32 + row * (size_t)W.K + (size_t)ch * 64;
 #pragma unroll
-    for (int r = 0; r < 8; ++r) {
-      const float w = F[r] * scale;  // exact: a 21-bit integer times a power of two
-      if (w32) w32[base + r] = w;
-      if (wbf) wbf[base + r] = __bfloat16_as_ushort(__float2bfloat16_rn(w));
+    for (int i = 0; i < 8; ++i) {
+      if (i >= nvalid) break;
+      float G[8];
+      const float scale = regen_chunk_block_r<P, 1>(tab.t, f, i, rowk, G);
+#pragma unroll
+      for (int r = 0; r < 8; ++r) dst[8 * i + r] = (G[r] - kMagic2) * scale;
     }
+  }
+}
+
+// bf16: the tensor-core tile producer's routine (regen_pair_bf16), one
+// thread per pair of blocks (b, b + 1) of a row, each written as the 16-byte
+// row the producer stores into shared memory.  A row with an odd block count
+// pairs its last block with an empty one whose output is discarded.
+template <int P>
+__global__ void decompress_bf16_kernel(const nslm_seed_matrix W, uint16_t *wbf) {
+  __shared__ StreamTables tab;
+  build_stream_tables(&tab);
+  __syncthreads();
+  const int nb = W.K / 8, npair = (nb + 1) / 2;
+  const size_t ntask = (size_t)W.N * npair;
+  for (size_t t = (size_t)blockIdx.x * blockDim.x + threadIdx.x; t < ntask;
+       t += (size_t)gridDim.x * blockDim.x) {
+    const size_t row = t / npair;
+    const int b = 2 * (int)(t - row * npair);
+    const bool two = b + 1 < nb;
+    const uint16_t *sr = W.seeds + row * nb, *qr = W.coefs + row * nb;
+    const uint32_t s2 = (uint32_t)sr[b] | (two ? (uint32_t)sr[b + 1] << 16 : 0u);
+    const uint32_t q2 = (uint32_t)qr[b] | (two ? (uint32_t)qr[b + 1] << 16 : 0u);
+    const uint8_t *cr = codes_row_of(W, P, row, nb);
+    uint32_t c2 = 0;
+    if (P == 4) c2 = cr[b / 2];
+    if (P == kP3C5) c2 = p3c5_code(cr, q2 & 0xFFFFu, b) | (two ? p3c5_code(cr, q2 >> 16, b + 1) << 4 : 0u);
+    uint4 *dst0 = reinterpret_cast<uint4 *>(wbf + row * (size_t)W.K + (size_t)b * 8);
+    uint4 spare;
+    regen_pair_bf16<P, 1>(tab.t, s2, q2, c2, row_scale_key(W.exp_bias[row]), dst0, two ? dst0 + 1 : &spare);
   }
 }
 
@@ -189,13 +231,21 @@ static int32_t decompress(const nslm_seed_matrix *W, float *w32, uint16_t *wbf, 
   if (!w32 && !wbf) return NSLM_ERR_ARG;
   if ((st = check_device())) return st;
   if (W->N == 0) return NSLM_OK;
-  const size_t nblk = (size_t)W->N * (W->K / 8);
+  if (!aligned16(w32 ? (const void *)w32 : (const void *)wbf)) return NSLM_ERR_ALIGN;
+  const int nb = W->K / 8;
+  const size_t ntask = (size_t)W->N * (w32 ? (nb + 7) / 8 : (nb + 1) / 2);
   const int threads = 256;
-  const int grid = (int)std::min<size_t>((nblk + threads - 1) / threads, (size_t)num_sms() * 8);
+  const int grid = (int)std::min<size_t>((ntask + threads - 1) / threads, (size_t)num_sms() * 8);
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  if (W->P == 4) decompress_kernel<4><<<grid, threads, 0, s>>>(*W, w32, wbf);
-  else if (W->P == kP3C5) decompress_kernel<kP3C5><<<grid, threads, 0, s>>>(*W, w32, wbf);
-  else decompress_kernel<3><<<grid, threads, 0, s>>>(*W, w32, wbf);
+  if (w32) {
+    if (W->P == 4) decompress_f32_kernel<4><<<grid, threads, 0, s>>>(*W, w32);
+    else if (W->P == kP3C5) decompress_f32_kernel<kP3C5><<<grid, threads, 0, s>>>(*W, w32);
+    else decompress_f32_kernel<3><<<grid, threads, 0, s>>>(*W, w32);
+  } else {
+    if (W->P == 4) decompress_bf16_kernel<4><<<grid, threads, 0, s>>>(*W, wbf);
+    else if (W->P == kP3C5) decompress_bf16_kernel<kP3C5><<<grid, threads, 0, s>>>(*W, wbf);
+    else decompress_bf16_kernel<3><<<grid, threads, 0, s>>>(*W, wbf);
+  }
   st = launch_status();
   if (st == NSLM_OK) g_launches = 1;
   return st;
@@ -215,12 +265,26 @@ const char *nslm_status_string(int32_t status) {
     case NSLM_ERR_SHAPE: return "unsupported shape";
     case NSLM_ERR_WORKSPACE: return "workspace missing or too small";
     case NSLM_ERR_CUDA: return "CUDA error";
+    case NSLM_ERR_TIMEOUT: return "a device-side wait gave up";
     case NSLM_ERR_UNSUPPORTED: return "device is not sm_100";
     default: return "unknown status";
   }
 }
 
 int32_t nslm_last_launch_count(void) { return g_launches; }
+
+int32_t nslm_device_status(const void *ws, nslm_stream_t stream) {
+  int32_t st = check_device();
+  if (st) return st;
+  const int32_t *word = static_cast<const int32_t *>(ws);
+  if (!word && (st = static_scratch_status_word(&word))) return st;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if ((st = cuda_status(cudaStreamSynchronize(s)))) return st;
+  int32_t v = 0;
+  if ((st = cuda_status(cudaMemcpyAsync(&v, word, sizeof(v), cudaMemcpyDeviceToHost, s)))) return st;
+  if ((st = cuda_status(cudaStreamSynchronize(s)))) return st;
+  return v == 0 ? NSLM_OK : NSLM_ERR_TIMEOUT;
+}
 
 size_t nslm_workspace_bytes(int32_t op, int32_t T, int32_t E, int32_t hidden, int32_t inter,
                             int32_t k, int32_t L) {

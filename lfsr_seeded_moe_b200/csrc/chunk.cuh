@@ -306,6 +306,38 @@ __device__ __forceinline__ float regen_chunk_block_r(const uint32_t *tl, const C
   return block_scale(code, rowk);
 }
 
+// Regenerate blocks (b, b+1) of one row as bf16 (round to nearest even of
+// the exact weight) and store them as two 16-byte rows: the tile producer of
+// the tensor-core path.  seeds2/coefs2 hold the two blocks' 16-bit fields;
+// code2 their two exponent nibbles (low nibble: block b) for P = 4 and the
+// 5-bit format, unused for P = 3 (the code is the top nibble of coefs); tl is
+// this lane's copy of R interleaved stream tables.
+template <int P, int R>
+__device__ __forceinline__ void regen_pair_bf16(const uint32_t *tl, uint32_t seeds2, uint32_t coefs2,
+                                                uint32_t code2, uint32_t rowk, uint4 *dst0, uint4 *dst1) {
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    const uint32_t q = h ? (coefs2 >> 16) : (coefs2 & 0xFFFFu);
+    const uint32_t b0 = h ? ((seeds2 >> 16) & 0xFFu) : (seeds2 & 0xFFu);
+    const uint32_t b1 = h ? (seeds2 >> 24) : ((seeds2 >> 8) & 0xFFu);
+    const uint32_t nxt = tl[R * b0] ^ tl[R * (256u + b1)];
+    const uint32_t v = h ? (seeds2 & 0xFFFF0000u) : (seeds2 << 16);
+    float G[8];
+    block_magic(v, nxt, coef_pairs2<P>(q), G);
+    const uint32_t code = (P == 3) ? (q >> 12) : ((code2 >> (4 * h)) & 0xFu);
+    const float s = block_scale(code, rowk);
+    const float off = -kMagic2 * s;
+    uint32_t packed[4];
+#pragma unroll
+    for (int r = 0; r < 8; r += 2) {
+      // (Mg + A) * s - Mg * s = A * s exactly (power-of-two scale)
+      const __nv_bfloat162 bb = __floats2bfloat162_rn(fmaf(G[r], s, off), fmaf(G[r + 1], s, off));
+      packed[r >> 1] = *reinterpret_cast<const uint32_t *>(&bb);
+    }
+    *(h ? dst1 : dst0) = make_uint4(packed[0], packed[1], packed[2], packed[3]);
+  }
+}
+
 // <G, x> - Mg * sum(x) for one staged vector, as a packed pair sum.
 __device__ __forceinline__ float block_dot(const float (&G)[8], const float4 &xa, const float4 &xb,
                                            const float2 &xn) {

@@ -66,35 +66,6 @@ struct GroupedParams {
 // the bank conflicts it removes.
 constexpr int kTabCopies = 1;
 
-// Regenerate blocks (b, b+1) of one row as bf16 and store them as two 16-byte
-// core-matrix rows.  seeds2/coefs2 hold the two blocks' 16-bit fields, code2
-// their two exponent nibbles; tl is this lane's table copy.
-template <int P>
-__device__ __forceinline__ void regen_pair_bf16(const uint32_t *tl, uint32_t seeds2, uint32_t coefs2,
-                                                uint32_t code2, uint32_t rowk, uint4 *dst0, uint4 *dst1) {
-#pragma unroll
-  for (int h = 0; h < 2; ++h) {
-    const uint32_t q = h ? (coefs2 >> 16) : (coefs2 & 0xFFFFu);
-    const uint32_t b0 = h ? ((seeds2 >> 16) & 0xFFu) : (seeds2 & 0xFFu);
-    const uint32_t b1 = h ? (seeds2 >> 24) : ((seeds2 >> 8) & 0xFFu);
-    const uint32_t nxt = tl[kTabCopies * b0] ^ tl[kTabCopies * (256u + b1)];
-    const uint32_t v = h ? (seeds2 & 0xFFFF0000u) : (seeds2 << 16);
-    float G[8];
-    block_magic(v, nxt, coef_pairs2<P>(q), G);
-    const uint32_t code = (P == 4) ? ((code2 >> (4 * h)) & 0xFu) : (q >> 12);
-    const float s = block_scale(code, rowk);
-    const float off = -kMagic2 * s;
-    uint32_t packed[4];
-#pragma unroll
-    for (int r = 0; r < 8; r += 2) {
-      // (Mg + A) * s - Mg * s = A * s exactly (power-of-two scale)
-      const __nv_bfloat162 bb = __floats2bfloat162_rn(fmaf(G[r], s, off), fmaf(G[r + 1], s, off));
-      packed[r >> 1] = *reinterpret_cast<const uint32_t *>(&bb);
-    }
-    *(h ? dst1 : dst0) = make_uint4(packed[0], packed[1], packed[2], packed[3]);
-  }
-}
-
 // Tile shapes: every thread owns two tasks per K slice -- two consecutive
 // blocks (16 weights) of the same row of both 128-row sub-tiles.  GATEUP tiles are
 // 128 rows of gate and the same 128 rows of up (two accumulators); the other
@@ -376,7 +347,7 @@ __global__ void __launch_bounds__(kCtaThreads, 1) grouped_seed_gemm_kernel(const
         for (int j = 0; j < 2; ++j) {
           uint4 *dst0 = reinterpret_cast<uint4 *>(atile + j * kBM * 128 + a_off);
           uint4 *dst1 = reinterpret_cast<uint4 *>(atile + j * kBM * 128 + a_off + 128);
-          regen_pair_bf16<P>(tl, f.s2[j], f.q2[j], f.c2[j], rowk[j], dst0, dst1);
+          regen_pair_bf16<P, kTabCopies>(tl, f.s2[j], f.q2[j], f.c2[j], rowk[j], dst0, dst1);
         }
         if (kt + 3 < ksteps) load_slice<P>(sp, qp, cpp, ok, kt + 3, f);
         cp_async_wait<1>();  // this slice's token rows (the next slice's may still be in flight)

@@ -22,15 +22,9 @@
 //    seed byte (computed at compile time; each CTA copies the 2 KB into
 //    shared memory).
 //
-// 2. Byte dot products.  For a window Z = W >> (1 + t), the integer
-//    d_t = sum_j c_j * byte_j(Z) is one dp4a (unsigned stream bytes times
-//    signed coefficient bytes).  Because s_{1+8j+r} = byte_j(W >> (1+r)) +
-//    256 * byte_j(W >> (9+r)),
-//        sum_j c_j * s_{1+8j+r} = d_r + 256 * d_{r+8},
-//    so 16 funnel shifts and 16 dp4a give all 8 A_r.  The centring term
-//    -32768 * sum_j c_j and a float "magic" offset ride in the dp4a
-//    accumulator, so A_r + 1.5 * 2^23 lands in an fp32 bit pattern and one
-//    subtraction recovers A_r exactly (no int-to-float convert).
+// 2. Two-way dot products.  The decode kernels and the tensor-core tile
+//    producer turn the stream and the coefficients into the 8 integers A_r
+//    with 15 funnel shifts and 16 dp2a per block (chunk.cuh, block_magic).
 //
 // Measured on this B200 (warp instructions per clock per SM): LOP3/SHF/PRMT
 // share one pipe at 2.0, DP4A/IMAD another at 2.0, and a mix of the two
@@ -40,9 +34,6 @@
 #include <cuda_runtime.h>
 
 namespace nslm {
-
-constexpr uint32_t kMagicBits = 0x4B400000u;  // 1.5 * 2^23 as fp32
-constexpr float kMagic = 12582912.0f;
 
 // ---------------------------------------------------------------- stream
 
@@ -149,21 +140,7 @@ __device__ __forceinline__ void stream_word(const StreamTables *tab, uint32_t se
   hi = nxt >> 16;
 }
 
-// ----------------------------------------------------------- coefficients
-
-// Packed coefficient nibbles -> four signed bytes [c0, c1, c2, c3]
-// (P = 3: byte 3 is 0; the top nibble there is the exponent code).
-template <int P>
-__device__ __forceinline__ uint32_t coef_bytes(uint32_t q16) {
-  if (P == 35) {  // three 5-bit fields: a set bit 4 adds 0xE0
-    const uint32_t v = (q16 & 0x1Fu) | ((q16 << 3) & 0x1F00u) | ((q16 << 6) & 0x1F0000u);
-    return v + (v & 0x101010u) * 14u;
-  }
-  uint32_t v = (q16 | (q16 << 12)) & 0x0F0F0F0Fu;            // [c0, c2, c1, c3]
-  v = __byte_perm(v, 0u, P == 4 ? 0x3120 : 0x4120);          // [c0, c1, c2, c3|0]
-  // two's-complement nibble -> byte: a set bit 3 adds 0xF0 (no carry out)
-  return v + (v & 0x08080808u) * 30u;
-}
+// ------------------------------------------------------- dot-product ops
 
 __device__ __forceinline__ int32_t dp4a_us(uint32_t a_u8x4, uint32_t b_s8x4, int32_t acc) {
   int32_t d;
@@ -191,23 +168,6 @@ __device__ __forceinline__ int32_t dp2a_hi_us(uint32_t a_u16x2, uint32_t b_s8x4,
 }
 
 // ----------------------------------------------------------------- block
-
-// The 8 weights of a block as fp32 (w_r = A_r exactly, before the power-of-
-// two scale): F[r] = (float)A_r.
-__device__ __forceinline__ void block_ints(uint32_t lo, uint32_t hi, uint32_t cb,
-                                           float (&F)[8]) {
-  int32_t csum = dp4a_ss(cb, 0x01010101u, 0);
-  int32_t base = (int32_t)kMagicBits - 32768 * csum;
-#pragma unroll
-  for (int r = 0; r < 8; ++r) {
-    uint32_t z0 = __funnelshift_r(lo, hi, 1 + r);   // W >> (1 + r)
-    uint32_t z1 = __funnelshift_r(lo, hi, 9 + r);   // W >> (9 + r)
-    int32_t d0 = dp4a_us(z0, cb, base);
-    int32_t d1 = dp4a_us(z1, cb, 0);
-    int32_t bits = d0 + 256 * d1;                   // bit pattern of kMagic + A_r
-    F[r] = __int_as_float(bits) - kMagic;
-  }
-}
 
 // Scale 2^(code + bias - 15) as an fp32 bit pattern: rowk = (bias + 112) << 23.
 __device__ __forceinline__ float block_scale(uint32_t code, uint32_t rowk) {

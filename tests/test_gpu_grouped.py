@@ -94,12 +94,27 @@ def test_batched_ffn_zipf_skew(nslm):
     assert O.normwise_rel_err(got, ref) <= TOL
 
 
+def _every_row_within(got, ref):
+    # every token row on its own scale, so an error confined to one tile of
+    # one expert cannot hide behind the other rows' magnitudes
+    assert np.all(np.isfinite(got))
+    errs = [O.normwise_rel_err(got[t], ref[t]) for t in range(got.shape[0])]
+    worst = int(np.argmax(errs))
+    assert errs[worst] <= TOL, (worst, errs[worst], O.elementwise_rel_err(got[worst], ref[worst]))
+    assert O.normwise_rel_err(got, ref) <= TOL
+
+
 def test_batched_ffn_layer_64_tokens(nslm):
-    # batched MoE layer: 64 tokens, 100 experts, hidden 2048, intermediate 1408, P=3, top-8
-    got, ref = _batched_case(nslm, 100, 2048, 1408, 3, 64, 8, 963, sample=[0, 1, 17, 42, 63])
-    assert O.normwise_rel_err(got, ref) <= TOL
+    # batched MoE layer: 64 tokens, 100 experts, hidden 2048, intermediate 1408, P=3, top-8;
+    # every token row against the oracle
+    got, ref = _batched_case(nslm, 100, 2048, 1408, 3, 64, 8, 963)
+    _every_row_within(got, ref)
 
 
-def test_batched_ffn_layer_512_tokens_zipf(nslm):
-    got, ref = _batched_case(nslm, 100, 2048, 1408, 3, 512, 8, 964, zipf=1.1, sample=[0, 255, 511])
-    assert O.normwise_rel_err(got, ref) <= TOL
+@pytest.mark.parametrize("zipf", [None, 1.1])
+def test_batched_ffn_layer_512_tokens(nslm, zipf):
+    # the benchmarked batched layers (uniform and Zipf s=1.1 routing), every
+    # token row against the oracle: hot experts take several N tiles, and the
+    # last ragged M tile and late tiles' epilogues are all compared
+    got, ref = _batched_case(nslm, 100, 2048, 1408, 3, 512, 8, 964, zipf=zipf)
+    _every_row_within(got, ref)

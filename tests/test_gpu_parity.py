@@ -61,13 +61,38 @@ def test_decompress_fp32_bit_exact_all_seeds(nslm, P):
 
 @pytest.mark.parametrize("P", [3, 4, 35])
 def test_decompress_bf16_bit_exact_all_seeds(nslm, P):
-    m = _all_seed_matrix(P, -20, 10)
+    # the tensor-core tile producer's routine, over every seed and biases
+    # -100..100 (every weight a normal bf16 number)
+    m = _all_seed_matrix(P)
     md = _dev(m)
-    w = torch.empty(m.N, m.K, dtype=torch.int16, device="cuda")
+    w = torch.full((m.N, m.K), -1, dtype=torch.int16, device="cuda")
     nslm.nslm_debug_decompress_bf16(md, w)
     torch.cuda.synchronize()
     ref = O.decompress_bf16(m.numpy())
     assert np.array_equal(w.cpu().numpy().view(np.uint16), ref)
+
+
+@pytest.mark.parametrize("P,N,K", [(3, 37, 8 * 13), (4, 29, 16 * 7), (3, 5, 8), (4, 3, 16)])
+def test_decompress_ragged_rows_bit_exact(nslm, P, N, K):
+    # rows whose block count is not a multiple of 8 (the decode kernels' ragged
+    # chunk loads) or is odd (the bf16 producer's last block pairs with an
+    # empty one); every entry is written, none past the end
+    m = synth.seed_matrix(N, K, P, (905, N, K, P))
+    m.exp_bias = torch.linspace(-100, 100, N).round().to(torch.int32)
+    md = _dev(m)
+    pad = 64
+    w = torch.full((N * K + pad,), float("nan"), dtype=torch.float32, device="cuda")
+    nslm.nslm_debug_decompress(md, w)
+    wb = torch.full((N * K + pad,), -1, dtype=torch.int16, device="cuda")
+    nslm.nslm_debug_decompress_bf16(md, wb)
+    torch.cuda.synchronize()
+    got = w.cpu().numpy()
+    ref = O.decompress(m.numpy(), np.float32).reshape(-1)
+    assert np.array_equal(got[:N * K].view(np.uint32), ref.view(np.uint32))
+    assert np.all(np.isnan(got[N * K:]))
+    gb = wb.cpu().numpy().view(np.uint16)
+    assert np.array_equal(gb[:N * K], O.decompress_bf16(m.numpy()).reshape(-1))
+    assert np.all(gb[N * K:] == 0xFFFF)
 
 
 GEMV_SHAPES = [(512, 1024), (2048, 4096), (4096, 2048), (1408, 2048), (2048, 1408)]
@@ -213,7 +238,7 @@ def test_ffn_one_token_all_ids_dropped_gives_zero(nslm):
 def test_ffn_decode_one_token_full_layer(nslm):
     # one MoE layer decode: 100 experts, hidden 2048, intermediate 1408, P=4, top-8
     y, ref = _ffn_case(nslm, 100, 2048, 1408, 4, 1, 8, 906)
-    assert O.normwise_rel_err(y, ref) <= TIGHT
+    assert O.normwise_rel_err(y, ref) <= TIGHT, O.elementwise_rel_err(y, ref)
 
 
 @pytest.mark.parametrize("T", [2, 5, 8])
@@ -228,7 +253,7 @@ def test_ffn_decode_batch8_full_layer(nslm):
     # experts, and the 64 routed h vectors are staged for the down projection
     # in several groups
     y, ref = _ffn_case(nslm, 100, 2048, 1408, 4, 8, 8, 940)
-    assert O.normwise_rel_err(y, ref) <= TIGHT
+    assert O.normwise_rel_err(y, ref) <= TIGHT, O.elementwise_rel_err(y, ref)
 
 
 @pytest.mark.parametrize("P", [3, 4])
@@ -366,12 +391,14 @@ def _stack_prefix(nslm, dl, logits, x, T, E, hidden, inter, k, n):
     return y.cpu().numpy().astype(np.float64)
 
 
-def test_stack_decode_batch8_full_layers_pinned(nslm):
-    # 8 tokens through two layers of the 100-expert 2048/1408 P=4 stack, each
-    # layer checked against the oracle on the GPU's own input
-    Lyr, E, hidden, inter, P, k, T = 2, 100, 2048, 1408, 4, 8, 8
+@pytest.mark.parametrize("T", [1, 8])
+def test_stack_decode_full_layers_pinned(nslm, T):
+    # the benchmarked stack configuration (100 experts, 2048/1408, P=4, top-8),
+    # one token and 8 tokens, through two layers of one persistent launch;
+    # each layer checked against the oracle on the GPU's own input
+    Lyr, E, hidden, inter, P, k = 2, 100, 2048, 1408, 4, 8
     layers = [synth.moe_layer(l, E, hidden, inter, P, config=943) for l in range(Lyr)]
-    logits = torch.stack([synth.router_logits((943, l), T, E) for l in range(Lyr)])
+    logits = torch.stack([synth.router_logits((943, l, T), T, E) for l in range(Lyr)])
     x, xh = _x((943, T), T, hidden)
     dl = [(_dev(m.gate), _dev(m.up), _dev(m.down)) for m in layers]
     ys = [_stack_prefix(nslm, dl, logits, x, T, E, hidden, inter, k, n) for n in (1, 2)]
@@ -380,7 +407,10 @@ def test_stack_decode_batch8_full_layers_pinned(nslm):
         xl = xh if l == 0 else O.rms_chain(ys[l - 1])
         ids, w = O.route_topk(logits[l].numpy(), k)
         ref = O.moe_ffn(g, u, d, E, hidden, inter, xl, ids, w, mode=0)
-        assert O.normwise_rel_err(ys[l], ref) <= TOL, l
+        # layer 0 to the fp32 decode path's own accuracy; later layers to the
+        # stated bar, since the GPU's fp32 normalisation of y and the oracle's
+        # fp64 one may round a few inputs to neighbouring bf16 values
+        assert O.normwise_rel_err(ys[l], ref) <= (TIGHT if l == 0 else TOL), (l, O.elementwise_rel_err(ys[l], ref))
     assert np.array_equal(ys[1], _stack_prefix(nslm, dl, logits, x, T, E, hidden, inter, k, 2))
 
 
