@@ -67,6 +67,9 @@ typedef struct CUstream_st *nslm_stream_t;
 #define NSLM_ERR_SHAPE (-3)       /* N, K, P or a size outside what is supported */
 #define NSLM_ERR_WORKSPACE (-4)   /* workspace missing or smaller than required */
 #define NSLM_ERR_CUDA (-5)        /* a CUDA call or launch failed */
+#define NSLM_ERR_TIMEOUT (-6)     /* a bounded device-side wait gave up; only
+                                     nslm_device_status returns it, once the
+                                     work it reports on has completed */
 #define NSLM_ERR_UNSUPPORTED (-7) /* the current device is not sm_100 */
 
 /* P = NSLM_P3C5: three coefficients of 5 bits ("NanoSeedLM: LLM inference
@@ -202,7 +205,11 @@ int32_t nslm_moe_seed_ffn_hybrid(const nslm_moe_layer *p3, int32_t E3, const nsl
  * call before capturing any stream.  All calls share the one array: calls
  * whose work overlaps on the GPU (e.g. on two streams at once) race and give
  * wrong results.  Each call rewrites what it reads, so the contents left by an
- * earlier call do no harm. */
+ * earlier call do no harm.  A grid-barrier wait that gives up (about 1 s) is
+ * reported by nslm_device_status(NULL, stream), not by the return value.
+ * The cached address belongs to the CUDA context it was looked up in: after
+ * cudaDeviceReset the library must be reloaded before this entry point is
+ * called again on that device. */
 int32_t nslm_moe_seed_ffn_static(const nslm_seed_matrix *gate, const nslm_seed_matrix *up,
                                  const nslm_seed_matrix *down, int32_t E, const uint16_t *x_bf16,
                                  const int32_t *ids, const float *w, int32_t T, int32_t k,
@@ -316,6 +323,20 @@ int32_t nslm_debug_wait_probe(int32_t kind, int32_t *out, int64_t cycles, nslm_s
 int32_t nslm_debug_decompress(const nslm_seed_matrix *W, float *w_out, nslm_stream_t stream);
 int32_t nslm_debug_decompress_bf16(const nslm_seed_matrix *W, uint16_t *w_out,
                                    nslm_stream_t stream);
+
+/* Device-side status of the calls that used workspace ws: NSLM_OK, or
+ * NSLM_ERR_TIMEOUT if a bounded wait of one of them gave up (the grid barrier
+ * of a persistent decode kernel, about 1 s, or a tensor-core pipeline wait,
+ * about 2 s).  Such a call has returned NSLM_OK to its caller, because the
+ * wait happens on the GPU after the call returned; its output is then
+ * incomplete.  The status is the first int32 of the workspace, which every
+ * decode or tensor-core call rewrites at its start, so it reports the last
+ * call that used ws.  ws = NULL reads the status of the built-in scratch of
+ * nslm_moe_seed_ffn_static instead.
+ * Not for the hot path: it waits for `stream` to finish (cudaStreamSynchronize)
+ * and then copies the 4-byte word to the host, so it cannot be captured in a
+ * CUDA graph.  Returns NSLM_ERR_CUDA if the stream reports an error. */
+int32_t nslm_device_status(const void *ws, nslm_stream_t stream);
 
 /* A static, human-readable name for a status code. */
 const char *nslm_status_string(int32_t status);

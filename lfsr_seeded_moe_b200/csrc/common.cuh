@@ -39,6 +39,10 @@ int32_t max_active_ctas(const void *kernel, int threads, size_t smem);
 
 int32_t check_matrix(const nslm_seed_matrix *W);
 
+// Device address of the status word (offset 0) of the built-in scratch array
+// of nslm_moe_seed_ffn_static on the current device.
+int32_t static_scratch_status_word(const int32_t **out);
+
 // Work layout of one seed matrix product: a CTA covers R rows x C chunks of
 // 8 blocks (64 weights); C = ceil(nb / 8).
 struct ChunkLayout {

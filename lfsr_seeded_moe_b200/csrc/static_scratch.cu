@@ -46,6 +46,14 @@ int32_t static_scratch_address(void **out) {
 }
 
 }  // namespace
+
+int32_t static_scratch_status_word(const int32_t **out) {
+  void *p = nullptr;
+  const int32_t st = static_scratch_address(&p);
+  if (st == NSLM_OK) *out = static_cast<const int32_t *>(p);
+  return st;
+}
+
 }  // namespace nslm
 
 using namespace nslm;

@@ -26,6 +26,7 @@ NSLM_ERR_ALIGN = -2
 NSLM_ERR_SHAPE = -3
 NSLM_ERR_WORKSPACE = -4
 NSLM_ERR_CUDA = -5
+NSLM_ERR_TIMEOUT = -6
 NSLM_ERR_UNSUPPORTED = -7
 
 NSLM_P3C5 = 35  # P = 3 with 5-bit coefficients
@@ -85,6 +86,7 @@ def _load():
         "nslm_debug_wait_probe": (i32, [i32, vp, ctypes.c_int64, vp]),
         "nslm_debug_decompress": (i32, [mp, vp, vp]),
         "nslm_debug_decompress_bf16": (i32, [mp, vp, vp]),
+        "nslm_device_status": (i32, [vp, vp]),
         "nslm_status_string": (ctypes.c_char_p, [i32]),
         "nslm_last_launch_count": (i32, []),
     }
@@ -148,6 +150,16 @@ def nslm_status_string(status: int) -> str:
 
 def nslm_last_launch_count() -> int:
     return int(_lib.nslm_last_launch_count())
+
+
+def nslm_device_status(ws=None, stream=None) -> int:
+    """NSLM_OK or NSLM_ERR_TIMEOUT for the last call that used ws (None: the
+    static-scratch entry point).  Waits for the stream; returns the status
+    rather than raising on NSLM_ERR_TIMEOUT (other errors raise)."""
+    rc = int(_lib.nslm_device_status(_p(ws), _s(stream)))
+    if rc not in (NSLM_OK, NSLM_ERR_TIMEOUT):
+        raise NslmError("nslm_device_status", rc)
+    return rc
 
 
 def nslm_workspace_bytes(op: int, T: int, E: int, hidden: int, inter: int, k: int, L: int = 0) -> int:

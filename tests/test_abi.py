@@ -18,7 +18,7 @@ def test_every_declared_symbol_is_exported():
 
 
 def test_status_strings():
-    for code in (0, -1, -2, -3, -4, -5, -7):
+    for code in (0, -1, -2, -3, -4, -5, -6, -7):
         assert nslm.nslm_status_string(code) not in ("", "unknown status")
     assert nslm.nslm_status_string(12345) == "unknown status"
 

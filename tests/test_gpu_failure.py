@@ -42,6 +42,9 @@ def test_grid_barrier_wait_gives_up_and_reports(nslm):
     torch.cuda.synchronize()
     assert time.time() - t0 < 5.0
     assert out.cpu().tolist() == [1, 0, 1, 0, 0]  # status 1, abort raised, the wait returned false
+    # out[0..3] are laid out as the head of a decode workspace: the status
+    # reader maps the give-up to NSLM_ERR_TIMEOUT
+    assert nslm.nslm_device_status(out) == nslm.NSLM_ERR_TIMEOUT
     _gemv_still_works(nslm)
 
 
@@ -50,6 +53,7 @@ def test_grid_barrier_wait_passes_once_arrived(nslm):
     nslm.nslm_debug_wait_probe(0, out, LIMIT)
     torch.cuda.synchronize()
     assert out.cpu().tolist() == [0, 1, 0, 0, 1]
+    assert nslm.nslm_device_status(out) == nslm.NSLM_OK
 
 
 def test_grid_barrier_wait_stops_at_the_abort_flag(nslm):
