@@ -67,25 +67,70 @@ def layer_packed_bytes_per_token() -> int:
 # ------------------------------------------------------------------ clocks
 
 class ClockSampler:
-    """Samples SM clocks and throttle reasons with nvidia-smi while running."""
+    """Samples SM clocks and throttle reasons while the timed region runs.
+
+    NVML is polled every 2 ms from a thread (so that even a region of a few
+    tens of milliseconds gets several samples), on the GPU that CUDA device
+    `dev` is (matched by UUID, since CUDA and NVML may number GPUs
+    differently); without NVML, nvidia-smi is run at its 20 ms interval.
+    Every sample is kept as one CSV row in nvidia-smi's field order."""
 
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    # NVML reason bits, in the order of the last four fields
+    BITS = (0x8, 0x40, 0x20, 0x4)
 
-    def __init__(self, gpu_index: int):
+    def __init__(self, gpu_index: int, uuid: str | None = None, period_s: float = 0.002):
         self.gpu = gpu_index
+        self.uuid = uuid
+        self.period = period_s
         self.proc = None
+        self.thread = None
+        self.stop = threading.Event()
         self.lines = []
 
+    def _nvml_handle(self):
+        import pynvml
+        pynvml.nvmlInit()
+        if self.uuid:
+            try:
+                return pynvml, pynvml.nvmlDeviceGetHandleByUUID(self.uuid)
+            except pynvml.NVMLError:
+                pass
+        return pynvml, pynvml.nvmlDeviceGetHandleByIndex(self.gpu)
+
+    def _poll(self, nv, h):
+        try:
+            mx = nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM)
+        except nv.NVMLError:
+            mx = "[N/A]"
+        while not self.stop.is_set():
+            try:
+                sm = nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM)
+                pw = nv.nvmlDeviceGetPowerUsage(h) / 1000.0
+                rs = nv.nvmlDeviceGetCurrentClocksEventReasons(h)
+                flags = ", ".join("Active" if rs & b else "Not Active" for b in self.BITS)
+                self.lines.append(f"{self.gpu}, {sm}, {mx}, {pw:.1f}, {rs:#x}, {flags}")
+            except nv.NVMLError:
+                pass
+            self.stop.wait(self.period)
+
     def __enter__(self):
+        try:
+            nv, h = self._nvml_handle()
+            self.thread = threading.Thread(target=self._poll, args=(nv, h), daemon=True)
+            self.thread.start()
+            return self
+        except Exception:  # no NVML: fall back to nvidia-smi
+            self.thread = None
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
                  "--format=csv,noheader,nounits", "-lms", "20"],
                 stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
-            self.t = threading.Thread(target=self._read, daemon=True)
-            self.t.start()
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
         except OSError:
             self.proc = None
         return self
@@ -95,12 +140,15 @@ class ClockSampler:
             self.lines.append(line.strip())
 
     def __exit__(self, *exc):
+        self.stop.set()
         if self.proc is not None:
             self.proc.terminate()
             try:
                 self.proc.wait(timeout=5)
             except subprocess.TimeoutExpired:
                 self.proc.kill()
+        if self.thread is not None:
+            self.thread.join(timeout=5)
 
     def summary(self):
         sm, mx, reasons = [], None, set()
@@ -121,6 +169,14 @@ class ClockSampler:
             return {"sm_mhz": None, "sm_max_mhz": mx, "reasons": [], "samples": 0}
         return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
                 "samples": len(sm)}
+
+
+def device_uuid(torch, dev) -> str | None:
+    """NVML's name of the GPU behind CUDA device `dev` ("GPU-<uuid>")."""
+    try:
+        return "GPU-" + str(torch.cuda.get_device_properties(dev).uuid)
+    except Exception:
+        return None
 
 
 # --------------------------------------------------------------- oracle leg
@@ -162,40 +218,114 @@ def oracle_layer_seconds(n_layers: int, T: int = 1, seed_tag: int = 0):
     return total
 
 
-def cpu_baseline(budget_s: float = 15.0, T: int = 1):
+def workload_config(T: int, world: int) -> dict:
+    """The workload both arms report (the same dict, key for key)."""
+    per_expert = layer_packed_bytes_per_token() // K_TOP
+    return {"workload": WORKLOAD, "batch_tokens": T, "layers": LAYERS, "experts": E,
+            "hidden": HIDDEN, "inter": INTER, "P": P, "top_k": K_TOP,
+            "packed_GB_resident": round(LAYERS * E * per_expert / 1e9, 3),
+            "l2": "inputs larger than L2 (1.75 GB of weights read per token)",
+            "parallelism": f"replicas x{world}"}
+
+
+def cpu_model() -> str:
+    try:
+        for ln in open("/proc/cpuinfo"):
+            if ln.startswith("model name"):
+                return ln.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    import platform
+    return platform.processor() or "unknown"
+
+
+def _oracle_gemvs(O, synth, np):
+    """The single small GEMV (512 x 1024, P=4) and the expert-sized sweep
+    (P=4 and P=3) on the oracle: us, weights/s and packed-GB/s equivalent."""
+    out = []
+    for Pv, (N, K) in [(4, GEMV_SMALL)] + [(Pv, nk) for Pv in (4, 3) for nk in GEMV_SHAPES]:
+        m = synth.seed_matrix(N, K, Pv, (11, N, K, Pv)).numpy()
+        x = synth.bf16_bits(synth.activations((11,), 1, K)).numpy().view(np.uint16)
+        reps = 4 if N * K < 2 ** 21 else 1
+        t0 = time.perf_counter()
+        for _ in range(reps):
+            O.seed_matvec(m, x)
+        t = (time.perf_counter() - t0) / reps
+        out.append({"P": Pv, "N": N, "K": K, "us": round(t * 1e6, 1), "weights_per_s": round(N * K / t, 1),
+                    "packed_GB_s": round(O.packed_bytes(N, K, Pv) / t / 1e9, 4)})
+    return out
+
+
+def cpu_baseline(budget_s: float = 12.0, T: int = 1):
+    """The oracle timed on this host's cores, with all threads and with one:
+    the seed GEMVs (the 512 x 1024 GEMV and the expert-sized sweep), one
+    decode layer (one token) and the 45-layer stack (one token, a sample of
+    layers scaled to 45).  The headline value is the stack's tokens/s on all
+    cores."""
+    import numpy as np
+
+    from lfsr_seeded_moe_b200 import synth
     from oracle import oracle as O
 
-    t1 = oracle_layer_seconds(1, T, seed_tag=1)
-    n = max(1, min(LAYERS, int(budget_s / max(t1, 1e-3))))
-    t = oracle_layer_seconds(n, T, seed_tag=2) if n > 1 else t1
-    per_layer = t / n
-    tok_s = T / (per_layer * LAYERS)
-    return {"value": tok_s, "unit": "tokens/s", "cores": O.threads_used(), "kind": "oracle",
-            "sample": f"{n} layer(s) x {T} token(s) of the 45-layer stack, oracle fp64, scaled to 45 layers "
-                      f"({per_layer:.3f} s per layer)"}
+    all_cores = O.threads_used()
+    runs = {}
+    try:
+        for threads, share in ((all_cores, 0.6), (1, 0.4)):
+            O.lib().omp_set_num_threads(threads)
+            gemv = _oracle_gemvs(O, synth, np)
+            t1 = oracle_layer_seconds(1, T, seed_tag=1)
+            n = max(1, min(LAYERS, int(share * budget_s / max(t1, 1e-3))))
+            t = oracle_layer_seconds(n, T, seed_tag=2) if n > 1 else t1
+            per_layer = t / n
+            runs[threads] = {
+                "threads": threads, "gemv": gemv,
+                "one_layer": {"us": round(t1 * 1e6, 1), "tokens_per_s": round(T / t1, 3),
+                              "weights_per_s": round(K_TOP * 3 * HIDDEN * INTER * T / t1, 1),
+                              "packed_GB_s": round(layer_packed_bytes_per_token() / t1 / 1e9, 4)},
+                "stack": {"tokens_per_s": T / (per_layer * LAYERS), "layers_timed": n,
+                          "s_per_layer": round(per_layer, 4),
+                          "packed_GB_s": round(layer_packed_bytes_per_token() / per_layer / 1e9, 4)},
+            }
+    finally:
+        O.lib().omp_set_num_threads(all_cores)
+    top = runs[all_cores]["stack"]
+    return {"value": top["tokens_per_s"], "unit": "tokens/s", "cores": all_cores, "kind": "oracle",
+            "nproc": os.cpu_count(), "cpu_model": cpu_model(),
+            "sample": f"{top['layers_timed']} layer(s) x {T} token(s) of the 45-layer stack on all "
+                      f"{all_cores} threads (oracle fp64, routed experts only), scaled to 45 layers; "
+                      f"per-config figures on all threads and on one in 'all_cores' / 'one_core'",
+            "all_cores": runs[all_cores], "one_core": runs[1]}
 
 
 def run_reference(args):
+    """The reference arm: the CPU oracle (the plain C definition of the method)
+    on this host's cores.  Each step is a bounded sample of the workload: one
+    layer of the 45-layer stack for the step's tokens (a different layer and
+    routing each step).  ms_per_step is that measured sample; value scales it to
+    the whole stack's tokens/s."""
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return 0
     from oracle import oracle as O
 
     T = args.batch
-    for _ in range(args.warmup):
-        oracle_layer_seconds(1, T, seed_tag=100)
+    world = int(os.environ.get("WORLD_SIZE", str(args.gpus)))
+    for i in range(args.warmup):
+        oracle_layer_seconds(1, T, seed_tag=100 + i)
     times = [oracle_layer_seconds(1, T, seed_tag=200 + i) for i in range(args.steps)]
     per_layer = sum(times) / len(times)
     tok_s = T / (per_layer * LAYERS)
+    sample = (f"each of {args.steps} step(s): one decode layer of the 45-layer stack for {T} token(s) on the "
+              f"oracle (fp64, {O.threads_used()} threads); tokens/s = tokens / (45 x the mean layer time)")
     line = {
         "impl": "reference", "metric": METRIC, "value": tok_s, "unit": "tokens/s",
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
-        "ms_per_step": per_layer * LAYERS * 1e3, "higher_is_better": True, "scaling": "weak",
+        "ms_per_step": round(per_layer * 1e3, 3), "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded SplitMix64 fields)",
-        "config": {"workload": WORKLOAD, "batch_tokens": T, "layers": LAYERS,
-                   "sample": "each step: one layer of the stack on the CPU oracle, scaled x45"},
+        "config": workload_config(T, world),
+        "step": "one of the stack's 45 layers (a bounded sample); ms_per_step is its measured time",
         "cpu_baseline": {"value": tok_s, "unit": "tokens/s", "cores": O.threads_used(), "kind": "oracle",
-                         "sample": f"{args.steps} step(s) of one decode layer, scaled to 45 layers"},
+                         "nproc": os.cpu_count(), "cpu_model": cpu_model(), "sample": sample},
         "e2e": {"value": tok_s, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line))
@@ -592,7 +722,7 @@ def main():
     if world > 1:
         dist.barrier()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    with ClockSampler(dev.index if dev.index is not None else 0) as clk:
+    with ClockSampler(dev.index if dev.index is not None else 0, device_uuid(torch, dev)) as clk:
         torch.cuda.synchronize()
         e0.record()
         for i in range(args.steps):
@@ -724,12 +854,8 @@ def main():
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(elapsed / args.steps * 1e3, 4),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
         "data": "synthetic (seeded SplitMix64 packed fields, bf16 N(0,1) activations, N(0,1) router logits)",
-        "config": {"workload": WORKLOAD, "batch_tokens": T, "layers": LAYERS, "experts": E,
-                   "hidden": HIDDEN, "inter": INTER, "P": P, "top_k": K_TOP,
-                   "packed_GB_resident": round(sum(L.gate.packed_bytes() + L.up.packed_bytes() + L.down.packed_bytes()
-                                                   for L in layers) / 1e9, 3),
-                   "l2": "inputs larger than L2 (1.75 GB of weights read per token)",
-                   "parallelism": f"replicas x{world}", "graph": "one CUDA graph per step"},
+        "config": workload_config(T, world),
+        "graph": "one CUDA graph per step",
         "clocks": clk.summary(),
         "e2e": e2e,
         "gpu_launches": launches_per_step * args.steps,

@@ -50,3 +50,31 @@ def test_layer_packed_bytes_per_token():
     expert = 3 * 2048 * 1408 // 8 * 9 // 2 + 4 * (1408 + 1408 + 2048)
     assert 3 * 2048 * 1408 // 8 * 9 // 2 == 4_866_048
     assert bench.layer_packed_bytes_per_token() == 8 * expert == 39_084_032
+
+
+def test_cpu_baseline_reports_every_config_on_all_cores_and_one():
+    # the oracle baseline: the seed GEMVs (512 x 1024 and the expert-sized
+    # sweep, P=4 and P=3), one decode layer and the 45-layer stack, each with
+    # all threads and with one, plus the host's core count and CPU model
+    got = bench.cpu_baseline(budget_s=0.5)
+    assert got["kind"] == "oracle" and got["unit"] == "tokens/s" and got["value"] > 0
+    assert got["nproc"] >= 1 and got["cpu_model"] and got["cores"] >= 1
+    assert got["all_cores"]["threads"] == got["cores"] and got["one_core"]["threads"] == 1
+    for run in (got["all_cores"], got["one_core"]):
+        shapes = {(g["P"], g["N"], g["K"]) for g in run["gemv"]}
+        assert (4, 512, 1024) in shapes
+        assert all((Pv, N, K) in shapes for Pv in (3, 4) for N, K in bench.GEMV_SHAPES)
+        assert all(g["weights_per_s"] > 0 and g["packed_GB_s"] > 0 for g in run["gemv"])
+        assert run["one_layer"]["tokens_per_s"] > 0 and run["stack"]["tokens_per_s"] > 0
+    assert got["value"] == got["all_cores"]["stack"]["tokens_per_s"]
+
+
+def test_clock_sampler_rows_from_nvml_reason_bits():
+    # the NVML poller writes rows in nvidia-smi's field order, one Active flag
+    # per reason bit (hw_slowdown 0x8, hw_thermal 0x40, sw_thermal 0x20,
+    # sw_power_cap 0x4), which summary() reads back
+    s = bench.ClockSampler(0)
+    for sm, mask in ((1965, 0x0), (1850, 0x4), (1900, 0x4)):
+        flags = ", ".join("Active" if mask & b else "Not Active" for b in bench.ClockSampler.BITS)
+        s.lines.append(f"0, {sm}, 1965, 900.0, {mask:#x}, {flags}")
+    assert s.summary() == {"sm_mhz": 1900.0, "sm_max_mhz": 1965.0, "reasons": ["sw_power_cap"], "samples": 3}

@@ -72,7 +72,12 @@ def test_reference_arm_line_on_rank_zero(monkeypatch, capsys):
     d = json.loads(lines[0])
     assert d["impl"] == "reference" and d["value"] > 0 and d["higher_is_better"] is True
     assert d["metric"] == "MoE seed-FFN decode tokens/s" and d["unit"] == "tokens/s"
-    assert d["steps"] == 1 and d["n_gpus"] == 1 and "workload" in d["config"]
+    assert d["steps"] == 1 and d["n_gpus"] == 1
+    assert d["config"] == bench.workload_config(1, 1)   # the GPU arm's config, key for key
+    # ms_per_step is the measured time of what a step ran (one layer), which
+    # the value scales to the 45-layer stack
+    assert d["value"] == pytest.approx(1e3 / (45 * d["ms_per_step"]), rel=1e-3)
     cb = d["cpu_baseline"]
     assert cb["kind"] == "oracle" and cb["cores"] >= 1 and cb["sample"] and cb["value"] == d["value"]
+    assert cb["nproc"] >= 1 and cb["cpu_model"]
     assert d["e2e"] == {"value": d["value"], "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}
