@@ -127,6 +127,21 @@ size_t nslm_workspace_bytes(int32_t op, int32_t T, int32_t E, int32_t hidden,
 int32_t nslm_seed_gemv(const nslm_seed_matrix *W, const uint16_t *x_bf16, int32_t M,
                        float *y, void *ws, size_t ws_bytes, nslm_stream_t stream);
 
+/* nslm_seed_gemv with flags (0 gives nslm_seed_gemv exactly):
+ *   NSLM_GEMV_FIELDS_READY  the caller declares that no kernel enqueued
+ *     earlier on `stream` writes W's seeds, coefs, codes or exp_bias.  The
+ *     product kernel is launched with programmatic dependent launch in both
+ *     forms and waits for its predecessor before it reads x or writes y; with
+ *     this flag its first weight-field copies are issued before that wait, so
+ *     they overlap the tail of the preceding kernel (e.g. the previous GEMV of
+ *     a decode step).  If the declaration is false the result is undefined.
+ *     It affects M = 1 with K % 64 == 0 (the one-vector kernel); other
+ *     shapes run as without it.
+ * Other bits return NSLM_ERR_ARG. */
+#define NSLM_GEMV_FIELDS_READY 1u
+int32_t nslm_seed_gemv_flags(const nslm_seed_matrix *W, const uint16_t *x_bf16, int32_t M,
+                             float *y, uint32_t flags, nslm_stream_t stream);
+
 /* Grouped seed GEMM over stacked experts, the batched (prefill) product of
  * "Qwen3.8-Flash-Next" prompt processing ("The prompt time ... the grouped
  * expert GEMMs", NanoSeedLM documentation index, Results).
@@ -316,6 +331,18 @@ int32_t nslm_pack_nibbles(const nslm_seed_matrix *in, uint8_t *nibbles, nslm_str
  * out[0] = 1 if it passed, 0 if it gave up.  cycles: the wait limit in SM
  * clocks (> 0).  out: device, 5 int32.  One launch of one CTA. */
 int32_t nslm_debug_wait_probe(int32_t kind, int32_t *out, int64_t cycles, nslm_stream_t stream);
+
+/* Test export: the bf16 hidden activations h = SiLU(gate x) * (up x) that the
+ * last nslm_moe_seed_ffn call with T > 8 (the tensor-core path) left in its
+ * workspace ws (ws_bytes, T, E, hidden, inter, k as in that call), written
+ * to h_out [T * k][inter] (bf16 bit patterns, DEVICE) in pair order: row
+ * t * k + q is token t's q-th routed expert.  Rows of pairs whose expert id was
+ * outside [0, E) are not written.  It lets a test take the kernel's own
+ * rounding of h to bf16 as given when it checks the down projection.  One
+ * launch; T <= 8 returns NSLM_ERR_SHAPE (the decode path keeps h in fp32). */
+int32_t nslm_debug_batched_hidden(const void *ws, size_t ws_bytes, int32_t T, int32_t E,
+                                  int32_t hidden, int32_t inter, int32_t k, uint16_t *h_out,
+                                  nslm_stream_t stream);
 
 /* Test exports: the regenerated weights themselves, written out densely.
  * w_out: fp32 [N][K] (exact) or bf16 bit patterns [N][K] (round to nearest

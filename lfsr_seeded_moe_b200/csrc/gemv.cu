@@ -147,7 +147,11 @@ struct Gemv1Params {
   FastDiv div_C;
 };
 
-template <int P>
+// EARLY: the caller has declared that no kernel before this one on the stream
+// writes the matrix's fields, so the first task's field copies are issued
+// before griddepcontrol.wait and overlap the tail of the preceding kernel;
+// the activations are read, and y written, only after the wait.
+template <int P, bool EARLY>
 __global__ void __launch_bounds__(kGemv1Threads) gemv1_kernel(const Gemv1Params p) {
   extern __shared__ float4 smem4[];
   const int tid = threadIdx.x, nthr = blockDim.x, warp = tid >> 5, lane = tid & 31;
@@ -160,11 +164,6 @@ __global__ void __launch_bounds__(kGemv1Threads) gemv1_kernel(const Gemv1Params 
   const int nrows = max(0, min(p.rpc, p.W.N - n0));
   const int ntask = nrows * p.C;
   const int nb = p.W.K >> 3;
-  // launched with programmatic stream serialization: wait here for the
-  // preceding kernel (its writes of W or x), then let the next one launch
-  asm volatile("griddepcontrol.wait;" ::: "memory");
-  asm volatile("griddepcontrol.launch_dependents;");
-
   // the 5-bit format's code bits (3 bytes per chunk, not 4-byte aligned) come
   // by plain loads into one register per buffer, one task ahead like the rest
   uint32_t cq0 = 0, cq1 = 0;
@@ -179,8 +178,19 @@ __global__ void __launch_bounds__(kGemv1Threads) gemv1_kernel(const Gemv1Params 
       else cq0 = v;
     }
   };
-  if (tid < ntask) fetch(tid, 0);
-  cp_async_commit();
+  // launched with programmatic stream serialization: wait here for the
+  // preceding kernel (its writes of W or x; with EARLY only of x), then let
+  // the next one launch
+  if (EARLY) {
+    if (tid < ntask) fetch(tid, 0);
+    cp_async_commit();
+  }
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  asm volatile("griddepcontrol.launch_dependents;");
+  if (!EARLY) {
+    if (tid < ntask) fetch(tid, 0);
+    cp_async_commit();
+  }
   // stream tables and activations: every load in flight before the first store
   {
     const uint4 *xrow = reinterpret_cast<const uint4 *>(p.x);
@@ -228,10 +238,8 @@ static size_t gemv1_smem(int C, int rpc, int threads) {
 
 using namespace nslm;
 
-extern "C" int32_t nslm_seed_gemv(const nslm_seed_matrix *W, const uint16_t *x_bf16, int32_t M,
-                                  float *y, void *ws, size_t ws_bytes, nslm_stream_t stream) {
-  (void)ws;
-  (void)ws_bytes;
+static int32_t seed_gemv(const nslm_seed_matrix *W, const uint16_t *x_bf16, int32_t M, float *y,
+                         bool fields_ready, nslm_stream_t stream) {
   g_launches = 0;
   int32_t st = check_matrix(W);
   if (st) return st;
@@ -258,7 +266,9 @@ extern "C" int32_t nslm_seed_gemv(const nslm_seed_matrix *W, const uint16_t *x_b
     const int threads = std::max(64, 32 * ceil_div(ceil_div(tasks, rounds), 32));
     const size_t smem = gemv1_smem(q.C, q.rpc, threads);
     if (smem <= 200 * 1024 && (int64_t)q.rpc * q.C < (1 << 22)) {
-      auto k = (W->P == 4) ? gemv1_kernel<4> : (W->P == kP3C5 ? gemv1_kernel<kP3C5> : gemv1_kernel<3>);
+      auto k = fields_ready
+                   ? ((W->P == 4) ? gemv1_kernel<4, true> : (W->P == kP3C5 ? gemv1_kernel<kP3C5, true> : gemv1_kernel<3, true>))
+                   : ((W->P == 4) ? gemv1_kernel<4, false> : (W->P == kP3C5 ? gemv1_kernel<kP3C5, false> : gemv1_kernel<3, false>));
       if ((st = ensure_smem((const void *)k, smem))) return st;
       ensure_stream_source(s);
       cudaLaunchConfig_t cfg{};
@@ -295,4 +305,18 @@ extern "C" int32_t nslm_seed_gemv(const nslm_seed_matrix *W, const uint16_t *x_b
                          : dispatch_gemv<3>(p, vec, grid, L.threads, smem, s);
   if (st == NSLM_OK) g_launches = 1;
   return st;
+}
+
+extern "C" int32_t nslm_seed_gemv(const nslm_seed_matrix *W, const uint16_t *x_bf16, int32_t M,
+                                  float *y, void *ws, size_t ws_bytes, nslm_stream_t stream) {
+  (void)ws;
+  (void)ws_bytes;
+  return seed_gemv(W, x_bf16, M, y, false, stream);
+}
+
+extern "C" int32_t nslm_seed_gemv_flags(const nslm_seed_matrix *W, const uint16_t *x_bf16, int32_t M,
+                                        float *y, uint32_t flags, nslm_stream_t stream) {
+  g_launches = 0;
+  if (flags & ~(uint32_t)NSLM_GEMV_FIELDS_READY) return NSLM_ERR_ARG;
+  return seed_gemv(W, x_bf16, M, y, (flags & NSLM_GEMV_FIELDS_READY) != 0, stream);
 }

@@ -475,6 +475,20 @@ __global__ void batched_reduce_kernel(const float *__restrict__ part, const int3
   }
 }
 
+// Test export: the bf16 hidden activations a batched FFN call left in its
+// workspace, moved from sorted order to pair order (h_out[t*k + q][inter]).
+__global__ void batched_hidden_kernel(const BatchedPlan bp, int E, int inter, uint16_t *__restrict__ h_out) {
+  const int n = bp.offsets[E];  // valid pairs
+  const int per = inter / 8;    // 16-byte pieces per row
+  const size_t total = (size_t)n * per;
+  for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < total; i += (size_t)gridDim.x * blockDim.x) {
+    const int pos = (int)(i / per), c = (int)(i - (size_t)pos * per);
+    const int pair = bp.pair_of[pos];
+    reinterpret_cast<uint4 *>(h_out + (size_t)pair * inter)[c] =
+        reinterpret_cast<const uint4 *>(bp.h + (size_t)pos * inter)[c];
+  }
+}
+
 // ---------------------------------------------------------------- host
 
 static int tmem_cols_for(int ncols) {
@@ -577,6 +591,26 @@ size_t grouped_ws_bytes(int E) {
 }  // namespace nslm
 
 using namespace nslm;
+
+extern "C" int32_t nslm_debug_batched_hidden(const void *ws, size_t ws_bytes, int32_t T, int32_t E,
+                                             int32_t hidden, int32_t inter, int32_t k, uint16_t *h_out,
+                                             nslm_stream_t stream) {
+  g_launches = 0;
+  if (!ws || !h_out) return NSLM_ERR_ARG;
+  if (T <= kMaxT || k < 1 || k > kMaxK || E < 1 || E > 1024 || hidden % kBK || inter % kBK || hidden <= 0 ||
+      inter <= 0)
+    return NSLM_ERR_SHAPE;
+  const BatchedPlan bp = batched_workspace(static_cast<char *>(const_cast<void *>(ws)), T, k, E, hidden, inter);
+  if (ws_bytes < bp.bytes) return NSLM_ERR_WORKSPACE;
+  if (!aligned16(ws) || !aligned16(h_out)) return NSLM_ERR_ALIGN;
+  int32_t st = check_device();
+  if (st) return st;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  batched_hidden_kernel<<<num_sms() * 4, 256, 0, s>>>(bp, E, inter, h_out);
+  st = launch_status();
+  if (st == NSLM_OK) g_launches = 1;
+  return st;
+}
 
 extern "C" int32_t nslm_seed_grouped_gemm(const nslm_seed_matrix *W, int32_t E,
                                           const uint16_t *x_bf16, const int32_t *offsets,

@@ -30,6 +30,7 @@ NSLM_ERR_TIMEOUT = -6
 NSLM_ERR_UNSUPPORTED = -7
 
 NSLM_P3C5 = 35  # P = 3 with 5-bit coefficients
+NSLM_GEMV_FIELDS_READY = 1
 
 NSLM_OP_GEMV = 0
 NSLM_OP_GROUPED_GEMM = 1
@@ -70,6 +71,7 @@ def _load():
     sig = {
         "nslm_workspace_bytes": (sz, [i32, i32, i32, i32, i32, i32, i32]),
         "nslm_seed_gemv": (i32, [mp, vp, i32, vp, vp, sz, vp]),
+        "nslm_seed_gemv_flags": (i32, [mp, vp, i32, vp, ctypes.c_uint32, vp]),
         "nslm_seed_grouped_gemm": (i32, [mp, i32, vp, vp, i32, vp, vp, sz, vp]),
         "nslm_moe_route_topk": (i32, [vp, i32, i32, i32, vp, vp, vp]),
         "nslm_moe_seed_ffn": (i32, [mp, mp, mp, i32, vp, vp, vp, i32, i32, vp, vp, sz, vp]),
@@ -84,6 +86,7 @@ def _load():
         "nslm_unpack_nibbles": (i32, [vp, mp, vp]),
         "nslm_pack_nibbles": (i32, [mp, vp, vp]),
         "nslm_debug_wait_probe": (i32, [i32, vp, ctypes.c_int64, vp]),
+        "nslm_debug_batched_hidden": (i32, [vp, sz, i32, i32, i32, i32, i32, vp, vp]),
         "nslm_debug_decompress": (i32, [mp, vp, vp]),
         "nslm_debug_decompress_bf16": (i32, [mp, vp, vp]),
         "nslm_device_status": (i32, [vp, vp]),
@@ -169,6 +172,12 @@ def nslm_workspace_bytes(op: int, T: int, E: int, hidden: int, inter: int, k: in
 def nslm_seed_gemv(W, x_bf16, M: int, y, ws=None, ws_bytes: int = 0, stream=None) -> None:
     _check("nslm_seed_gemv", _lib.nslm_seed_gemv(ctypes.byref(_mat(W)), _p(x_bf16), M, _p(y),
                                                   _p(ws), ws_bytes, _s(stream)))
+
+
+def nslm_seed_gemv_flags(W, x_bf16, M: int, y, flags: int = 0, stream=None) -> None:
+    """nslm_seed_gemv with flags (NSLM_GEMV_FIELDS_READY: W is not written by earlier kernels)."""
+    _check("nslm_seed_gemv_flags", _lib.nslm_seed_gemv_flags(ctypes.byref(_mat(W)), _p(x_bf16), M, _p(y),
+                                                              int(flags), _s(stream)))
 
 
 def nslm_seed_grouped_gemm(W, E: int, x_bf16, offsets, R: int, y, ws=None, ws_bytes: int = 0,
@@ -260,6 +269,13 @@ def nslm_pack_nibbles(W, nibbles, stream=None) -> None:
 def nslm_debug_wait_probe(kind: int, out, cycles: int, stream=None) -> None:
     """Run one bounded device wait (see include/nslm.h) with results in out (5 int32)."""
     _check("nslm_debug_wait_probe", _lib.nslm_debug_wait_probe(int(kind), _p(out), int(cycles), _s(stream)))
+
+
+def nslm_debug_batched_hidden(ws, ws_bytes: int, T: int, E: int, hidden: int, inter: int, k: int, h_out,
+                              stream=None) -> None:
+    """bf16 h [T*k][inter] (pair order) left in ws by the last tensor-core FFN call."""
+    _check("nslm_debug_batched_hidden",
+           _lib.nslm_debug_batched_hidden(_p(ws), ws_bytes, T, E, hidden, inter, k, _p(h_out), _s(stream)))
 
 
 def nslm_debug_decompress(W, w_out, stream=None) -> None:

@@ -32,6 +32,11 @@ def _gemv(W, x=0x7000000, M=1, y=0x8000000):
     return nslm.raw().nslm_seed_gemv(ctypes.byref(W), x, M, y, 0, 0, 0)
 
 
+def test_gemv_flags_rejects_unknown_bits():
+    rc = nslm.raw().nslm_seed_gemv_flags(ctypes.byref(_mat()), 0x7000000, 1, 0x8000000, 2, 0)
+    assert rc == nslm.NSLM_ERR_ARG
+
+
 def test_gemv_argument_checks():
     assert _gemv(_mat(P=5)) == nslm.NSLM_ERR_SHAPE
     assert _gemv(_mat(K=24, P=4)) == nslm.NSLM_ERR_SHAPE      # P=4 needs K % 16 == 0

@@ -111,6 +111,26 @@ def test_gemv_matches_oracle(nslm, P, N, K):
     assert err <= TOL and err <= TIGHT, err
 
 
+@pytest.mark.parametrize("P", [3, 4, 35])
+def test_gemv_fields_ready_chain_matches_oracle(nslm, P):
+    # back-to-back GEMVs with NSLM_GEMV_FIELDS_READY (each one's weight copies
+    # start before its predecessor ends); the activations of the second are
+    # written by the kernel just before it, which the flag must still wait for
+    N, K = 2048, 4096
+    ms = [synth.seed_matrix(N, K, P, (904, c, P)) for c in range(3)]
+    x, xh = _x((904, P), 1, K)
+    ys = [_out(1, N) for _ in ms]
+    x2 = torch.empty_like(x)
+    for i, m in enumerate(ms):
+        if i == 1:
+            x2.copy_(x)                       # a kernel that writes the next GEMV's input
+        nslm.nslm_seed_gemv_flags(_dev(m), x2 if i >= 1 else x, 1, ys[i], nslm.NSLM_GEMV_FIELDS_READY)
+    torch.cuda.synchronize()
+    for m, y in zip(ms, ys):
+        ref = O.seed_matvec(m.numpy(), xh)
+        assert O.normwise_rel_err(y.cpu().numpy(), ref) <= TIGHT
+
+
 @pytest.mark.parametrize("M", [2, 3, 8])
 @pytest.mark.parametrize("P", [3, 4, 35])
 def test_gemv_multi_token(nslm, M, P):
