@@ -344,6 +344,21 @@ int32_t nslm_debug_batched_hidden(const void *ws, size_t ws_bytes, int32_t T, in
                                   int32_t hidden, int32_t inter, int32_t k, uint16_t *h_out,
                                   nslm_stream_t stream);
 
+/* Test exports of the bounds-check build (libnslm built with
+ * -DNSLM_BOUNDS_CHECK=1: python -m lfsr_seeded_moe_b200.build --bounds-check).
+ * There every checked global access of the kernels compares its index with
+ * the extent it was given; an index outside records a site number (1-2 field
+ * copies by offset, 3-4 field loads by row, 5-6 the tensor-core producer's
+ * field and token-row loads, 7-9 the tensor-core epilogue's stores, 10 the
+ * decode kernels' h stores) and the access is skipped, so nothing traps.
+ * nslm_debug_bounds_status waits for the device, then returns the first site
+ * recorded since the previous call (0: none) and clears it.
+ * nslm_debug_bounds_probe(W) launches one field copy one chunk past the end
+ * of W (P = 4, K % 64 == 0, N >= 1), which its check refuses as site 1.  In
+ * the normal build both return NSLM_ERR_UNSUPPORTED and launch nothing. */
+int32_t nslm_debug_bounds_status(void);
+int32_t nslm_debug_bounds_probe(const nslm_seed_matrix *W, nslm_stream_t stream);
+
 /* Test exports: the regenerated weights themselves, written out densely.
  * w_out: fp32 [N][K] (exact) or bf16 bit patterns [N][K] (round to nearest
  * even of the exact value).  Not on the hot path. */

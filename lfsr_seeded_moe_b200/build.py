@@ -1,6 +1,6 @@
 """Build libnslm.so (the CUDA library) in-tree for sm_100a with nvcc.
 
-    python -m lfsr_seeded_moe_b200.build [--force] [--stream-source l2next|l2basis]
+    python -m lfsr_seeded_moe_b200.build [--force] [--stream-source l2next|l2basis] [--bounds-check]
 
 The shared library lands in lfsr_seeded_moe_b200/_build/libnslm.so; it is
 rebuilt when any source under csrc/ or include/ is newer than it.
@@ -8,7 +8,10 @@ rebuilt when any source under csrc/ or include/ is newer than it.
 decode kernels take a block's stream bits from an L2-resident 65,536-entry
 table (l2next: the 32 bits after each seed; l2basis: the 16 shifted words of
 each seed) in place of the shared-memory GF(2) tables; the binding loads it
-when NSLM_STREAM_SOURCE names it.
+when NSLM_LIB_VARIANT names it.  --bounds-check builds _build/boundscheck/
+with -DNSLM_BOUNDS_CHECK=1: every checked global access compares its index
+with its extent and records the site instead of making the access (the
+tests run the small parity cases on it).
 """
 from __future__ import annotations
 
@@ -39,6 +42,8 @@ def _inputs():
 
 
 STREAM_SOURCES = {"l2next": 1, "l2basis": 2}
+VARIANT_DEFS = {"l2next": ["-DNSLM_STREAM_SOURCE=1"], "l2basis": ["-DNSLM_STREAM_SOURCE=2"],
+                "boundscheck": ["-DNSLM_BOUNDS_CHECK=1"]}
 
 
 def lib_path(stream_source: str | None = None) -> str:
@@ -60,7 +65,7 @@ def build(force: bool = False, verbose: bool = False, extra_flags=None,
         return lib
     out_dir = os.path.dirname(lib)
     os.makedirs(out_dir, exist_ok=True)
-    defs = [f"-DNSLM_STREAM_SOURCE={STREAM_SOURCES[stream_source]}"] if stream_source else []
+    defs = VARIANT_DEFS[stream_source] if stream_source else []
     jobs = []
     for src in sources():
         obj = os.path.join(out_dir, os.path.basename(src)[:-3] + ".o")
@@ -89,5 +94,7 @@ if __name__ == "__main__":
     src = sys.argv[sys.argv.index("--stream-source") + 1] if "--stream-source" in sys.argv else None
     if src is not None and src not in STREAM_SOURCES:
         raise SystemExit(f"--stream-source must be one of {sorted(STREAM_SOURCES)}")
+    if "--bounds-check" in sys.argv:
+        src = "boundscheck"
     print(build(force="--force" in sys.argv, verbose=True, stream_source=src,
                 extra_flags=["-Xptxas", "-v"] if "--ptxas-v" in sys.argv else None))

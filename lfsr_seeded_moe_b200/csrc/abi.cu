@@ -179,8 +179,8 @@ __global__ void decompress_f32_kernel(const nslm_seed_matrix W, float *w32) {
     const uint16_t *sr = W.seeds + row * nb, *qr = W.coefs + row * nb;
     const uint8_t *cr = codes_row_of(W, P, row, nb);
     ChunkFields f;
-    if (nb % 8 == 0) load_chunk<P, true>(sr, qr, cr, nb, ch, f);
-    else load_chunk<P, false>(sr, qr, cr, nb, ch, f);
+    if (nb % 8 == 0) load_chunk<P, true>(sr, qr, cr, nb, ch, f, row, (size_t)W.N);
+    else load_chunk<P, false>(sr, qr, cr, nb, ch, f, row, (size_t)W.N);
     const uint32_t rowk = row_scale_key(W.exp_bias[row]);
     const int nvalid = min(8, nb - 8 * ch);
     float *dst = w32 + row * (size_t)W.K + (size_t)ch * 64;
@@ -251,6 +251,30 @@ static int32_t decompress(const nslm_seed_matrix *W, float *w32, uint16_t *wbf, 
   return st;
 }
 
+NSLM_BOUNDS_ACCESSOR(abi)
+
+#if NSLM_BOUNDS_CHECK
+int32_t bounds_error_gemv();
+int32_t bounds_error_grouped();
+int32_t bounds_error_moe();
+int32_t bounds_error_stack1();
+int32_t bounds_error_stackb();
+int32_t bounds_error_probe();
+int32_t bounds_error_all() {
+  int32_t (*const fns[])() = {bounds_error_abi, bounds_error_gemv, bounds_error_grouped, bounds_error_moe,
+                              bounds_error_stack1, bounds_error_stackb, bounds_error_probe};
+  int32_t first = 0;
+  for (auto f : fns) {
+    const int32_t v = f();
+    if (v < 0) return NSLM_ERR_CUDA;
+    if (first == 0) first = v;
+  }
+  return first;
+}
+#else
+int32_t bounds_error_all() { return NSLM_ERR_UNSUPPORTED; }
+#endif
+
 }  // namespace nslm
 
 using namespace nslm;
@@ -272,6 +296,13 @@ const char *nslm_status_string(int32_t status) {
 }
 
 int32_t nslm_last_launch_count(void) { return g_launches; }
+
+int32_t nslm_debug_bounds_status(void) {
+  int32_t st = check_device();
+  if (st) return st;
+  if ((st = cuda_status(cudaDeviceSynchronize()))) return st;
+  return bounds_error_all();
+}
 
 int32_t nslm_device_status(const void *ws, nslm_stream_t stream) {
   int32_t st = check_device();

@@ -17,6 +17,7 @@
 #include <cuda_bf16.h>
 
 #include "../../include/nslm.h"
+#include "common.cuh"
 #include "regen.cuh"
 
 namespace nslm {
@@ -131,12 +132,18 @@ struct ChunkFields {
 };
 
 // Loads with an evict-first hint: every packed byte is read once per call.
+// row / nrows: the row's index in its matrix and the matrix's row count (for
+// the bounds-check build; a chunk outside the matrix loads as zero fields).
 template <int P, bool VEC>
 __device__ __forceinline__ void load_chunk(const uint16_t *__restrict__ seeds_row,
                                            const uint16_t *__restrict__ coefs_row,
                                            const uint8_t *__restrict__ codes_row, int nb,
-                                           int ch, ChunkFields &f) {
+                                           int ch, ChunkFields &f, size_t row = 0, size_t nrows = 1) {
   const int b0 = ch * 8;
+  if (!in_bounds(row, nrows, 4) || !in_bounds((size_t)b0 + (VEC ? 7 : 0), (size_t)nb, 3)) {
+    f = ChunkFields{};
+    return;
+  }
   if (VEC) {
     uint4 s = __ldcs(reinterpret_cast<const uint4 *>(seeds_row + b0));
     uint4 q = __ldcs(reinterpret_cast<const uint4 *>(coefs_row + b0));
@@ -165,6 +172,11 @@ __device__ __forceinline__ void load_chunk(const uint16_t *__restrict__ seeds_ro
   }
 }
 
+// The scale key of a row's exponent bias (bounds-checked like the fields).
+__device__ __forceinline__ uint32_t load_bias_key(const nslm_seed_matrix &W, size_t row) {
+  return row_scale_key(in_bounds(row, (size_t)W.N, 4) ? __ldg(W.exp_bias + row) : 0);
+}
+
 // Shared-memory landing slots for the fields of one whole chunk per thread
 // (structure of arrays over the n threads of a CTA, so that a warp's 16-byte
 // reads are contiguous): seeds, coefs, codes word, exponent bias.
@@ -185,6 +197,7 @@ struct FieldSlots {
 template <int P>
 __device__ __forceinline__ void fetch_chunk(const nslm_seed_matrix &W, size_t grow, int nb, int ch,
                                             const FieldSlots &fs, int i) {
+  if (!in_bounds(grow, (size_t)W.N, 2) || !in_bounds((size_t)ch * 8 + 7, (size_t)nb, 1)) return;
   cp_async16(fs.s + i, W.seeds + grow * nb + ch * 8);
   cp_async16(fs.q + i, W.coefs + grow * nb + ch * 8);
   if (P == 4) cp_async4(fs.c + i, W.codes + grow * (nb / 2) + ch * 4);
@@ -196,6 +209,8 @@ __device__ __forceinline__ void fetch_chunk(const nslm_seed_matrix &W, size_t gr
 template <int P>
 __device__ __forceinline__ void fetch_chunk_off(const nslm_seed_matrix &W, uint32_t off, uint32_t row,
                                                 const FieldSlots &fs, int i) {
+  if (!in_bounds((size_t)off + 7, (size_t)W.N * (size_t)(W.K >> 3), 1) || !in_bounds(row, (size_t)W.N, 2))
+    return;
   cp_async16(fs.s + i, W.seeds + off);
   cp_async16(fs.q + i, W.coefs + off);
   if (P == 4) cp_async4(fs.c + i, W.codes + (off >> 1));

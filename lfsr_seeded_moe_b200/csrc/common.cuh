@@ -55,4 +55,51 @@ ChunkLayout chunk_layout(int32_t K, int32_t N, int32_t target_ctas, int32_t max_
 
 __host__ __device__ inline int32_t ceil_div(int32_t a, int32_t b) { return (a + b - 1) / b; }
 
+// ------------------------------------------------------------ bounds checks
+//
+// A build with -DNSLM_BOUNDS_CHECK=1 (python -m lfsr_seeded_moe_b200.build
+// --bounds-check) compares the index of every checked global access with the
+// extent its kernel was given.  An index outside records the site's number in
+// a device word (the first site wins) and the access is skipped: nothing traps
+// and no address outside a buffer is formed.  nslm_debug_bounds_status reads
+// and clears the word.  In the normal build the checks compile to nothing.
+// Site numbers: 1-2 field copies by offset, 3-4 field loads by row, 5-6 the
+// tensor-core producer's field and token-row loads, 7-9 the tensor-core
+// epilogue's stores, 10-11 the decode kernels' h and y stores, 12 the GEMV's
+// y store, 99 the self-test probe.
+#ifndef NSLM_BOUNDS_CHECK
+#define NSLM_BOUNDS_CHECK 0
+#endif
+#if NSLM_BOUNDS_CHECK
+static __device__ int32_t g_bounds_error;  // one per translation unit
+// Host accessor of this translation unit's word: returns it, then clears it.
+#define NSLM_BOUNDS_ACCESSOR(tu)                                                  \
+  int32_t bounds_error_##tu() {                                                   \
+    int32_t v = 0, z = 0;                                                         \
+    if (cudaMemcpyFromSymbol(&v, g_bounds_error, sizeof(v)) != cudaSuccess) return -1; \
+    if (cudaMemcpyToSymbol(g_bounds_error, &z, sizeof(z)) != cudaSuccess) return -1;   \
+    return v;                                                                     \
+  }
+#else
+#define NSLM_BOUNDS_ACCESSOR(tu)
+#endif
+
+// True when idx < n; otherwise (bounds-check build) records `site` and
+// returns false so that the caller skips the access.
+__device__ __forceinline__ bool in_bounds(size_t idx, size_t n, int site) {
+#if NSLM_BOUNDS_CHECK
+  if (idx >= n) {
+    atomicCAS(&g_bounds_error, 0, site);
+    return false;
+  }
+#else
+  (void)idx;
+  (void)n;
+  (void)site;
+#endif
+  return true;
+}
+
+int32_t bounds_error_all();  // the first recorded site over all translation units (and clears them)
+
 }  // namespace nslm

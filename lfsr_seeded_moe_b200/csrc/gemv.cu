@@ -57,7 +57,7 @@ __global__ void __launch_bounds__(512) seed_gemv_kernel(const GemvParams p) {
                          P == 4    ? p.codes + (size_t)row * (p.nb / 2)
                          : P == 35 ? p.codes + (size_t)row * (3 * p.nb / 8)
                                    : nullptr,
-                         p.nb, ch, f);
+                         p.nb, ch, f, (size_t)row, (size_t)p.N);
       const uint32_t rowk = row_scale_key(__ldg(p.exp_bias + row));
       chunk_dot<P, M, VEC, CPAD>(tab, f, p.nb, ch, rowk, xs4, xn2, cpad, 0, acc);
     }
@@ -233,6 +233,8 @@ static size_t gemv1_smem(int C, int rpc, int threads) {
   return sizeof(StreamTables) + FieldSlots::bytes(2 * threads) + cm_bytes(C) + 16 +
          (size_t)rpc * C * sizeof(float);
 }
+
+NSLM_BOUNDS_ACCESSOR(gemv)
 
 }  // namespace nslm
 

@@ -45,7 +45,8 @@ enum GMode { GMODE_GEMM = 0, GMODE_GATEUP = 1, GMODE_DOWN = 2 };
 struct GroupedParams {
   nslm_seed_matrix A0, A1;  // A1: up projection (GATEUP only)
   int32_t E, rows, K, nb;
-  int32_t R;                // B rows available
+  int32_t R;                // sorted rows (GEMM: rows of x and y; FFN: routed pairs)
+  int32_t x_rows;           // rows of x (bounds checks)
   const uint16_t *x;        // bf16 B rows [R][K]
   const int32_t *row_of;    // sorted row -> B row (null: identity)
   const int32_t *offsets;   // [E + 1] sorted-row offsets per expert
@@ -93,10 +94,16 @@ struct SliceFields {  // packed fields of one thread's two tasks for one K slice
   uint32_t s2[2], q2[2], c2[2];
 };
 
+// (bp: the thread's block pair, nw: 32-bit words per row of seeds, for the
+// bounds-check build)
 template <int P>
 __device__ __forceinline__ void load_slice(const uint32_t *const (&sp)[2], const uint32_t *const (&qp)[2],
                                            const uint8_t *const (&cp)[2], const bool (&ok)[2], int kt,
-                                           SliceFields &f) {
+                                           SliceFields &f, int bp, int nw) {
+  if (!in_bounds((size_t)(4 * kt + bp), (size_t)nw, 5)) {
+    f = SliceFields{};
+    return;
+  }
 #pragma unroll
   for (int j = 0; j < 2; ++j) {
     f.s2[j] = ok[j] ? __ldcs(sp[j] + 4 * kt) : 0u;
@@ -240,7 +247,7 @@ __global__ void __launch_bounds__(kCtaThreads, 1) grouped_seed_gemm_kernel(const
             if (!rok || n >= ti.n_valid) continue;
             const size_t sr = (size_t)(ti.r_begin + n);
             const float hv = __fdividef(g[j], 1.f + __expf(-g[j])) * up[j];
-            p.h[sr * p.rows + row] = __bfloat16_as_ushort(__float2bfloat16_rn(hv));
+            if (in_bounds(sr, (size_t)p.R, 7)) p.h[sr * p.rows + row] = __bfloat16_as_ushort(__float2bfloat16_rn(hv));
           }
         }
       } else {
@@ -257,10 +264,11 @@ __global__ void __launch_bounds__(kCtaThreads, 1) grouped_seed_gemm_kernel(const
               if (!rok || n >= ti.n_valid) continue;
               const size_t sr = (size_t)(ti.r_begin + n);
               if (MODE == GMODE_GEMM) {
-                p.y[sr * p.rows + row] = v[j];
+                if (in_bounds(sr, (size_t)p.R, 8)) p.y[sr * p.rows + row] = v[j];
               } else {
-                p.part[(size_t)s_epr[MODE == GMODE_DOWN ? ew : 0][MODE == GMODE_DOWN ? n : 0] * p.rows + row] =
-                    s_epw[MODE == GMODE_DOWN ? ew : 0][MODE == GMODE_DOWN ? n : 0] * v[j];
+                const size_t pr = (size_t)s_epr[MODE == GMODE_DOWN ? ew : 0][MODE == GMODE_DOWN ? n : 0];
+                if (in_bounds(pr, (size_t)p.R, 9))
+                  p.part[pr * p.rows + row] = s_epw[MODE == GMODE_DOWN ? ew : 0][MODE == GMODE_DOWN ? n : 0] * v[j];
               }
             }
           }
@@ -285,11 +293,15 @@ __global__ void __launch_bounds__(kCtaThreads, 1) grouped_seed_gemm_kernel(const
         const nslm_seed_matrix &W = (MODE == GMODE_GATEUP && j) ? p.A1 : p.A0;
         const int grow = ti.m0 + (MODE == GMODE_GATEUP ? 0 : j * kBM) + trow;
         ok[j] = grow < p.rows;
-        const size_t wr = (size_t)ti.e * p.rows + (ok[j] ? grow : 0);
+        size_t wr = (size_t)ti.e * p.rows + (ok[j] ? grow : 0);
+        if (!in_bounds(wr, (size_t)W.N, 5)) {
+          ok[j] = false;
+          wr = 0;
+        }
         sp[j] = reinterpret_cast<const uint32_t *>(W.seeds + wr * p.nb) + bp;
         qp[j] = reinterpret_cast<const uint32_t *>(W.coefs + wr * p.nb) + bp;
         cpp[j] = (P == 4) ? W.codes + wr * (p.nb / 2) + bp : nullptr;
-        rowk[j] = row_scale_key(__ldg(W.exp_bias + wr));
+        rowk[j] = load_bias_key(W, wr);
       }
       const size_t a_off = ((trow >> 3) * 8 + 2 * bp) * 128 + (trow & 7) * 16;
       // token rows this thread copies: chunks (n, kc) for n = trow, trow + 128 and kc = bp, bp + 4
@@ -300,8 +312,12 @@ __global__ void __launch_bounds__(kCtaThreads, 1) grouped_seed_gemm_kernel(const
         const int n = trow + 128 * i;
 #pragma unroll
         for (int h = 0; h < 2; ++h) bdst[i][h] = ((n >> 3) * 8 + bp + 4 * h) * 128 + (n & 7) * 16;
-        const bool v = n < ti.n_valid;
-        const int xr = v ? (p.row_of ? p.row_of[ti.r_begin + n] : ti.r_begin + n) : 0;
+        bool v = n < ti.n_valid;
+        int xr = v ? (p.row_of ? p.row_of[ti.r_begin + n] : ti.r_begin + n) : 0;
+        if (v && !in_bounds((size_t)xr, (size_t)p.x_rows, 6)) {
+          v = false;
+          xr = 0;
+        }
         brow[i] = p.x + (size_t)xr * p.K;
         bbytes[i] = v ? 16u : 0u;  // zero-fill rows past n_valid
       }
@@ -332,9 +348,10 @@ __global__ void __launch_bounds__(kCtaThreads, 1) grouped_seed_gemm_kernel(const
       // uses set kt % 3 and reloads it for slice kt + 3 (the loop is unrolled
       // by three, so no set is ever copied while its loads are in flight)
       SliceFields f0, f1, f2;
-      load_slice<P>(sp, qp, cpp, ok, 0, f0);
-      if (ksteps > 1) load_slice<P>(sp, qp, cpp, ok, 1, f1);
-      if (ksteps > 2) load_slice<P>(sp, qp, cpp, ok, 2, f2);
+      const int nw = p.nb / 2;
+      load_slice<P>(sp, qp, cpp, ok, 0, f0, bp, nw);
+      if (ksteps > 1) load_slice<P>(sp, qp, cpp, ok, 1, f1, bp, nw);
+      if (ksteps > 2) load_slice<P>(sp, qp, cpp, ok, 2, f2, bp, nw);
       auto slice = [&](SliceFields &f, int kt) {
         const int stage = it % kStages;
         // the stage of slice it was claimed when its token rows were copied
@@ -349,7 +366,7 @@ __global__ void __launch_bounds__(kCtaThreads, 1) grouped_seed_gemm_kernel(const
           uint4 *dst1 = reinterpret_cast<uint4 *>(atile + j * kBM * 128 + a_off + 128);
           regen_pair_bf16<P, kTabCopies>(tl, f.s2[j], f.q2[j], f.c2[j], rowk[j], dst0, dst1);
         }
-        if (kt + 3 < ksteps) load_slice<P>(sp, qp, cpp, ok, kt + 3, f);
+        if (kt + 3 < ksteps) load_slice<P>(sp, qp, cpp, ok, kt + 3, f, bp, nw);
         cp_async_wait<1>();  // this slice's token rows (the next slice's may still be in flight)
         umma::fence_proxy_async();
         umma::mbar_arrive(umma::smem_u32(&full_bar[stage]));
@@ -561,7 +578,7 @@ int32_t launch_batched_ffn(const FfnDims &d, const nslm_seed_matrix *gate, const
   {
     GroupedParams p{};
     p.A0 = *gate; p.A1 = *up; p.E = d.E; p.rows = d.inter; p.K = d.hidden; p.nb = d.hidden / 8;
-    p.R = TK; p.x = x_bf16; p.row_of = bp.row_of; p.offsets = bp.offsets; p.tile_start = bp.tiles_gu;
+    p.R = TK; p.x_rows = T; p.x = x_bf16; p.row_of = bp.row_of; p.offsets = bp.offsets; p.tile_start = bp.tiles_gu;
     p.mtiles = mt_gu; p.bn = bn; p.tmem_cols = tmem_cols_for(2 * bn); p.status = bp.status; p.h = bp.h;
     // the gathered rows index x (T rows), not the sorted rows: bound by T via row_of
     if (int32_t st = launch_grouped(p, d.P, GMODE_GATEUP, s)) return st;
@@ -570,7 +587,7 @@ int32_t launch_batched_ffn(const FfnDims &d, const nslm_seed_matrix *gate, const
   {
     GroupedParams p{};
     p.A0 = *down; p.E = d.E; p.rows = d.hidden; p.K = d.inter; p.nb = d.inter / 8;
-    p.R = TK; p.x = bp.h; p.row_of = nullptr; p.offsets = bp.offsets; p.tile_start = bp.tiles_dn;
+    p.R = TK; p.x_rows = TK; p.x = bp.h; p.row_of = nullptr; p.offsets = bp.offsets; p.tile_start = bp.tiles_dn;
     p.mtiles = mt_dn; p.bn = bn; p.tmem_cols = tmem_cols_for(2 * bn); p.status = bp.status;
     p.part = bp.part; p.pair_of = bp.pair_of; p.pair_w = w;
     if (int32_t st = launch_grouped(p, d.P, GMODE_DOWN, s)) return st;
@@ -587,6 +604,8 @@ int32_t launch_batched_ffn(const FfnDims &d, const nslm_seed_matrix *gate, const
 size_t grouped_ws_bytes(int E) {
   return ((size_t)(E + 2) * sizeof(int32_t) + 255) / 256 * 256;
 }
+
+NSLM_BOUNDS_ACCESSOR(grouped)
 
 }  // namespace nslm
 
@@ -639,7 +658,7 @@ extern "C" int32_t nslm_seed_grouped_gemm(const nslm_seed_matrix *W, int32_t E,
   tile_prefix_kernel<<<1, 1024, 0, s>>>(offsets, E, mtiles, bn, R, tile_start, status);
   if ((st = launch_status())) return st;
   GroupedParams p{};
-  p.A0 = *W; p.E = E; p.rows = rows; p.K = W->K; p.nb = W->K / 8; p.R = R; p.x = x_bf16;
+  p.A0 = *W; p.E = E; p.rows = rows; p.K = W->K; p.nb = W->K / 8; p.R = R; p.x_rows = R; p.x = x_bf16;
   p.row_of = nullptr; p.offsets = offsets; p.tile_start = tile_start; p.mtiles = mtiles; p.bn = bn;
   p.tmem_cols = tmem_cols_for(2 * bn); p.status = status; p.y = y;
   st = launch_grouped(p, W->P, GMODE_GEMM, s);

@@ -181,7 +181,7 @@ __device__ __forceinline__ void gate_up_body(const GateUpParams &p, const Stream
     const int orow = g * p.R + r2;
     if (orow < p.inter) {
       const float gs = s_sum[(2 * m) * p.R + r2], us = s_sum[(2 * m + 1) * p.R + r2];
-      p.h[(size_t)s_pair[m] * p.inter + orow] = gs / (1.f + expf(-gs)) * us;
+      if (in_bounds((size_t)s_pair[m], (size_t)p.T * p.k, 10)) p.h[(size_t)s_pair[m] * p.inter + orow] = gs / (1.f + expf(-gs)) * us;
     }
   }
 }
@@ -218,11 +218,11 @@ __global__ void __launch_bounds__(256) ffn_gate_up_kernel(const GateUpParams p) 
   if (active) {
     const size_t grow = (size_t)e * p.inter + row;
     load_chunk<P, VEC>(p.gate.seeds + grow * nb, p.gate.coefs + grow * nb,
-                       codes_row<P>(p.gate.codes, grow, nb), nb, ch, fg);
+                       codes_row<P>(p.gate.codes, grow, nb), nb, ch, fg, grow, (size_t)p.gate.N);
     load_chunk<P, VEC>(p.up.seeds + grow * nb, p.up.coefs + grow * nb,
-                       codes_row<P>(p.up.codes, grow, nb), nb, ch, fu);
-    rowkg = row_scale_key(__ldg(p.gate.exp_bias + grow));
-    rowku = row_scale_key(__ldg(p.up.exp_bias + grow));
+                       codes_row<P>(p.up.codes, grow, nb), nb, ch, fu, grow, (size_t)p.up.N);
+    rowkg = load_bias_key(p.gate, grow);
+    rowku = load_bias_key(p.up, grow);
   }
   if (tid < M) {
     const int pr = pl->pair[p0 + tid];
@@ -329,8 +329,8 @@ __global__ void __launch_bounds__(512) ffn_down_kernel(const DownParams p) {
   if (active && s0 < s1) {
     const size_t grow = (size_t)pl->expert[s0] * p.hidden + row;
     load_chunk<P, VEC>(p.down.seeds + grow * nb, p.down.coefs + grow * nb,
-                       codes_row<P>(p.down.codes, grow, nb), nb, ch, f);
-    rowk = row_scale_key(__ldg(p.down.exp_bias + grow));
+                       codes_row<P>(p.down.codes, grow, nb), nb, ch, f, grow, (size_t)p.down.N);
+    rowk = load_bias_key(p.down, grow);
   }
   build_stream_tables(tab);
   __syncthreads();
@@ -353,8 +353,8 @@ __global__ void __launch_bounds__(512) ffn_down_kernel(const DownParams p) {
     if (active && s + 1 < s1) {
       const size_t grow = (size_t)pl->expert[s + 1] * p.hidden + row;
       load_chunk<P, VEC>(p.down.seeds + grow * nb, p.down.coefs + grow * nb,
-                         codes_row<P>(p.down.codes, grow, nb), nb, ch, fn);
-      rowkn = row_scale_key(__ldg(p.down.exp_bias + grow));
+                         codes_row<P>(p.down.codes, grow, nb), nb, ch, fn, grow, (size_t)p.down.N);
+      rowkn = load_bias_key(p.down, grow);
     }
     if (active) {
       const int v0 = stage_all ? a0 : 0;
@@ -539,5 +539,7 @@ int32_t launch_route_plan(const float *logits, const int32_t *ids, const float *
                                       n_counters, sync, std::max(1, std::min(slot_cap, T)));
   return launch_status();
 }
+
+NSLM_BOUNDS_ACCESSOR(moe)
 
 }  // namespace nslm

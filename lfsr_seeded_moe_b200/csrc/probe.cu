@@ -3,6 +3,7 @@
 // after their limit and report it, instead of hanging.  One CTA waits for an
 // event that nothing produces (or, for the positive case, one that already
 // happened) with the kernels' own wait routines and a caller-chosen limit.
+#include "chunk.cuh"
 #include "common.cuh"
 #include "persist.cuh"
 #include "umma.cuh"
@@ -34,6 +35,22 @@ __global__ void mbar_wait_probe_kernel(int32_t *out, long long cycles, int arriv
 }
 
 }  // namespace
+// The bounds-check build's self-test: a field copy one chunk past the end of
+// W, which the copy's own check refuses (site 1) before any address is formed.
+__global__ void bounds_probe_kernel(const nslm_seed_matrix W) {
+#if NSLM_BOUNDS_CHECK
+  __shared__ __align__(16) unsigned char slots[64];
+  const FieldSlots fs(slots, 1);
+  const uint32_t nb = (uint32_t)(W.K >> 3);
+  if (threadIdx.x == 0) fetch_chunk_off<4>(W, (uint32_t)W.N * nb, 0u, fs, 0);
+  cp_async_wait_all();
+#else
+  (void)W;
+#endif
+}
+
+NSLM_BOUNDS_ACCESSOR(probe)
+
 }  // namespace nslm
 
 using namespace nslm;
@@ -49,4 +66,22 @@ extern "C" int32_t nslm_debug_wait_probe(int32_t kind, int32_t *out, int64_t cyc
   st = launch_status();
   if (st == NSLM_OK) g_launches = 1;
   return st;
+}
+
+extern "C" int32_t nslm_debug_bounds_probe(const nslm_seed_matrix *W, nslm_stream_t stream) {
+  g_launches = 0;
+#if NSLM_BOUNDS_CHECK
+  int32_t st = check_matrix(W);
+  if (st) return st;
+  if (W->P != 4 || W->N < 1 || W->K % 64) return NSLM_ERR_SHAPE;
+  if ((st = check_device())) return st;
+  bounds_probe_kernel<<<1, 32, 0, reinterpret_cast<cudaStream_t>(stream)>>>(*W);
+  st = launch_status();
+  if (st == NSLM_OK) g_launches = 1;
+  return st;
+#else
+  (void)W;
+  (void)stream;
+  return NSLM_ERR_UNSUPPORTED;
+#endif
 }

@@ -52,6 +52,7 @@ struct Stack1Params {
   float *rms_part;        // [grid] sums of y^2 over each CTA's rows, written with y
   uint32_t barrier_base;  // arrivals recorded by earlier launches of the same call
   int32_t n, hidden, inter;
+  int32_t h_rows;         // rows of h (the routed pairs; bounds checks)
   int32_t Ch, Ci;         // 64-weight chunks per row of gate/up (hidden) and down (inter)
   int32_t J;              // chunk rounds per lane in phase A: ceil(Ch / 32)
   int32_t rpc;            // output rows per CTA in phase B
@@ -150,11 +151,13 @@ __global__ void __launch_bounds__(kStack1MaxThreads, 1) stack1_kernel(const __gr
       fetch_chunk_off<P>(Lm.up, off, r32, fs, (2 * buf + 1) * nthr + tid);
     } else {
       load_chunk<P, false>(Lm.gate.seeds + grow * nbh, Lm.gate.coefs + grow * nbh,
-                           P == 4 ? Lm.gate.codes + grow * (nbh / 2) : nullptr, nbh, c, fg);
+                           P == 4 ? Lm.gate.codes + grow * (nbh / 2) : nullptr, nbh, c, fg, grow,
+                           (size_t)Lm.gate.N);
       load_chunk<P, false>(Lm.up.seeds + grow * nbh, Lm.up.coefs + grow * nbh,
-                           P == 4 ? Lm.up.codes + grow * (nbh / 2) : nullptr, nbh, c, fu);
-      kg = row_scale_key(__ldg(Lm.gate.exp_bias + grow));
-      ku = row_scale_key(__ldg(Lm.up.exp_bias + grow));
+                           P == 4 ? Lm.up.codes + grow * (nbh / 2) : nullptr, nbh, c, fu, grow,
+                           (size_t)Lm.up.N);
+      kg = load_bias_key(Lm.gate, grow);
+      ku = load_bias_key(Lm.up, grow);
     }
   };
   // ---- phase B task geometry (row, routed expert, chunk) of this CTA's rows
@@ -174,8 +177,9 @@ __global__ void __launch_bounds__(kStack1MaxThreads, 1) stack1_kernel(const __gr
       fetch_chunk_off<P>(Lm.down, r32 * (uint32_t)nbi + 8u * (uint32_t)c, r32, fs, buf * nthr + tid);
     } else {
       load_chunk<P, false>(Lm.down.seeds + grow * nbi, Lm.down.coefs + grow * nbi,
-                           P == 4 ? Lm.down.codes + grow * (nbi / 2) : nullptr, nbi, c, f);
-      k = row_scale_key(__ldg(Lm.down.exp_bias + grow));
+                           P == 4 ? Lm.down.codes + grow * (nbi / 2) : nullptr, nbi, c, f, grow,
+                           (size_t)Lm.down.N);
+      k = load_bias_key(Lm.down, grow);
     }
   };
 
@@ -236,7 +240,8 @@ __global__ void __launch_bounds__(kStack1MaxThreads, 1) stack1_kernel(const __gr
           const float g = warp_sum(ag.x + ag.y), u = warp_sum(au.x + au.y);
           // SiLU with the fast exp and divide (relative error ~1e-6; an exp
           // that overflows gives the limit 0)
-          if (lane == 0) __stcg(p.h + (size_t)s_pair[slot] * p.inter + row, __fdividef(g, 1.f + __expf(-g)) * u);
+          if (lane == 0 && in_bounds((size_t)s_pair[slot], (size_t)p.h_rows, 10))
+            __stcg(p.h + (size_t)s_pair[slot] * p.inter + row, __fdividef(g, 1.f + __expf(-g)) * u);
           ag = au = make_float2(0.f, 0.f);
         }
       }
@@ -389,6 +394,7 @@ static int32_t launch_stack1_t(const FfnDims &d, const nslm_moe_layer *layers, i
   const int grid = num_sms() * per_sm;
   Stack1Params p{};
   p.h = h;
+  p.h_rows = k;
   p.y_mid = y_mid;
   p.sync = sync;
   p.rms_part = rms_part;
@@ -446,5 +452,7 @@ int32_t launch_stack1(const FfnDims &d, const nslm_moe_layer *layers, int n, con
   return vec ? launch_stack1_t<3, true>(d, layers, n, plans, x0, y_in, k, h, y_mid, y_out, sync, rms_part, s, launches)
              : launch_stack1_t<3, false>(d, layers, n, plans, x0, y_in, k, h, y_mid, y_out, sync, rms_part, s, launches);
 }
+
+NSLM_BOUNDS_ACCESSOR(stack1)
 
 }  // namespace nslm

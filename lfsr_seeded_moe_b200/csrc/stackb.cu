@@ -315,7 +315,8 @@ __global__ void __launch_bounds__(kStackBThreads, 1) stackb_kernel(const __grid_
               const float g = warp_sum(ag[m].x + ag[m].y), u = warp_sum(au[m].x + au[m].y);
               // SiLU with the fast exp and divide (relative error ~1e-6; an
               // exp that overflows gives the limit 0)
-              if (lane == 0) __stcg(p.h + (size_t)s_pid[q0 + m] * p.inter + row, __fdividef(g, 1.f + __expf(-g)) * u);
+              if (lane == 0 && in_bounds((size_t)s_pid[q0 + m], (size_t)p.T * p.k, 10))
+                __stcg(p.h + (size_t)s_pid[q0 + m] * p.inter + row, __fdividef(g, 1.f + __expf(-g)) * u);
             }
             ag[m] = au[m] = make_float2(0.f, 0.f);
           }
@@ -588,6 +589,8 @@ int32_t launch_stackb(const FfnDims &d, const nslm_moe_layer *layers, int n, con
     return launch_stackb_t<4>(d, sh, layers, n, plans, x0, y_in, T, k, h, y_mid, y_out, sync, rms_part, s, launches);
   return launch_stackb_t<3>(d, sh, layers, n, plans, x0, y_in, T, k, h, y_mid, y_out, sync, rms_part, s, launches);
 }
+
+NSLM_BOUNDS_ACCESSOR(stackb)
 
 }  // namespace nslm
 

@@ -13,10 +13,12 @@ import os
 import re
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-# NSLM_STREAM_SOURCE=l2next or l2basis loads an ablation build of the library
-# (`python -m lfsr_seeded_moe_b200.build --stream-source l2next`), whose
-# decode kernels read the stream bits from an L2-resident 65,536-entry table
-_SOURCE = os.environ.get("NSLM_STREAM_SOURCE", "")
+# NSLM_LIB_VARIANT loads a variant build of the library from _build/<variant>/:
+# l2next or l2basis (`python -m lfsr_seeded_moe_b200.build --stream-source
+# l2next`), whose decode kernels read the stream bits from an L2-resident
+# 65,536-entry table, or boundscheck (`... build --bounds-check`), whose
+# kernels check their indices; NSLM_STREAM_SOURCE is an older name for it.
+_SOURCE = os.environ.get("NSLM_LIB_VARIANT", "") or os.environ.get("NSLM_STREAM_SOURCE", "")
 LIB_PATH = os.path.join(_HERE, "_build", *([_SOURCE] if _SOURCE else []), "libnslm.so")
 HEADER_PATH = os.path.join(os.path.dirname(_HERE), "include", "nslm.h")
 
@@ -86,6 +88,8 @@ def _load():
         "nslm_unpack_nibbles": (i32, [vp, mp, vp]),
         "nslm_pack_nibbles": (i32, [mp, vp, vp]),
         "nslm_debug_wait_probe": (i32, [i32, vp, ctypes.c_int64, vp]),
+        "nslm_debug_bounds_status": (i32, []),
+        "nslm_debug_bounds_probe": (i32, [mp, vp]),
         "nslm_debug_batched_hidden": (i32, [vp, sz, i32, i32, i32, i32, i32, vp, vp]),
         "nslm_debug_decompress": (i32, [mp, vp, vp]),
         "nslm_debug_decompress_bf16": (i32, [mp, vp, vp]),
@@ -276,6 +280,18 @@ def nslm_debug_batched_hidden(ws, ws_bytes: int, T: int, E: int, hidden: int, in
     """bf16 h [T*k][inter] (pair order) left in ws by the last tensor-core FFN call."""
     _check("nslm_debug_batched_hidden",
            _lib.nslm_debug_batched_hidden(_p(ws), ws_bytes, T, E, hidden, inter, k, _p(h_out), _s(stream)))
+
+
+def nslm_debug_bounds_status() -> int:
+    """First bounds-check site recorded since the last call (0: none); bounds-check build only."""
+    rc = int(_lib.nslm_debug_bounds_status())
+    if rc < 0:
+        raise NslmError("nslm_debug_bounds_status", rc)
+    return rc
+
+
+def nslm_debug_bounds_probe(W, stream=None) -> None:
+    _check("nslm_debug_bounds_probe", _lib.nslm_debug_bounds_probe(ctypes.byref(_mat(W)), _s(stream)))
 
 
 def nslm_debug_decompress(W, w_out, stream=None) -> None:

@@ -6,6 +6,8 @@ import numpy as np
 import pytest
 import torch
 
+import guard
+
 from oracle import oracle as O
 from lfsr_seeded_moe_b200 import synth
 
@@ -64,10 +66,10 @@ def _pinned(m):
 
 def _empty_cache(S, rows, K, P):
     nb = K // 8
-    return synth.SeedMatrix(torch.zeros(S * rows, nb, dtype=torch.int16, device="cuda"),
-                            torch.zeros(S * rows, nb, dtype=torch.int16, device="cuda"),
-                            torch.zeros(S * rows, nb // 2, dtype=torch.uint8, device="cuda") if P == 4 else None,
-                            torch.zeros(S * rows, dtype=torch.int32, device="cuda"), rows, K, P, S)
+    return synth.SeedMatrix(guard.buffer((S * rows, nb), torch.int16, fill=0),
+                            guard.buffer((S * rows, nb), torch.int16, fill=0),
+                            guard.buffer((S * rows, nb // 2), torch.uint8, fill=0) if P == 4 else None,
+                            guard.buffer((S * rows,), torch.int32, fill=0), rows, K, P, S)
 
 
 @pytest.mark.parametrize("T,P", [(1, 4), (2, 3)])
@@ -76,11 +78,11 @@ def test_expert_cache_lru_and_layers(nslm, T, P):
     layers = [synth.moe_layer(l, E, hidden, inter, P, config=960 + P) for l in range(L)]
     host = [tuple(_pinned(getattr(m, n)) for n in ("gate", "up", "down")) for m in layers]
     cache = (_empty_cache(S, inter, hidden, P), _empty_cache(S, inter, hidden, P), _empty_cache(S, hidden, inter, P))
-    state = torch.zeros(nslm.nslm_expert_cache_state_bytes(S), dtype=torch.uint8, device="cuda")
+    state = guard.buffer(nslm.nslm_expert_cache_state_bytes(S), torch.uint8, fill=0)
     ref = _LRU(S)
     rng = np.random.default_rng(961)
     wsb = nslm.nslm_workspace_bytes(nslm.NSLM_OP_MOE_FFN, T, S, hidden, inter, k)
-    ws = torch.empty(wsb, dtype=torch.uint8, device="cuda")
+    ws = guard.buffer(wsb, torch.uint8)
     for step in range(5):
         for l in range(L):
             ids = np.stack([rng.choice(E, k, replace=False) for _ in range(T)]).astype(np.int32)
@@ -88,13 +90,13 @@ def test_expert_cache_lru_and_layers(nslm, T, P):
                 ids[0, 2] = -1  # a dropped pair
             w = rng.uniform(0.05, 0.4, (T, k)).astype(np.float32)
             dids = torch.from_numpy(ids).cuda()
-            slots = torch.full((T, k), -7, dtype=torch.int32, device="cuda")
+            slots = guard.buffer((T, k), torch.int32, fill=-7)
             nslm.nslm_expert_cache_fetch(host[l], E, l, cache, S, state, dids, T, k, slots)
             want, _ = ref.step(l, E, ids.reshape(-1).tolist())
             assert slots.cpu().numpy().reshape(-1).tolist() == want, (step, l)
             xb = synth.activations((962, step, l), T, hidden)
             xd, wd = xb.cuda(), torch.from_numpy(w).cuda()
-            y = torch.full((T, hidden), float("nan"), device="cuda")
+            y = guard.buffer((T, hidden), torch.float32, fill=float("nan"))
             nslm.nslm_moe_seed_ffn(cache[0], cache[1], cache[2], S, xd, slots, wd, T, k, y, ws, wsb)
             torch.cuda.synchronize()
             g, u, d = (getattr(layers[l], n).numpy() for n in ("gate", "up", "down"))

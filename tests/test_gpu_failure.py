@@ -8,6 +8,8 @@ import numpy as np
 import pytest
 import torch
 
+import guard
+
 from oracle import oracle as O
 from lfsr_seeded_moe_b200 import synth
 
@@ -27,7 +29,7 @@ def nslm():
 def _gemv_still_works(nslm):
     m = synth.seed_matrix(64, 256, 4, (980,))
     x = synth.activations((980,), 1, 256)
-    y = torch.empty(1, 64, device="cuda")
+    y = guard.buffer((1, 64), torch.float32, fill=float("nan"))
     md = m.to("cuda")
     nslm.nslm_seed_gemv(md, x.cuda(), 1, y)
     torch.cuda.synchronize()

@@ -10,6 +10,8 @@ import numpy as np
 import pytest
 import torch
 
+import guard
+
 from oracle import oracle as O
 from lfsr_seeded_moe_b200 import synth
 
@@ -42,9 +44,9 @@ def test_grouped_gemm_matches_bf16_oracle(nslm, P, rows, K, counts):
     W = synth.seed_matrix(rows, K, P, (960, rows, K, P), E)
     xb = synth.activations((960, R), R, K)
     offs = np.concatenate([[0], np.cumsum(counts)]).astype(np.int32)
-    y = torch.full((R, rows), float("nan"), device="cuda")
+    y = guard.buffer((R, rows), torch.float32, fill=float("nan"))
     wsb = nslm.nslm_workspace_bytes(nslm.NSLM_OP_GROUPED_GEMM, R, E, K, rows, 1)
-    ws = torch.zeros(wsb, dtype=torch.uint8, device="cuda")
+    ws = guard.buffer(wsb, torch.uint8, fill=0)
     nslm.nslm_seed_grouped_gemm(W.to("cuda"), E, xb.cuda(), torch.from_numpy(offs).cuda(), R, y, ws, wsb)
     torch.cuda.synchronize()
     assert _status(ws) == 0
@@ -65,9 +67,9 @@ def _batched_case(nslm, E, hidden, inter, P, T, k, tag, zipf=None, sample=None):
     xb = synth.activations((tag, T), T, hidden)
     logits = synth.router_logits((tag, T), T, E, zipf)
     ids, w = O.route_topk(logits.numpy(), k)
-    y = torch.full((T, hidden), float("nan"), device=dev)
+    y = guard.buffer((T, hidden), torch.float32, fill=float("nan"))
     wsb = nslm.nslm_workspace_bytes(nslm.NSLM_OP_MOE_FFN, T, E, hidden, inter, k)
-    ws = torch.zeros(wsb, dtype=torch.uint8, device=dev)
+    ws = guard.buffer(wsb, torch.uint8, fill=0)
     w32 = w.astype(np.float32)
     nslm.nslm_moe_seed_ffn(L.gate.to(dev), L.up.to(dev), L.down.to(dev), E, xb.to(dev),
                            torch.from_numpy(ids).to(dev), torch.from_numpy(w32).to(dev), T, k, y, ws, wsb)
@@ -112,13 +114,13 @@ def _split_case(nslm, E, hidden, inter, P, T, k, tag, zipf=None):
     xb = synth.activations((tag, T), T, hidden)
     logits = synth.router_logits((tag, T), T, E, zipf)
     ids, w = O.route_topk(logits.numpy(), k)
-    y = torch.full((T, hidden), float("nan"), device=dev)
+    y = guard.buffer((T, hidden), torch.float32, fill=float("nan"))
     wsb = nslm.nslm_workspace_bytes(nslm.NSLM_OP_MOE_FFN, T, E, hidden, inter, k)
-    ws = torch.zeros(wsb, dtype=torch.uint8, device=dev)
+    ws = guard.buffer(wsb, torch.uint8, fill=0)
     w32 = w.astype(np.float32)
     nslm.nslm_moe_seed_ffn(L.gate.to(dev), L.up.to(dev), L.down.to(dev), E, xb.to(dev),
                            torch.from_numpy(ids).to(dev), torch.from_numpy(w32).to(dev), T, k, y, ws, wsb)
-    hg = torch.full((T * k, inter), -1, dtype=torch.int16, device=dev)
+    hg = guard.buffer((T * k, inter), torch.int16, fill=-1)
     nslm.nslm_debug_batched_hidden(ws, wsb, T, E, hidden, inter, k, hg)
     torch.cuda.synchronize()
     assert _status(ws) == 0

@@ -4,6 +4,8 @@ import numpy as np
 import pytest
 import torch
 
+import guard
+
 from oracle import oracle as O
 from lfsr_seeded_moe_b200 import synth
 
@@ -36,7 +38,7 @@ def test_unpack_and_pack_match_the_oracle_layout(nslm, P, N, K):
     if P == 4:
         assert torch.equal(out.codes.cpu(), m.codes)
     # and back
-    nb = torch.full(nib.shape, 0xEE, dtype=torch.uint8, device="cuda")
+    nb = guard.buffer(nib.shape, torch.uint8, fill=0xEE)
     md = m.to("cuda")
     nslm.nslm_pack_nibbles(md, nb)
     torch.cuda.synchronize()
@@ -53,8 +55,8 @@ def test_unpacked_pack_gives_the_same_products(nslm):
     out.seeds, out.exp_bias = m.seeds.cuda(), m.exp_bias.cuda()
     nslm.nslm_unpack_nibbles(nib, out)
     x = synth.activations((712,), 1, K).cuda()
-    y0 = torch.empty(1, N, device="cuda")
-    y1 = torch.empty(1, N, device="cuda")
+    y0 = guard.buffer((1, N), torch.float32, fill=float("nan"))
+    y1 = guard.buffer((1, N), torch.float32, fill=float("nan"))
     md = m.to("cuda")
     nslm.nslm_seed_gemv(nslm.matrix(md), x, 1, y0)
     nslm.nslm_seed_gemv(nslm.matrix(out), x, 1, y1)

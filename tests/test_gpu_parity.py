@@ -7,6 +7,8 @@ import numpy as np
 import pytest
 import torch
 
+import guard
+
 from oracle import oracle as O
 from lfsr_seeded_moe_b200 import synth
 
@@ -26,7 +28,7 @@ def nslm():
 
 def _out(*shape):
     """Output buffer pre-filled with NaN, so an entry the kernel never wrote fails."""
-    return torch.full(shape, float("nan"), dtype=torch.float32, device="cuda")
+    return guard.buffer(shape, torch.float32, fill=float("nan"))
 
 
 def _dev(m):
@@ -65,7 +67,7 @@ def test_decompress_bf16_bit_exact_all_seeds(nslm, P):
     # -100..100 (every weight a normal bf16 number)
     m = _all_seed_matrix(P)
     md = _dev(m)
-    w = torch.full((m.N, m.K), -1, dtype=torch.int16, device="cuda")
+    w = guard.buffer((m.N, m.K), torch.int16, fill=-1)
     nslm.nslm_debug_decompress_bf16(md, w)
     torch.cuda.synchronize()
     ref = O.decompress_bf16(m.numpy())
@@ -81,9 +83,9 @@ def test_decompress_ragged_rows_bit_exact(nslm, P, N, K):
     m.exp_bias = torch.linspace(-100, 100, N).round().to(torch.int32)
     md = _dev(m)
     pad = 64
-    w = torch.full((N * K + pad,), float("nan"), dtype=torch.float32, device="cuda")
+    w = guard.buffer((N * K + pad,), torch.float32, fill=float("nan"))
     nslm.nslm_debug_decompress(md, w)
-    wb = torch.full((N * K + pad,), -1, dtype=torch.int16, device="cuda")
+    wb = guard.buffer((N * K + pad,), torch.int16, fill=-1)
     nslm.nslm_debug_decompress_bf16(md, wb)
     torch.cuda.synchronize()
     got = w.cpu().numpy()
@@ -180,7 +182,7 @@ def test_route_topk_matches_oracle(nslm):
     logits = synth.router_logits((905,), T, E)
     logits[3, :] = 0.5                          # all tied
     logits[4, 7] = logits[4, 90] = 5.0          # tie at the top
-    ids = torch.empty(T, k, dtype=torch.int32, device="cuda")
+    ids = guard.buffer((T, k), torch.int32)
     w = _out(T, k)
     nslm.nslm_moe_route_topk(logits.cuda(), T, E, k, ids, w)
     torch.cuda.synchronize()
@@ -198,7 +200,7 @@ def _ffn_case(nslm, E, hidden, inter, P, T, k, tag, zipf=None):
     w = torch.from_numpy(rw.astype(np.float32)).cuda()
     y = _out(T, hidden)
     wsb = nslm.nslm_workspace_bytes(nslm.NSLM_OP_MOE_FFN, T, E, hidden, inter, k)
-    ws = torch.empty(wsb, dtype=torch.uint8, device="cuda")
+    ws = guard.buffer(wsb, torch.uint8)
     nslm.nslm_moe_seed_ffn(_dev(L.gate), _dev(L.up), _dev(L.down), E, x, ids, w, T, k, y, ws, wsb)
     torch.cuda.synchronize()
     g, u, d = (getattr(L, n).numpy() for n in ("gate", "up", "down"))
@@ -210,7 +212,7 @@ def _ffn_with_ids(nslm, L, E, hidden, inter, x, rid, w32, k):
     T = rid.shape[0]
     y = _out(T, hidden)
     wsb = nslm.nslm_workspace_bytes(nslm.NSLM_OP_MOE_FFN, T, E, hidden, inter, k)
-    ws = torch.empty(wsb, dtype=torch.uint8, device="cuda")
+    ws = guard.buffer(wsb, torch.uint8)
     nslm.nslm_moe_seed_ffn(_dev(L.gate), _dev(L.up), _dev(L.down), E, x, torch.from_numpy(rid).cuda(),
                            torch.from_numpy(w32).cuda(), T, k, y, ws, wsb)
     torch.cuda.synchronize()
@@ -340,7 +342,7 @@ def test_ffn_hybrid_p3_p4_experts(nslm, T):
     w32 = rng.uniform(0.05, 0.3, (T, k)).astype(np.float32)
     y = _out(T, hidden)
     wsb = nslm.nslm_workspace_bytes(nslm.NSLM_OP_MOE_FFN_HYBRID, T, E, hidden, inter, k)
-    ws = torch.empty(wsb, dtype=torch.uint8, device="cuda")
+    ws = guard.buffer(wsb, torch.uint8)
     d3 = tuple(_dev(getattr(L3, n)) for n in ("gate", "up", "down"))
     d4 = tuple(_dev(getattr(L4, n)) for n in ("gate", "up", "down"))
     nslm.nslm_moe_seed_ffn_hybrid(d3, E3, d4, E4, x, torch.from_numpy(rid).cuda(), torch.from_numpy(w32).cuda(),
@@ -392,7 +394,7 @@ def test_stack_decode_matches_oracle(nslm, T):
     dl = [(_dev(m.gate), _dev(m.up), _dev(m.down)) for m in layers]
     y = _out(T, hidden)
     wsb = nslm.nslm_workspace_bytes(nslm.NSLM_OP_MOE_STACK, T, E, hidden, inter, k, Lyr)
-    ws = torch.empty(wsb, dtype=torch.uint8, device="cuda")
+    ws = guard.buffer(wsb, torch.uint8)
     nslm.nslm_moe_stack_decode(dl, Lyr, E, k, logits.cuda().contiguous(), x, T, y, ws, wsb)
     torch.cuda.synchronize()
     hl = [tuple(getattr(m, n).numpy() for n in ("gate", "up", "down")) for m in layers]
@@ -404,7 +406,7 @@ def _stack_prefix(nslm, dl, logits, x, T, E, hidden, inter, k, n):
     """Output of the first n layers of a stack (status word checked)."""
     y = _out(T, hidden)
     wsb = nslm.nslm_workspace_bytes(nslm.NSLM_OP_MOE_STACK, T, E, hidden, inter, k, n)
-    ws = torch.zeros(wsb, dtype=torch.uint8, device="cuda")
+    ws = guard.buffer(wsb, torch.uint8, fill=0)
     nslm.nslm_moe_stack_decode(dl[:n], n, E, k, logits[:n].cuda().contiguous(), x, T, y, ws, wsb)
     torch.cuda.synchronize()
     assert int(ws[:4].view(torch.int32).item()) == 0

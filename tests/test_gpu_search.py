@@ -9,6 +9,8 @@ import numpy as np
 import pytest
 import torch
 
+import guard
+
 from oracle import oracle as O
 from lfsr_seeded_moe_b200 import synth
 
@@ -29,9 +31,9 @@ class _Out:
     def __init__(self, N, K, P, bias):
         nb = K // 8
         self.N, self.K, self.P = N, K, P
-        self.seeds = torch.full((N, nb), -1, dtype=torch.int16, device="cuda")
-        self.coefs = torch.full((N, nb), -1, dtype=torch.int16, device="cuda")
-        self.codes = torch.full((N, nb // 2), 0xEE, dtype=torch.uint8, device="cuda") if P == 4 else None
+        self.seeds = guard.buffer((N, nb), torch.int16, fill=-1)
+        self.coefs = guard.buffer((N, nb), torch.int16, fill=-1)
+        self.codes = guard.buffer((N, nb // 2), torch.uint8, fill=0xEE) if P == 4 else None
         self.exp_bias = torch.as_tensor(np.asarray(bias, np.int32)).cuda()
 
     def fields(self):
@@ -50,7 +52,7 @@ class _Out:
 def _run(nslm, w, P, bias, lo, hi, imp=None):
     N, K = w.shape
     out = _Out(N, K, P, bias)
-    err = torch.full((N, K // 8), float("nan"), dtype=torch.float64, device="cuda")
+    err = guard.buffer((N, K // 8), torch.float64, fill=float("nan"))
     dimp = None if imp is None else torch.as_tensor(imp, dtype=torch.float32).cuda()
     nslm.nslm_seed_search(torch.as_tensor(w, dtype=torch.float32).cuda(), out, lo, hi, err, imp=dimp)
     torch.cuda.synchronize()

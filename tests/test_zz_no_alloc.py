@@ -14,6 +14,8 @@ import numpy as np
 import pytest
 import torch
 
+import guard
+
 from oracle import oracle as O
 from lfsr_seeded_moe_b200 import synth
 
@@ -47,16 +49,16 @@ def test_static_scratch_matches_workspace_entry_point_and_oracle_twice(nslm, E, 
     xb = synth.activations((950, T), T, hidden)
     x = xb.to(dev)
     logits = synth.router_logits((950, T), T, E)
-    ids = torch.empty(T, k, dtype=torch.int32, device=dev)
-    w = torch.empty(T, k, dtype=torch.float32, device=dev)
+    ids = guard.buffer((T, k), torch.int32)
+    w = guard.buffer((T, k), torch.float32)
     nslm.nslm_moe_route_topk(logits.to(dev), T, E, k, ids, w)
 
-    ref = torch.full((T, hidden), float("nan"), device=dev)
+    ref = guard.buffer((T, hidden), torch.float32, fill=float("nan"))
     wsb = nslm.nslm_workspace_bytes(nslm.NSLM_OP_MOE_FFN, T, E, hidden, inter, k)
-    ws = torch.empty(wsb, dtype=torch.uint8, device=dev)
+    ws = guard.buffer(wsb, torch.uint8)
     nslm.nslm_moe_seed_ffn(L.gate, L.up, L.down, E, x, ids, w, T, k, ref, ws, wsb)
 
-    outs = [torch.full((T, hidden), float("nan"), device=dev) for _ in range(2)]
+    outs = [guard.buffer((T, hidden), torch.float32, fill=float("nan")) for _ in range(2)]
     nslm.nslm_moe_seed_ffn_static(L.gate, L.up, L.down, E, x, ids, w, T, k, outs[0])
     torch.cuda.synchronize()
     free_before = torch.cuda.mem_get_info()[0]
