@@ -17,7 +17,8 @@ clocks seen during the timed region and the CPU oracle's time on a sample.
 Extra objects, each skippable by its flag: one_layer_decode (one layer's
 latency and HBM fraction), stack_batch8 (the same stack at 8 tokens a step,
 --no-batch8), batched (the tcgen05 grouped GEMM layer at 64 and 512 tokens,
---no-batched), host_experts (experts kept in pinned host memory behind the
+--no-batched), stack_p3c5 (the one-token stack in the 5-bit P=3 format,
+--no-p3c5), host_experts (experts kept in pinned host memory behind the
 device expert cache, one GPU only, --no-host-experts) and seed_search (the
 seed/coefficient search, plain and importance-weighted, --no-search).
 --profile runs one small case of a single kernel family for ncu and prints
@@ -59,20 +60,53 @@ def peaks():
     return FALLBACK_HBM_GBS, "fallback"
 
 
-def layer_packed_bytes_per_token() -> int:
-    per_expert = 2 * (INTER * (HIDDEN // 8) * 4.5 + 4 * INTER) + (HIDDEN * (INTER // 8) * 4.5 + 4 * HIDDEN)
+def layer_packed_bytes_per_token(per_block: float = 4.5) -> int:
+    """Packed bytes one token reads in one layer: 8 experts' gate, up and down
+    fields (per_block bytes per 8-weight block: 4.5 for P=4, 4.375 for the
+    5-bit P=3 format) plus an int32 exponent bias per row."""
+    per_expert = 2 * (INTER * (HIDDEN // 8) * per_block + 4 * INTER) + (HIDDEN * (INTER // 8) * per_block + 4 * HIDDEN)
     return int(K_TOP * per_expert)
 
 
 # ------------------------------------------------------------------ clocks
 
+_POLLER = r"""
+import sys, time
+import pynvml as nv
+uuid, index, period = sys.argv[1], int(sys.argv[2]), float(sys.argv[3])
+nv.nvmlInit()
+try:
+    h = nv.nvmlDeviceGetHandleByUUID(uuid) if uuid else nv.nvmlDeviceGetHandleByIndex(index)
+except nv.NVMLError:
+    h = nv.nvmlDeviceGetHandleByIndex(index)
+try:
+    mx = nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM)
+except nv.NVMLError:
+    mx = "[N/A]"
+bits = (0x8, 0x40, 0x20, 0x4)
+print("ready", flush=True)
+while True:
+    try:
+        sm = nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM)
+        pw = nv.nvmlDeviceGetPowerUsage(h) / 1000.0
+        rs = nv.nvmlDeviceGetCurrentClocksEventReasons(h)
+        flags = ", ".join("Active" if rs & b else "Not Active" for b in bits)
+        print(f"{time.monotonic():.6f}|{index}, {sm}, {mx}, {pw:.1f}, {rs:#x}, {flags}", flush=True)
+    except nv.NVMLError:
+        pass
+    time.sleep(period)
+"""
+
+
 class ClockSampler:
     """Samples SM clocks and throttle reasons while the timed region runs.
 
-    NVML is polled every 2 ms from a thread (so that even a region of a few
-    tens of milliseconds gets several samples), on the GPU that CUDA device
-    `dev` is (matched by UUID, since CUDA and NVML may number GPUs
-    differently); without NVML, nvidia-smi is run at its 20 ms interval.
+    A child process polls NVML every 2 ms (a process of its own, so that the
+    timed loop, which holds the interpreter lock, cannot starve it) on the GPU
+    that CUDA device `dev` is (matched by UUID, since CUDA and NVML may number
+    GPUs differently) and stamps each sample with the monotonic clock; only
+    samples inside the marked window (mark_start / mark_end around the timed
+    region) are kept.  Without NVML, nvidia-smi runs at its 20 ms interval.
     Every sample is kept as one CSV row in nvidia-smi's field order."""
 
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
@@ -87,43 +121,23 @@ class ClockSampler:
         self.period = period_s
         self.proc = None
         self.thread = None
-        self.stop = threading.Event()
-        self.lines = []
-
-    def _nvml_handle(self):
-        import pynvml
-        pynvml.nvmlInit()
-        if self.uuid:
-            try:
-                return pynvml, pynvml.nvmlDeviceGetHandleByUUID(self.uuid)
-            except pynvml.NVMLError:
-                pass
-        return pynvml, pynvml.nvmlDeviceGetHandleByIndex(self.gpu)
-
-    def _poll(self, nv, h):
-        try:
-            mx = nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM)
-        except nv.NVMLError:
-            mx = "[N/A]"
-        while not self.stop.is_set():
-            try:
-                sm = nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM)
-                pw = nv.nvmlDeviceGetPowerUsage(h) / 1000.0
-                rs = nv.nvmlDeviceGetCurrentClocksEventReasons(h)
-                flags = ", ".join("Active" if rs & b else "Not Active" for b in self.BITS)
-                self.lines.append(f"{self.gpu}, {sm}, {mx}, {pw:.1f}, {rs:#x}, {flags}")
-            except nv.NVMLError:
-                pass
-            self.stop.wait(self.period)
+        self.stamped = []   # (monotonic time, row) from the NVML poller
+        self.lines = []     # rows kept for the summary
+        self.t0 = self.t1 = None
 
     def __enter__(self):
         try:
-            nv, h = self._nvml_handle()
-            self.thread = threading.Thread(target=self._poll, args=(nv, h), daemon=True)
+            self.proc = subprocess.Popen([sys.executable, "-c", _POLLER, self.uuid or "", str(self.gpu), str(self.period)],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            if self.proc.stdout.readline().strip() != "ready":
+                raise OSError("no NVML poller")
+            self.thread = threading.Thread(target=self._read_stamped, daemon=True)
             self.thread.start()
             return self
-        except Exception:  # no NVML: fall back to nvidia-smi
-            self.thread = None
+        except OSError:
+            if self.proc is not None:
+                self.proc.kill()
+            self.proc = None
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
@@ -135,13 +149,27 @@ class ClockSampler:
             self.proc = None
         return self
 
+    def mark_start(self):
+        self.t0 = time.monotonic()
+
+    def mark_end(self):
+        self.t1 = time.monotonic()
+
+    def _read_stamped(self):
+        for line in self.proc.stdout:
+            t, _, row = line.strip().partition("|")
+            try:
+                self.stamped.append((float(t), row))
+            except ValueError:
+                pass
+
     def _read(self):
         for line in self.proc.stdout:
             self.lines.append(line.strip())
 
     def __exit__(self, *exc):
-        self.stop.set()
         if self.proc is not None:
+            time.sleep(2 * self.period)  # the samples of the window's last moments
             self.proc.terminate()
             try:
                 self.proc.wait(timeout=5)
@@ -149,6 +177,15 @@ class ClockSampler:
                 self.proc.kill()
         if self.thread is not None:
             self.thread.join(timeout=5)
+        self.keep_window()
+
+    def keep_window(self):
+        """Keep the stamped samples taken inside [mark_start, mark_end]."""
+        if self.stamped:
+            t0 = self.t0 if self.t0 is not None else float("-inf")
+            t1 = self.t1 if self.t1 is not None else float("inf")
+            self.lines.extend(row for t, row in self.stamped if t0 <= t <= t1)
+            self.stamped = []
 
     def summary(self):
         sm, mx, reasons = [], None, set()
@@ -531,6 +568,46 @@ def stack_batch_leg(torch, nslm, synth, dev, arr, hbm, T: int, steps: int, rank:
             "note": "one cooperative launch for all 45 layers (plus the routing launch); inputs > L2"}
 
 
+def stack_p3c5_leg(torch, nslm, synth, dev, hbm, steps: int, rank: int):
+    """The 45-layer one-token stack with every expert in the 5-bit P=3 format
+    (4.375 bits per weight), on the same persistent kernel, 8 cycled inputs."""
+    Pf, S = nslm.NSLM_P3C5, 8
+    layers = [synth.moe_layer(l, E, HIDDEN, INTER, Pf, device=dev, config=5) for l in range(LAYERS)]
+    arr = nslm.moe_layers([(L.gate, L.up, L.down) for L in layers])
+    logits = [torch.stack([synth.router_logits((5, l, rank, s), 1, E) for l in range(LAYERS)]).to(dev).contiguous()
+              for s in range(S)]
+    xs = [synth.activations((5, rank, s), 1, HIDDEN).to(dev).contiguous() for s in range(S)]
+    y = torch.empty(1, HIDDEN, device=dev)
+    wsb = nslm.nslm_workspace_bytes(nslm.NSLM_OP_MOE_STACK, 1, E, HIDDEN, INTER, K_TOP, LAYERS)
+    ws = torch.zeros(wsb, dtype=torch.uint8, device=dev)
+    graphs = []
+    for s in range(S):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            nslm.nslm_moe_stack_decode(arr, LAYERS, E, K_TOP, logits[s], xs[s], 1, y, ws, wsb)
+        graphs.append(g)
+    for i in range(3):
+        graphs[i % S].replay()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for i in range(steps):
+        graphs[i % S].replay()
+    e1.record()
+    torch.cuda.synchronize()
+    t = e0.elapsed_time(e1) * 1e-3 / steps
+    status = int(ws[:4].view(torch.int32).item())
+    nbytes = LAYERS * layer_packed_bytes_per_token(4.375)
+    graphs.clear()
+    del layers, arr
+    torch.cuda.empty_cache()
+    return {"format": "P=3 with 5-bit coefficients (4.375 bits per weight)", "batch_tokens": 1,
+            "value": round(1.0 / t, 2), "unit": "tokens/s", "ms_per_step": round(t * 1e3, 4), "steps": steps,
+            "status": status, "packed_GB_per_step": round(nbytes / 1e9, 3),
+            "hbm_frac": round(nbytes / t / 1e9 / hbm, 4),
+            "note": "one cooperative launch for all 45 layers (plus the routing launch); inputs > L2"}
+
+
 def host_experts_leg(torch, nslm, synth, dev, n_layers: int = 8, slots: int = 400, tokens: int = 32):
     """One-token decode with the routed experts in pinned host memory behind the
     VRAM expert cache (LRU, copies by the device from host memory): per token and
@@ -686,6 +763,7 @@ def main():
     ap.add_argument("--no-search", action="store_true")
     ap.add_argument("--no-batch8", action="store_true", help="skip the 8-token stack leg")
     ap.add_argument("--no-host-experts", action="store_true", help="skip the host-memory expert cache leg")
+    ap.add_argument("--no-p3c5", action="store_true", help="skip the 5-bit P=3 stack leg")
     ap.add_argument("--profile", choices=["layer", "layer8", "batched", "gemv", "search"],
                     help="run a small fixed workload for an ncu capture and exit")
     args = ap.parse_args()
@@ -741,11 +819,13 @@ def main():
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     with ClockSampler(dev.index if dev.index is not None else 0, device_uuid(torch, dev)) as clk:
         torch.cuda.synchronize()
+        clk.mark_start()
         e0.record()
         for i in range(args.steps):
             graphs[i % S].replay()
         e1.record()
         torch.cuda.synchronize()
+        clk.mark_end()
     if world > 1:
         dist.barrier()
     elapsed = slowest_rank_time(e0.elapsed_time(e1) * 1e-3, world, dev)
@@ -860,6 +940,10 @@ def main():
     if T == 1 and not args.no_batch8:
         batch8 = stack_batch_leg(torch, nslm, synth, dev, arr, hbm, 8, max(10, args.steps // 4), rank)
 
+    p3c5 = None
+    if T == 1 and not args.no_p3c5:
+        p3c5 = stack_p3c5_leg(torch, nslm, synth, dev, hbm, max(10, args.steps // 4), rank)
+
     host_experts = None
     if T == 1 and world == 1 and not args.no_host_experts:  # pins 3.9 GB of host memory per process
         host_experts = host_experts_leg(torch, nslm, synth, dev)
@@ -887,6 +971,8 @@ def main():
     line["one_layer_decode"] = one_layer
     if batch8 is not None:
         line["stack_batch8"] = batch8
+    if p3c5 is not None:
+        line["stack_p3c5"] = p3c5
     if host_experts is not None:
         line["host_experts"] = host_experts
     if search is not None:

@@ -79,11 +79,10 @@ typedef struct CUstream_st *nslm_stream_t;
  * complement in bits 0-4, 5-9, 10-14 and bit 0 of the exponent code in bit 15;
  * codes: u8 [N][3 K / 64] holds code bits 1..3 of block b of a row at bits
  * 3b .. 3b+2 of the row's bit string, least significant bit first.  K must be
- * a multiple of 64.  Taken by nslm_seed_gemv, the debug decompression, and
- * the decode FFN and layer stack for T <= 8 (on the per-layer kernels, not
- * the persistent ones); the tensor-core FFN path (T > 8), grouped GEMM,
- * search, expert cache, nibbles and hybrid entry points return
- * NSLM_ERR_SHAPE for it. */
+ * a multiple of 64.  Taken by nslm_seed_gemv, the debug decompression, the
+ * decode FFN and layer stack (T <= 8, persistent and per-layer kernels), the
+ * tensor-core FFN path (T > 8) and nslm_seed_grouped_gemm; the search, expert
+ * cache, nibbles and hybrid entry points return NSLM_ERR_SHAPE for it. */
 #define NSLM_P3C5 35
 
 /* One packed seed matrix (see the layout above).  For a stack of E experts,

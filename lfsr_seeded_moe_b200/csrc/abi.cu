@@ -383,7 +383,7 @@ int32_t nslm_moe_seed_ffn(const nslm_seed_matrix *gate, const nslm_seed_matrix *
   if (k < 1 || k > kMaxK || T < 0) return NSLM_ERR_SHAPE;
   if (!aligned16(x_bf16) || !aligned16(y)) return NSLM_ERR_ALIGN;
   if (T == 0) return NSLM_OK;
-  if (T > kMaxT && (d.hidden % 64 || d.inter % 64 || E > 1024 || d.P == kP3C5)) return NSLM_ERR_SHAPE;
+  if (T > kMaxT && (d.hidden % 64 || d.inter % 64 || E > 1024)) return NSLM_ERR_SHAPE;
   const size_t need = nslm_workspace_bytes(NSLM_OP_MOE_FFN, T, E, d.hidden, d.inter, k, 0);
   if (!ws || ws_bytes < need) return NSLM_ERR_WORKSPACE;
   if (!aligned16(ws)) return NSLM_ERR_ALIGN;

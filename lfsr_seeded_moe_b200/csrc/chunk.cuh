@@ -172,6 +172,16 @@ __device__ __forceinline__ void load_chunk(const uint16_t *__restrict__ seeds_ro
   }
 }
 
+// The 5-bit format's 24 code bits (bits 1..3 of 8 blocks' codes) of chunk
+// `chunk` of a matrix (counted over all rows): 3 bytes at 3 * chunk, which are
+// not 4-byte aligned, so they come by plain loads into a register, not into
+// the cp.async field slots.
+__device__ __forceinline__ uint32_t load_codes3(const nslm_seed_matrix &W, size_t chunk) {
+  if (!in_bounds(chunk, (size_t)W.N * (size_t)(W.K >> 6), 1)) return 0u;
+  const uint8_t *q = W.codes + 3 * chunk;
+  return (uint32_t)__ldcs(q) | ((uint32_t)__ldcs(q + 1) << 8) | ((uint32_t)__ldcs(q + 2) << 16);
+}
+
 // The scale key of a row's exponent bias (bounds-checked like the fields).
 __device__ __forceinline__ uint32_t load_bias_key(const nslm_seed_matrix &W, size_t row) {
   return row_scale_key(in_bounds(row, (size_t)W.N, 4) ? __ldg(W.exp_bias + row) : 0);

@@ -109,6 +109,16 @@ __device__ __forceinline__ void load_slice(const uint32_t *const (&sp)[2], const
     f.s2[j] = ok[j] ? __ldcs(sp[j] + 4 * kt) : 0u;
     f.q2[j] = ok[j] ? __ldcs(qp[j] + 4 * kt) : 0u;
     f.c2[j] = (P == 4 && ok[j]) ? (uint32_t)__ldcs(cp[j] + 4 * kt) : 0u;
+    if (P == kP3C5 && ok[j]) {
+      // the pair's 6 code bits (bits 1..3 of two codes) at bit 6 bp of the
+      // slice's 3 bytes: one byte for bp = 0, 3, two for bp = 1, 2; cp is the
+      // row's codes; bit 0 of each code is bit 15 of its coefs half
+      const uint8_t *cb = cp[j] + 3 * kt + ((6 * bp) >> 3);
+      uint32_t t = __ldcs(cb);
+      if (bp == 1 || bp == 2) t |= (uint32_t)__ldcs(cb + 1) << 8;
+      const uint32_t c6 = (t >> ((6 * bp) & 7)) & 0x3Fu, q = f.q2[j];
+      f.c2[j] = (((q >> 15) & 1u) | ((c6 & 7u) << 1)) | ((((q >> 31) & 1u) | ((c6 >> 3) << 1)) << 4);
+    }
   }
 }
 
@@ -300,7 +310,8 @@ __global__ void __launch_bounds__(kCtaThreads, 1) grouped_seed_gemm_kernel(const
         }
         sp[j] = reinterpret_cast<const uint32_t *>(W.seeds + wr * p.nb) + bp;
         qp[j] = reinterpret_cast<const uint32_t *>(W.coefs + wr * p.nb) + bp;
-        cpp[j] = (P == 4) ? W.codes + wr * (p.nb / 2) + bp : nullptr;
+        cpp[j] = (P == 4) ? W.codes + wr * (p.nb / 2) + bp
+                 : (P == kP3C5) ? W.codes + wr * (size_t)(3 * p.nb / 8) : nullptr;
         rowk[j] = load_bias_key(W, wr);
       }
       const size_t a_off = ((trow >> 3) * 8 + 2 * bp) * 128 + (trow & 7) * 16;
@@ -528,6 +539,11 @@ static int32_t launch_grouped_t(const GroupedParams &p, cudaStream_t s) {
 }
 
 int32_t launch_grouped(const GroupedParams &p, int P, int mode, cudaStream_t s) {
+  if (P == kP3C5) {
+    if (mode == GMODE_GEMM) return launch_grouped_t<kP3C5, GMODE_GEMM>(p, s);
+    if (mode == GMODE_GATEUP) return launch_grouped_t<kP3C5, GMODE_GATEUP>(p, s);
+    return launch_grouped_t<kP3C5, GMODE_DOWN>(p, s);
+  }
   if (P == 4) {
     if (mode == GMODE_GEMM) return launch_grouped_t<4, GMODE_GEMM>(p, s);
     if (mode == GMODE_GATEUP) return launch_grouped_t<4, GMODE_GATEUP>(p, s);
@@ -638,7 +654,6 @@ extern "C" int32_t nslm_seed_grouped_gemm(const nslm_seed_matrix *W, int32_t E,
   g_launches = 0;
   int32_t st = check_matrix(W);
   if (st) return st;
-  if (W->P == kP3C5) return NSLM_ERR_SHAPE;  // the tensor-core path takes P = 3 and P = 4
   if (!x_bf16 || !offsets || !y) return NSLM_ERR_ARG;
   if (E < 1 || E > 1024 || R < 0) return NSLM_ERR_SHAPE;
   if (W->N % E != 0) return NSLM_ERR_SHAPE;

@@ -127,6 +127,10 @@ __global__ void __launch_bounds__(kStack1MaxThreads, 1) stack1_kernel(const __gr
   const int n0 = blockIdx.x * p.rpc;
   const int nrows = max(0, min(p.rpc, p.hidden - n0));
 
+  // code bits of the 5-bit format: fetched into these registers with the
+  // other fields of the next task, taken over at the start of its step
+  uint32_t nqg = 0, nqu = 0, nqd = 0;
+
   // ---- phase A task geometry (a step = one chunk round of one routed row)
   auto a_steps = [&](int nslots) {
     const int ntask = nslots * p.inter;
@@ -149,6 +153,10 @@ __global__ void __launch_bounds__(kStack1MaxThreads, 1) stack1_kernel(const __gr
       const uint32_t r32 = (uint32_t)grow, off = r32 * (uint32_t)nbh + 8u * (uint32_t)c;
       fetch_chunk_off<P>(Lm.gate, off, r32, fs, (2 * buf) * nthr + tid);
       fetch_chunk_off<P>(Lm.up, off, r32, fs, (2 * buf + 1) * nthr + tid);
+      if (P == kP3C5) {
+        nqg = load_codes3(Lm.gate, off >> 3);
+        nqu = load_codes3(Lm.up, off >> 3);
+      }
     } else {
       load_chunk<P, false>(Lm.gate.seeds + grow * nbh, Lm.gate.coefs + grow * nbh,
                            P == 4 ? Lm.gate.codes + grow * (nbh / 2) : nullptr, nbh, c, fg, grow,
@@ -175,6 +183,7 @@ __global__ void __launch_bounds__(kStack1MaxThreads, 1) stack1_kernel(const __gr
     if (VEC) {
       const uint32_t r32 = (uint32_t)grow;
       fetch_chunk_off<P>(Lm.down, r32 * (uint32_t)nbi + 8u * (uint32_t)c, r32, fs, buf * nthr + tid);
+      if (P == kP3C5) nqd = load_codes3(Lm.down, r32 * (uint32_t)(nbi >> 3) + (uint32_t)c);
     } else {
       load_chunk<P, false>(Lm.down.seeds + grow * nbi, Lm.down.coefs + grow * nbi,
                            P == 4 ? Lm.down.codes + grow * (nbi / 2) : nullptr, nbi, c, f, grow,
@@ -224,11 +233,16 @@ __global__ void __launch_bounds__(kStack1MaxThreads, 1) stack1_kernel(const __gr
         ChunkFields cg = fg, cu = fu;
         uint32_t ckg = kg, cku = ku;
         if (VEC) {
+          const uint32_t cqg = nqg, cqu = nqu;  // this step's 5-bit-format code bits
           if (step + 1 < nsteps) a_fetch(Lm, s_expert, step + 1, (step + 1) & 1, fg, fu, kg, ku);
           cp_async_commit();
           cp_async_wait<1>();
           read_chunk<P>(fs, (2 * (step & 1)) * nthr + tid, cg, ckg);
           read_chunk<P>(fs, (2 * (step & 1) + 1) * nthr + tid, cu, cku);
+          if (P == kP3C5) {
+            cg.codes = cqg;
+            cu.codes = cqu;
+          }
         } else if (step + 1 < nsteps) {
           a_fetch(Lm, s_expert, step + 1, 0, fg, fu, kg, ku);
         }
@@ -284,10 +298,12 @@ __global__ void __launch_bounds__(kStack1MaxThreads, 1) stack1_kernel(const __gr
         ChunkFields cf = fd;
         uint32_t ck = kd;
         if (VEC) {
+          const uint32_t cqd = nqd;  // this task's 5-bit-format code bits
           if (t + nthr < bt) b_fetch(Lm, dSC, SC, t + nthr, (it + 1) & 1, fd, kd);
           cp_async_commit();
           cp_async_wait<1>();
           read_chunk<P>(fs, (it & 1) * nthr + tid, cf, ck);
+          if (P == kP3C5) cf.codes = cqd;
         } else if (t + nthr < bt) {
           b_fetch(Lm, dSC, SC, t + nthr, 0, fd, kd);
         }
@@ -369,7 +385,7 @@ static size_t stack1_smem(const FfnDims &d, int k, int threads) {
 
 bool stack1_supported(const FfnDims &d, int k) {
   if (k < 1 || k > kMaxK) return false;
-  if (d.P != 3 && d.P != 4) return false;  // the 5-bit format runs on the per-layer kernels
+  if (d.P != 3 && d.P != 4 && d.P != kP3C5) return false;
   // 32-bit element offsets into the field streams
   if ((int64_t)d.E * d.inter * (d.hidden / 8) >= (1ll << 31) || (int64_t)d.E * d.hidden * (d.inter / 8) >= (1ll << 31))
     return false;
@@ -446,6 +462,8 @@ int32_t launch_stack1(const FfnDims &d, const nslm_moe_layer *layers, int n, con
                       const uint16_t *x0, const float *y_in, int k, float *h, float *y_mid,
                       float *y_out, int32_t *sync, float *rms_part, cudaStream_t s, int &launches) {
   const bool vec = d.hidden % 64 == 0 && d.inter % 64 == 0;
+  if (d.P == kP3C5)  // K % 64 == 0 for both projections: whole chunks always
+    return launch_stack1_t<kP3C5, true>(d, layers, n, plans, x0, y_in, k, h, y_mid, y_out, sync, rms_part, s, launches);
   if (d.P == 4)
     return vec ? launch_stack1_t<4, true>(d, layers, n, plans, x0, y_in, k, h, y_mid, y_out, sync, rms_part, s, launches)
                : launch_stack1_t<4, false>(d, layers, n, plans, x0, y_in, k, h, y_mid, y_out, sync, rms_part, s, launches);

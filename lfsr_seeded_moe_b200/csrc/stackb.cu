@@ -155,6 +155,9 @@ __global__ void __launch_bounds__(kStackBThreads, 1) stackb_kernel(const __grid_
     row = t - slot * p.inter;
     c = lane + 32 * (step - i * p.J);
   };
+  // code bits of the 5-bit format: fetched into these registers with the
+  // other fields of the next task, taken over at the start of its step
+  uint32_t nqg = 0, nqu = 0, nqd = 0;
   auto a_fetch = [&](const LayerMatsB &Lm, const int *expert, int step, int buf) {
     int slot, row, c;
     a_locate(step, slot, row, c);
@@ -163,6 +166,10 @@ __global__ void __launch_bounds__(kStackBThreads, 1) stackb_kernel(const __grid_
     const uint32_t off = r32 * (uint32_t)nbh + 8u * (uint32_t)c;
     fetch_chunk_off<P>(Lm.gate, off, r32, fsA, (2 * buf) * nthr + tid);
     fetch_chunk_off<P>(Lm.up, off, r32, fsA, (2 * buf + 1) * nthr + tid);
+    if (P == kP3C5) {
+      nqg = load_codes3(Lm.gate, off >> 3);
+      nqu = load_codes3(Lm.up, off >> 3);
+    }
   };
   // ---- phase B task geometry: task t of group g = (slot s, row r, chunk pair q);
   // its step 0 takes chunk q, step 1 chunk q + Cq
@@ -187,6 +194,7 @@ __global__ void __launch_bounds__(kStackBThreads, 1) stackb_kernel(const __grid_
     if (r < 0 || c >= p.Ci) return;
     const uint32_t r32 = (uint32_t)s_expert[s] * (uint32_t)p.hidden + (uint32_t)(n0 + r);
     fetch_chunk_off<P>(Lm.down, r32 * (uint32_t)nbi + 8u * (uint32_t)c, r32, fsB, buf * nthr + tid);
+    if (P == kP3C5) nqd = load_codes3(Lm.down, r32 * (uint32_t)(nbi >> 3) + (uint32_t)c);
   };
 
   uint32_t nbar = 0;  // grid barriers passed in this launch
@@ -285,6 +293,7 @@ __global__ void __launch_bounds__(kStackBThreads, 1) stackb_kernel(const __grid_
       for (int step = 0; step < nsteps; ++step) {
         int slot, row, c;
         a_locate(step, slot, row, c);
+        const uint32_t cqg = nqg, cqu = nqu;  // this step's 5-bit-format code bits
         if (step + 1 < nsteps) a_fetch(Lm, s_expert, step + 1, (step + 1) & 1);
         cp_async_commit();
         cp_async_wait<1>();
@@ -292,6 +301,10 @@ __global__ void __launch_bounds__(kStackBThreads, 1) stackb_kernel(const __grid_
         uint32_t ckg, cku;
         read_chunk<P>(fsA, (2 * (step & 1)) * nthr + tid, cg, ckg);
         read_chunk<P>(fsA, (2 * (step & 1) + 1) * nthr + tid, cu, cku);
+        if (P == kP3C5) {
+          cg.codes = cqg;
+          cu.codes = cqu;
+        }
         const int q0 = s_start[slot], M = min(MT, s_start[slot + 1] - q0);
         int off[MT];
 #pragma unroll
@@ -373,6 +386,7 @@ __global__ void __launch_bounds__(kStackBThreads, 1) stackb_kernel(const __grid_
         for (int k = 0; k < n; ++k) {
           int r, s, q, c;
           b_locate(g, k, r, s, q, c);
+          const uint32_t cqd = nqd;  // this task's 5-bit-format code bits
           if (k + 1 < n) {
             b_fetch(Lm, g, k + 1, (it + 1) & 1);
           } else if (g + 1 < s_ngroups && b_nsteps(g + 1) > 0) {
@@ -384,6 +398,7 @@ __global__ void __launch_bounds__(kStackBThreads, 1) stackb_kernel(const __grid_
           ChunkFields cf;
           uint32_t ck;
           read_chunk<P>(fsB, (it & 1) * nthr + tid, cf, ck);
+          if (P == kP3C5) cf.codes = cqd;
           ++it;
           const int q0 = s_start[s], M = min(MT, s_start[s + 1] - q0);
           if ((k & 1) == 0) {
@@ -506,7 +521,7 @@ bool stackb_shape(const FfnDims &d, int T, int k, StackBShape &sh) {
 }  // namespace
 
 bool stackb_supported(const FfnDims &d, int T, int k) {
-  if (d.P != 3 && d.P != 4) return false;  // the 5-bit format runs on the per-layer kernels
+  if (d.P != 3 && d.P != 4 && d.P != kP3C5) return false;
   StackBShape sh{};
   if (!stackb_shape(d, T, k, sh)) return false;
   // 32-bit element offsets into the field streams
@@ -587,6 +602,9 @@ int32_t launch_stackb(const FfnDims &d, const nslm_moe_layer *layers, int n, con
   if (!stackb_shape(d, T, k, sh)) return NSLM_ERR_SHAPE;
   if (d.P == 4)
     return launch_stackb_t<4>(d, sh, layers, n, plans, x0, y_in, T, k, h, y_mid, y_out, sync, rms_part, s, launches);
+  if (d.P == kP3C5)
+    return launch_stackb_t<kP3C5>(d, sh, layers, n, plans, x0, y_in, T, k, h, y_mid, y_out, sync, rms_part, s,
+                                  launches);
   return launch_stackb_t<3>(d, sh, layers, n, plans, x0, y_in, T, k, h, y_mid, y_out, sync, rms_part, s, launches);
 }
 

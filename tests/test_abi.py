@@ -147,21 +147,20 @@ def test_expert_cache_argument_checks():
 
 def test_p3c5_format_checks():
     # P = 35 (three 5-bit coefficients): K a multiple of 64 and a codes stream;
-    # taken by the GEMV and decompression, refused by the FFN, grouped GEMM
-    # and search entry points
+    # taken by the GEMV, decompression, FFN (decode and tensor-core paths) and
+    # grouped GEMM, refused by the search
     assert _gemv(_mat(K=96, P=35)) == nslm.NSLM_ERR_SHAPE
     assert _gemv(_mat(K=128, P=35, codes=False)) == nslm.NSLM_ERR_ARG
     E, hidden, inter = 4, 256, 128
     f = nslm.raw().nslm_moe_seed_ffn
     g, u, d = _mat(E * inter, hidden, P=35), _mat(E * inter, hidden, P=35), _mat(E * hidden, inter, P=35)
     ws = nslm.nslm_workspace_bytes(nslm.NSLM_OP_MOE_FFN, 16, E, hidden, inter, 2)
-    # T <= 8 runs the per-layer decode kernels: the arguments pass (without a
-    # device the call then stops at the device check); T > 8 is refused
-    st1 = f(ctypes.byref(g), ctypes.byref(u), ctypes.byref(d), E, 0x7000000, 0x7100000, 0x7200000, 1, 2,
-            0x7300000, 0x7400000, ws, 0)
-    assert st1 not in (nslm.NSLM_ERR_SHAPE, nslm.NSLM_ERR_ARG, nslm.NSLM_ERR_ALIGN, nslm.NSLM_ERR_WORKSPACE)
-    assert f(ctypes.byref(g), ctypes.byref(u), ctypes.byref(d), E, 0x7000000, 0x7100000, 0x7200000, 16, 2,
-             0x7300000, 0x7400000, ws, 0) == nslm.NSLM_ERR_SHAPE
+    # both the decode (T <= 8) and the tensor-core (T > 8) paths take the
+    # arguments (without a device the call then stops at the device check)
+    for T in (1, 16):
+        st = f(ctypes.byref(g), ctypes.byref(u), ctypes.byref(d), E, 0x7000000, 0x7100000, 0x7200000, T, 2,
+               0x7300000, 0x7400000, ws, 0)
+        assert st not in (nslm.NSLM_ERR_SHAPE, nslm.NSLM_ERR_ARG, nslm.NSLM_ERR_ALIGN, nslm.NSLM_ERR_WORKSPACE)
     # a layer mixing formats is refused
     assert f(ctypes.byref(g), ctypes.byref(_mat(E * inter, hidden, P=4)), ctypes.byref(d), E, 0x7000000, 0x7100000,
              0x7200000, 1, 2, 0x7300000, 0x7400000, ws, 0) == nslm.NSLM_ERR_SHAPE

@@ -78,3 +78,14 @@ def test_clock_sampler_rows_from_nvml_reason_bits():
         flags = ", ".join("Active" if mask & b else "Not Active" for b in bench.ClockSampler.BITS)
         s.lines.append(f"0, {sm}, 1965, 900.0, {mask:#x}, {flags}")
     assert s.summary() == {"sm_mhz": 1900.0, "sm_max_mhz": 1965.0, "reasons": ["sw_power_cap"], "samples": 3}
+
+
+def test_clock_sampler_keeps_only_the_timed_window():
+    # samples stamped by the poller process before and after the timed region
+    # are dropped; those inside it are summarised
+    s = bench.ClockSampler(0)
+    row = "0, {}, 1965, 900.0, 0x0, Not Active, Not Active, Not Active, Not Active"
+    s.stamped = [(0.5, row.format(1200)), (1.0, row.format(1965)), (1.2, row.format(1950)), (2.5, row.format(700))]
+    s.t0, s.t1 = 0.9, 2.0
+    s.keep_window()
+    assert s.summary() == {"sm_mhz": 1957.5, "sm_max_mhz": 1965.0, "reasons": [], "samples": 2}

@@ -32,7 +32,7 @@ def _status(ws):
     return int(ws[:4].view(torch.int32).item())
 
 
-@pytest.mark.parametrize("P", [3, 4])
+@pytest.mark.parametrize("P", [3, 4, 35])
 @pytest.mark.parametrize("rows,K,counts", [
     (256, 512, [0, 5, 40, 300]),      # an empty expert; one expert over 256 rows (two N tiles)
     (200, 192, [17, 1, 64]),          # ragged row tile (200 = 128 + 72), K of three slices
@@ -82,7 +82,7 @@ def _batched_case(nslm, E, hidden, inter, P, T, k, tag, zipf=None, sample=None):
     return y.cpu().numpy()[toks], ref
 
 
-@pytest.mark.parametrize("P", [3, 4])
+@pytest.mark.parametrize("P", [3, 4, 35])
 @pytest.mark.parametrize("T", [9, 64])
 def test_batched_ffn_small(nslm, P, T):
     got, ref = _batched_case(nslm, 16, 256, 128, P, T, 4, 961)

@@ -360,13 +360,21 @@ def test_ffn_hybrid_p3_p4_experts(nslm, T):
 
 @pytest.mark.parametrize("T", [1, 3])
 def test_ffn_decode_p3c5_layer(nslm, T):
-    # the 5-bit P=3 format through the decode FFN (the per-layer kernels)
+    # the 5-bit P=3 format through the decode FFN (the persistent kernels:
+    # T = 1 one-token, T = 3 batched)
     y, ref = _ffn_case(nslm, 10, 512, 256, 35, T, 4, 947 + T)
     assert O.normwise_rel_err(y, ref) <= TIGHT
 
 
-def test_stack_decode_p3c5(nslm):
-    Lyr, E, hidden, inter, P, k, T = 4, 8, 256, 128, 35, 2, 2
+def test_ffn_decode_p3c5_full_layer(nslm):
+    # the benchmarked layer shape (100 experts, 2048/1408, top-8) in the 5-bit format, one token
+    y, ref = _ffn_case(nslm, 100, 2048, 1408, 35, 1, 8, 949)
+    assert O.normwise_rel_err(y, ref) <= TIGHT, O.elementwise_rel_err(y, ref)
+
+
+@pytest.mark.parametrize("T", [1, 2])
+def test_stack_decode_p3c5(nslm, T):
+    Lyr, E, hidden, inter, P, k = 4, 8, 256, 128, 35, 2
     layers = [synth.moe_layer(l, E, hidden, inter, P, config=948) for l in range(Lyr)]
     logits = torch.stack([synth.router_logits((948, l), T, E) for l in range(Lyr)])
     x, xh = _x((948, T), T, hidden)
