@@ -181,9 +181,10 @@ __global__ void __launch_bounds__(kGemv1Threads) gemv1_kernel(const Gemv1Params 
   // launched with programmatic stream serialization: wait here for the
   // preceding kernel (its writes of W or x; with EARLY only of x), then let
   // the next one launch
-  if (EARLY) {
+  if (EARLY) {  // the stream tables come from constant data: built before the wait too
     if (tid < ntask) fetch(tid, 0);
     cp_async_commit();
+    for (int i = tid; i < 512; i += nthr) tab->t[i] = kStreamTab.t[i];
   }
   asm volatile("griddepcontrol.wait;" ::: "memory");
   asm volatile("griddepcontrol.launch_dependents;");
@@ -196,7 +197,8 @@ __global__ void __launch_bounds__(kGemv1Threads) gemv1_kernel(const Gemv1Params 
     const uint4 *xrow = reinterpret_cast<const uint4 *>(p.x);
     uint4 xv = make_uint4(0, 0, 0, 0);
     if (tid < nb) xv = __ldg(xrow + tid);
-    for (int i = tid; i < 512; i += nthr) tab->t[i] = kStreamTab.t[i];
+    if (!EARLY)
+      for (int i = tid; i < 512; i += nthr) tab->t[i] = kStreamTab.t[i];
     for (int b = tid; b < nb; b += nthr) {
       if (b != tid) xv = __ldg(xrow + b);
       float4 lo, hi;
