@@ -709,7 +709,8 @@ def search_leg(torch, nslm, dev, with_cpu: bool):
 
 def profile_workload(kind: str, reps: int):
     """A small fixed workload for ncu captures (no timing, no JSON): `reps`
-    calls of one decode layer (T=1 or T=8, P=4), of one batched layer (T=512, P=3),
+    calls of one decode layer (T=1 or T=8, P=4; T=1 in the 5-bit format), of
+    one batched layer (T=512, P=3),
     of one seed GEMV (2048 x 4096, P=4) or of the seed search of a 16 x 256
     fp32 matrix over all seeds."""
     import torch
@@ -733,7 +734,7 @@ def profile_workload(kind: str, reps: int):
             nslm.nslm_seed_gemv(nslm.matrix(m), x, 1, y)
         torch.cuda.synchronize()
         return
-    T, Pv, cfg = {"layer": (1, 4, 2), "layer8": (8, 4, 2)}.get(kind, (512, 3, 3))
+    T, Pv, cfg = {"layer": (1, 4, 2), "layer8": (8, 4, 2), "layer_p3c5": (1, nslm.NSLM_P3C5, 2)}.get(kind, (512, 3, 3))
     L = synth.moe_layer(0, E, HIDDEN, INTER, Pv, device=dev, config=cfg)
     logits = synth.router_logits((cfg, T), T, E).to(dev)
     ids = torch.empty(T, K_TOP, dtype=torch.int32, device=dev)
@@ -764,7 +765,7 @@ def main():
     ap.add_argument("--no-batch8", action="store_true", help="skip the 8-token stack leg")
     ap.add_argument("--no-host-experts", action="store_true", help="skip the host-memory expert cache leg")
     ap.add_argument("--no-p3c5", action="store_true", help="skip the 5-bit P=3 stack leg")
-    ap.add_argument("--profile", choices=["layer", "layer8", "batched", "gemv", "search"],
+    ap.add_argument("--profile", choices=["layer", "layer8", "layer_p3c5", "batched", "gemv", "search"],
                     help="run a small fixed workload for an ncu capture and exit")
     args = ap.parse_args()
     if args.profile:
