@@ -39,6 +39,19 @@ import threading
 import time
 
 ROOT = os.path.dirname(os.path.abspath(__file__))
+
+# the sources the one-token decode kernel is compiled from: a traffic figure
+# recorded under profiles/ is used only while their digest is unchanged
+KERNEL_SOURCES = ("stack1.cu", "stack1.cuh", "chunk.cuh", "regen.cuh", "persist.cuh", "common.cuh", "moe.cuh")
+
+
+def kernel_sources_sha256() -> str:
+    import hashlib
+    h = hashlib.sha256()
+    for name in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, "lfsr_seeded_moe_b200", "csrc", name), "rb") as f:
+            h.update(name.encode() + b"\0" + f.read())
+    return h.hexdigest()
 if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
@@ -875,12 +888,17 @@ def main():
     traffic = None
     tr_path = os.path.join(ROOT, "profiles", "ffn_decode_layer_traffic.txt")
     if os.path.exists(tr_path) and T == 1:
+        rec = {}
         for ln in open(tr_path):
-            if ln.startswith("dram_bytes_per_layer_call:"):
-                try:  # one layer's DRAM bytes (ncu), scaled to the launch's 45 layers
-                    traffic = int(ln.split(":")[1].split()[0]) * LAYERS
-                except ValueError:
-                    traffic = None
+            if ":" in ln and not ln.startswith("#"):
+                key, val = ln.split(":", 1)
+                rec[key.strip()] = val.split()[0] if val.split() else ""
+        # the counters hold only for the kernel source they were taken on
+        if rec.get("kernel_sources_sha256") == kernel_sources_sha256():
+            try:  # one layer's DRAM bytes (ncu), scaled to the launch's 45 layers
+                traffic = int(rec["dram_bytes_per_layer_call"]) * LAYERS
+            except (KeyError, ValueError):
+                traffic = None
     # one layer through nslm_moe_seed_ffn (routing plan + the persistent
     # kernel for one layer), for context: per-call overheads included
     nslm.nslm_moe_route_topk(logits[0][0], T, E, K_TOP, ids, wts)

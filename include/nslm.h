@@ -327,8 +327,13 @@ int32_t nslm_pack_nibbles(const nslm_seed_matrix *in, uint8_t *nibbles, nslm_str
  * out[2] = 1.  out[4] = 1 if the wait passed, 0 if it gave up.
  * kind 1 / 2: the mbarrier wait of the tensor-core pipeline on a barrier
  * whose phase nothing completes (1) or that one arrival completed first (2);
- * out[0] = 1 if it passed, 0 if it gave up.  cycles: the wait limit in SM
- * clocks (> 0).  out: device, 5 int32.  One launch of one CTA. */
+ * out[0] = 1 if it passed, 0 if it gave up.  kind 3: the wait of the
+ * one-token stack on a tagged 64-bit word (fp32 bits low, layer tag high),
+ * here the word at out[6..7] (caller-initialised, out 8-byte aligned) waited
+ * on for tag 1, with out[0..3] as the status words of kind 0; out[4] = 1 if it
+ * passed, 0 if it gave up (then out[0] = 1, out[2] = 1); out[5] = the value
+ * bits it saw.  cycles: the wait limit in SM clocks (> 0).  out: device, 5
+ * int32 (8 for kind 3).  One launch of one CTA. */
 int32_t nslm_debug_wait_probe(int32_t kind, int32_t *out, int64_t cycles, nslm_stream_t stream);
 
 /* Test export: the bf16 hidden activations h = SiLU(gate x) * (up x) that the

@@ -364,7 +364,8 @@ int32_t nslm_moe_route_topk(const float *logits, int32_t T, int32_t E, int32_t k
   for (int t0 = 0; t0 < T; t0 += kMaxT) {
     const int tn = std::min(kMaxT, T - t0);
     st = launch_route_plan(logits + (size_t)t0 * E, nullptr, nullptr, tn, E, k, 1, nullptr,
-                           ids + (size_t)t0 * k, w + (size_t)t0 * k, nullptr, 0, nullptr, tn, s);
+                           ids + (size_t)t0 * k, w + (size_t)t0 * k, nullptr, 0, nullptr, tn, nullptr, 0,
+                           s);
     if (st) return st;
     ++g_launches;
   }
@@ -397,7 +398,7 @@ int32_t nslm_moe_seed_ffn(const nslm_seed_matrix *gate, const nslm_seed_matrix *
   }
   const FfnWorkspace fw = ffn_workspace(reinterpret_cast<char *>(ws), T, k, d.hidden, d.inter, 1);
   if ((st = launch_route_plan(nullptr, ids, w, T, E, k, 1, fw.plans, nullptr, nullptr, fw.counters,
-                              d.hidden, fw.sync, decode_slot_cap(d, T, k), s)))
+                              d.hidden, fw.sync, decode_slot_cap(d, T, k), nullptr, 0, s)))
     return st;
   int launches = 1;
   const nslm_moe_layer layer{*gate, *up, *down};
@@ -428,7 +429,8 @@ int32_t nslm_moe_stack_decode(const nslm_moe_layer *layers, int32_t L, int32_t E
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   const FfnWorkspace fw = ffn_workspace(reinterpret_cast<char *>(ws), T, k, d.hidden, d.inter, L);
   if ((st = launch_route_plan(logits, nullptr, nullptr, T, E, k, L, fw.plans, nullptr, nullptr,
-                              fw.counters, d.hidden, fw.sync, decode_slot_cap(d, T, k), s)))
+                              fw.counters, d.hidden, fw.sync, decode_slot_cap(d, T, k),
+                              T == 1 && L > 1 ? fw.ytag : nullptr, fw.n_ytag, s)))
     return st;
   int launches = 1;
   st = launch_decode_stack(d, layers, L, x0_bf16, T, k, fw, y, s, launches);

@@ -77,10 +77,12 @@ __global__ void __launch_bounds__(256) route_plan_kernel(const float *__restrict
                                                          int E, int k, SlotPlan *plans,
                                                          int32_t *ids_out, float *w_out,
                                                          int32_t *counters, int n_counters,
-                                                         int32_t *sync, int slot_cap) {
+                                                         int32_t *sync, int slot_cap,
+                                                         uint64_t *tags, int n_tags) {
   const int layer = blockIdx.x;
   if (counters && layer == 0)
     for (int i = threadIdx.x; i < n_counters; i += blockDim.x) counters[i] = 0;
+  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < n_tags; i += gridDim.x * blockDim.x) tags[i] = 0;
   if (sync && layer == 0 && threadIdx.x < kSyncWords) sync[threadIdx.x] = 0;
   __shared__ int32_t s_ids[kMaxPairs];
   __shared__ float s_w[kMaxPairs];
@@ -450,6 +452,9 @@ FfnWorkspace ffn_workspace(char *base, int T, int k, int hidden, int inter, int 
   off += round256((size_t)kSlotGroups * T * hidden * sizeof(float));
   w.y_mid = reinterpret_cast<float *>(base ? base + off : nullptr);
   off += round256((size_t)T * hidden * sizeof(float));
+  w.ytag = reinterpret_cast<uint64_t *>(base ? base + off : nullptr);
+  w.n_ytag = hidden + kMaxNormParts;
+  off += round256((size_t)w.n_ytag * sizeof(uint64_t));
   w.bytes = off;
   return w;
 }
@@ -534,9 +539,11 @@ int32_t launch_decode_layer(const FfnDims &d, const nslm_seed_matrix *gate,
 
 int32_t launch_route_plan(const float *logits, const int32_t *ids, const float *w, int T, int E,
                           int k, int L, SlotPlan *plans, int32_t *ids_out, float *w_out,
-                          int32_t *counters, int n_counters, int32_t *sync, int slot_cap, cudaStream_t s) {
+                          int32_t *counters, int n_counters, int32_t *sync, int slot_cap,
+                          uint64_t *tags, int n_tags, cudaStream_t s) {
   route_plan_kernel<<<L, 256, 0, s>>>(logits, ids, w, T, E, k, plans, ids_out, w_out, counters,
-                                      n_counters, sync, std::max(1, std::min(slot_cap, T)));
+                                      n_counters, sync, std::max(1, std::min(slot_cap, T)), tags,
+                                      tags ? n_tags : 0);
   return launch_status();
 }
 

@@ -52,6 +52,12 @@ struct FfnWorkspace {
   float *h;            // [T*k][inter]
   float *y_part;       // [slot groups][T][hidden]
   float *y_mid;        // [T][hidden] (layer stack)
+  // one-token layer stack: y rows, then the per-CTA norm partials, between
+  // layers as 64-bit words (value bits low, 32-bit layer tag high), zeroed
+  // by the routing kernel at the start of every one-token call of two or
+  // more layers (a one-layer call does not read them)
+  uint64_t *ytag;      // [hidden + kMaxNormParts]
+  int32_t n_ytag;
   size_t bytes;
 };
 FfnWorkspace ffn_workspace(char *base, int T, int k, int hidden, int inter, int L);
@@ -62,7 +68,8 @@ size_t hybrid_extra_bytes(int T, int k, int hidden);
 
 int32_t launch_route_plan(const float *logits, const int32_t *ids, const float *w, int T, int E,
                           int k, int L, SlotPlan *plans, int32_t *ids_out, float *w_out,
-                          int32_t *counters, int n_counters, int32_t *sync, int slot_cap, cudaStream_t s);
+                          int32_t *counters, int n_counters, int32_t *sync, int slot_cap,
+                          uint64_t *tags, int n_tags, cudaStream_t s);
 int32_t launch_decode_layer(const FfnDims &d, const nslm_seed_matrix *gate,
                             const nslm_seed_matrix *up, const nslm_seed_matrix *down,
                             const SlotPlan *plan, const uint16_t *x_bf16, const float *y_prev,

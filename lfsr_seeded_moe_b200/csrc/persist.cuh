@@ -67,4 +67,44 @@ static __device__ bool grid_wait(int32_t *sync, uint32_t target, int *s_ok,
   return *s_ok != 0;
 }
 
+// Values handed from one layer to the next as 64-bit words: the fp32 bits in
+// the low half, the tag of the layer that wrote them in the high half.  An
+// aligned 64-bit access is single-copy atomic, so a reader that sees the tag
+// it expects also sees the value stored with it: no fence, flag or barrier
+// is needed between the writer and the reader of one word.
+__device__ __forceinline__ void st_tagged(uint64_t *p, float v, uint32_t tag) {
+  const uint64_t w = ((uint64_t)tag << 32) | __float_as_uint(v);
+  asm volatile("st.relaxed.gpu.global.b64 [%0], %1;" ::"l"(p), "l"(w) : "memory");
+}
+__device__ __forceinline__ uint64_t ld_tagged(const uint64_t *p) {
+  uint64_t w;
+  asm volatile("ld.relaxed.gpu.global.b64 %0, [%1];" : "=l"(w) : "l"(p) : "memory");
+  return w;
+}
+__device__ __forceinline__ void ld_tagged2(const uint64_t *p, uint64_t &a, uint64_t &b) {
+  asm volatile("ld.relaxed.gpu.global.v2.b64 {%0, %1}, [%2];" : "=l"(a), "=l"(b) : "l"(p) : "memory");
+}
+__device__ __forceinline__ bool has_tag(uint64_t w, uint32_t tag) { return (uint32_t)(w >> 32) == tag; }
+__device__ __forceinline__ float tagged_value(uint64_t w) { return __uint_as_float((uint32_t)w); }
+
+// Call `ready()` (which reloads what it checks) until it returns true.  Gives
+// up, returning false, when another CTA has raised the abort flag or after
+// max_cycles, raising the flag and recording status 1 itself, as grid_wait.
+template <class F>
+__device__ bool poll_bounded(int32_t *sync, F &&ready, long long max_cycles = kBarrierWaitCycles) {
+  if (ready()) return true;
+  const long long t0 = clock64();
+  for (uint32_t it = 1;; ++it) {
+    if (ready()) return true;
+    if ((it & 63) == 0) {
+      if (ld_acquire(sync + 2) != 0) return false;
+      if (clock64() - t0 > max_cycles) {
+        atomicExch(sync + 2, 1);
+        atomicCAS(sync, 0, 1);
+        return false;
+      }
+    }
+  }
+}
+
 }  // namespace nslm

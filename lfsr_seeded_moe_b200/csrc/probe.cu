@@ -19,6 +19,25 @@ __global__ void grid_wait_probe_kernel(int32_t *out, long long cycles) {
   if (threadIdx.x == 0) out[4] = ok ? 1 : 0;
 }
 
+// The tagged-word wait of the one-token stack on the 64-bit word at out[6..7]
+// (value bits, tag), waiting for tag 1 with out[0..3] as the sync words;
+// out[4] = 1 if the wait succeeded, 0 if it gave up; out[5] = the value bits
+// it saw.
+__global__ void tag_wait_probe_kernel(int32_t *out, long long cycles) {
+  if (threadIdx.x != 0) return;
+  const uint64_t *word = reinterpret_cast<const uint64_t *>(out + 6);
+  uint64_t w = 0;
+  const bool ok = poll_bounded(
+      out,
+      [&] {
+        w = ld_tagged(word);
+        return has_tag(w, 1u);
+      },
+      cycles);
+  out[4] = ok ? 1 : 0;
+  out[5] = (int32_t)(uint32_t)w;
+}
+
 // out[0] = 1 if the mbarrier wait succeeded, 0 if it gave up; `arrive` = 1
 // completes the barrier's phase before the wait.
 __global__ void mbar_wait_probe_kernel(int32_t *out, long long cycles, int arrive) {
@@ -57,11 +76,13 @@ using namespace nslm;
 
 extern "C" int32_t nslm_debug_wait_probe(int32_t kind, int32_t *out, int64_t cycles, nslm_stream_t stream) {
   g_launches = 0;
-  if (!out || cycles <= 0 || (kind != 0 && kind != 1 && kind != 2)) return NSLM_ERR_ARG;
+  if (!out || cycles <= 0 || kind < 0 || kind > 3) return NSLM_ERR_ARG;
+  if (kind == 3 && reinterpret_cast<uintptr_t>(out) % 8) return NSLM_ERR_ALIGN;
   int32_t st = check_device();
   if (st) return st;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   if (kind == 0) grid_wait_probe_kernel<<<1, 32, 0, s>>>(out, (long long)cycles);
+  else if (kind == 3) tag_wait_probe_kernel<<<1, 32, 0, s>>>(out, (long long)cycles);
   else mbar_wait_probe_kernel<<<1, 32, 0, s>>>(out, (long long)cycles, kind == 2 ? 1 : 0);
   st = launch_status();
   if (st == NSLM_OK) g_launches = 1;

@@ -5,9 +5,10 @@
 // projections, SiLU, a down projection, and the routing-weighted sum.  The
 // weights are regenerated in registers ("What I changed: September 2026").
 //
-// One launch runs all layers.  Each CTA (one per SM, 26 warps) keeps its
-// stream tables for the whole stack and alternates two phases, separated by
-// grid barriers (the launch is cooperative, so every CTA is resident):
+// One launch runs all layers.  Each CTA (one per SM, up to 20 warps) keeps
+// its stream tables and every layer's routing plan for the whole stack and
+// alternates two phases (the launch is cooperative, so every CTA is
+// resident):
 //
 //   A (gate/up)  every CTA stages the layer input x (layer 0: the bf16 token;
 //                later layers: bf16(y / rms(y)) of the previous layer's fp32
@@ -19,11 +20,19 @@
 //                tasks, partials go to shared memory and one warp per row adds
 //                them in a fixed order (deterministic, no atomics on data).
 //
+// A grid barrier separates A from B: every CTA needs all of h.  From B to the
+// next layer's A there is no barrier: each y row, and each CTA's sum of y^2
+// over its rows, is stored as a 64-bit word tagged with the layer, and the
+// next layer's staging polls exactly the words it reads until their tags
+// match.  (A CTA cannot overwrite h before every CTA has read it: it starts
+// the next phase A only after reading every CTA's y, which each CTA writes
+// after staging h.)
+//
 // Weight fields are copied with cp.async into per-thread shared-memory slots
 // one task ahead, and the first task of the next phase is fetched before the
-// barrier, so barrier latency overlaps the first loads.  Every barrier wait
-// is bounded: a CTA that gives up raises the abort flag (all others stop at
-// their next wait) and records status 1 in the workspace.
+// wait, so the wait overlaps the first loads.  Every wait is bounded: a CTA
+// that gives up raises the abort flag (all others stop at their next wait)
+// and records status 1 in the workspace.
 #include <algorithm>
 
 #include "chunk.cuh"
@@ -43,14 +52,13 @@ struct LayerMats {
 
 struct Stack1Params {
   const SlotPlan *plans;  // [n] this launch's layers
-  const uint16_t *x0;     // bf16 [hidden]: input of the first layer, or null
-  const float *y_in;      // fp32 [hidden]: the previous layer's output when x0 is null
+  const uint16_t *x0;     // bf16 [hidden]: input of layer 0 (the first launch), else null
   float *h;               // [k][inter] by pair
-  float *y_mid;           // [hidden] fp32 between layers
-  float *y_out;           // [hidden] output of the last layer
+  uint64_t *ytag;         // [hidden] y rows, then [grid] sums of y^2, tagged (zeroed per call)
+  float *y_out;           // [hidden] output of the last layer if this launch ends the stack, else null
   int32_t *sync;          // status, barrier arrivals, abort
-  float *rms_part;        // [grid] sums of y^2 over each CTA's rows, written with y
   uint32_t barrier_base;  // arrivals recorded by earlier launches of the same call
+  uint32_t l0;            // index in the stack of this launch's first layer
   int32_t n, hidden, inter;
   int32_t h_rows;         // rows of h (the routed pairs; bounds checks)
   int32_t Ch, Ci;         // 64-weight chunks per row of gate/up (hidden) and down (inter)
@@ -66,36 +74,71 @@ __device__ __forceinline__ bool stack_wait(const Stack1Params &p, uint32_t e, in
   return grid_wait(p.sync, p.barrier_base + (e + 1) * gridDim.x, s_ok);
 }
 
-// Stage x = bf16(y / sqrt(mean(y^2) + 1e-6)) chunk-major.  The sum of squares
-// is the fixed-order sum of the per-CTA partials that were written with y.
-__device__ void stage_norm_y(float4 *xs4, float2 *xn2, const float *y, const float *part, int G, int K,
-                             float *scratch) {
+// Stage x = bf16(y / sqrt(mean(y^2) + 1e-6)) chunk-major from the tagged y
+// rows and per-CTA sums of squares of layer `tag` - 1, polling each word until
+// it carries `tag`.  The sum of squares is the fixed-order sum of the G
+// partials.  The last warp polls the partials while the others poll their
+// first block of 8 rows.  False if a wait gave up.
+__device__ bool stage_norm_tagged(float4 *xs4, float2 *xn2, const uint64_t *ytag, uint32_t tag, int G, int K,
+                                  int32_t *sync, float *scratch) {
   const int tid = threadIdx.x, nthr = blockDim.x, nb = K >> 3;
-  const float4 *row = reinterpret_cast<const float4 *>(y);
-  float4 lo = make_float4(0.f, 0.f, 0.f, 0.f), hi = lo;
-  if (tid < nb) {  // the first block of this thread, in flight during the sum
-    lo = __ldcg(row + 2 * tid);
-    hi = __ldcg(row + 2 * tid + 1);
-  }
-  if (tid < 32) {
+  bool ok = true;
+  uint64_t w[8];
+  auto poll_block = [&](int b) {
+    return poll_bounded(sync, [&] {
+      const uint64_t *src = ytag + 8 * b;
+#pragma unroll
+      for (int j = 0; j < 8; j += 2) ld_tagged2(src + j, w[j], w[j + 1]);
+      bool all = true;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) all &= has_tag(w[j], tag);
+      return all;
+    });
+  };
+  if (tid < nb) ok &= poll_block(tid);  // the first block of this thread
+  if (tid >= nthr - 32) {
+    const int lane = tid & 31;
+    // the first 256 partials with all loads in flight, then any others; the
+    // per-lane order of the additions is that of one strided loop
+    float v[8];
+    ok &= poll_bounded(sync, [&] {
+      bool all = true;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        v[j] = 0.f;
+        if (lane + 32 * j < G) {
+          const uint64_t u = ld_tagged(ytag + K + lane + 32 * j);
+          all &= has_tag(u, tag);
+          v[j] = tagged_value(u);
+        }
+      }
+      return all;
+    });
     float ss = 0.f;
-    for (int i = tid; i < G; i += 32) ss += __ldcg(part + i);
+#pragma unroll
+    for (int j = 0; j < 8; ++j) ss += v[j];
+    for (int i = lane + 256; i < G; i += 32) {
+      uint64_t u = 0;
+      ok &= poll_bounded(sync, [&] {
+        u = ld_tagged(ytag + K + i);
+        return has_tag(u, tag);
+      });
+      ss += tagged_value(u);
+    }
     ss = warp_sum(ss);
-    if (tid == 0) scratch[32] = sqrtf(ss / (float)K + 1e-6f);
+    if (lane == 0) scratch[32] = sqrtf(ss / (float)K + 1e-6f);
   }
   __syncthreads();
   const float r = scratch[32];
   for (int b = tid; b < nb; b += nthr) {
-    if (b != tid) {
-      lo = __ldcg(row + 2 * b);
-      hi = __ldcg(row + 2 * b + 1);
-    }
-#define NSLM_NORM(v) __bfloat162float(__float2bfloat16_rn(__fdiv_rn((v), r)))
-    const float4 a = make_float4(NSLM_NORM(lo.x), NSLM_NORM(lo.y), NSLM_NORM(lo.z), NSLM_NORM(lo.w));
-    const float4 c = make_float4(NSLM_NORM(hi.x), NSLM_NORM(hi.y), NSLM_NORM(hi.z), NSLM_NORM(hi.w));
+    if (b != tid) ok &= poll_block(b);
+#define NSLM_NORM(u) __bfloat162float(__float2bfloat16_rn(__fdiv_rn(tagged_value(u), r)))
+    const float4 a = make_float4(NSLM_NORM(w[0]), NSLM_NORM(w[1]), NSLM_NORM(w[2]), NSLM_NORM(w[3]));
+    const float4 c = make_float4(NSLM_NORM(w[4]), NSLM_NORM(w[5]), NSLM_NORM(w[6]), NSLM_NORM(w[7]));
 #undef NSLM_NORM
     cm_store_block(xs4, xn2, b, a, c);
   }
+  return ok;
 }
 
 template <int P, bool VEC>
@@ -112,13 +155,12 @@ __global__ void __launch_bounds__(kStack1MaxThreads, 1) stack1_kernel(const __gr
   const FieldSlots fs(xn2 + (size_t)kCmXn * p.stage_slots + (p.stage_slots & 1), 4 * nthr);
   float *red = reinterpret_cast<float *>(fs.b + 4 * nthr);  // phase B partials
   __shared__ float scratch[33];
-  __shared__ int s_row0, s_ok, s_nslots;
+  __shared__ int s_ok, s_nslots;
   __shared__ int s_expert[kMaxK], s_pair[kMaxK];
   __shared__ float s_w[kMaxK];
-  __shared__ int s_next_expert[kMaxK], s_next_nslots;  // the next layer's plan, for its prefetch
-
-  build_stream_tables_rep<kTabCopies>(tab);
-  if (tid == 0) s_row0 = 0;
+  // every layer's routed slots (expert, pair, weight), read once at the start
+  __shared__ int s_pl_n[kMaxFusedLayers], s_pl_expert[kMaxFusedLayers][kMaxK], s_pl_pair[kMaxFusedLayers][kMaxK];
+  __shared__ float s_pl_w[kMaxFusedLayers][kMaxK];
 
   const int nbh = p.hidden >> 3, nbi = p.inter >> 3;
   // phase A warp number: consecutive tasks go to different CTAs, so every SM
@@ -197,33 +239,48 @@ __global__ void __launch_bounds__(kStack1MaxThreads, 1) stack1_kernel(const __gr
   uint32_t kg = 0, ku = 0, kd = 0;
   uint32_t nbar = 0;  // barriers passed in this launch
 
-  // first fields of layer 0, phase A
+  // first fields of layer 0, phase A, straight from the plan in global memory
   if (a_steps(min(p.plans->n_slots, kMaxK)) > 0) a_fetch(p.layer[0], p.plans->expert, 0, 0, fg, fu, kg, ku);
   if (VEC) cp_async_commit();
-  __syncthreads();  // tables
+  // the plans, by the highest threads, while the lowest stage layer 0's input
+  for (int i = nthr - 1 - tid; i < p.n * kMaxK; i += nthr) {
+    const int l = i / kMaxK, j = i - l * kMaxK;
+    const SlotPlan *pl = p.plans + l;
+    const int ns = pl->n_slots, st = pl->start[j], ex = pl->expert[j];  // j < kMaxK: in the arrays
+    if (j == 0) s_pl_n[l] = min(ns, kMaxK);
+    if (j < ns) {
+      const int pr = pl->pair[st];
+      s_pl_expert[l][j] = ex;
+      s_pl_pair[l][j] = pr;
+      s_pl_w[l][j] = pl->w[pr];
+    }
+  }
+  if (p.x0) {  // layer 0's input, bf16 -> fp32 chunk-major
+    const uint4 *row = reinterpret_cast<const uint4 *>(p.x0);
+    for (int b = tid; b < nbh; b += nthr) {
+      float4 lo, hi;
+      bf16x8_to_f32(__ldg(row + b), lo, hi);
+      cm_store_block(xs4, xn2, b, lo, hi);
+    }
+  }
+  build_stream_tables_rep<kTabCopies>(tab);
+  __syncthreads();  // tables, plans, layer 0's input
 
   for (int l = 0; l < p.n; ++l) {
     const LayerMats &Lm = p.layer[l];
-    const SlotPlan *pl = p.plans + l;
-    __syncthreads();  // smem plan and staging reuse
-    if (tid < kMaxK && tid < pl->n_slots) {
-      const int pr = pl->pair[pl->start[tid]];
-      s_expert[tid] = pl->expert[tid];
-      s_pair[tid] = pr;
-      s_w[tid] = pl->w[pr];
+    const uint32_t g = p.l0 + (uint32_t)l;  // index of this layer in the stack
+    __syncthreads();  // plan and staging reuse
+    if (tid < s_pl_n[l]) {
+      s_expert[tid] = s_pl_expert[l][tid];
+      s_pair[tid] = s_pl_pair[l][tid];
+      s_w[tid] = s_pl_w[l][tid];
     }
-    if (tid == 0) s_nslots = min(pl->n_slots, kMaxK);
-    if (l + 1 < p.n) {
-      if (tid < kMaxK && tid < pl[1].n_slots) s_next_expert[tid] = pl[1].expert[tid];
-      if (tid == 0) s_next_nslots = min(pl[1].n_slots, kMaxK);
-    }
+    if (tid == 0) s_nslots = s_pl_n[l];
 
     // =========================== phase A: gate/up + SiLU
-    if (l == 0 && p.x0)
-      stage_activations<true>(xs4, xn2, p.x0, nullptr, &s_row0, 1, p.hidden, p.Ch, scratch);
-    else
-      stage_norm_y(xs4, xn2, l == 0 ? p.y_in : p.y_mid, p.rms_part, gridDim.x, p.hidden, scratch);
-    __syncthreads();
+    // layer 0's input was staged at the start
+    const bool staged = g == 0 || stage_norm_tagged(xs4, xn2, p.ytag, g, gridDim.x, p.hidden, p.sync, scratch);
+    if (__syncthreads_or(!staged)) break;
     {
       const int nsteps = a_steps(s_nslots);
       float2 ag = make_float2(0.f, 0.f), au = make_float2(0.f, 0.f);
@@ -313,32 +370,36 @@ __global__ void __launch_bounds__(kStack1MaxThreads, 1) stack1_kernel(const __gr
         red[t] = s_w[s] * (acc.x + acc.y);
       }
       __syncthreads();
-      float *yl = (l == p.n - 1) ? p.y_out : p.y_mid;
+      // the stack's output in plain fp32; between layers tagged words
+      const bool last = l == p.n - 1 && p.y_out;
       float *rowy = red + p.rpc * p.stage_slots;  // this CTA's outputs, for the norm partial
       for (int r = warp; r < nrows; r += nwarps) {
         float sum = 0.f;
         for (int q = lane; q < SC; q += 32) sum += red[r * SC + q];
         sum = warp_sum(sum);
         if (lane == 0) {
-          __stcg(yl + n0 + r, sum);
+          if (last)
+            __stcg(p.y_out + n0 + r, sum);
+          else
+            st_tagged(p.ytag + n0 + r, sum, g + 1);
           rowy[r] = sum;
         }
       }
-      __syncthreads();
-      if (warp == 0) {  // sum of squares of this CTA's rows, fixed order
-        float ss = 0.f;
-        for (int r = lane; r < nrows; r += 32) ss = fmaf(rowy[r], rowy[r], ss);
-        ss = warp_sum(ss);
-        if (lane == 0) __stcg(p.rms_part + blockIdx.x, ss);
+      if (!last) {
+        __syncthreads();
+        if (warp == 0) {  // sum of squares of this CTA's rows, fixed order
+          float ss = 0.f;
+          for (int r = lane; r < nrows; r += 32) ss = fmaf(rowy[r], rowy[r], ss);
+          ss = warp_sum(ss);
+          if (lane == 0) st_tagged(p.ytag + p.hidden + blockIdx.x, ss, g + 1);
+        }
       }
     }
     if (l + 1 == p.n) break;
-    // arrive; fetch the next layer's first phase A fields while the others arrive
-    grid_arrive(p.sync);
+    // the next layer's first phase A fields, in flight while its input arrives
     if (VEC) cp_async_wait<0>();
-    if (a_steps(s_next_nslots) > 0) a_fetch(p.layer[l + 1], s_next_expert, 0, 0, fg, fu, kg, ku);
+    if (a_steps(s_pl_n[l + 1]) > 0) a_fetch(p.layer[l + 1], s_pl_expert[l + 1], 0, 0, fg, fu, kg, ku);
     if (VEC) cp_async_commit();
-    if (!stack_wait(p, nbar++, &s_ok)) break;
   }
   if (VEC) cp_async_wait<0>();
 }
@@ -393,14 +454,15 @@ bool stack1_supported(const FfnDims &d, int k) {
   if (d.inter >= (1 << 16) || d.hidden >= (1 << 16)) return false;
   if ((int64_t)k * ceil_div(d.inter / 8, 8) >= (1 << 16)) return false;
   if ((int64_t)k * d.inter * ceil_div(d.hidden / 64, 32) >= (1 << 22)) return false;
-  return stack1_smem(d, k, stack1_threads(d, k)) <= 224 * 1024;
+  // dynamic shared memory plus ~7 KB of static (the per-layer plans) within 227 KB
+  return stack1_smem(d, k, stack1_threads(d, k)) <= 220 * 1024;
 }
 
 template <int P, bool VEC>
 static int32_t launch_stack1_t(const FfnDims &d, const nslm_moe_layer *layers, int n,
-                               const SlotPlan *plans, const uint16_t *x0, const float *y_in, int k,
-                               float *h, float *y_mid, float *y_out, int32_t *sync, float *rms_part,
-                               cudaStream_t s, int &launches) {
+                               const SlotPlan *plans, const uint16_t *x0, int k, float *h,
+                               uint64_t *ytag, float *y_out, int32_t *sync, cudaStream_t s,
+                               int &launches) {
   const int threads = stack1_threads(d, k);
   const size_t smem = stack1_smem(d, k, threads);
   auto kern = stack1_kernel<P, VEC>;
@@ -411,9 +473,8 @@ static int32_t launch_stack1_t(const FfnDims &d, const nslm_moe_layer *layers, i
   Stack1Params p{};
   p.h = h;
   p.h_rows = k;
-  p.y_mid = y_mid;
+  p.ytag = ytag;
   p.sync = sync;
-  p.rms_part = rms_part;
   p.hidden = d.hidden;
   p.inter = d.inter;
   p.Ch = ceil_div(d.hidden / 8, 8);
@@ -434,9 +495,9 @@ static int32_t launch_stack1_t(const FfnDims &d, const nslm_moe_layer *layers, i
     const int m = std::min(kMaxFusedLayers, n - l0);
     p.plans = plans + l0;
     p.x0 = l0 == 0 ? x0 : nullptr;
-    p.y_in = l0 == 0 ? y_in : y_mid;
-    p.y_out = (l0 + m == n) ? y_out : y_mid;
+    p.y_out = (l0 + m == n) ? y_out : nullptr;
     p.n = m;
+    p.l0 = (uint32_t)l0;
     p.barrier_base = base;
     for (int i = 0; i < m; ++i)
       p.layer[i] = LayerMats{layers[l0 + i].gate, layers[l0 + i].up, layers[l0 + i].down};
@@ -453,22 +514,23 @@ static int32_t launch_stack1_t(const FfnDims &d, const nslm_moe_layer *layers, i
     ensure_stream_source(s);
     if ((st = cuda_status(cudaLaunchKernelEx(&cfg, kern, p)))) return st;
     ++launches;
-    base += (uint32_t)(2 * m - 1) * (uint32_t)grid;
+    base += (uint32_t)m * (uint32_t)grid;  // one grid barrier per layer
   }
   return NSLM_OK;
 }
 
 int32_t launch_stack1(const FfnDims &d, const nslm_moe_layer *layers, int n, const SlotPlan *plans,
-                      const uint16_t *x0, const float *y_in, int k, float *h, float *y_mid,
-                      float *y_out, int32_t *sync, float *rms_part, cudaStream_t s, int &launches) {
+                      const uint16_t *x0, int k, float *h, uint64_t *ytag, float *y_out, int32_t *sync,
+                      cudaStream_t s, int &launches) {
+  if (!x0 || !ytag) return NSLM_ERR_ARG;
   const bool vec = d.hidden % 64 == 0 && d.inter % 64 == 0;
   if (d.P == kP3C5)  // K % 64 == 0 for both projections: whole chunks always
-    return launch_stack1_t<kP3C5, true>(d, layers, n, plans, x0, y_in, k, h, y_mid, y_out, sync, rms_part, s, launches);
+    return launch_stack1_t<kP3C5, true>(d, layers, n, plans, x0, k, h, ytag, y_out, sync, s, launches);
   if (d.P == 4)
-    return vec ? launch_stack1_t<4, true>(d, layers, n, plans, x0, y_in, k, h, y_mid, y_out, sync, rms_part, s, launches)
-               : launch_stack1_t<4, false>(d, layers, n, plans, x0, y_in, k, h, y_mid, y_out, sync, rms_part, s, launches);
-  return vec ? launch_stack1_t<3, true>(d, layers, n, plans, x0, y_in, k, h, y_mid, y_out, sync, rms_part, s, launches)
-             : launch_stack1_t<3, false>(d, layers, n, plans, x0, y_in, k, h, y_mid, y_out, sync, rms_part, s, launches);
+    return vec ? launch_stack1_t<4, true>(d, layers, n, plans, x0, k, h, ytag, y_out, sync, s, launches)
+               : launch_stack1_t<4, false>(d, layers, n, plans, x0, k, h, ytag, y_out, sync, s, launches);
+  return vec ? launch_stack1_t<3, true>(d, layers, n, plans, x0, k, h, ytag, y_out, sync, s, launches)
+             : launch_stack1_t<3, false>(d, layers, n, plans, x0, k, h, ytag, y_out, sync, s, launches);
 }
 
 NSLM_BOUNDS_ACCESSOR(stack1)

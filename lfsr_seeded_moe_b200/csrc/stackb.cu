@@ -623,8 +623,7 @@ int decode_slot_cap(const FfnDims &d, int T, int k) {
 int32_t launch_decode_stack(const FfnDims &d, const nslm_moe_layer *layers, int L, const uint16_t *x0,
                             int T, int k, const FfnWorkspace &fw, float *y, cudaStream_t s, int &launches) {
   if (T == 1 && stack1_supported(d, k))
-    return launch_stack1(d, layers, L, fw.plans, x0, nullptr, k, fw.h, fw.y_mid, y, fw.sync, fw.rms_part, s,
-                         launches);
+    return launch_stack1(d, layers, L, fw.plans, x0, k, fw.h, fw.ytag, y, fw.sync, s, launches);
   if (T > 1 && stackb_supported(d, T, k))
     return launch_stackb(d, layers, L, fw.plans, x0, nullptr, T, k, fw.h, fw.y_mid, y, fw.sync, fw.rms_part,
                          s, launches);

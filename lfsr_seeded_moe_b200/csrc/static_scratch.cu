@@ -84,7 +84,7 @@ extern "C" int32_t nslm_moe_seed_ffn_static(const nslm_seed_matrix *gate, const 
   // counters on every call, so whatever an earlier call left in the array is
   // harmless; h and the partial sums are written before they are read.
   if ((st = launch_route_plan(nullptr, ids, w, T, E, k, 1, fw.plans, nullptr, nullptr, fw.counters,
-                              d.hidden, fw.sync, decode_slot_cap(d, T, k), s)))
+                              d.hidden, fw.sync, decode_slot_cap(d, T, k), nullptr, 0, s)))
     return st;
   int launches = 1;
   const nslm_moe_layer layer{*gate, *up, *down};

@@ -172,7 +172,9 @@ def test_wait_probe_argument_checks():
     f = nslm.raw().nslm_debug_wait_probe
     assert f(0, 0, 1000, 0) == nslm.NSLM_ERR_ARG          # no output buffer
     assert f(0, 0x9000000, 0, 0) == nslm.NSLM_ERR_ARG     # no limit
-    assert f(3, 0x9000000, 1000, 0) == nslm.NSLM_ERR_ARG  # unknown kind
+    assert f(4, 0x9000000, 1000, 0) == nslm.NSLM_ERR_ARG  # unknown kind
+    assert f(-1, 0x9000000, 1000, 0) == nslm.NSLM_ERR_ARG
+    assert f(3, 0x9000004, 1000, 0) == nslm.NSLM_ERR_ALIGN  # the tagged word must be 8-byte aligned
 
 
 def test_hybrid_argument_checks():

@@ -77,3 +77,40 @@ def test_mbarrier_wait_gives_up_and_passes(nslm):
     torch.cuda.synchronize()
     assert int(out[0].item()) == 1
     _gemv_still_works(nslm)
+
+
+def _tag_words(tag, value_bits, abort=0):
+    # status, arrivals, abort, spare, passed, seen, then one 64-bit word
+    # (value bits, tag) at out[6..7]
+    return torch.tensor([0, 0, abort, 0, 7, 7, value_bits, tag], dtype=torch.int32, device="cuda")
+
+
+def test_tagged_word_wait_gives_up_and_reports(nslm):
+    out = _tag_words(0, 12345)  # the tag the wait expects (1) never arrives
+    t0 = time.time()
+    nslm.nslm_debug_wait_probe(3, out, LIMIT)
+    torch.cuda.synchronize()
+    assert time.time() - t0 < 5.0
+    got = out.cpu().tolist()
+    assert got[:5] == [1, 0, 1, 0, 0]  # status 1, abort raised, the wait returned false
+    assert nslm.nslm_device_status(out) == nslm.NSLM_ERR_TIMEOUT
+    _gemv_still_works(nslm)
+
+
+def test_tagged_word_wait_passes_and_sees_the_value(nslm):
+    bits = int(np.float32(-2.5).view(np.int32))
+    out = _tag_words(1, bits)
+    nslm.nslm_debug_wait_probe(3, out, LIMIT)
+    torch.cuda.synchronize()
+    got = out.cpu().tolist()
+    assert got[:6] == [0, 0, 0, 0, 1, bits]
+    assert nslm.nslm_device_status(out) == nslm.NSLM_OK
+
+
+def test_tagged_word_wait_stops_at_the_abort_flag(nslm):
+    out = _tag_words(0, 0, abort=1)
+    t0 = time.time()
+    nslm.nslm_debug_wait_probe(3, out, 2_000_000_000)
+    torch.cuda.synchronize()
+    assert time.time() - t0 < 0.5
+    assert out.cpu().tolist()[:5] == [0, 0, 1, 0, 0]
