@@ -65,7 +65,9 @@ struct Stack1Params {
   int32_t J;              // chunk rounds per lane in phase A: ceil(Ch / 32)
   int32_t rpc;            // output rows per CTA in phase B
   int32_t stage_slots;    // chunk slots of the staging area
-  FastDiv div_inter, div_J, div_Ci, div_nbi;
+  int32_t region_bytes;   // bytes of the staging region (chunk-major x / h, or the table form's tables)
+  int32_t f3_np;          // table form: passes of 128 block positions over the hidden dimension
+  FastDiv div_inter, div_J, div_Ci, div_nbi, div_W;
   FastDiv div_SC[kMaxK + 1];  // by S * Ci for S routed experts
   LayerMats layer[kMaxFusedLayers];
 };
@@ -74,11 +76,132 @@ __device__ __forceinline__ bool stack_wait(const Stack1Params &p, uint32_t e, in
   return grid_wait(p.sync, p.barrier_base + (e + 1) * gridDim.x, s_ok);
 }
 
+// ---------------------------------------------------------------- table form
+//
+// Phase A can take its dot products from tables of x instead of the staged
+// x itself.  With S the 48-bit stream of a block (seed, then the next 32
+// register bits; s_t = the 16 bits of S from bit t), beta_q = the byte of S
+// from bit 1 + 8q, and A_r = sum_j c_j (s_{1+8j+r} - 32768) (the integer part
+// of weight r), the dot product of the block with its 8 inputs x_r is exactly
+//
+//   sum_r x_r A_r = A0 A_0 + 32768 (A0 - X) C
+//                 + sum_j c_j (T[beta_j & 127] - 65536 T[beta_{j+2} & 127]),
+//
+// with A0 = sum_r x_r 2^-r, X = sum_r x_r, C = sum_j c_j and the 128-entry
+// table T[b] = -sum_{r=1..7} x_r 2^-r (b mod 2^r) of the block position: the
+// bits 7..15 of each s_{1+8j+r} enter every r with weight 2^(m-r), i.e.
+// through A0, and the low 7 bits of the two neighbouring bytes through T (the
+// bits of beta_{j+2} carry the same weights as those of beta_j, times
+// -65536).  Every row of a layer shares x, so one CTA builds the tables of
+// 128 positions (64 KB) and all its rows use them: six table reads per block
+// replace the eight per-weight dot products.  The integer A_0 comes from two
+// dp2a as in the direct form; T is built and read in fp32.
+//
+// Layout: position o of a pass (0..127) keeps T/2 at byte (o / 64) * 32768 +
+// b * 256 + w * 4, with word w = 32 (o % 2) + (o % 64) / 2: lane l, which
+// takes positions 64 i + 2 l + t (one 32-bit word of seeds), reads word
+// 32 t + l, in its own bank, and forms the address with one byte permute;
+// constants (A0 / 2, 16384 (A0 - X)) per position follow the tables.
+constexpr int kF3Positions = 128;                       // block positions per pass
+constexpr int kF3TableBytes = kF3Positions * 128 * 4;   // 64 KB
+constexpr int kF3MaxTasks = 4;                          // routed rows per warp it takes
+
+// Tables and constants of the pass's 128 positions from their inputs xp
+// (fp32, 8 per position).  Entry b of position o is the sum of the d_k of
+// the set bits k of b, d_k = -(1/2) 2^k sum_{r>k} x_r 2^-r.
+__device__ void f3_build(char *tab, float2 *cst, const float *xp, int tid, int nthr) {
+  for (int job = tid; job < kF3Positions * 8; job += nthr) {
+    const int o = job & (kF3Positions - 1), m = job >> 7;  // a warp: 32 positions, one entry range
+    const float4 xa = *reinterpret_cast<const float4 *>(xp + 8 * o);
+    const float4 xb = *reinterpret_cast<const float4 *>(xp + 8 * o + 4);
+    const float x[8] = {xa.x, xa.y, xa.z, xa.w, xb.x, xb.y, xb.z, xb.w};
+    float d[7], S = 0.f;
+#pragma unroll
+    for (int k = 6; k >= 0; --k) {
+      S = fmaf(x[k + 1], 1.f / (float)(2 << k), S);  // sum_{r>k} x_r 2^-r
+      d[k] = -0.5f * (float)(1 << k) * S;
+    }
+    float base = 0.f;
+    if (m & 1) base += d[4];
+    if (m & 2) base += d[5];
+    if (m & 4) base += d[6];
+    float L[16];
+    L[0] = 0.f;
+#pragma unroll
+    for (int k = 0; k < 4; ++k)
+#pragma unroll
+      for (int e = 0; e < (1 << k); ++e) L[e + (1 << k)] = L[e] + d[k];
+    char *dst = tab + (o >> 6) * 32768 + (32 * (o & 1) + ((o & 63) >> 1)) * 4 + 16 * m * 256;
+#pragma unroll
+    for (int e = 0; e < 16; ++e) *reinterpret_cast<float *>(dst + e * 256) = base + L[e];
+    if (m == 0) {
+      float a0 = 0.f, xs = 0.f;
+#pragma unroll
+      for (int r = 0; r < 8; ++r) {
+        a0 = fmaf(x[r], 1.f / (float)(1 << r), a0);
+        xs += x[r];
+      }
+      cst[o] = make_float2(0.5f * a0, 16384.f * (a0 - xs));
+    }
+  }
+}
+
+// sum_r x_r A_r of one block from its seed and 16-bit coefficient word; tb:
+// its table block plus 128 t (bytes), lc: 4 * lane, a0h / yh: its constants.
+template <int P>
+__device__ __forceinline__ float f3_block(const uint32_t *tl, uint32_t seed, uint32_t q16, uint32_t lc,
+                                          const char *tb, float a0h, float yh) {
+  const uint32_t nxt = tl[seed & 0xFFu] ^ tl[256u + (seed >> 8)];
+  const uint32_t v = seed << 16;
+  const uint32_t z1 = __funnelshift_r(v, nxt, 17), z9 = __funnelshift_r(v, nxt, 25), z17 = nxt >> 1;
+  const uint32_t cp2 = coef_pairs2<P>(q16);                                 // [2c0, 2c2, 2c1, 2c3]
+  const int32_t c2 = dp4a_ss(cp2, 0x01010101u, 0);                          // 2 C
+  const int32_t i0 = dp2a_hi_us(z9, cp2, dp2a_lo_us(z1, cp2, -32768 * c2));  // 2 A_0
+  const uint32_t m1 = z1 & 0x7F7F7F7Fu, m17 = z17 & 0x7F7F7F7Fu;
+#define NSLM_T(m, k) (*reinterpret_cast<const float *>(tb + __byte_perm((m), lc, 0x5504u | ((k) << 4))))
+  const float t0 = NSLM_T(m1, 0), t1 = NSLM_T(m1, 1), t2 = NSLM_T(m1, 2), t3 = NSLM_T(m1, 3);
+  const float t4 = NSLM_T(m17, 2);
+  float acc = fmaf(yh, (float)c2, a0h * (float)i0);
+  acc = fmaf((float)(int8_t)(cp2 & 0xFFu), fmaf(-65536.f, t2, t0), acc);
+  acc = fmaf((float)(int8_t)((cp2 >> 16) & 0xFFu), fmaf(-65536.f, t3, t1), acc);
+  acc = fmaf((float)(int8_t)((cp2 >> 8) & 0xFFu), fmaf(-65536.f, t4, t2), acc);
+  if (P == 4) acc = fmaf((float)(int8_t)(cp2 >> 24), fmaf(-65536.f, NSLM_T(m17, 3), t3), acc);
+#undef NSLM_T
+  return acc;
+}
+
+// This lane's share of one row's dot product over a pass: positions
+// 64 i + 2 lane + t (i, t in {0, 1}) of the 128 whose fields the warp's lanes
+// 0..15 copied, in order, to the slots from `slot`.
+template <int P>
+__device__ __forceinline__ float f3_row(const uint32_t *tl, const FieldSlots &fs, int slot, int lane,
+                                        const char *tab, const float (&a0h)[2][2], const float (&yh)[2][2]) {
+  const uint32_t *sw = reinterpret_cast<const uint32_t *>(fs.s + slot);
+  const uint32_t *qw = reinterpret_cast<const uint32_t *>(fs.q + slot);
+  const uint8_t *cb = reinterpret_cast<const uint8_t *>(fs.c + slot);
+  const uint32_t rowk = row_scale_key(fs.b[slot]);
+  float acc = 0.f;
+#pragma unroll
+  for (int i = 0; i < 2; ++i) {
+    const uint32_t s2 = sw[32 * i + lane], q2 = qw[32 * i + lane];
+    const uint32_t cbyte = (P == 4) ? (uint32_t)cb[32 * i + lane] : 0u;
+#pragma unroll
+    for (int t = 0; t < 2; ++t) {
+      const uint32_t seed = t ? (s2 >> 16) : (s2 & 0xFFFFu), q = t ? (q2 >> 16) : (q2 & 0xFFFFu);
+      const uint32_t code = (P == 4) ? ((cbyte >> (4 * t)) & 0xFu) : (q >> 12);
+      const float tot = f3_block<P>(tl, seed, q, 4u * (uint32_t)lane, tab + i * 32768 + 128 * t, a0h[i][t], yh[i][t]);
+      acc = fmaf(block_scale(code, rowk), tot, acc);
+    }
+  }
+  return acc;
+}
+
 // Stage x = bf16(y / sqrt(mean(y^2) + 1e-6)) chunk-major from the tagged y
 // rows and per-CTA sums of squares of layer `tag` - 1, polling each word until
 // it carries `tag`.  The sum of squares is the fixed-order sum of the G
 // partials.  The last warp polls the partials while the others poll their
 // first block of 8 rows.  False if a wait gave up.
+template <bool PLAIN>
 __device__ bool stage_norm_tagged(float4 *xs4, float2 *xn2, const uint64_t *ytag, uint32_t tag, int G, int K,
                                   int32_t *sync, float *scratch) {
   const int tid = threadIdx.x, nthr = blockDim.x, nb = K >> 3;
@@ -136,13 +259,19 @@ __device__ bool stage_norm_tagged(float4 *xs4, float2 *xn2, const uint64_t *ytag
     const float4 a = make_float4(NSLM_NORM(w[0]), NSLM_NORM(w[1]), NSLM_NORM(w[2]), NSLM_NORM(w[3]));
     const float4 c = make_float4(NSLM_NORM(w[4]), NSLM_NORM(w[5]), NSLM_NORM(w[6]), NSLM_NORM(w[7]));
 #undef NSLM_NORM
-    cm_store_block(xs4, xn2, b, a, c);
+    if (PLAIN) {  // fp32 in order, for the table form's tables
+      reinterpret_cast<float4 *>(xs4)[2 * b] = a;
+      reinterpret_cast<float4 *>(xs4)[2 * b + 1] = c;
+    } else {
+      cm_store_block(xs4, xn2, b, a, c);
+    }
   }
   return ok;
 }
 
-template <int P, bool VEC>
+template <int P, bool VEC, bool F3>
 __global__ void __launch_bounds__(kStack1MaxThreads, 1) stack1_kernel(const __grid_constant__ Stack1Params p) {
+  static_assert(!F3 || (VEC && (P == 3 || P == 4)), "the table form takes whole chunks of P = 3 or 4");
   extern __shared__ float4 smem4[];
   const int tid = threadIdx.x, nthr = blockDim.x, lane = tid & 31, warp = tid >> 5;
   const int nwarps = nthr >> 5;
@@ -152,7 +281,12 @@ __global__ void __launch_bounds__(kStack1MaxThreads, 1) stack1_kernel(const __gr
   float4 *xs4 = smem4 + kTabCopies * sizeof(StreamTables) / 16;
   float2 *xn2 = reinterpret_cast<float2 *>(xs4 + (size_t)kCmX4 * p.stage_slots);
   // field slots: phase A [2 buffers][gate, up][threads], phase B [2 buffers][threads]
-  const FieldSlots fs(xn2 + (size_t)kCmXn * p.stage_slots + (p.stage_slots & 1), 4 * nthr);
+  const FieldSlots fs(reinterpret_cast<char *>(xs4) + p.region_bytes, 4 * nthr);
+  // table form (phase A): tables, constants, per-task partial sums, x in order
+  char *f3tab = reinterpret_cast<char *>(xs4);
+  float2 *f3cst = reinterpret_cast<float2 *>(f3tab + kF3TableBytes);
+  float2 *f3part = f3cst + kF3Positions;
+  float *xplain = reinterpret_cast<float *>(f3part + nwarps * kF3MaxTasks * 32);
   float *red = reinterpret_cast<float *>(fs.b + 4 * nthr);  // phase B partials
   __shared__ float scratch[33];
   __shared__ int s_ok, s_nslots;
@@ -210,6 +344,22 @@ __global__ void __launch_bounds__(kStack1MaxThreads, 1) stack1_kernel(const __gr
       ku = load_bias_key(Lm.up, grow);
     }
   };
+  // ---- table form: a warp's routed rows (tasks) and, per pass, one step a task
+  auto f3_tasks = [&](int nslots) {
+    const int ntask = nslots * p.inter;
+    return gw < ntask ? (int)fdiv((uint32_t)(ntask - 1 - gw), p.div_W) + 1 : 0;
+  };
+  // copy the fields of task `it`, pass `pass` (lanes 0..15: chunks 16 pass + lane)
+  auto f3_fetch = [&](const LayerMats &Lm, const int32_t *expert, int it, int pass, int buf) {
+    if (lane >= kF3Positions / 8) return;
+    const int t = gw + it * W;
+    const int slot = (int)fdiv(t, p.div_inter), row = t - slot * p.inter;
+    const uint32_t r32 = (uint32_t)((size_t)expert[slot] * p.inter + row);
+    const uint32_t off = r32 * (uint32_t)nbh + 8u * (uint32_t)(16 * pass + lane);
+    fetch_chunk_off<P>(Lm.gate, off, r32, fs, (2 * buf) * nthr + tid);
+    fetch_chunk_off<P>(Lm.up, off, r32, fs, (2 * buf + 1) * nthr + tid);
+  };
+
   // ---- phase B task geometry (row, routed expert, chunk) of this CTA's rows
   auto b_locate = [&](int t, FastDiv dSC, int SC, int &r, int &s, int &c, int &q) {
     r = (int)fdiv(t, dSC);
@@ -240,7 +390,11 @@ __global__ void __launch_bounds__(kStack1MaxThreads, 1) stack1_kernel(const __gr
   uint32_t nbar = 0;  // barriers passed in this launch
 
   // first fields of layer 0, phase A, straight from the plan in global memory
-  if (a_steps(min(p.plans->n_slots, kMaxK)) > 0) a_fetch(p.layer[0], p.plans->expert, 0, 0, fg, fu, kg, ku);
+  if (F3) {
+    if (f3_tasks(min(p.plans->n_slots, kMaxK)) > 0) f3_fetch(p.layer[0], p.plans->expert, 0, 0, 0);
+  } else if (a_steps(min(p.plans->n_slots, kMaxK)) > 0) {
+    a_fetch(p.layer[0], p.plans->expert, 0, 0, fg, fu, kg, ku);
+  }
   if (VEC) cp_async_commit();
   // the plans, by the highest threads, while the lowest stage layer 0's input
   for (int i = nthr - 1 - tid; i < p.n * kMaxK; i += nthr) {
@@ -255,12 +409,17 @@ __global__ void __launch_bounds__(kStack1MaxThreads, 1) stack1_kernel(const __gr
       s_pl_w[l][j] = pl->w[pr];
     }
   }
-  if (p.x0) {  // layer 0's input, bf16 -> fp32 chunk-major
+  if (p.x0) {  // layer 0's input, bf16 -> fp32 chunk-major (table form: in order)
     const uint4 *row = reinterpret_cast<const uint4 *>(p.x0);
     for (int b = tid; b < nbh; b += nthr) {
       float4 lo, hi;
       bf16x8_to_f32(__ldg(row + b), lo, hi);
-      cm_store_block(xs4, xn2, b, lo, hi);
+      if (F3) {
+        reinterpret_cast<float4 *>(xplain)[2 * b] = lo;
+        reinterpret_cast<float4 *>(xplain)[2 * b + 1] = hi;
+      } else {
+        cm_store_block(xs4, xn2, b, lo, hi);
+      }
     }
   }
   build_stream_tables_rep<kTabCopies>(tab);
@@ -279,9 +438,56 @@ __global__ void __launch_bounds__(kStack1MaxThreads, 1) stack1_kernel(const __gr
 
     // =========================== phase A: gate/up + SiLU
     // layer 0's input was staged at the start
-    const bool staged = g == 0 || stage_norm_tagged(xs4, xn2, p.ytag, g, gridDim.x, p.hidden, p.sync, scratch);
+    const bool staged =
+        g == 0 || stage_norm_tagged<F3>(F3 ? reinterpret_cast<float4 *>(xplain) : xs4, xn2, p.ytag, g,
+                                        gridDim.x, p.hidden, p.sync, scratch);
     if (__syncthreads_or(!staged)) break;
-    {
+    if (F3) {
+      // the table form: per pass of 128 block positions, the CTA builds their
+      // tables, then every warp runs its tasks over them; lane partial sums
+      // carry over passes in shared memory, so every row sums in one order
+      const int ntk = f3_tasks(s_nslots);
+      float2 *part = f3part + warp * kF3MaxTasks * 32 + lane;
+      for (int pass = 0; pass < p.f3_np; ++pass) {
+        if (pass > 0) __syncthreads();  // the previous pass's tables are read
+        f3_build(f3tab, f3cst, xplain + pass * kF3Positions * 8, tid, nthr);
+        __syncthreads();
+        float a0h[2][2], yh[2][2];
+#pragma unroll
+        for (int i = 0; i < 2; ++i)
+#pragma unroll
+          for (int t = 0; t < 2; ++t) {
+            const float2 c = f3cst[64 * i + 2 * lane + t];
+            a0h[i][t] = c.x;
+            yh[i][t] = c.y;
+          }
+        for (int it = 0; it < ntk; ++it) {
+          const int step = pass * ntk + it;
+          __syncwarp();  // every lane has read the buffer the next copies refill
+          if (it + 1 < ntk) f3_fetch(Lm, s_expert, it + 1, pass, (step + 1) & 1);
+          else if (pass + 1 < p.f3_np) f3_fetch(Lm, s_expert, 0, pass + 1, (step + 1) & 1);
+          cp_async_commit();
+          cp_async_wait<1>();
+          __syncwarp();  // the step's copies, made by lanes 0..15, seen by all
+          const float pg = f3_row<P>(tl, fs, (2 * (step & 1)) * nthr + warp * 32, lane, f3tab, a0h, yh);
+          const float pu = f3_row<P>(tl, fs, (2 * (step & 1) + 1) * nthr + warp * 32, lane, f3tab, a0h, yh);
+          if (pass == 0) {
+            part[it * 32] = make_float2(pg, pu);
+          } else {
+            const float2 o = part[it * 32];
+            part[it * 32] = make_float2(o.x + pg, o.y + pu);
+          }
+        }
+      }
+      for (int it = 0; it < ntk; ++it) {
+        const float2 v = part[it * 32];
+        const float gs = warp_sum(v.x), us = warp_sum(v.y);
+        const int t = gw + it * W;
+        const int slot = (int)fdiv(t, p.div_inter), row = t - slot * p.inter;
+        if (lane == 0 && in_bounds((size_t)s_pair[slot], (size_t)p.h_rows, 10))
+          __stcg(p.h + (size_t)s_pair[slot] * p.inter + row, __fdividef(gs, 1.f + __expf(-gs)) * us);
+      }
+    } else {
       const int nsteps = a_steps(s_nslots);
       float2 ag = make_float2(0.f, 0.f), au = make_float2(0.f, 0.f);
       for (int step = 0; step < nsteps; ++step) {
@@ -398,7 +604,11 @@ __global__ void __launch_bounds__(kStack1MaxThreads, 1) stack1_kernel(const __gr
     if (l + 1 == p.n) break;
     // the next layer's first phase A fields, in flight while its input arrives
     if (VEC) cp_async_wait<0>();
-    if (a_steps(s_pl_n[l + 1]) > 0) a_fetch(p.layer[l + 1], s_pl_expert[l + 1], 0, 0, fg, fu, kg, ku);
+    if (F3) {
+      if (f3_tasks(s_pl_n[l + 1]) > 0) f3_fetch(p.layer[l + 1], s_pl_expert[l + 1], 0, 0, 0);
+    } else if (a_steps(s_pl_n[l + 1]) > 0) {
+      a_fetch(p.layer[l + 1], s_pl_expert[l + 1], 0, 0, fg, fu, kg, ku);
+    }
     if (VEC) cp_async_commit();
   }
   if (VEC) cp_async_wait<0>();
@@ -437,11 +647,43 @@ static int stack1_threads(const FfnDims &d, int k) {
   return 32 * best;
 }
 
-static size_t stack1_smem(const FfnDims &d, int k, int threads) {
+// The table form of phase A is an ablation build (-DNSLM_STACK1_F3=1, the
+// "tableform" library variant): measured on B200 for the 100-expert
+// 2048/1408 layer it executes ~85 warp instructions per phase A block against
+// the direct form's ~77 (the byte permutes, int -> float conversions and
+// address arithmetic of six lookups outweigh the eight dot products they
+// replace), 38.1 against 36.0 us per layer.
+#ifndef NSLM_STACK1_F3
+#define NSLM_STACK1_F3 0
+#endif
+
+// Bytes of the staging region: chunk-major x (phase A) and h (phase B), or
+// with the table form the tables, constants, partial sums and x in order.
+static size_t stack1_region_bytes(const FfnDims &d, int k, int threads, bool f3) {
   const int Ch = ceil_div(d.hidden / 8, 8), Ci = ceil_div(d.inter / 8, 8);
   const int slots = std::max(Ch, k * Ci);
-  return kTabCopies * sizeof(StreamTables) + cm_bytes(slots) + 16 + FieldSlots::bytes(4 * threads) +
-         (size_t)stack1_rows_per_cta(d) * (slots + 1) * sizeof(float);
+  size_t r = cm_bytes(slots) + (size_t)(slots & 1) * sizeof(float2);
+  if (f3)
+    r = std::max(r, (size_t)kF3TableBytes + kF3Positions * sizeof(float2) +
+                        (size_t)(threads / 32) * kF3MaxTasks * 32 * sizeof(float2) + (size_t)d.hidden * sizeof(float));
+  return (r + 15) / 16 * 16;
+}
+
+static size_t stack1_smem(const FfnDims &d, int k, int threads, bool f3 = false) {
+  const int Ch = ceil_div(d.hidden / 8, 8), Ci = ceil_div(d.inter / 8, 8);
+  const int slots = std::max(Ch, k * Ci);
+  return kTabCopies * sizeof(StreamTables) + stack1_region_bytes(d, k, threads, f3) +
+         FieldSlots::bytes(4 * threads) + (size_t)stack1_rows_per_cta(d) * (slots + 1) * sizeof(float);
+}
+
+// Whether phase A takes the table form: whole chunks of P = 3 or 4, passes of
+// 128 block positions, at most kF3MaxTasks routed rows per warp, and room.
+static bool stack1_f3(const FfnDims &d, int k, int threads) {
+  if (!NSLM_STACK1_F3 || (d.P != 3 && d.P != 4)) return false;
+  if (d.hidden % (8 * kF3Positions) || d.inter % 64) return false;
+  const long long warps = (long long)num_sms() * (threads / 32);
+  if (((long long)k * d.inter + warps - 1) / warps > kF3MaxTasks) return false;
+  return stack1_smem(d, k, threads, true) <= 210 * 1024;
 }
 
 bool stack1_supported(const FfnDims &d, int k) {
@@ -458,14 +700,14 @@ bool stack1_supported(const FfnDims &d, int k) {
   return stack1_smem(d, k, stack1_threads(d, k)) <= 220 * 1024;
 }
 
-template <int P, bool VEC>
+template <int P, bool VEC, bool F3>
 static int32_t launch_stack1_t(const FfnDims &d, const nslm_moe_layer *layers, int n,
                                const SlotPlan *plans, const uint16_t *x0, int k, float *h,
                                uint64_t *ytag, float *y_out, int32_t *sync, cudaStream_t s,
                                int &launches) {
   const int threads = stack1_threads(d, k);
-  const size_t smem = stack1_smem(d, k, threads);
-  auto kern = stack1_kernel<P, VEC>;
+  const size_t smem = stack1_smem(d, k, threads, F3);
+  auto kern = stack1_kernel<P, VEC, F3>;
   int32_t st = ensure_smem((const void *)kern, smem);
   if (st) return st;
   const int per_sm = max_active_ctas((const void *)kern, threads, smem);
@@ -482,6 +724,12 @@ static int32_t launch_stack1_t(const FfnDims &d, const nslm_moe_layer *layers, i
   p.J = ceil_div(p.Ch, 32);
   p.rpc = ceil_div(d.hidden, grid);
   p.stage_slots = std::max(p.Ch, k * p.Ci);
+  p.region_bytes = (int32_t)stack1_region_bytes(d, k, threads, F3);
+  p.f3_np = F3 ? d.hidden / (8 * kF3Positions) : 0;
+  p.div_W = make_fastdiv((uint32_t)(grid * (threads / 32)));
+  if (F3 && ((long long)k * d.inter + (long long)grid * (threads / 32) - 1) / ((long long)grid * (threads / 32)) >
+                kF3MaxTasks)
+    return NSLM_ERR_SHAPE;
   p.div_inter = make_fastdiv((uint32_t)d.inter);
   p.div_J = make_fastdiv((uint32_t)p.J);
   p.div_Ci = make_fastdiv((uint32_t)p.Ci);
@@ -524,13 +772,12 @@ int32_t launch_stack1(const FfnDims &d, const nslm_moe_layer *layers, int n, con
                       cudaStream_t s, int &launches) {
   if (!x0 || !ytag) return NSLM_ERR_ARG;
   const bool vec = d.hidden % 64 == 0 && d.inter % 64 == 0;
-  if (d.P == kP3C5)  // K % 64 == 0 for both projections: whole chunks always
-    return launch_stack1_t<kP3C5, true>(d, layers, n, plans, x0, k, h, ytag, y_out, sync, s, launches);
-  if (d.P == 4)
-    return vec ? launch_stack1_t<4, true>(d, layers, n, plans, x0, k, h, ytag, y_out, sync, s, launches)
-               : launch_stack1_t<4, false>(d, layers, n, plans, x0, k, h, ytag, y_out, sync, s, launches);
-  return vec ? launch_stack1_t<3, true>(d, layers, n, plans, x0, k, h, ytag, y_out, sync, s, launches)
-             : launch_stack1_t<3, false>(d, layers, n, plans, x0, k, h, ytag, y_out, sync, s, launches);
+  const bool f3 = vec && stack1_f3(d, k, stack1_threads(d, k));
+#define NSLM_L(P_, V_, F_) launch_stack1_t<P_, V_, F_>(d, layers, n, plans, x0, k, h, ytag, y_out, sync, s, launches)
+  if (d.P == kP3C5) return NSLM_L(kP3C5, true, false);  // K % 64 == 0 for both projections: whole chunks
+  if (d.P == 4) return f3 ? NSLM_L(4, true, true) : vec ? NSLM_L(4, true, false) : NSLM_L(4, false, false);
+  return f3 ? NSLM_L(3, true, true) : vec ? NSLM_L(3, true, false) : NSLM_L(3, false, false);
+#undef NSLM_L
 }
 
 NSLM_BOUNDS_ACCESSOR(stack1)
