@@ -886,6 +886,7 @@ def main():
     step_bytes /= len(logits)
     achieved = step_bytes / step_s / 1e9
     traffic = None
+    warp_instr = None
     tr_path = os.path.join(ROOT, "profiles", "ffn_decode_layer_traffic.txt")
     if os.path.exists(tr_path) and T == 1:
         rec = {}
@@ -899,6 +900,10 @@ def main():
                 traffic = int(rec["dram_bytes_per_layer_call"]) * LAYERS
             except (KeyError, ValueError):
                 traffic = None
+            try:  # one layer's executed warp instructions (ncu), for the issue view
+                warp_instr = int(rec["warp_instructions_per_layer_call"])
+            except (KeyError, ValueError):
+                warp_instr = None
     # one layer through nslm_moe_seed_ffn (routing plan + the persistent
     # kernel for one layer), for context: per-call overheads included
     nslm.nslm_moe_route_topk(logits[0][0], T, E, K_TOP, ids, wts)
@@ -935,6 +940,20 @@ def main():
                 "traffic_note": "one layer's ncu DRAM bytes x the launch's layers",
                 "single_layer_call_us": round(layer_s * 1e6, 3),
                 "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)" if peak_kind == "measured" else "fallback"}
+    if warp_instr is not None:
+        # the bound in practice: the instruction stream that regenerates the
+        # weights.  Achieved lane-instructions per second over the timed
+        # launch (one layer's ncu count x its layers) against the issue peak:
+        # 4 schedulers x 32 lanes x one instruction per clock per SM at the
+        # median SM clock sampled under load
+        mhz = clk.summary().get("sm_mhz") or clk.summary().get("sm_max_mhz")
+        if mhz:
+            lanes_s = warp_instr * 32.0 * LAYERS / step_s
+            peak_alu = torch.cuda.get_device_properties(dev).multi_processor_count * 128 * mhz * 1e6
+            roofline["alu"] = {"bound": "alu", "unit": "lane-instructions/s", "achieved": round(lanes_s, 1),
+                               "peak": round(peak_alu, 1), "frac": round(lanes_s / peak_alu, 4),
+                               "warp_instructions_per_layer": warp_instr,
+                               "peak_basis": f"SMs x 128 lanes x 1 instruction/clock x {mhz} MHz (median under load)"}
     del g
     torch.cuda.empty_cache()
 

@@ -28,6 +28,10 @@
 // the next phase A only after reading every CTA's y, which each CTA writes
 // after staging h.)
 //
+// Phase B stages the routed h by one 256-byte bulk asynchronous copy per
+// 64-value chunk (global -> shared, completing on an mbarrier; no multicast),
+// then forms the block sums from shared memory.
+//
 // Weight fields are copied with cp.async into per-thread shared-memory slots
 // one task ahead, and the first task of the next phase is fetched before the
 // wait, so the wait overlaps the first loads.  Every wait is bounded: a CTA
@@ -39,6 +43,7 @@
 #include "common.cuh"
 #include "persist.cuh"
 #include "stack1.cuh"
+#include "umma.cuh"
 
 namespace nslm {
 
@@ -290,6 +295,7 @@ __global__ void __launch_bounds__(kStack1MaxThreads, 1) stack1_kernel(const __gr
   float *red = reinterpret_cast<float *>(fs.b + 4 * nthr);  // phase B partials
   __shared__ float scratch[33];
   __shared__ int s_ok, s_nslots;
+  __shared__ __align__(8) uint64_t s_hbar;  // completion of the bulk copies of h (one phase a layer)
   __shared__ int s_expert[kMaxK], s_pair[kMaxK];
   __shared__ float s_w[kMaxK];
   // every layer's routed slots (expert, pair, weight), read once at the start
@@ -423,7 +429,11 @@ __global__ void __launch_bounds__(kStack1MaxThreads, 1) stack1_kernel(const __gr
     }
   }
   build_stream_tables_rep<kTabCopies>(tab);
-  __syncthreads();  // tables, plans, layer 0's input
+  if (tid == 0) {
+    umma::mbar_init(umma::smem_u32(&s_hbar), 1);
+    umma::mbar_init_fence();
+  }
+  __syncthreads();  // tables, plans, layer 0's input, the barrier's init
 
   for (int l = 0; l < p.n; ++l) {
     const LayerMats &Lm = p.layer[l];
@@ -535,24 +545,56 @@ __global__ void __launch_bounds__(kStack1MaxThreads, 1) stack1_kernel(const __gr
     // =========================== phase B: down + weighted combine
     {
       const FastDiv dSC = p.div_SC[s_nslots];
-      // all routed h blocks, two per thread per round with both loads in flight
       const int nhb = s_nslots * nbi;
-      for (int i = tid; i < nhb; i += 2 * nthr) {
-        const int i2 = i + nthr;
-        const int s = (int)fdiv(i, p.div_nbi), b = i - s * nbi;
-        const float4 *src = reinterpret_cast<const float4 *>(p.h + (size_t)s_pair[s] * p.inter) + 2 * b;
-        const float4 a0 = __ldcg(src), a1 = __ldcg(src + 1);
-        float4 c0, c1;
-        int s2 = 0, b2 = 0;
-        if (i2 < nhb) {
-          s2 = (int)fdiv(i2, p.div_nbi);
-          b2 = i2 - s2 * nbi;
-          const float4 *src2 = reinterpret_cast<const float4 *>(p.h + (size_t)s_pair[s2] * p.inter) + 2 * b2;
-          c0 = __ldcg(src2);
-          c1 = __ldcg(src2 + 1);
+      if (VEC) {
+        // all routed h chunks (64 values, 256 contiguous bytes each, as is
+        // their chunk-major slot) by bulk asynchronous copies completing on
+        // s_hbar; then the block sums from shared memory
+        const int nch = s_nslots * p.Ci;
+        const uint32_t hbar = umma::smem_u32(&s_hbar);
+        if (tid == 0) {
+          asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(hbar),
+                       "r"((uint32_t)nch * 256u) : "memory");
         }
-        cm_store_block(xs4, xn2, s * p.Ci * 8 + b, a0, a1);
-        if (i2 < nhb) cm_store_block(xs4, xn2, s2 * p.Ci * 8 + b2, c0, c1);
+        for (int q = tid; q < nch; q += nthr) {
+          const int s = (int)fdiv(q, p.div_Ci), c = q - s * p.Ci;
+          const float *src = p.h + (size_t)s_pair[s] * p.inter + 64 * c;
+          asm volatile("fence.proxy.async.global;" ::: "memory");
+          asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+          asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], 256, [%2];"
+                       ::"r"(umma::smem_u32(xs4 + kCmX4 * q)), "l"(src), "r"(hbar) : "memory");
+        }
+        const bool hok = umma::mbar_wait_bounded(hbar, (uint32_t)(l & 1), kBarrierWaitCycles);
+        if (!hok && tid == 0) {
+          atomicExch(p.sync + 2, 1);
+          atomicCAS(p.sync, 0, 1);
+        }
+        if (__syncthreads_or(!hok)) break;
+        for (int i = tid; i < nhb; i += nthr) {
+          const int q = i >> 3, b = i & 7;  // chunk-major: blocks of a chunk consecutive
+          const float4 lo = xs4[kCmX4 * q + 2 * b], hi = xs4[kCmX4 * q + 2 * b + 1];
+          const float sum = ((lo.x + lo.y) + (lo.z + lo.w)) + ((hi.x + hi.y) + (hi.z + hi.w));
+          xn2[kCmXn * q + b] = make_float2(-kMagic2 * sum, 0.f);
+        }
+      } else {
+        // all routed h blocks, two per thread per round with both loads in flight
+        for (int i = tid; i < nhb; i += 2 * nthr) {
+          const int i2 = i + nthr;
+          const int s = (int)fdiv(i, p.div_nbi), b = i - s * nbi;
+          const float4 *src = reinterpret_cast<const float4 *>(p.h + (size_t)s_pair[s] * p.inter) + 2 * b;
+          const float4 a0 = __ldcg(src), a1 = __ldcg(src + 1);
+          float4 c0, c1;
+          int s2 = 0, b2 = 0;
+          if (i2 < nhb) {
+            s2 = (int)fdiv(i2, p.div_nbi);
+            b2 = i2 - s2 * nbi;
+            const float4 *src2 = reinterpret_cast<const float4 *>(p.h + (size_t)s_pair[s2] * p.inter) + 2 * b2;
+            c0 = __ldcg(src2);
+            c1 = __ldcg(src2 + 1);
+          }
+          cm_store_block(xs4, xn2, s * p.Ci * 8 + b, a0, a1);
+          if (i2 < nhb) cm_store_block(xs4, xn2, s2 * p.Ci * 8 + b2, c0, c1);
+        }
       }
       __syncthreads();
       for (int t = tid, it = 0; t < bt; t += nthr, ++it) {
