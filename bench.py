@@ -720,6 +720,64 @@ def search_leg(torch, nslm, dev, with_cpu: bool):
     return res
 
 
+def anatomy(reps: int):
+    """Per-layer anatomy of the one-token 45-layer launch from the trace build
+    (`python -m lfsr_seeded_moe_b200.build --trace`; loaded here through
+    NSLM_LIB_VARIANT=trace): medians over the middle layers of the global-timer
+    stamps at each CTA's phase boundaries, in microseconds.  Prints one JSON
+    line.  The trace build adds two block barriers a layer, so its layer time
+    runs slightly above the default build's."""
+    os.environ.setdefault("NSLM_LIB_VARIANT", "trace")
+    import numpy as np
+    import torch
+
+    from lfsr_seeded_moe_b200 import nslm, synth
+
+    if not nslm.LIB_PATH.endswith(os.path.join("trace", "libnslm.so")):
+        raise SystemExit(f"--profile anatomy needs the trace build, loaded {nslm.LIB_PATH}")
+    dev = torch.device("cuda", 0)
+    layers = [synth.moe_layer(l, E, HIDDEN, INTER, 4, device=dev, config=4) for l in range(LAYERS)]
+    arr = nslm.moe_layers([(m.gate, m.up, m.down) for m in layers])
+    lg = torch.stack([synth.router_logits((4, l, 0, 0), 1, E) for l in range(LAYERS)]).to(dev).contiguous()
+    x = synth.activations((4, 0, 0), 1, HIDDEN).to(dev).contiguous()
+    y = torch.empty(1, HIDDEN, device=dev)
+    wsb = nslm.nslm_workspace_bytes(nslm.NSLM_OP_MOE_STACK, 1, E, HIDDEN, INTER, K_TOP, LAYERS)
+    ws = torch.zeros(wsb, dtype=torch.uint8, device=dev)
+    for _ in range(max(2, reps)):
+        nslm.nslm_moe_stack_decode(arr, LAYERS, E, K_TOP, lg, x, 1, y, ws, wsb)
+    torch.cuda.synchronize()
+    assert nslm.nslm_device_status(ws) == nslm.NSLM_OK
+    t = nslm.nslm_debug_stack_trace().astype(np.float64) / 1e3  # us
+    G = torch.cuda.get_device_properties(dev).multi_processor_count
+    t = t[:, :G, :LAYERS]
+    full = slice(0, max(1, G - 2))  # CTAs with a full share of output rows
+    med = lambda a: float(np.median(a))
+    rows = {}
+    for l in range(2, LAYERS - 2):
+        s0, s1, s2, s3, s4, s5, s6 = (t[k, :, l] for k in range(7))
+        seg = {
+            "stage_x": med(s1 - s0),
+            "phase_A_median_cta": med(s2 - s1),
+            "phase_A_tail": float(np.max(s2)) - med(s2),
+            "barrier_after_last_arrival": med(s3) - float(np.max(s2)),
+            "stage_h": med(s5 - s3),
+            "phase_B_tasks": med((s6 - s5)[full]),
+            "row_sums_and_y_stores": med((s4 - s6)[full]),
+            "phase_B_tail": float(np.max(s4)) - med(s4),
+            "phase_B_end_to_next_layer": med(t[0, :, l + 1] - s4),
+            "layer": med(t[0, :, l + 1] - s0),
+        }
+        for k, v in seg.items():
+            rows.setdefault(k, []).append(v)
+    out = {"workload": "45-layer one-token decode stack, 100 experts, 2048/1408, P=4, top-8 (trace build)",
+           "unit": "us", "layers_used": f"2..{LAYERS - 3}", "ctas": G}
+    for k, v in rows.items():
+        out[k] = round(float(np.median(v)), 2)
+    lat = np.array([t[2, :, l] - np.median(t[2, :, l]) for l in range(2, LAYERS - 2)]).mean(0)
+    out["phase_A_latest_ctas"] = {int(c): round(float(lat[c]), 2) for c in np.argsort(-lat)[:6]}
+    print(json.dumps(out))
+
+
 def profile_workload(kind: str, reps: int):
     """A small fixed workload for ncu captures (no timing, no JSON): `reps`
     calls of one decode layer (T=1 or T=8, P=4; T=1 in the 5-bit format), of
@@ -778,9 +836,11 @@ def main():
     ap.add_argument("--no-batch8", action="store_true", help="skip the 8-token stack leg")
     ap.add_argument("--no-host-experts", action="store_true", help="skip the host-memory expert cache leg")
     ap.add_argument("--no-p3c5", action="store_true", help="skip the 5-bit P=3 stack leg")
-    ap.add_argument("--profile", choices=["layer", "layer8", "layer_p3c5", "batched", "gemv", "search"],
+    ap.add_argument("--profile", choices=["layer", "layer8", "layer_p3c5", "batched", "gemv", "search", "anatomy"],
                     help="run a small fixed workload for an ncu capture and exit")
     args = ap.parse_args()
+    if args.profile == "anatomy":
+        return anatomy(args.steps)
     if args.profile:
         return profile_workload(args.profile, args.steps)
     if args.impl == "reference":

@@ -363,6 +363,18 @@ int32_t nslm_debug_batched_hidden(const void *ws, size_t ws_bytes, int32_t T, in
 int32_t nslm_debug_bounds_status(void);
 int32_t nslm_debug_bounds_probe(const nslm_seed_matrix *W, nslm_stream_t stream);
 
+/* Test export of the trace build of the library (-DNSLM_STACK1_TRACE=1:
+ * python -m lfsr_seeded_moe_b200.build --trace).  There the one-token
+ * persistent decode kernel (nslm_moe_stack_decode and nslm_moe_seed_ffn at
+ * T = 1) stamps the device's global nanosecond timer at the phase boundaries
+ * of every layer: stamp k of CTA c at layer l of a launch is out[(k * 256 +
+ * c) * 64 + l] (k: 0 layer start, 1 input x staged, 2 the CTA's gate/up phase
+ * done, 3 past the grid barrier, 5 h staged, 6 thread 0's down tasks done,
+ * 4 the CTA's down phase done; CTAs below 256, layers below 64 of the last
+ * launch).  out: HOST, n_words >= 8 * 256 * 64 uint64.  Synchronises the
+ * device.  In the normal build returns NSLM_ERR_UNSUPPORTED. */
+int32_t nslm_debug_stack_trace(uint64_t *out, size_t n_words);
+
 /* Test exports: the regenerated weights themselves, written out densely.
  * w_out: fp32 [N][K] (exact) or bf16 bit patterns [N][K] (round to nearest
  * even of the exact value).  Not on the hot path. */

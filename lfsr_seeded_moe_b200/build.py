@@ -1,7 +1,7 @@
 """Build libnslm.so (the CUDA library) in-tree for sm_100a with nvcc.
 
     python -m lfsr_seeded_moe_b200.build [--force] [--stream-source l2next|l2basis] [--bounds-check]
-                                         [--table-form]
+                                         [--table-form] [--trace]
 
 The shared library lands in lfsr_seeded_moe_b200/_build/libnslm.so; it is
 rebuilt when any source under csrc/ or include/ is newer than it.
@@ -15,7 +15,9 @@ with its extent and records the site instead of making the access (the
 tests run the small parity cases on it).  --table-form builds
 _build/tableform/ with -DNSLM_STACK1_F3=1: phase A of the one-token stack
 takes its dot products from per-position tables of x (an ablation; slower on
-B200, kept tested and measurable).
+B200, kept tested and measurable).  --trace builds _build/trace/ with
+-DNSLM_STACK1_TRACE=1: the one-token decode kernel stamps the global timer
+at its phase boundaries (`bench.py --profile anatomy` reads them).
 """
 from __future__ import annotations
 
@@ -47,7 +49,8 @@ def _inputs():
 
 STREAM_SOURCES = {"l2next": 1, "l2basis": 2}
 VARIANT_DEFS = {"l2next": ["-DNSLM_STREAM_SOURCE=1"], "l2basis": ["-DNSLM_STREAM_SOURCE=2"],
-                "boundscheck": ["-DNSLM_BOUNDS_CHECK=1"], "tableform": ["-DNSLM_STACK1_F3=1"]}
+                "boundscheck": ["-DNSLM_BOUNDS_CHECK=1"], "tableform": ["-DNSLM_STACK1_F3=1"],
+                "trace": ["-DNSLM_STACK1_TRACE=1"]}
 
 
 def lib_path(stream_source: str | None = None) -> str:
@@ -102,5 +105,7 @@ if __name__ == "__main__":
         src = "boundscheck"
     if "--table-form" in sys.argv:
         src = "tableform"
+    if "--trace" in sys.argv:
+        src = "trace"
     print(build(force="--force" in sys.argv, verbose=True, stream_source=src,
                 extra_flags=["-Xptxas", "-v"] if "--ptxas-v" in sys.argv else None))

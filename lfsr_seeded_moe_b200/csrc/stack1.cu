@@ -51,6 +51,36 @@ namespace {
 
 constexpr int kTabCopies = 1;  // interleaved stream-table copies (bank conflicts / kTabCopies)
 
+}  // namespace
+
+// Trace build (-DNSLM_STACK1_TRACE=1, the "trace" library variant): thread 0
+// of every CTA stamps the global timer at the phase boundaries of each layer
+// (stamp k of CTA c, layer l at g_stack1_trace[k][c][l]), with a block
+// barrier before the stamps that mark a whole CTA's end of a phase.  The
+// default build has none of it.
+#ifndef NSLM_STACK1_TRACE
+#define NSLM_STACK1_TRACE 0
+#endif
+constexpr int kTraceStamps = 8, kTraceCtas = 256, kTraceLayers = 64;
+#if NSLM_STACK1_TRACE
+__device__ unsigned long long g_stack1_trace[kTraceStamps][kTraceCtas][kTraceLayers];
+#define NSLM_TRACE(k, sync_first)                                                              \
+  do {                                                                                         \
+    if (sync_first) __syncthreads();                                                           \
+    if (threadIdx.x == 0 && blockIdx.x < kTraceCtas && l < kTraceLayers) {                     \
+      unsigned long long t_;                                                                   \
+      asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t_));                                   \
+      g_stack1_trace[k][blockIdx.x][l] = t_;                                                   \
+    }                                                                                          \
+  } while (0)
+#else
+#define NSLM_TRACE(k, sync_first) \
+  do {                            \
+  } while (0)
+#endif
+
+namespace {
+
 struct LayerMats {
   nslm_seed_matrix gate, up, down;
 };
@@ -445,6 +475,7 @@ __global__ void __launch_bounds__(kStack1MaxThreads, 1) stack1_kernel(const __gr
       s_w[tid] = s_pl_w[l][tid];
     }
     if (tid == 0) s_nslots = s_pl_n[l];
+    NSLM_TRACE(0, false);  // layer start
 
     // =========================== phase A: gate/up + SiLU
     // layer 0's input was staged at the start
@@ -452,6 +483,7 @@ __global__ void __launch_bounds__(kStack1MaxThreads, 1) stack1_kernel(const __gr
         g == 0 || stage_norm_tagged<F3>(F3 ? reinterpret_cast<float4 *>(xplain) : xs4, xn2, p.ytag, g,
                                         gridDim.x, p.hidden, p.sync, scratch);
     if (__syncthreads_or(!staged)) break;
+    NSLM_TRACE(1, false);  // x staged
     if (F3) {
       // the table form: per pass of 128 block positions, the CTA builds their
       // tables, then every warp runs its tasks over them; lane partial sums
@@ -533,6 +565,7 @@ __global__ void __launch_bounds__(kStack1MaxThreads, 1) stack1_kernel(const __gr
         }
       }
     }
+    NSLM_TRACE(2, true);  // this CTA's phase A done
     // arrive; fetch phase B's first fields (weights only) while the others arrive
     const int SC = s_nslots * p.Ci;
     const int bt = nrows * SC;
@@ -541,6 +574,7 @@ __global__ void __launch_bounds__(kStack1MaxThreads, 1) stack1_kernel(const __gr
     if (tid < bt) b_fetch(Lm, p.div_SC[s_nslots], SC, tid, 0, fd, kd);
     if (VEC) cp_async_commit();
     if (!stack_wait(p, nbar++, &s_ok)) break;
+    NSLM_TRACE(3, false);  // past the grid barrier
 
     // =========================== phase B: down + weighted combine
     {
@@ -597,6 +631,7 @@ __global__ void __launch_bounds__(kStack1MaxThreads, 1) stack1_kernel(const __gr
         }
       }
       __syncthreads();
+      NSLM_TRACE(5, false);  // h staged
       for (int t = tid, it = 0; t < bt; t += nthr, ++it) {
         int r, s, c, q;
         b_locate(t, dSC, SC, r, s, c, q);
@@ -617,6 +652,7 @@ __global__ void __launch_bounds__(kStack1MaxThreads, 1) stack1_kernel(const __gr
         chunk_dot_cm<P, VEC, kTabCopies>(tl, cf, nvalid, ck, xs4 + kCmX4 * q, xn2 + kCmXn * q, acc);
         red[t] = s_w[s] * (acc.x + acc.y);
       }
+      NSLM_TRACE(6, false);  // thread 0's phase B tasks done
       __syncthreads();
       // the stack's output in plain fp32; between layers tagged words
       const bool last = l == p.n - 1 && p.y_out;
@@ -643,6 +679,7 @@ __global__ void __launch_bounds__(kStack1MaxThreads, 1) stack1_kernel(const __gr
         }
       }
     }
+    NSLM_TRACE(4, true);  // this CTA's phase B done (y and its sum of squares stored)
     if (l + 1 == p.n) break;
     // the next layer's first phase A fields, in flight while its input arrives
     if (VEC) cp_async_wait<0>();
@@ -825,3 +862,17 @@ int32_t launch_stack1(const FfnDims &d, const nslm_moe_layer *layers, int n, con
 NSLM_BOUNDS_ACCESSOR(stack1)
 
 }  // namespace nslm
+
+// The trace build's stamps (see NSLM_STACK1_TRACE), copied to host memory.
+extern "C" int32_t nslm_debug_stack_trace(uint64_t *out, size_t n_words) {
+#if NSLM_STACK1_TRACE
+  if (!out) return NSLM_ERR_ARG;
+  if (n_words < (size_t)nslm::kTraceStamps * nslm::kTraceCtas * nslm::kTraceLayers) return NSLM_ERR_SHAPE;
+  if (int32_t st = nslm::check_device()) return st;
+  return nslm::cuda_status(cudaMemcpyFromSymbol(out, nslm::g_stack1_trace, sizeof(nslm::g_stack1_trace)));
+#else
+  (void)out;
+  (void)n_words;
+  return NSLM_ERR_UNSUPPORTED;
+#endif
+}

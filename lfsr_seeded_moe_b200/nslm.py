@@ -90,6 +90,7 @@ def _load():
         "nslm_debug_wait_probe": (i32, [i32, vp, ctypes.c_int64, vp]),
         "nslm_debug_bounds_status": (i32, []),
         "nslm_debug_bounds_probe": (i32, [mp, vp]),
+        "nslm_debug_stack_trace": (i32, [vp, sz]),
         "nslm_debug_batched_hidden": (i32, [vp, sz, i32, i32, i32, i32, i32, vp, vp]),
         "nslm_debug_decompress": (i32, [mp, vp, vp]),
         "nslm_debug_decompress_bf16": (i32, [mp, vp, vp]),
@@ -288,6 +289,14 @@ def nslm_debug_bounds_status() -> int:
     if rc < 0:
         raise NslmError("nslm_debug_bounds_status", rc)
     return rc
+
+
+def nslm_debug_stack_trace():
+    """The trace build's stamps as a uint64 numpy array [8][256][64] (ns)."""
+    import numpy as np
+    out = np.zeros((8, 256, 64), np.uint64)
+    _check("nslm_debug_stack_trace", _lib.nslm_debug_stack_trace(out.ctypes.data, out.size))
+    return out
 
 
 def nslm_debug_bounds_probe(W, stream=None) -> None:

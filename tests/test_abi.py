@@ -214,3 +214,10 @@ def test_header_compiles_as_c99(tmp_path):
         r = subprocess.run([gcc, *args, "-I", inc, "-fsyntax-only", str(src)], capture_output=True, text=True)
         assert r.returncode == 0, r.stderr
 
+
+
+def test_stack_trace_is_a_trace_build_export():
+    # the normal build has no trace: the export refuses without touching its buffer
+    import numpy as np
+    out = np.zeros(8, np.uint64)
+    assert nslm.raw().nslm_debug_stack_trace(out.ctypes.data, out.size) == nslm.NSLM_ERR_UNSUPPORTED
