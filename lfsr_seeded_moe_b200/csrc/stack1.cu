@@ -32,9 +32,12 @@
 // 64-value chunk (global -> shared, completing on an mbarrier; no multicast),
 // then forms the block sums from shared memory.
 //
-// Weight fields are copied with cp.async into per-thread shared-memory slots
-// one task ahead, and the first task of the next phase is fetched before the
-// wait, so the wait overlaps the first loads.  Every wait is bounded: a CTA
+// Weight fields land in per-thread shared-memory slots one task ahead: in
+// phase A by bulk asynchronous copies (lane 0 of each warp copies the step's
+// seeds, coefficients and code words of both matrices, completing on the
+// warp's barrier of that buffer), in phase B by cp.async.  The first task of
+// the next phase is fetched before the wait, so the wait overlaps the first
+// loads.  Every wait is bounded: a CTA
 // that gives up raises the abort flag (all others stop at their next wait)
 // and records status 1 in the workspace.
 #include <algorithm>
@@ -304,9 +307,10 @@ __device__ bool stage_norm_tagged(float4 *xs4, float2 *xn2, const uint64_t *ytag
   return ok;
 }
 
-template <int P, bool VEC, bool F3>
+template <int P, bool VEC, bool F3, bool BA>
 __global__ void __launch_bounds__(kStack1MaxThreads, 1) stack1_kernel(const __grid_constant__ Stack1Params p) {
   static_assert(!F3 || (VEC && (P == 3 || P == 4)), "the table form takes whole chunks of P = 3 or 4");
+  static_assert(!BA || (VEC && !F3), "bulk phase A copies take whole chunks, direct form");
   extern __shared__ float4 smem4[];
   const int tid = threadIdx.x, nthr = blockDim.x, lane = tid & 31, warp = tid >> 5;
   const int nwarps = nthr >> 5;
@@ -326,6 +330,8 @@ __global__ void __launch_bounds__(kStack1MaxThreads, 1) stack1_kernel(const __gr
   __shared__ float scratch[33];
   __shared__ int s_ok, s_nslots;
   __shared__ __align__(8) uint64_t s_hbar;  // completion of the bulk copies of h (one phase a layer)
+  // BA: completion of each warp's bulk copies of its phase A fields, per buffer
+  __shared__ __align__(8) uint64_t s_fbar[kStack1MaxThreads / 32][2];
   __shared__ int s_expert[kMaxK], s_pair[kMaxK];
   __shared__ float s_w[kMaxK];
   // every layer's routed slots (expert, pair, weight), read once at the start
@@ -380,6 +386,72 @@ __global__ void __launch_bounds__(kStack1MaxThreads, 1) stack1_kernel(const __gr
       ku = load_bias_key(Lm.up, grow);
     }
   };
+  // ---- BA: a warp's phase A fields by bulk asynchronous copies, lane 0
+  // issuing per matrix one copy each of the step's seeds, coefficients and
+  // code words (the lanes' chunks are consecutive, so their slots and the
+  // fields in global memory are both contiguous), completing on the warp's
+  // barrier of that buffer; the row's exponent bias goes to a register.  Copy
+  // n (counted over the launch) lands in buffer n % 2, phase (n / 2) % 2.
+  uint32_t nfetch = 0, nread = 0, nbg = 0, nbu = 0;
+  auto a_fetch_bulk = [&](const LayerMats &Lm, const int32_t *expert, int step) {
+    int slot, row, c;
+    a_locate(step, slot, row, c);
+    const int cb = c - lane, nch = min(32, p.Ch - cb);  // this step's chunks: cb .. cb + nch - 1
+    const uint32_t r32 = (uint32_t)((size_t)expert[slot] * p.inter + row);
+    nbg = load_bias_key(Lm.gate, r32);
+    nbu = load_bias_key(Lm.up, r32);
+    if (P == kP3C5 && c < p.Ch) {
+      const uint32_t off = r32 * (uint32_t)nbh + 8u * (uint32_t)c;
+      nqg = load_codes3(Lm.gate, off >> 3);
+      nqu = load_codes3(Lm.up, off >> 3);
+    }
+    const uint32_t buf = nfetch++ & 1u;
+    __syncwarp();  // every lane has read the buffer's previous fields
+    if (lane == 0) {
+      const uint32_t bar = umma::smem_u32(&s_fbar[warp][buf]);
+      const uint32_t sb = 16u * (uint32_t)nch, cbytes = (P == 4) ? 4u * (uint32_t)nch : 0u;
+      const size_t first = (size_t)r32 * nbh + 8u * (uint32_t)cb;
+      if (!in_bounds(first + 8u * (uint32_t)nch - 1, (size_t)Lm.gate.N * nbh, 1) ||
+          !in_bounds(r32, (size_t)Lm.gate.N, 2)) {
+        umma::mbar_arrive(bar);  // nothing copied: the phase completes on the arrival alone
+      } else {
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(2u * (2u * sb + cbytes))
+                     : "memory");
+#pragma unroll
+        for (int m = 0; m < 2; ++m) {
+          const nslm_seed_matrix &W = m ? Lm.up : Lm.gate;
+          const int sl = (2 * (int)buf + m) * nthr + warp * 32;
+#define NSLM_BULK(dst, src, n)                                                                                   \
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(  \
+                   umma::smem_u32(dst)),                                                                         \
+               "l"(src), "r"(n), "r"(bar)                                                                        \
+               : "memory")
+          NSLM_BULK(fs.s + sl, W.seeds + first, sb);
+          NSLM_BULK(fs.q + sl, W.coefs + first, sb);
+          if (P == 4) NSLM_BULK(fs.c + sl, W.codes + first / 2, cbytes);
+#undef NSLM_BULK
+        }
+      }
+    }
+  };
+  // wait for copy nread and read this lane's fields of it; false on timeout
+  auto a_read_bulk = [&](ChunkFields &fg_, ChunkFields &fu_) {
+    const uint32_t buf = nread & 1u, par = (nread >> 1) & 1u;
+    ++nread;
+    if (!umma::mbar_wait_bounded(umma::smem_u32(&s_fbar[warp][buf]), par, kBarrierWaitCycles)) return false;
+#pragma unroll
+    for (int m = 0; m < 2; ++m) {
+      ChunkFields &f = m ? fu_ : fg_;
+      const int sl = (2 * (int)buf + m) * nthr + tid;
+      const uint4 sv = fs.s[sl], qv = fs.q[sl];
+      f.s[0] = sv.x; f.s[1] = sv.y; f.s[2] = sv.z; f.s[3] = sv.w;
+      f.q[0] = qv.x; f.q[1] = qv.y; f.q[2] = qv.z; f.q[3] = qv.w;
+      f.codes = (P == 4) ? fs.c[sl] : 0u;
+    }
+    return true;
+  };
+
   // ---- table form: a warp's routed rows (tasks) and, per pass, one step a task
   auto f3_tasks = [&](int nslots) {
     const int ntask = nslots * p.inter;
@@ -425,11 +497,23 @@ __global__ void __launch_bounds__(kStack1MaxThreads, 1) stack1_kernel(const __gr
   uint32_t kg = 0, ku = 0, kd = 0;
   uint32_t nbar = 0;  // barriers passed in this launch
 
+  // the barriers, initialised and fenced by one thread before any copy uses them
+  if (tid == 0) {
+    umma::mbar_init(umma::smem_u32(&s_hbar), 1);
+    if (BA)
+      for (int w = 0; w < nwarps; ++w)
+        for (int b = 0; b < 2; ++b) umma::mbar_init(umma::smem_u32(&s_fbar[w][b]), 1);
+    umma::mbar_init_fence();
+  }
+  __syncthreads();
   // first fields of layer 0, phase A, straight from the plan in global memory
   if (F3) {
     if (f3_tasks(min(p.plans->n_slots, kMaxK)) > 0) f3_fetch(p.layer[0], p.plans->expert, 0, 0, 0);
   } else if (a_steps(min(p.plans->n_slots, kMaxK)) > 0) {
-    a_fetch(p.layer[0], p.plans->expert, 0, 0, fg, fu, kg, ku);
+    if (BA)
+      a_fetch_bulk(p.layer[0], p.plans->expert, 0);
+    else
+      a_fetch(p.layer[0], p.plans->expert, 0, 0, fg, fu, kg, ku);
   }
   if (VEC) cp_async_commit();
   // the plans, by the highest threads, while the lowest stage layer 0's input
@@ -459,11 +543,7 @@ __global__ void __launch_bounds__(kStack1MaxThreads, 1) stack1_kernel(const __gr
     }
   }
   build_stream_tables_rep<kTabCopies>(tab);
-  if (tid == 0) {
-    umma::mbar_init(umma::smem_u32(&s_hbar), 1);
-    umma::mbar_init_fence();
-  }
-  __syncthreads();  // tables, plans, layer 0's input, the barrier's init
+  __syncthreads();  // tables, plans, layer 0's input
 
   for (int l = 0; l < p.n; ++l) {
     const LayerMats &Lm = p.layer[l];
@@ -532,12 +612,30 @@ __global__ void __launch_bounds__(kStack1MaxThreads, 1) stack1_kernel(const __gr
     } else {
       const int nsteps = a_steps(s_nslots);
       float2 ag = make_float2(0.f, 0.f), au = make_float2(0.f, 0.f);
+      bool aok = true;
       for (int step = 0; step < nsteps; ++step) {
         int slot, row, c;
         a_locate(step, slot, row, c);
         ChunkFields cg = fg, cu = fu;
         uint32_t ckg = kg, cku = ku;
-        if (VEC) {
+        if (BA) {
+          ckg = nbg;
+          cku = nbu;
+          const uint32_t cqg = nqg, cqu = nqu;  // this step's 5-bit-format code bits
+          if (!a_read_bulk(cg, cu)) {
+            if (lane == 0) {
+              atomicExch(p.sync + 2, 1);
+              atomicCAS(p.sync, 0, 1);
+            }
+            aok = false;
+            break;
+          }
+          if (P == kP3C5) {
+            cg.codes = cqg;
+            cu.codes = cqu;
+          }
+          if (step + 1 < nsteps) a_fetch_bulk(Lm, s_expert, step + 1);
+        } else if (VEC) {
           const uint32_t cqg = nqg, cqu = nqu;  // this step's 5-bit-format code bits
           if (step + 1 < nsteps) a_fetch(Lm, s_expert, step + 1, (step + 1) & 1, fg, fu, kg, ku);
           cp_async_commit();
@@ -564,6 +662,7 @@ __global__ void __launch_bounds__(kStack1MaxThreads, 1) stack1_kernel(const __gr
           ag = au = make_float2(0.f, 0.f);
         }
       }
+      if (BA && __syncthreads_or(!aok)) break;
     }
     NSLM_TRACE(2, true);  // this CTA's phase A done
     // arrive; fetch phase B's first fields (weights only) while the others arrive
@@ -686,7 +785,10 @@ __global__ void __launch_bounds__(kStack1MaxThreads, 1) stack1_kernel(const __gr
     if (F3) {
       if (f3_tasks(s_pl_n[l + 1]) > 0) f3_fetch(p.layer[l + 1], s_pl_expert[l + 1], 0, 0, 0);
     } else if (a_steps(s_pl_n[l + 1]) > 0) {
-      a_fetch(p.layer[l + 1], s_pl_expert[l + 1], 0, 0, fg, fu, kg, ku);
+      if (BA)
+        a_fetch_bulk(p.layer[l + 1], s_pl_expert[l + 1], 0);
+      else
+        a_fetch(p.layer[l + 1], s_pl_expert[l + 1], 0, 0, fg, fu, kg, ku);
     }
     if (VEC) cp_async_commit();
   }
@@ -735,6 +837,9 @@ static int stack1_threads(const FfnDims &d, int k) {
 #ifndef NSLM_STACK1_F3
 #define NSLM_STACK1_F3 0
 #endif
+#ifndef NSLM_STACK1_BULK_A
+#define NSLM_STACK1_BULK_A 1  // phase A's weight fields by bulk copies where they apply
+#endif
 
 // Bytes of the staging region: chunk-major x (phase A) and h (phase B), or
 // with the table form the tables, constants, partial sums and x in order.
@@ -779,14 +884,14 @@ bool stack1_supported(const FfnDims &d, int k) {
   return stack1_smem(d, k, stack1_threads(d, k)) <= 220 * 1024;
 }
 
-template <int P, bool VEC, bool F3>
+template <int P, bool VEC, bool F3, bool BA>
 static int32_t launch_stack1_t(const FfnDims &d, const nslm_moe_layer *layers, int n,
                                const SlotPlan *plans, const uint16_t *x0, int k, float *h,
                                uint64_t *ytag, float *y_out, int32_t *sync, cudaStream_t s,
                                int &launches) {
   const int threads = stack1_threads(d, k);
   const size_t smem = stack1_smem(d, k, threads, F3);
-  auto kern = stack1_kernel<P, VEC, F3>;
+  auto kern = stack1_kernel<P, VEC, F3, BA>;
   int32_t st = ensure_smem((const void *)kern, smem);
   if (st) return st;
   const int per_sm = max_active_ctas((const void *)kern, threads, smem);
@@ -852,10 +957,17 @@ int32_t launch_stack1(const FfnDims &d, const nslm_moe_layer *layers, int n, con
   if (!x0 || !ytag) return NSLM_ERR_ARG;
   const bool vec = d.hidden % 64 == 0 && d.inter % 64 == 0;
   const bool f3 = vec && stack1_f3(d, k, stack1_threads(d, k));
-#define NSLM_L(P_, V_, F_) launch_stack1_t<P_, V_, F_>(d, layers, n, plans, x0, k, h, ytag, y_out, sync, s, launches)
-  if (d.P == kP3C5) return NSLM_L(kP3C5, true, false);  // K % 64 == 0 for both projections: whole chunks
-  if (d.P == 4) return f3 ? NSLM_L(4, true, true) : vec ? NSLM_L(4, true, false) : NSLM_L(4, false, false);
-  return f3 ? NSLM_L(3, true, true) : vec ? NSLM_L(3, true, false) : NSLM_L(3, false, false);
+  // phase A fields by bulk copies: whole chunks whose P = 4 code words make
+  // 16-byte multiples (hidden % 256 == 0)
+  const bool ba = vec && !f3 && NSLM_STACK1_BULK_A && d.hidden % 256 == 0;
+#define NSLM_L(P_, V_, F_, B_) \
+  launch_stack1_t<P_, V_, F_, B_>(d, layers, n, plans, x0, k, h, ytag, y_out, sync, s, launches)
+  if (d.P == kP3C5) return ba ? NSLM_L(kP3C5, true, false, true) : NSLM_L(kP3C5, true, false, false);
+  if (d.P == 4)
+    return f3 ? NSLM_L(4, true, true, false) : ba ? NSLM_L(4, true, false, true)
+               : vec ? NSLM_L(4, true, false, false) : NSLM_L(4, false, false, false);
+  return f3 ? NSLM_L(3, true, true, false) : ba ? NSLM_L(3, true, false, true)
+            : vec ? NSLM_L(3, true, false, false) : NSLM_L(3, false, false, false);
 #undef NSLM_L
 }
 
