@@ -386,53 +386,55 @@ __global__ void __launch_bounds__(kStack1MaxThreads, 1) stack1_kernel(const __gr
       ku = load_bias_key(Lm.up, grow);
     }
   };
-  // ---- BA: a warp's phase A fields by bulk asynchronous copies, lane 0
-  // issuing per matrix one copy each of the step's seeds, coefficients and
-  // code words (the lanes' chunks are consecutive, so their slots and the
-  // fields in global memory are both contiguous), completing on the warp's
-  // barrier of that buffer; the row's exponent bias goes to a register.  Copy
-  // n (counted over the launch) lands in buffer n % 2, phase (n / 2) % 2.
+  // ---- BA: a warp's phase A fields by bulk asynchronous copies: per matrix
+  // one copy each of the step's seeds, coefficients and code words (the
+  // lanes' chunks are consecutive, so their slots and the fields in global
+  // memory are both contiguous), one lane a copy, all in one instruction,
+  // completing on the warp's barrier of that buffer.  The row's exponent bias
+  // goes to a register as the raw word (its scale key is formed when the step
+  // is read, so nothing waits for the load here).  Copy n (counted over the
+  // launch) lands in buffer n % 2, phase (n / 2) % 2.
   uint32_t nfetch = 0, nread = 0, nbg = 0, nbu = 0;
   auto a_fetch_bulk = [&](const LayerMats &Lm, const int32_t *expert, int step) {
     int slot, row, c;
     a_locate(step, slot, row, c);
     const int cb = c - lane, nch = min(32, p.Ch - cb);  // this step's chunks: cb .. cb + nch - 1
     const uint32_t r32 = (uint32_t)((size_t)expert[slot] * p.inter + row);
-    nbg = load_bias_key(Lm.gate, r32);
-    nbu = load_bias_key(Lm.up, r32);
+    nbg = in_bounds(r32, (size_t)Lm.gate.N, 4) ? (uint32_t)__ldg(Lm.gate.exp_bias + r32) : 0u;
+    nbu = in_bounds(r32, (size_t)Lm.up.N, 4) ? (uint32_t)__ldg(Lm.up.exp_bias + r32) : 0u;
     if (P == kP3C5 && c < p.Ch) {
       const uint32_t off = r32 * (uint32_t)nbh + 8u * (uint32_t)c;
       nqg = load_codes3(Lm.gate, off >> 3);
       nqu = load_codes3(Lm.up, off >> 3);
     }
     const uint32_t buf = nfetch++ & 1u;
+    const uint32_t bar = umma::smem_u32(&s_fbar[warp][buf]);
+    const uint32_t sb = 16u * (uint32_t)nch, cbytes = (P == 4) ? 4u * (uint32_t)nch : 0u;
+    const size_t first = (size_t)r32 * nbh + 8u * (uint32_t)cb;
+    const bool inside = in_bounds(first + 8u * (uint32_t)nch - 1, (size_t)Lm.gate.N * nbh, 1) &&
+                        in_bounds(r32, (size_t)Lm.gate.N, 2);
     __syncwarp();  // every lane has read the buffer's previous fields
     if (lane == 0) {
-      const uint32_t bar = umma::smem_u32(&s_fbar[warp][buf]);
-      const uint32_t sb = 16u * (uint32_t)nch, cbytes = (P == 4) ? 4u * (uint32_t)nch : 0u;
-      const size_t first = (size_t)r32 * nbh + 8u * (uint32_t)cb;
-      if (!in_bounds(first + 8u * (uint32_t)nch - 1, (size_t)Lm.gate.N * nbh, 1) ||
-          !in_bounds(r32, (size_t)Lm.gate.N, 2)) {
-        umma::mbar_arrive(bar);  // nothing copied: the phase completes on the arrival alone
-      } else {
-        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+      if (inside)
         asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(2u * (2u * sb + cbytes))
                      : "memory");
-#pragma unroll
-        for (int m = 0; m < 2; ++m) {
-          const nslm_seed_matrix &W = m ? Lm.up : Lm.gate;
-          const int sl = (2 * (int)buf + m) * nthr + warp * 32;
-#define NSLM_BULK(dst, src, n)                                                                                   \
-  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(  \
-                   umma::smem_u32(dst)),                                                                         \
-               "l"(src), "r"(n), "r"(bar)                                                                        \
-               : "memory")
-          NSLM_BULK(fs.s + sl, W.seeds + first, sb);
-          NSLM_BULK(fs.q + sl, W.coefs + first, sb);
-          if (P == 4) NSLM_BULK(fs.c + sl, W.codes + first / 2, cbytes);
-#undef NSLM_BULK
-        }
-      }
+      else
+        umma::mbar_arrive(bar);  // nothing copied: the phase completes on the arrival alone
+    }
+    __syncwarp();  // the expected bytes are set before any copy completes
+    constexpr int kFields = (P == 4) ? 3 : 2;  // seeds, coefficients (, code words) per matrix
+    if (inside && lane < 2 * kFields) {
+      const int m = lane / kFields, fld = lane - m * kFields;
+      const nslm_seed_matrix &W = m ? Lm.up : Lm.gate;
+      const int sl = (2 * (int)buf + m) * nthr + warp * 32;
+      const void *dst = fld == 0 ? (const void *)(fs.s + sl) : fld == 1 ? (const void *)(fs.q + sl) : (const void *)(fs.c + sl);
+      const void *src = fld == 0 ? (const void *)(W.seeds + first)
+                        : fld == 1 ? (const void *)(W.coefs + first) : (const void *)(W.codes + first / 2);
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+      asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                       umma::smem_u32(dst)),
+                   "l"(src), "r"(fld == 2 ? cbytes : sb), "r"(bar)
+                   : "memory");
     }
   };
   // wait for copy nread and read this lane's fields of it; false on timeout
@@ -619,8 +621,8 @@ __global__ void __launch_bounds__(kStack1MaxThreads, 1) stack1_kernel(const __gr
         ChunkFields cg = fg, cu = fu;
         uint32_t ckg = kg, cku = ku;
         if (BA) {
-          ckg = nbg;
-          cku = nbu;
+          ckg = row_scale_key((int32_t)nbg);
+          cku = row_scale_key((int32_t)nbu);
           const uint32_t cqg = nqg, cqu = nqu;  // this step's 5-bit-format code bits
           if (!a_read_bulk(cg, cu)) {
             if (lane == 0) {
