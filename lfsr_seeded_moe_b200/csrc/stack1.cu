@@ -33,13 +33,14 @@
 // then forms the block sums from shared memory.
 //
 // Weight fields land in per-thread shared-memory slots one task ahead: in
-// phase A by bulk asynchronous copies (lane 0 of each warp copies the step's
-// seeds, coefficients and code words of both matrices, completing on the
-// warp's barrier of that buffer), in phase B by cp.async.  The first task of
-// the next phase is fetched before the wait, so the wait overlaps the first
-// loads.  Every wait is bounded: a CTA
-// that gives up raises the abort flag (all others stop at their next wait)
-// and records status 1 in the workspace.
+// phase A (hidden % 256 == 0) by bulk asynchronous copies, six lanes of each
+// warp copying the step's seeds, coefficients and code words of both
+// matrices in one instruction, completing on the warp's barrier of that
+// buffer; otherwise, and in phase B, by cp.async.  The first task of the
+// next phase is fetched before the wait, so the wait overlaps the first
+// loads.  Every wait is bounded: a CTA that gives up raises the abort flag
+// (all others stop at their next wait) and records status 1 in the
+// workspace.
 #include <algorithm>
 
 #include "chunk.cuh"

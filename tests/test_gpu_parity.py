@@ -224,6 +224,9 @@ def _ffn_with_ids(nslm, L, E, hidden, inter, x, rid, w32, k):
     (12, 272, 120, 3, 8),      # ragged rows in both projections
     (8, 4160, 208, 4, 2),      # 65 chunks per gate row (two rounds per lane), ragged down rows
     (4, 64, 64, 4, 1),         # one chunk per row, one expert per token
+    (6, 4096, 128, 4, 2),      # two full rounds of bulk-copied gate/up chunks per lane
+    (5, 2560, 192, 3, 3),      # bulk copies: a full round, then 8 chunks
+    (4, 2304, 128, 4, 2),      # bulk copies: a full round, then 4 chunks (16 bytes of codes)
 ])
 def test_ffn_one_token_shapes(nslm, E, hidden, inter, P, k):
     tag = 920 + hidden
