@@ -65,8 +65,8 @@ constexpr int kTabCopies = 1;  // interleaved stream-table copies (bank conflict
 #ifndef NSLM_STACK1_TRACE
 #define NSLM_STACK1_TRACE 0
 #endif
-constexpr int kTraceStamps = 8, kTraceCtas = 256, kTraceLayers = 64;
 #if NSLM_STACK1_TRACE
+constexpr int kTraceStamps = 8, kTraceCtas = 256, kTraceLayers = 64;
 __device__ unsigned long long g_stack1_trace[kTraceStamps][kTraceCtas][kTraceLayers];
 #define NSLM_TRACE(k, sync_first)                                                              \
   do {                                                                                         \
