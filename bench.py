@@ -45,6 +45,27 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 KERNEL_SOURCES = ("stack1.cu", "stack1.cuh", "chunk.cuh", "regen.cuh", "persist.cuh", "common.cuh", "moe.cuh")
 
 
+def layer_record(path: str | None = None) -> dict:
+    """The per-layer ncu record of the one-token kernel (profiles/
+    ffn_decode_layer_traffic.txt): its integer fields, and whether its
+    digest matches the kernel sources as they are now (the figures hold only
+    then)."""
+    path = path or os.path.join(ROOT, "profiles", "ffn_decode_layer_traffic.txt")
+    rec = {}
+    if os.path.exists(path):
+        for ln in open(path):
+            if ":" in ln and not ln.startswith("#"):
+                key, val = ln.split(":", 1)
+                rec[key.strip()] = val.split()[0] if val.split() else ""
+    out = {"matches": bool(rec) and rec.get("kernel_sources_sha256") == kernel_sources_sha256()}
+    for key in ("dram_bytes_per_layer_call", "warp_instructions_per_layer_call"):
+        try:
+            out[key] = int(rec[key])
+        except (KeyError, ValueError):
+            out[key] = None
+    return out
+
+
 def kernel_sources_sha256() -> str:
     import hashlib
     h = hashlib.sha256()
@@ -947,23 +968,11 @@ def main():
     achieved = step_bytes / step_s / 1e9
     traffic = None
     warp_instr = None
-    tr_path = os.path.join(ROOT, "profiles", "ffn_decode_layer_traffic.txt")
-    if os.path.exists(tr_path) and T == 1:
-        rec = {}
-        for ln in open(tr_path):
-            if ":" in ln and not ln.startswith("#"):
-                key, val = ln.split(":", 1)
-                rec[key.strip()] = val.split()[0] if val.split() else ""
-        # the counters hold only for the kernel source they were taken on
-        if rec.get("kernel_sources_sha256") == kernel_sources_sha256():
-            try:  # one layer's DRAM bytes (ncu), scaled to the launch's 45 layers
-                traffic = int(rec["dram_bytes_per_layer_call"]) * LAYERS
-            except (KeyError, ValueError):
-                traffic = None
-            try:  # one layer's executed warp instructions (ncu), for the issue view
-                warp_instr = int(rec["warp_instructions_per_layer_call"])
-            except (KeyError, ValueError):
-                warp_instr = None
+    rec = layer_record()
+    if T == 1 and rec["matches"]:  # the counters hold only for the kernel source they were taken on
+        if rec["dram_bytes_per_layer_call"] is not None:  # one layer's DRAM bytes, x the launch's 45 layers
+            traffic = rec["dram_bytes_per_layer_call"] * LAYERS
+        warp_instr = rec["warp_instructions_per_layer_call"]  # one layer's warp instructions (issue view)
     # one layer through nslm_moe_seed_ffn (routing plan + the persistent
     # kernel for one layer), for context: per-call overheads included
     nslm.nslm_moe_route_topk(logits[0][0], T, E, K_TOP, ids, wts)

@@ -89,3 +89,19 @@ def test_clock_sampler_keeps_only_the_timed_window():
     s.t0, s.t1 = 0.9, 2.0
     s.keep_window()
     assert s.summary() == {"sm_mhz": 1957.5, "sm_max_mhz": 1965.0, "reasons": [], "samples": 2}
+
+
+def test_layer_record_holds_only_for_the_sources_it_names(tmp_path):
+    import bench
+    d = bench.kernel_sources_sha256()
+    assert len(d) == 64 and d == bench.kernel_sources_sha256()
+    good = tmp_path / "rec.txt"
+    good.write_text(f"dram_bytes_per_layer_call: 123\nwarp_instructions_per_layer_call: 45\n"
+                    f"kernel_sources_sha256: {d}\n# a comment: 7\n")
+    r = bench.layer_record(str(good))
+    assert r == {"matches": True, "dram_bytes_per_layer_call": 123, "warp_instructions_per_layer_call": 45}
+    stale = tmp_path / "stale.txt"
+    stale.write_text("dram_bytes_per_layer_call: 123\nkernel_sources_sha256: unrecorded\n")
+    r = bench.layer_record(str(stale))
+    assert r["matches"] is False and r["warp_instructions_per_layer_call"] is None
+    assert bench.layer_record(str(tmp_path / "missing.txt"))["matches"] is False
