@@ -422,14 +422,18 @@ def job_throughput(world: int, steps: int, tokens_per_step: int, elapsed_s: floa
 
 # ------------------------------------------------------------------- GPU leg
 
-def gemv_sweep(torch, nslm, synth, dev, hbm):
+def gemv_sweep(torch, nslm, synth, dev, hbm, shapes=None):
     """The single small GEMV (512 x 1024, P=4) and the expert-sized sweep for
     P=4, P=3 and the 5-bit P=3 format (35), batch 1.  Each shape is timed over
     rotating weight copies in one CUDA graph (more than 4x L2 where 400 copies
     reach it; the small GEMV's copies stay largely in L2): the cold (HBM)
-    figures.  The warm figures repeat one copy, which then sits in L2."""
+    figures.  The warm figures repeat one copy, which then sits in L2.
+    `shapes` ([(N, K), ...]) replaces the whole list, small GEMV included."""
     out = []
-    cases = [(4, GEMV_SMALL)] + [(Pv, nk) for Pv in (4, 3, 35) for nk in GEMV_SHAPES]
+    if shapes:
+        cases = [(Pv, nk) for Pv in (4, 3, 35) for nk in shapes]
+    else:
+        cases = [(4, GEMV_SMALL)] + [(Pv, nk) for Pv in (4, 3, 35) for nk in GEMV_SHAPES]
     for Pv, (N, K) in cases:
         m0 = synth.seed_matrix(N, K, Pv, (11, N, K, Pv), device=dev)
         nbytes = m0.packed_bytes()
@@ -843,6 +847,17 @@ def profile_workload(kind: str, reps: int):
         raise SystemExit("batched layer reported a non-zero status")
 
 
+def _gemv_shapes(text: str):
+    """'8192x8192,2048x4096' -> [(8192, 8192), (2048, 4096)]."""
+    out = []
+    for part in text.split(","):
+        n, k = part.lower().split("x")
+        out.append((int(n), int(k)))
+    if not out or any(n < 1 or k < 8 or k % 8 for n, k in out):
+        raise argparse.ArgumentTypeError("shapes are NxK with N >= 1 and K a positive multiple of 8")
+    return out
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -851,6 +866,8 @@ def main():
     ap.add_argument("--batch", type=int, default=1, help="decode tokens per step (1..8)")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-gemv", action="store_true")
+    ap.add_argument("--gemv-shapes", type=_gemv_shapes, default=None,
+                    help="NxK[,NxK...]: the GEMV leg's shapes instead of its default sweep")
     ap.add_argument("--no-batched", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--no-search", action="store_true")
@@ -1038,7 +1055,7 @@ def main():
 
     gemv = None
     if not args.no_gemv:
-        gemv = {"metric": GEMV_METRIC, "shapes": gemv_sweep(torch, nslm, synth, dev, hbm),
+        gemv = {"metric": GEMV_METRIC, "shapes": gemv_sweep(torch, nslm, synth, dev, hbm, args.gemv_shapes),
                 "note": "batch 1, each shape timed over rotating copies (> 4x L2) in a CUDA graph (cold, HBM); "
                         "fields_ready_*: the same chain through nslm_seed_gemv_flags(NSLM_GEMV_FIELDS_READY); "
                         "warm_L2_*: one copy repeated, L2-resident; pct_of_nominal_8TBs: of the nominal 8 TB/s"}

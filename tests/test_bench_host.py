@@ -105,3 +105,15 @@ def test_layer_record_holds_only_for_the_sources_it_names(tmp_path):
     r = bench.layer_record(str(stale))
     assert r["matches"] is False and r["warp_instructions_per_layer_call"] is None
     assert bench.layer_record(str(tmp_path / "missing.txt"))["matches"] is False
+
+
+def test_gemv_shapes_option_parses_and_rejects():
+    import argparse
+
+    import pytest
+
+    assert bench._gemv_shapes("8192x8192") == [(8192, 8192)]
+    assert bench._gemv_shapes("2048X4096,1408x2048") == [(2048, 4096), (1408, 2048)]
+    for bad in ("0x64", "16x12", "16x0", "16"):
+        with pytest.raises((argparse.ArgumentTypeError, ValueError)):
+            bench._gemv_shapes(bad)
