@@ -7,6 +7,7 @@
 // loops over row groups (grid-stride), so the activations are staged into
 // shared memory once per CTA.  Partial sums of the chunks of a row are added
 // in shared memory (fixed order, so results are deterministic).
+#include <type_traits>
 #include <algorithm>
 
 #include "chunk.cuh"
@@ -135,16 +136,23 @@ static int32_t dispatch_gemv(const GemvParams &p, bool vec, int grid, int thread
 // per-thread shared-memory slots) and has no barrier between tasks.  A CTA
 // owns a range of rows; its threads take (row, chunk) tasks, partial sums go
 // to shared memory and one warp per row adds them in a fixed order.
-// The rows are split over two CTAs per SM of at most 14 warps (up to 72
-// registers each): two smaller CTAs end at different times, so the next
-// GEMV's CTAs (launched early by programmatic dependent launch) take an SM's
-// free slot sooner, and the unrolled block loop gets the registers to overlap
-// its table lookups.  Measured on B200, 2048x4096 P=4 in a chain of GEMVs with
-// NSLM_GEMV_FIELDS_READY: 5.07 us with one CTA of up to 32 warps per SM, 4.69
-// with two; 3.25 -> 2.71 us at 512x1024.
+// CTAS = 2: the rows are split over two CTAs per SM of at most 14 warps (up
+// to 72 registers each).  Two smaller CTAs end at different times, so the
+// next GEMV's CTAs (launched early by programmatic dependent launch) take an
+// SM's free slot sooner, and the unrolled block loop gets the registers to
+// overlap its table lookups.  Measured on B200 in a chain of GEMVs with
+// NSLM_GEMV_FIELDS_READY: 2048x4096 P=4 5.07 us with one CTA of up to 32
+// warps per SM, 4.69 with two; 512x1024 3.25 -> 2.71 us.
+// CTAS = 1: one CTA of up to 32 warps (48 registers) per SM, for rows so long
+// that two CTAs' shared memory does not fit on an SM; there the extra warps
+// pay (2048x16384 P=4: 14.9 us against 15.3 with 14 warps, P=3 with 5-bit
+// coefficients 15.6 against 17.4).
 
-constexpr int kGemv1Threads = 448;   // at most; a CTA's (row, chunk) tasks in as few rounds as fit
-constexpr int kGemv1CtasPerSm = 2;   // CTAs per SM the row split and the register budget plan for
+template <int CTAS> struct Gemv1Shape;
+template <> struct Gemv1Shape<2> { static constexpr int kThreads = 448, kMinCtas = 2; };
+template <> struct Gemv1Shape<1> { static constexpr int kThreads = 1024, kMinCtas = 0; };  // 0: no minimum
+constexpr size_t kSmemPerSm = 228 * 1024;     // shared memory of one B200 SM
+constexpr size_t kSmemReservedPerCta = 1024;  // of which the system takes per resident CTA
 
 struct Gemv1Params {
   nslm_seed_matrix W;
@@ -159,8 +167,8 @@ struct Gemv1Params {
 // writes the matrix's fields, so the first task's field copies are issued
 // before griddepcontrol.wait and overlap the tail of the preceding kernel;
 // the activations are read, and y written, only after the wait.
-template <int P, bool EARLY>
-__global__ void __launch_bounds__(kGemv1Threads, kGemv1CtasPerSm) gemv1_kernel(const Gemv1Params p) {
+template <int P, bool EARLY, int CTAS>
+__global__ void __launch_bounds__(Gemv1Shape<CTAS>::kThreads, Gemv1Shape<CTAS>::kMinCtas) gemv1_kernel(const Gemv1Params p) {
   extern __shared__ float4 smem4[];
   const int tid = threadIdx.x, nthr = blockDim.x, warp = tid >> 5, lane = tid & 31;
   StreamTables *tab = reinterpret_cast<StreamTables *>(smem4);
@@ -271,16 +279,31 @@ static int32_t seed_gemv(const nslm_seed_matrix *W, const uint16_t *x_bf16, int3
     q.x = x_bf16;
     q.y = y;
     q.C = W->K / 64;
-    q.rpc = std::max(1, ceil_div(W->N, kGemv1CtasPerSm * sms));
     q.div_C = make_fastdiv((uint32_t)q.C);
-    const int tasks = q.rpc * q.C;
-    const int rounds = ceil_div(tasks, kGemv1Threads);
-    const int threads = std::max(64, 32 * ceil_div(ceil_div(tasks, rounds), 32));
-    const size_t smem = gemv1_smem(q.C, q.rpc, threads);
+    // two CTAs per SM where their shared memory fits on one SM together;
+    // otherwise (long rows) one larger CTA per SM, so that the grid still
+    // runs in one wave
+    int threads = 0, per_sm = 2;
+    size_t smem = 0;
+    for (per_sm = 2; per_sm >= 1; --per_sm) {
+      q.rpc = std::max(1, ceil_div(W->N, per_sm * sms));
+      const int tasks = q.rpc * q.C;
+      const int rounds = ceil_div(tasks, per_sm == 2 ? Gemv1Shape<2>::kThreads : Gemv1Shape<1>::kThreads);
+      threads = std::max(64, 32 * ceil_div(ceil_div(tasks, rounds), 32));
+      smem = gemv1_smem(q.C, q.rpc, threads);
+      if (per_sm == 1 || 2 * (smem + kSmemReservedPerCta) <= kSmemPerSm) break;
+    }
     if (smem <= 200 * 1024 && (int64_t)q.rpc * q.C < (1 << 22)) {
-      auto k = fields_ready
-                   ? ((W->P == 4) ? gemv1_kernel<4, true> : (W->P == kP3C5 ? gemv1_kernel<kP3C5, true> : gemv1_kernel<3, true>))
-                   : ((W->P == 4) ? gemv1_kernel<4, false> : (W->P == kP3C5 ? gemv1_kernel<kP3C5, false> : gemv1_kernel<3, false>));
+      auto pick = [&](auto ctas) {
+        constexpr int C2 = decltype(ctas)::value;
+        return fields_ready ? ((W->P == 4)       ? gemv1_kernel<4, true, C2>
+                               : (W->P == kP3C5) ? gemv1_kernel<kP3C5, true, C2>
+                                                 : gemv1_kernel<3, true, C2>)
+                            : ((W->P == 4)       ? gemv1_kernel<4, false, C2>
+                               : (W->P == kP3C5) ? gemv1_kernel<kP3C5, false, C2>
+                                                 : gemv1_kernel<3, false, C2>);
+      };
+      auto k = per_sm == 2 ? pick(std::integral_constant<int, 2>{}) : pick(std::integral_constant<int, 1>{});
       if ((st = ensure_smem((const void *)k, smem))) return st;
       ensure_stream_source(s);
       cudaLaunchConfig_t cfg{};

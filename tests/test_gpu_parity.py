@@ -113,6 +113,21 @@ def test_gemv_matches_oracle(nslm, P, N, K):
     assert err <= TOL and err <= TIGHT, err
 
 
+@pytest.mark.parametrize("P", [4, 35])
+def test_gemv_long_rows_matches_oracle(nslm, P):
+    # 16,384-weight rows: two CTAs' shared memory no longer fit on one SM, so
+    # the one-vector kernel runs one CTA per SM (eight rounds of tasks each)
+    N, K = 2048, 16384
+    m = synth.seed_matrix(N, K, P, (905, N, K, P))
+    x, xh = _x((905, K), 1, K)
+    y = _out(1, N)
+    nslm.nslm_seed_gemv(_dev(m), x, 1, y)
+    torch.cuda.synchronize()
+    ref = O.seed_matvec(m.numpy(), xh)
+    err = O.normwise_rel_err(y.cpu().numpy(), ref)
+    assert err <= TOL and err <= TIGHT, (err, O.elementwise_rel_err(y.cpu().numpy(), ref))
+
+
 @pytest.mark.parametrize("P", [3, 4, 35])
 def test_gemv_fields_ready_chain_matches_oracle(nslm, P):
     # back-to-back GEMVs with NSLM_GEMV_FIELDS_READY (each one's weight copies
